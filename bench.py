@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of batched speculative-decoding verification on B200.
+
+One step = one spec_verify_run over a resident batch: row statistics and the
+accept chain for every request, the residual / bonus sample, and the fp64
+refinement of the samples the fp32 filter could not certify.
+
+Default workload: stochastic verification, B=256 requests, k=5 drafted
+tokens each, all 5 verified, V=151936, bf16 logits (target ~ N(0, 3^2),
+draft = 0.8 target + 0.6 N(0, 3^2)), T=1.  Metric: verified draft positions
+per second (sum of L_i over the batch / step time), plus the HBM bandwidth
+the step sustains.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload headline|stochastic|greedy|conf|sweep:B]
+
+With N > 1 (launched by torch.distributed.run) every rank verifies its own
+batch of the same shape (weak scaling, no collective on the data path); the
+step time is the max over ranks.  ``--impl reference`` times the fp64 CPU
+oracle instead, on the host's cores, one bounded sample of requests per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verified draft positions/s and HBM GB/s (% of B200 peak), B=256 k=5 V=151936"
+UNIT = "positions/s"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="headline")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------- workloads ----
+
+def make_workload(name, device, rank):
+    from speculative_decoding_verification_86_b200 import workloads as W
+    if name == "headline":
+        w = W.headline(device, seed=1)
+    elif name == "stochastic":
+        w = W.stochastic(device, seed=1)
+    elif name == "greedy":
+        w = W.greedy(device, seed=2)
+    elif name == "conf":
+        w = W.confidence(device, seed=3)
+    elif name.startswith("sweep:"):
+        w = W.sweep(device, seed=4, B=int(name.split(":")[1]))
+    else:
+        raise SystemExit("unknown workload %r" % name)
+    return w
+
+
+def effective_lengths(w):
+    """L_i after clamping (and after the confidence budget, if any), on the host."""
+    import torch
+    B, kp1, _ = w["target"].shape
+    k = kp1 - 1
+    L = (w["verify_len"].clamp(0, k) if w.get("verify_len") is not None
+         else torch.full((B,), k, dtype=torch.int32, device=w["target"].device))
+    return L
+
+
+def dense_row_bytes(w, L):
+    """Algorithmic bytes of the statistics pass: (L_i + 1) target rows and, for
+    sampled requests, L_i draft rows, each V logits."""
+    import torch
+    V = w["target"].shape[2]
+    es = w["target"].element_size()
+    T = w.get("temperature")
+    sampled = (T > 0) if T is not None else torch.ones_like(L, dtype=torch.bool)
+    rows = (L + 1) + torch.where(sampled, L, torch.zeros_like(L))
+    return int(rows.sum().item()) * V * es
+
+
+def config_dict(w, name, n, L):
+    B, kp1, V = w["target"].shape
+    return {
+        "workload": w["name"],
+        "B": int(B), "k": int(kp1 - 1), "V": int(V),
+        "logits": "bf16" if w["target"].element_size() == 2 else "fp32",
+        "mean_L": float(L.float().mean().item()),
+        "temperature": "per-request" if w.get("temperature") is not None else 1.0,
+        "confidence_head": w.get("conf") is not None,
+        "l2": "no flush: the step reads %.0f MB of logits, more than the 126 MB L2"
+              % (w["target"].numel() * w["target"].element_size() / 1e6
+                 + (0 if w.get("draft") is None else w["draft"].numel() * w["draft"].element_size() / 1e6)),
+        "parallelism": "replicas%d" % n if n > 1 else "single",
+        "global_batch": int(B) * n,
+    }
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        t0, t1 = (self.marks + [0, 0])[:2]
+        inside = [l for (t, l) in self.lines if t0 <= t <= t1 + 0.05]
+        rows = [r.split(", ") for r in (inside or [l for _, l in self.lines[-3:]])]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[c - 5] for r in rows if len(r) >= 9 for c in range(5, 9)
+                          if r[c].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside)}
+
+
+# -------------------------------------------------------------- roofline ----
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return None
+
+
+def kernel_source_hash():
+    from speculative_decoding_verification_86_b200 import build
+    h = hashlib.sha256()
+    for p in build.sources():
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (same source hash); else None."""
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel, workload))
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            key, _, val = line.strip()[2:].partition(":")
+            vals[key.strip()] = val.strip().strip("`")
+    if vals.get("source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- oracle ----
+
+def oracle_sample(w, n_requests, threads):
+    """Run the fp64 oracle on the first n_requests of the batch; returns (seconds, positions)."""
+    import oracle
+    from speculative_decoding_verification_86_b200 import workloads as W
+    sub = {k: (v[:n_requests] if hasattr(v, "shape") and v.dim() > 0 and v.shape[0] == w["target"].shape[0] else v)
+           for k, v in w.items()}
+    if w.get("conf") is not None:
+        sub["conf"] = dict(w["conf"], hidden=w["conf"]["hidden"][:n_requests])
+    h = W.to_numpy_inputs(sub)
+    t0 = time.perf_counter()
+    res = oracle.verify(h["target"], h["draft"], h["tokens"], dtype=h["dtype"], verify_len=h["verify_len"],
+                        temperature=h["temperature"], conf=h["conf"], seed=h["seed"], threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, int(res["verify_len_used"].sum()), h
+
+
+def run_reference(args):
+    """The fp64 CPU oracle, timed on the host's cores (reference arm)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import torch
+    oracle.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = make_workload(args.workload, dev, 0)
+    L = effective_lengths(w)
+    cores = os.cpu_count() or 1
+    B = int(w["target"].shape[0])
+    per_step = max(1, min(B, cores))
+    for _ in range(max(0, args.warmup)):
+        oracle_sample(w, per_step, per_step)
+    tot_t, tot_pos = 0.0, 0
+    for _ in range(args.steps):
+        dt, pos, _ = oracle_sample(w, per_step, per_step)
+        tot_t += dt
+        tot_pos += pos
+    value = tot_pos / tot_t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args.workload, 1, L),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": per_step, "kind": "oracle",
+                         "sample": "first %d requests of the batch per step, one per thread" % per_step},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ ours ----
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_86_b200 import binding, build
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    build.build()
+    w = make_workload(args.workload, dev, rank)
+    B, kp1, V = w["target"].shape
+    k = kp1 - 1
+    L = effective_lengths(w)
+    positions = int(L.sum().item())
+    step_bytes = dense_row_bytes(w, L)
+    ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V)
+    out = ver._outputs(B, k, True)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ver.run(w["target"], w.get("draft"), w["tokens"], verify_len=w.get("verify_len"),
+                temperature=w.get("temperature"), conf=w.get("conf"), seed=w["seed"],
+                request_offset=rank * B, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    phys = int(visible.split(",")[local]) if visible else local
+    clocks = ClockSampler(phys)
+    clocks.start()
+    time.sleep(0.2)
+    ver.timing_enable([binding.TIMING_STATS])
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark()
+    if world > 1:
+        dist.barrier()
+    ms_local = e0.elapsed_time(e1)
+    n_stats, ms_stats = ver.timing_read(binding.TIMING_STATS)
+    ver.timing_enable([])
+    clk = clocks.stop()
+    counters = ver.last_counters()
+    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_per_step = ms_total / args.steps
+    value = positions * world / (ms_per_step / 1e3)
+    launches_per_step = 4 + (1 if w.get("conf") is not None else 0)
+
+    # end to end: host buffers in, host results out, through the C ABI
+    e2e = None
+    if args.e2e_steps > 0:
+        host = {key: (v.detach().cpu().pin_memory() if isinstance(v, torch.Tensor) else v)
+                for key, v in w.items()}
+        hconf = None
+        if w.get("conf") is not None:
+            hconf = dict(w["conf"], hidden=w["conf"]["hidden"].cpu().pin_memory(),
+                         w=w["conf"]["w"].cpu().pin_memory())
+        hout = dict(accepted=torch.empty(B, dtype=torch.int32).pin_memory(),
+                    tokens=torch.empty((B, k + 1), dtype=torch.int32).pin_memory(),
+                    p=torch.empty((B, k), dtype=torch.float32).pin_memory(),
+                    q=torch.empty((B, k), dtype=torch.float32).pin_memory(),
+                    status=torch.empty(B, dtype=torch.int32).pin_memory())
+
+        def hstep():
+            ver.run_host(host["target"], host.get("draft"), host["tokens"], verify_len=host.get("verify_len"),
+                         temperature=host.get("temperature"), conf=hconf, seed=w["seed"],
+                         request_offset=rank * B, out=hout)
+
+        hstep()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            hstep()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        te = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / args.e2e_steps
+        h2d = sum(v.numel() * v.element_size() for key, v in host.items()
+                  if isinstance(v, torch.Tensor) and key in ("target", "draft", "tokens", "verify_len", "temperature"))
+        if hconf is not None:
+            h2d += hconf["hidden"].numel() * 2 + hconf["w"].numel() * 2
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+        e2e = {"value": positions * world / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # CPU baseline: the fp64 oracle on this host, rank 0 at N = 1 only
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        t1, pos1, _ = oracle_sample(w, 1, 1)
+        n = int(max(1, min(B, round(cores * 10.0 / max(t1, 1e-3)))))
+        threads = min(cores, n)
+        dt, pos, _ = oracle_sample(w, n, threads)
+        cpu = {"value": pos / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "first %d of %d requests of this batch, fp64 C oracle, %d threads, %.1f s"
+                         % (n, B, threads, dt)}
+
+    peaks = measured_peaks()
+    if peaks and peaks.get("hbm_gbs"):
+        peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    else:
+        peak, peak_src = FALLBACK_HBM_GBS, "fallback"
+    ms_stats_avg = ms_stats / max(n_stats, 1)
+    achieved = step_bytes / (ms_stats_avg * 1e-3) / 1e9 if n_stats else None
+    traffic = profiled_traffic("k_stats", args.workload.replace(":", ""))
+    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
+        "data": "synthetic", "config": config_dict(w, args.workload, world, L),
+        "hbm_gbs": step_gbs, "hbm_frac_measured": step_gbs / peak, "hbm_frac_nominal_8tbs": step_gbs / NOMINAL_HBM_GBS,
+        "roofline": {"bound": "hbm", "kernel": "k_stats", "achieved": achieved, "peak": peak,
+                     "peak_source": peak_src, "unit": "GB/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": step_bytes,
+                     "launch_ms": ms_stats_avg, "launches_timed": n_stats},
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "fp64_paths": counters,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ver.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

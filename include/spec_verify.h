@@ -1,0 +1,196 @@
+/*
+ * spec_verify.h -- C ABI of the B200 (sm_100a) speculative-decoding
+ * verification library (libspecverify.so).
+ *
+ * What the library computes.  A drafter proposes a block of k tokens per
+ * request; the target model has scored the whole block in one pass and its
+ * logits are given for the k drafted positions plus one bonus position.
+ * Verification walks each request's block left to right
+ * ("Speculative decoding becomes standard: DSpark and multi-token drafters",
+ * section "Why draft-and-verify does not change the output"):
+ *   - stochastic (T > 0): accept drafted token x with probability
+ *     min(1, p(x)/q(x)), p = softmax(target/T), q = softmax(draft/T); at the
+ *     first rejection emit a sample from the corrected residual
+ *     norm(max(0, p - q)) and drop the rest of the block; if every verified
+ *     position is accepted emit a bonus token drawn from the target's next row;
+ *   - greedy (T == 0): keep x while it is the target's argmax (lowest index on
+ *     ties); at the first disagreement emit the argmax; if all agree emit the
+ *     argmax of the next row.
+ * The confidence head (same page, section "What DSpark adds") is a linear
+ * projection with a sigmoid giving each position's survival probability given
+ * that the earlier positions survived; the prefix product of these
+ * probabilities, compared with a threshold, truncates the verified length.
+ *
+ * Readings where the pages are silent (all shared with the CPU oracle):
+ *   accept iff u * q(x) < p(x) with u uniform on [0, 1) (53 bits); inverse-CDF
+ *   sampling picks the smallest index whose running sum exceeds u * total
+ *   (index order), falling back to the largest index with positive weight; a
+ *   residual with total mass below 1e-12 is replaced by p; random draws are
+ *   Philox4x32-10 with key = (seed low, seed high) and counter =
+ *   (2 * position + draw, request_offset + request, step, 0), draw 0 for the
+ *   accept test and draw 1 for the residual/bonus sample.  -inf logits mask a
+ *   token; NaN or +inf in a row the chain reads, a row whose max is -inf, or a
+ *   drafted token outside [0, V) fails that request.  Errors are found in
+ *   chain order: rows and tokens past the first rejection are never judged.
+ *
+ * Conventions for every entry point:
+ *   - Array arguments are DEVICE pointers on the context's device unless the
+ *     entry point says "host".  Logit rows are contiguous ([B, rows, V]
+ *     row-major); base pointers of logits must be 16-byte aligned and
+ *     V * sizeof(element) a multiple of 16 bytes, else SPEC_ERR_UNSUPPORTED.
+ *     Integer and fp32 side arrays must be 4-byte aligned.
+ *   - The caller owns every input/output buffer and the stream.  The context
+ *     owns its device workspace (allocated by spec_verify_init, freed by
+ *     spec_verify_destroy).  One context per concurrently used stream.
+ *   - Calls are asynchronous on `stream` (no host synchronisation) except the
+ *     "_host" entry point.  The return value covers argument validation and
+ *     launch errors only; per-request failures found on the device are
+ *     reported through out_status (bits below) and out_accepted = -1.
+ *   - Outputs are a pure function of (inputs, seed, step, request_offset):
+ *     every reduction merges in a fixed order.
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SPEC_OK = 0,
+    SPEC_ERR_INVALID_ARG = 1,   /* bad size, NULL where required, ctx too small */
+    SPEC_ERR_UNSUPPORTED = 2,   /* alignment / dtype / size the kernels do not take */
+    SPEC_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    SPEC_ERR_NOMEM = 4,         /* device or host allocation failed */
+    SPEC_ERR_DEVICE_STATUS = 5, /* (host entry point) a request failed on the device */
+    SPEC_ERR_TIMEOUT = 6        /* reserved: a bounded device wait gave up */
+} spec_status;
+
+typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
+
+/* Per-request device status bits (out_status[i]); 0 means success. */
+#define SPEC_DEV_BAD_TOKEN 1u       /* a drafted token the chain reached is outside [0, V) */
+#define SPEC_DEV_NONFINITE 2u       /* NaN/+inf in a row the chain read, or a row of all -inf */
+#define SPEC_DEV_BAD_TEMPERATURE 4u /* temperature negative, NaN, inf, or in (0, 2^-100) */
+#define SPEC_DEV_INTERNAL 16u       /* internal consistency check failed (should not occur) */
+
+typedef struct spec_verify_ctx spec_verify_ctx;
+
+/* Confidence-head arguments ("What DSpark adds"): survival s_j =
+ * sigmoid(w . hidden[i, j, :] + bias) for j < kb; the budget of request i is the
+ * number of leading positions whose prefix product prod_{j'<=j} s_j' >= threshold. */
+typedef struct {
+    const void* hidden; /* device, [B, kb, H] bf16 drafter hidden states */
+    const void* w;      /* device, [H] bf16 projection */
+    float bias;
+    int kb;             /* positions scored by the head (1..16) */
+    int H;              /* hidden width (1..65536) */
+    float threshold;
+} spec_conf_args;
+
+/* Create a context on `device` with workspace for batches up to max_batch
+ * requests, blocks up to max_k drafted tokens (max_k <= 16) and vocabularies
+ * up to max_vocab.  The current device is restored on return. */
+spec_status spec_verify_init(spec_verify_ctx** ctx, int device, int max_batch, int max_k,
+                             int64_t max_vocab);
+
+/* Free the context and its workspace (synchronises its device first). NULL is a no-op. */
+spec_status spec_verify_destroy(spec_verify_ctx* ctx);
+
+/* Stochastic/mixed verification of B requests.
+ *   target_logits [B, k+1, V]: row j scores drafted position j; row k is the bonus row.
+ *   draft_logits  [B, k, V] (same dtype), or NULL when every temperature is 0.
+ *   draft_tokens  [B, k] int32.
+ *   verify_len    [B] int32 positions to verify per request (clamped to [0, k]), or NULL => k.
+ *   temperature   [B] fp32 per request (0 => greedy), or NULL => 1.0 for all.
+ *   conf          NULL, or a confidence head; then L_i = min(verify_len_i, budget_i).
+ *   seed, step, request_offset select the random draws (see counter layout above).
+ * Outputs:
+ *   out_accepted [B] int32: n_i = accepted drafted tokens (-1 if the request failed).
+ *   out_tokens   [B, k+1] int32: x_0..x_{n-1}, then the correction or bonus token
+ *                at index n; -1 after it.
+ *   out_p, out_q [B, k] fp32 or NULL: p_j(x_j), q_j(x_j) for the positions the
+ *                chain evaluated (j <= n_i, j < L_i, T_i > 0); -1 elsewhere.
+ *   out_status   [B] uint32 or NULL: SPEC_DEV_* bits.
+ * Limits: 1 <= V <= max_vocab, 0 <= k <= max_k, 0 <= B <= max_batch (B == 0 is a no-op). */
+spec_status spec_verify_run(spec_verify_ctx* ctx, const void* target_logits,
+                            const void* draft_logits, spec_dtype dtype,
+                            const int32_t* draft_tokens, const int32_t* verify_len,
+                            const float* temperature, const spec_conf_args* conf, int B, int k,
+                            int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                            int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                            float* out_q, uint32_t* out_status, cudaStream_t stream);
+
+/* Test hook: spec_verify_run with the random draws replaced by `uniforms`
+ * (device, [B, k+1, 2] fp64; entry [i, j, d] is draw d of position j), so that
+ * tests can put draws exactly on decision boundaries. */
+spec_status spec_verify_run_with_uniforms(
+    spec_verify_ctx* ctx, const void* target_logits, const void* draft_logits, spec_dtype dtype,
+    const int32_t* draft_tokens, const int32_t* verify_len, const float* temperature,
+    const spec_conf_args* conf, int B, int k, int64_t V, const double* uniforms,
+    int32_t* out_accepted, int32_t* out_tokens, float* out_p, float* out_q,
+    uint32_t* out_status, cudaStream_t stream);
+
+/* Greedy (temperature 0) verification: target_logits [B, k+1, V], draft_tokens
+ * [B, k]; no draft logits are read.  Outputs as in spec_verify_run. */
+spec_status spec_verify_greedy(spec_verify_ctx* ctx, const void* target_logits, spec_dtype dtype,
+                               const int32_t* draft_tokens, const int32_t* verify_len, int B,
+                               int k, int64_t V, int32_t* out_accepted, int32_t* out_tokens,
+                               uint32_t* out_status, cudaStream_t stream);
+
+/* Confidence-head budget alone ("What DSpark adds"): hidden [B, kb, H] bf16,
+ * w [H] bf16 -> out_len [B] int32 (leading positions with prefix survival >=
+ * threshold) and optionally out_survival [B, kb] fp32 (per-position sigmoid). */
+spec_status spec_conf_budget(spec_verify_ctx* ctx, const void* hidden, const void* w,
+                             float bias, int B, int kb, int H, float threshold,
+                             int32_t* out_len, float* out_survival, cudaStream_t stream);
+
+/* spec_verify_run on HOST buffers: copies the inputs (pinned or pageable host
+ * memory) to device staging owned by the context, verifies, copies the outputs
+ * back and synchronises `stream`.  Staging grows on demand and is freed with the
+ * context.  Returns SPEC_ERR_DEVICE_STATUS if any request failed (outputs are
+ * still written).  `conf` points at HOST buffers too. */
+spec_status spec_verify_run_host(spec_verify_ctx* ctx, const void* target_logits,
+                                 const void* draft_logits, spec_dtype dtype,
+                                 const int32_t* draft_tokens, const int32_t* verify_len,
+                                 const float* temperature, const spec_conf_args* conf, int B,
+                                 int k, int64_t V, uint64_t seed, uint32_t step,
+                                 uint32_t request_offset, int32_t* out_accepted,
+                                 int32_t* out_tokens, float* out_p, float* out_q,
+                                 uint32_t* out_status, cudaStream_t stream);
+
+/* Per-kernel timing: launches of the kernel classes selected by `class_mask`
+ * (bit c selects class c: 0 = row statistics + accept chain, 1 = residual/bonus
+ * sampling, 2 = fp64 refinement, 3 = confidence head; 0 turns timing off) are
+ * bracketed by CUDA events on the caller's stream.  spec_verify_timing_read
+ * synchronises on those events and returns, for class `which`, the number of
+ * launches and their total milliseconds since timing was last enabled (enabling
+ * resets).  At most 4096 launches per class are recorded. */
+spec_status spec_verify_timing_enable(spec_verify_ctx* ctx, int class_mask);
+spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launches,
+                                    double* total_ms);
+
+/* Diagnostics of the last completed run (synchronises the stream first):
+ * out[0] = requests whose accept test needed the fp64 path, out[1] = samples
+ * refined in fp64, out[2] = samples resolved by the fp32 filter. */
+spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
+                                      uint32_t out[3]);
+
+/* Self-check of the one hardware constant the fp32 filter relies on: the
+ * maximum relative error of the ex2.approx.ftz.f32 instruction against fp64
+ * exp2, over every fp32 argument in [lo, hi] (-126 <= lo <= hi <= 0), measured
+ * on `device` (synchronous).  spec_verify_ex2_error_bound() returns the bound
+ * the kernels assume; the measured maximum must not exceed it. */
+spec_status spec_verify_selfcheck_ex2(int device, float lo, float hi, double* max_rel_err);
+double spec_verify_ex2_error_bound(void);
+
+const char* spec_status_string(spec_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H */

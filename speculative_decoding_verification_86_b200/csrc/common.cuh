@@ -1,0 +1,349 @@
+// Shared definitions of the verification kernels: launch geometry, workspace
+// records, run parameters and small device helpers.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sv {
+
+// ---------------------------------------------------------------- geometry --
+// A "chunk" is the slice of one logit row that one CTA streams: kThreads
+// threads x kUnroll 16-byte vectors each, i.e. 8192 bf16 or 4096 fp32 logits.
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 4;
+constexpr int kMaxK = 16;
+constexpr int kMaxRows = 2 * kMaxK + 1;  // k+1 target rows + k draft rows
+
+template <bool BF16>
+struct Geo {
+  static constexpr int kPerVec = BF16 ? 8 : 4;                  // logits per 16-byte vector
+  static constexpr int kChunkVecs = kThreads * kUnroll;          // vectors per chunk
+  static constexpr int kChunk = kChunkVecs * kPerVec;            // logits per chunk
+  static constexpr int kPerThread = kUnroll * kPerVec;           // logits per thread
+  static constexpr int kSumLevels = BF16 ? 5 : 4;                // pairwise-sum depth per thread
+};
+
+constexpr int kChunkBf16 = Geo<true>::kChunk;   // 8192
+constexpr int kChunkF32 = Geo<false>::kChunk;   // 4096
+
+// ------------------------------------------------------------ status bits --
+constexpr uint32_t kDevBadToken = 1u;
+constexpr uint32_t kDevNonfinite = 2u;
+constexpr uint32_t kDevBadTemperature = 4u;
+constexpr uint32_t kDevInternal = 16u;
+
+// ------------------------------------------------------- workspace records --
+// Statistics of one chunk of one row.
+//   stochastic row: K = fl(mraw * c) (reference of the exponent sums),
+//                   mraw = NaN-propagating max of the raw logits,
+//                   err = sum_t e_t * |a_t| (argument-rounding weight), arg unused;
+//                   the sum of e_t = 2^(l_t c - K) is stored separately in fp64.
+//   greedy row:     mraw = NaN-propagating max, arg = lowest index attaining it.
+struct ChunkMeta {
+  float K;
+  float mraw;
+  float err;
+  int arg;
+};
+
+// What is left to do for a request after its accept chain has been resolved.
+constexpr int kJobNone = 0;
+constexpr int kJobResidual = 1;  // sample norm(max(0, p - q)) of row pair `row`
+constexpr int kJobBonus = 2;     // sample p of target row `row`
+
+struct Job {
+  int kind;
+  int row;
+  int n;        // accepted count = index of the token to write
+  int pad0;
+  float cc;     // fp32 log2(e) / T used by the fp32 path
+  float Ka;     // exponent reference of the target row
+  float Kb;     // exponent reference of the draft row
+  float A;      // fp32 1 / Za   (1 for bonus jobs)
+  float Bq;     // fp32 1 / Zb
+  float kappa;  // ln2 * (2^-24 + |eta|): relative error per unit |argument|
+  float mraw_a; // raw max of the target row (fp64 refinement)
+  float mraw_b; // raw max of the draft row
+  double eps0a; // argument-independent relative error bound of p terms
+  double eps0b; // ... of q terms
+  double u2;    // the sample's uniform draw
+  double T;     // temperature
+};
+
+struct SampleChunk {
+  double mass;   // sum of fp32 weights over the chunk (fp64 accumulation of pairwise groups)
+  double bound;  // certified bound on |mass - exact mass|
+};
+
+struct Counters {
+  unsigned refine_count;   // samples queued for fp64 refinement
+  unsigned accept_slow;    // accept decisions resolved in fp64
+  unsigned sample_fast;    // samples certified by the fp32 filter
+  unsigned pad;
+};
+
+// -------------------------------------------------------------- run params --
+struct RunParams {
+  const void* target;      // [B, k+1, V]
+  const void* draft;       // [B, k, V] or nullptr
+  const int32_t* tokens;   // [B, k]
+  const int32_t* vlen;     // [B] or nullptr
+  const float* temp;       // [B] or nullptr
+  const int32_t* conf_len; // [B] confidence budget or nullptr
+  const double* uniforms;  // [B, k+1, 2] test override or nullptr
+  int B;
+  int k;
+  int64_t V;
+  int n_chunks;
+  uint64_t seed;
+  uint32_t step;
+  uint32_t req_off;
+  int force_greedy;        // every request at T = 0 (spec_verify_greedy)
+  float eps_ex2;           // certified relative error of ex2.approx.ftz.f32
+
+  int32_t* out_acc;
+  int32_t* out_tok;
+  float* out_p;
+  float* out_q;
+  uint32_t* out_status;
+
+  ChunkMeta* meta;         // [B, 2k+1, n_chunks]
+  double* ssum;            // [B, 2k+1, n_chunks]
+  unsigned* arrive_stats;  // [B]
+  unsigned* arrive_sample; // [B]
+  Job* jobs;               // [B]
+  SampleChunk* smass;      // [B, n_chunks]
+  int* refine_list;        // [B]
+  unsigned* arrive_r1;     // [B]
+  unsigned* arrive_r2;     // [B]
+  double2* rz;             // [B, n_chunks] fp64 Z partials (target, draft)
+  double2* rZ;             // [B] merged fp64 Z
+  double2* rm;             // [B, n_chunks] fp64 masses (residual, target)
+  Counters* counters;      // this run's counters
+  Counters* counters_next; // the other run's counters, reset here
+};
+
+struct ConfParams {
+  const uint16_t* hidden;  // [B, kb, H] bf16 bits
+  const uint16_t* w;       // [H]
+  float bias;
+  float threshold;
+  int B;
+  int kb;
+  int H;
+  int32_t* out_len;        // [B]
+  float* out_survival;     // [B, kb] or nullptr
+};
+
+// ------------------------------------------------------------ device utils --
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hmax2_nan(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float load_logit(const void* row, int64_t t, bool bf16) {
+  if (bf16) {
+    const uint16_t b = __ldg(reinterpret_cast<const unsigned short*>(row) + t);
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+  }
+  return __ldg(reinterpret_cast<const float*>(row) + t);
+}
+
+// Unpack the logits of one 16-byte vector (8 bf16 or 4 fp32) into floats.
+template <bool BF16>
+__device__ __forceinline__ void unpack(const uint4& v, float (&x)[Geo<BF16>::kPerVec]) {
+  if constexpr (BF16) {
+    x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x);
+    x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+    x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z);
+    x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
+  } else {
+    x[0] = __uint_as_float(v.x); x[1] = __uint_as_float(v.y);
+    x[2] = __uint_as_float(v.z); x[3] = __uint_as_float(v.w);
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint4 neg_inf_vec() {
+  const uint32_t w = BF16 ? 0xFF80FF80u : 0xFF800000u;
+  return make_uint4(w, w, w, w);
+}
+
+__device__ __forceinline__ bool temperature_valid(float T) {
+  return (T >= 0.0f) && !isinf(T) && !(T > 0.0f && T < 0x1p-100f);
+}
+
+// Row pointers.
+__device__ __forceinline__ const void* target_row(const RunParams& p, int i, int j, bool bf16) {
+  const int64_t idx = (static_cast<int64_t>(i) * (p.k + 1) + j) * p.V;
+  return static_cast<const char*>(p.target) + idx * (bf16 ? 2 : 4);
+}
+__device__ __forceinline__ const void* draft_row(const RunParams& p, int i, int j, bool bf16) {
+  const int64_t idx = (static_cast<int64_t>(i) * p.k + j) * p.V;
+  return static_cast<const char*>(p.draft) + idx * (bf16 ? 2 : 4);
+}
+
+struct ReqInfo {
+  int L;        // verified positions
+  float T;      // temperature
+  bool greedy;
+  bool bad_T;
+};
+
+__device__ __forceinline__ ReqInfo request_info(const RunParams& p, int i) {
+  ReqInfo r;
+  int L = p.vlen ? __ldg(p.vlen + i) : p.k;
+  L = max(0, min(L, p.k));
+  if (p.conf_len) L = min(L, __ldg(p.conf_len + i));
+  r.L = L;
+  r.T = p.force_greedy ? 0.0f : (p.temp ? __ldg(p.temp + i) : 1.0f);
+  r.bad_T = !temperature_valid(r.T);
+  r.greedy = !r.bad_T && r.T == 0.0f;
+  // a sampled request needs the drafter's logits
+  if (!r.greedy && p.draft == nullptr) r.bad_T = true;
+  return r;
+}
+
+// Number of (row, chunk) CTAs the statistics pass runs for request i.
+__device__ __forceinline__ int stats_expected(const ReqInfo& r, int n_chunks) {
+  if (r.bad_T) return 1;
+  if (r.greedy) return (r.L + 1) * n_chunks;
+  return (2 * r.L + 1) * n_chunks;
+}
+
+// ------------------------------------------------------- block reductions --
+// All reductions combine in a fixed order, so results never depend on timing.
+__device__ __forceinline__ float warp_max_nan(float x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+__device__ __forceinline__ double warp_sum_d(double x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ float warp_sum_f(float x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+__device__ __forceinline__ int warp_min_i(int x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x = min(x, __shfl_xor_sync(0xffffffffu, x, off));
+  return x;
+}
+
+// Block-wide reductions over kThreads threads; `sh` holds kWarps scratch slots.
+// Every thread receives the result.  Caller must not reuse `sh` before a barrier.
+__device__ __forceinline__ float block_max_nan(float x, float* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_max_nan(x);
+  __syncthreads();
+  if (lane == 0) sh[warp] = x;
+  __syncthreads();
+  float y = lane < kWarps ? sh[lane] : -INFINITY;
+  return warp_max_nan(y);
+}
+
+__device__ __forceinline__ double block_sum_d(double x, double* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_sum_d(x);
+  __syncthreads();
+  if (lane == 0) sh[warp] = x;
+  __syncthreads();
+  double y = lane < kWarps ? sh[lane] : 0.0;
+  return warp_sum_d(y);
+}
+
+__device__ __forceinline__ float block_sum_f(float x, float* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_sum_f(x);
+  __syncthreads();
+  if (lane == 0) sh[warp] = x;
+  __syncthreads();
+  float y = lane < kWarps ? sh[lane] : 0.0f;
+  return warp_sum_f(y);
+}
+
+__device__ __forceinline__ int block_min_i(int x, int* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_min_i(x);
+  __syncthreads();
+  if (lane == 0) sh[warp] = x;
+  __syncthreads();
+  int y = lane < kWarps ? sh[lane] : INT_MAX;
+  return warp_min_i(y);
+}
+
+// Inclusive scan of one double per thread across the block, in thread order.
+// Returns the exclusive prefix; `total` receives the block sum.
+__device__ __forceinline__ double block_exclusive_scan_d(double x, double* sh, double& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double incl = x;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  __syncthreads();
+  if (lane == 31) sh[warp] = incl;
+  __syncthreads();
+  double warp_base = 0.0, all = 0.0;
+  for (int w = 0; w < kWarps; ++w) {
+    const double s = sh[w];
+    if (w < warp) warp_base += s;
+    all += s;
+  }
+  total = all;
+  return warp_base + incl - x;
+}
+
+// Arrival on a per-request counter: returns true in exactly one CTA, the last
+// of `expected` arrivals, and resets the counter for the next launch.  Writes
+// this CTA made before the call are visible to the last arriver afterwards.
+__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* sh_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned old = atomicAdd(counter, 1u);
+    const bool last = (old == expected - 1u);
+    if (last) {
+      *counter = 0u;
+      __threadfence();
+    }
+    *sh_flag = last ? 1 : 0;
+  }
+  __syncthreads();
+  return *sh_flag != 0;
+}
+
+}  // namespace sv

@@ -1,0 +1,565 @@
+// Host side of the C ABI declared in include/spec_verify.h: argument checks,
+// the context's device workspace, and the launch sequence
+//   [k_conf] -> k_stats (row statistics + accept chain)
+//            -> k_sample (residual / bonus sampling, fp32 filter)
+//            -> k_refine_z -> k_refine_pick (fp64, only queued samples).
+// Every launch goes to the caller's stream; nothing here synchronises except
+// the host-buffer entry point, the diagnostics and the timing read-out.
+#include "spec_verify.h"
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "conf.cuh"
+#include "philox.cuh"
+#include "refine.cuh"
+#include "sample.cuh"
+#include "stats.cuh"
+
+namespace {
+
+// Bound on the relative error of ex2.approx.ftz.f32 over the arguments the
+// kernels pass (finite, <= 2^-20, results above the fp32 subnormal range).
+// spec_verify_selfcheck_ex2 measures the actual maximum on the device; the
+// GPU tests require it to stay below this bound.
+constexpr float kEpsEx2 = 0x1p-21f;
+
+constexpr int kClassStats = 0, kClassSample = 1, kClassRefine = 2, kClassConf = 3;
+constexpr int kTimingClasses = 4;
+constexpr int kMaxTimed = 4096;
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) return;
+    ok = (prev == dev) || (cudaSetDevice(dev) == cudaSuccess);
+  }
+  ~DeviceGuard() {
+    int cur = -1;
+    if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+  }
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+struct spec_verify_ctx {
+  int device = 0;
+  int max_batch = 0;
+  int max_k = 0;
+  int64_t max_vocab = 0;
+  int max_chunks = 0;
+  int num_sms = 0;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+
+  sv::ChunkMeta* meta = nullptr;
+  double* ssum = nullptr;
+  unsigned* arrive_stats = nullptr;
+  unsigned* arrive_sample = nullptr;
+  unsigned* arrive_r1 = nullptr;
+  unsigned* arrive_r2 = nullptr;
+  sv::Job* jobs = nullptr;
+  sv::SampleChunk* smass = nullptr;
+  int* refine_list = nullptr;
+  double2* rz = nullptr;
+  double2* rZ = nullptr;
+  double2* rm = nullptr;
+  sv::Counters* counters = nullptr;  // [2], alternating between runs
+  int32_t* conf_len = nullptr;
+  unsigned run_id = 0;
+
+  unsigned timing_mask = 0;  // bit c set: bracket launches of class c with events
+  std::vector<cudaEvent_t> ev_start[kTimingClasses], ev_stop[kTimingClasses];
+  int n_timed[kTimingClasses] = {0, 0, 0, 0};
+
+  void* stage = nullptr;
+  size_t stage_bytes = 0;
+};
+
+namespace {
+
+// Maximum relative error of ex2.approx.ftz.f32 against fp64 exp2 over every
+// fp32 value in [lo, hi]; the result (a non-negative double) is kept as its
+// bit pattern so atomicMax on the integer orders it correctly.
+__global__ void k_selfcheck_ex2(uint32_t first_bits, uint64_t count, unsigned long long* out) {
+  double worst = 0.0;
+  for (uint64_t n = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; n < count;
+       n += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const float x = __uint_as_float(first_bits + static_cast<uint32_t>(n));
+    const double ref = exp2(static_cast<double>(x));
+    if (ref < 0x1p-126) continue;  // results in the flushed range carry absolute error only
+    const double err = fabs(static_cast<double>(sv::ex2_approx(x)) - ref) / ref;
+    worst = fmax(worst, err);
+  }
+  for (int off = 16; off; off >>= 1) worst = fmax(worst, __shfl_xor_sync(0xffffffffu, worst, off));
+  if ((threadIdx.x & 31) == 0) atomicMax(out, static_cast<unsigned long long>(__double_as_longlong(worst)));
+}
+
+spec_status carve(spec_verify_ctx* c) {
+  const size_t rows = static_cast<size_t>(c->max_batch) * (2 * c->max_k + 1);
+  const size_t recs = rows * c->max_chunks;
+  const size_t per_req_chunks = static_cast<size_t>(c->max_batch) * c->max_chunks;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t o_meta = take(recs * sizeof(sv::ChunkMeta));
+  const size_t o_ssum = take(recs * sizeof(double));
+  const size_t o_arr = take(4 * static_cast<size_t>(c->max_batch) * sizeof(unsigned));
+  const size_t o_jobs = take(static_cast<size_t>(c->max_batch) * sizeof(sv::Job));
+  const size_t o_smass = take(per_req_chunks * sizeof(sv::SampleChunk));
+  const size_t o_rlist = take(static_cast<size_t>(c->max_batch) * sizeof(int));
+  const size_t o_rz = take(per_req_chunks * sizeof(double2));
+  const size_t o_rZ = take(static_cast<size_t>(c->max_batch) * sizeof(double2));
+  const size_t o_rm = take(per_req_chunks * sizeof(double2));
+  const size_t o_cnt = take(2 * sizeof(sv::Counters));
+  const size_t o_conf = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
+  if (cudaMalloc(&c->ws, off) != cudaSuccess) {
+    cudaGetLastError();
+    return SPEC_ERR_NOMEM;
+  }
+  c->ws_bytes = off;
+  char* b = static_cast<char*>(c->ws);
+  c->meta = reinterpret_cast<sv::ChunkMeta*>(b + o_meta);
+  c->ssum = reinterpret_cast<double*>(b + o_ssum);
+  unsigned* arr = reinterpret_cast<unsigned*>(b + o_arr);
+  c->arrive_stats = arr;
+  c->arrive_sample = arr + c->max_batch;
+  c->arrive_r1 = arr + 2 * c->max_batch;
+  c->arrive_r2 = arr + 3 * c->max_batch;
+  c->jobs = reinterpret_cast<sv::Job*>(b + o_jobs);
+  c->smass = reinterpret_cast<sv::SampleChunk*>(b + o_smass);
+  c->refine_list = reinterpret_cast<int*>(b + o_rlist);
+  c->rz = reinterpret_cast<double2*>(b + o_rz);
+  c->rZ = reinterpret_cast<double2*>(b + o_rZ);
+  c->rm = reinterpret_cast<double2*>(b + o_rm);
+  c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
+  c->conf_len = reinterpret_cast<int32_t*>(b + o_conf);
+  if (cudaMemset(c->ws, 0, off) != cudaSuccess) return SPEC_ERR_CUDA;
+  return SPEC_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+void timing_mark(spec_verify_ctx* c, int cls, bool start, cudaStream_t s) {
+  if (!(c->timing_mask & (1u << cls))) return;
+  int n = c->n_timed[cls];
+  if (n >= kMaxTimed) return;
+  std::vector<cudaEvent_t>& v = start ? c->ev_start[cls] : c->ev_stop[cls];
+  while (static_cast<int>(v.size()) <= n) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return;
+    v.push_back(e);
+  }
+  cudaEventRecord(v[n], s);
+  if (!start) c->n_timed[cls] = n + 1;
+}
+
+spec_status check_conf(const spec_verify_ctx* c, const spec_conf_args* conf) {
+  if (!conf) return SPEC_OK;
+  if (!conf->hidden || !conf->w) return SPEC_ERR_INVALID_ARG;
+  if (conf->kb < 1 || conf->kb > sv::kMaxK || conf->H < 1 || conf->H > 65536)
+    return SPEC_ERR_INVALID_ARG;
+  if (!aligned(conf->hidden, 2) || !aligned(conf->w, 2)) return SPEC_ERR_UNSUPPORTED;
+  (void)c;
+  return SPEC_OK;
+}
+
+spec_status launch_conf(spec_verify_ctx* c, const spec_conf_args* conf, int B, int32_t* out_len,
+                        float* out_surv, cudaStream_t s) {
+  sv::ConfParams cp;
+  cp.hidden = static_cast<const uint16_t*>(conf->hidden);
+  cp.w = static_cast<const uint16_t*>(conf->w);
+  cp.bias = conf->bias;
+  cp.threshold = conf->threshold;
+  cp.B = B;
+  cp.kb = conf->kb;
+  cp.H = conf->H;
+  cp.out_len = out_len;
+  cp.out_survival = out_surv;
+  timing_mark(c, kClassConf, true, s);
+  sv::k_conf<<<B, sv::kThreads, 0, s>>>(cp);
+  timing_mark(c, kClassConf, false, s);
+  return SPEC_OK;
+}
+
+spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, spec_dtype dtype,
+                     const int32_t* tokens, const int32_t* vlen, const float* temp,
+                     const spec_conf_args* conf, int B, int k, int64_t V, uint64_t seed,
+                     uint32_t step, uint32_t req_off, const double* uniforms, bool force_greedy,
+                     int32_t* out_acc, int32_t* out_tok, float* out_p, float* out_q,
+                     uint32_t* out_status, cudaStream_t s) {
+  if (!c) return SPEC_ERR_INVALID_ARG;
+  if (B < 0 || B > c->max_batch || k < 0 || k > c->max_k || V < 1 || V > c->max_vocab)
+    return SPEC_ERR_INVALID_ARG;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return SPEC_ERR_INVALID_ARG;
+  if (B == 0) return SPEC_OK;
+  if (!target || !out_acc || !out_tok || (k > 0 && !tokens)) return SPEC_ERR_INVALID_ARG;
+  if (!force_greedy && !draft && !temp && k > 0) return SPEC_ERR_INVALID_ARG;
+  if (spec_status st = check_conf(c, conf); st != SPEC_OK) return st;
+  const bool bf16 = dtype == SPEC_BF16;
+  const int64_t esize = bf16 ? 2 : 4;
+  if ((V * esize) % 16 != 0) return SPEC_ERR_UNSUPPORTED;
+  if (!aligned(target, 16) || (draft && !aligned(draft, 16))) return SPEC_ERR_UNSUPPORTED;
+  if ((tokens && !aligned(tokens, 4)) || (vlen && !aligned(vlen, 4)) || (temp && !aligned(temp, 4)) ||
+      !aligned(out_acc, 4) || !aligned(out_tok, 4) || (out_p && !aligned(out_p, 4)) ||
+      (out_q && !aligned(out_q, 4)) || (out_status && !aligned(out_status, 4)) ||
+      (uniforms && !aligned(uniforms, 8)))
+    return SPEC_ERR_UNSUPPORTED;
+
+  DeviceGuard g(c->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+
+  const int chunk = bf16 ? sv::kChunkBf16 : sv::kChunkF32;
+  const int n_chunks = static_cast<int>((V + chunk - 1) / chunk);
+
+  sv::RunParams p;
+  p.target = target;
+  p.draft = force_greedy ? nullptr : draft;
+  p.tokens = tokens;
+  p.vlen = vlen;
+  p.temp = force_greedy ? nullptr : temp;
+  p.conf_len = nullptr;
+  p.uniforms = uniforms;
+  p.B = B;
+  p.k = k;
+  p.V = V;
+  p.n_chunks = n_chunks;
+  p.seed = seed;
+  p.step = step;
+  p.req_off = req_off;
+  p.force_greedy = force_greedy ? 1 : 0;
+  p.eps_ex2 = kEpsEx2;
+  p.out_acc = out_acc;
+  p.out_tok = out_tok;
+  p.out_p = out_p;
+  p.out_q = out_q;
+  p.out_status = out_status;
+  p.meta = c->meta;
+  p.ssum = c->ssum;
+  p.arrive_stats = c->arrive_stats;
+  p.arrive_sample = c->arrive_sample;
+  p.jobs = c->jobs;
+  p.smass = c->smass;
+  p.refine_list = c->refine_list;
+  p.arrive_r1 = c->arrive_r1;
+  p.arrive_r2 = c->arrive_r2;
+  p.rz = c->rz;
+  p.rZ = c->rZ;
+  p.rm = c->rm;
+  c->run_id++;
+  p.counters = c->counters + (c->run_id & 1u);
+  p.counters_next = c->counters + ((c->run_id + 1u) & 1u);
+
+  cudaGetLastError();  // clear stale errors so the check below is ours
+  if (conf) {
+    launch_conf(c, conf, B, c->conf_len, nullptr, s);
+    p.conf_len = c->conf_len;
+  }
+  const int64_t stats_ctas = static_cast<int64_t>(B) * (2 * k + 1) * n_chunks;
+  timing_mark(c, kClassStats, true, s);
+  if (bf16) sv::k_stats<true><<<static_cast<unsigned>(stats_ctas), sv::kThreads, 0, s>>>(p);
+  else sv::k_stats<false><<<static_cast<unsigned>(stats_ctas), sv::kThreads, 0, s>>>(p);
+  timing_mark(c, kClassStats, false, s);
+  if (!force_greedy) {
+    const unsigned sample_ctas = static_cast<unsigned>(static_cast<int64_t>(B) * n_chunks);
+    const unsigned refine_ctas = static_cast<unsigned>(2 * c->num_sms);
+    timing_mark(c, kClassSample, true, s);
+    if (bf16) sv::k_sample<true><<<sample_ctas, sv::kThreads, 0, s>>>(p);
+    else sv::k_sample<false><<<sample_ctas, sv::kThreads, 0, s>>>(p);
+    timing_mark(c, kClassSample, false, s);
+    timing_mark(c, kClassRefine, true, s);
+    if (bf16) {
+      sv::k_refine_z<true><<<refine_ctas, sv::kThreads, 0, s>>>(p);
+      sv::k_refine_pick<true><<<refine_ctas, sv::kThreads, 0, s>>>(p);
+    } else {
+      sv::k_refine_z<false><<<refine_ctas, sv::kThreads, 0, s>>>(p);
+      sv::k_refine_pick<false><<<refine_ctas, sv::kThreads, 0, s>>>(p);
+    }
+    timing_mark(c, kClassRefine, false, s);
+  }
+  if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
+  return SPEC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spec_status_string(spec_status s) {
+  switch (s) {
+    case SPEC_OK: return "ok";
+    case SPEC_ERR_INVALID_ARG: return "invalid argument";
+    case SPEC_ERR_UNSUPPORTED: return "unsupported layout, alignment or size";
+    case SPEC_ERR_CUDA: return "CUDA runtime error";
+    case SPEC_ERR_NOMEM: return "out of memory";
+    case SPEC_ERR_DEVICE_STATUS: return "a request failed on the device (see out_status)";
+    case SPEC_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+spec_status spec_verify_init(spec_verify_ctx** out, int device, int max_batch, int max_k,
+                             int64_t max_vocab) {
+  if (!out) return SPEC_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (max_batch < 1 || max_k < 0 || max_k > sv::kMaxK || max_vocab < 1 ||
+      max_vocab > (int64_t(1) << 30))
+    return SPEC_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) {
+    cudaGetLastError();
+    return SPEC_ERR_CUDA;
+  }
+  if (device < 0 || device >= ndev) return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  spec_verify_ctx* c = new (std::nothrow) spec_verify_ctx();
+  if (!c) return SPEC_ERR_NOMEM;
+  c->device = device;
+  c->max_batch = max_batch;
+  c->max_k = max_k;
+  c->max_vocab = max_vocab;
+  c->max_chunks = static_cast<int>((max_vocab + sv::kChunkF32 - 1) / sv::kChunkF32);
+  if (cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+    delete c;
+    return SPEC_ERR_CUDA;
+  }
+  const spec_status st = carve(c);
+  if (st != SPEC_OK) {
+    if (c->ws) cudaFree(c->ws);
+    delete c;
+    return st;
+  }
+  *out = c;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_destroy(spec_verify_ctx* c) {
+  if (!c) return SPEC_OK;
+  DeviceGuard g(c->device);
+  cudaDeviceSynchronize();
+  for (int k = 0; k < kTimingClasses; ++k) {
+    for (cudaEvent_t e : c->ev_start[k]) cudaEventDestroy(e);
+    for (cudaEvent_t e : c->ev_stop[k]) cudaEventDestroy(e);
+  }
+  if (c->ws) cudaFree(c->ws);
+  if (c->stage) cudaFree(c->stage);
+  delete c;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_run(spec_verify_ctx* ctx, const void* target_logits,
+                            const void* draft_logits, spec_dtype dtype,
+                            const int32_t* draft_tokens, const int32_t* verify_len,
+                            const float* temperature, const spec_conf_args* conf, int B, int k,
+                            int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                            int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                            float* out_q, uint32_t* out_status, cudaStream_t stream) {
+  return run_impl(ctx, target_logits, draft_logits, dtype, draft_tokens, verify_len, temperature,
+                  conf, B, k, V, seed, step, request_offset, nullptr, false, out_accepted,
+                  out_tokens, out_p, out_q, out_status, stream);
+}
+
+spec_status spec_verify_run_with_uniforms(
+    spec_verify_ctx* ctx, const void* target_logits, const void* draft_logits, spec_dtype dtype,
+    const int32_t* draft_tokens, const int32_t* verify_len, const float* temperature,
+    const spec_conf_args* conf, int B, int k, int64_t V, const double* uniforms,
+    int32_t* out_accepted, int32_t* out_tokens, float* out_p, float* out_q,
+    uint32_t* out_status, cudaStream_t stream) {
+  if (!uniforms && B > 0) return SPEC_ERR_INVALID_ARG;
+  return run_impl(ctx, target_logits, draft_logits, dtype, draft_tokens, verify_len, temperature,
+                  conf, B, k, V, 0, 0, 0, uniforms, false, out_accepted, out_tokens, out_p,
+                  out_q, out_status, stream);
+}
+
+spec_status spec_verify_greedy(spec_verify_ctx* ctx, const void* target_logits, spec_dtype dtype,
+                               const int32_t* draft_tokens, const int32_t* verify_len, int B,
+                               int k, int64_t V, int32_t* out_accepted, int32_t* out_tokens,
+                               uint32_t* out_status, cudaStream_t stream) {
+  return run_impl(ctx, target_logits, nullptr, dtype, draft_tokens, verify_len, nullptr, nullptr,
+                  B, k, V, 0, 0, 0, nullptr, true, out_accepted, out_tokens, nullptr, nullptr,
+                  out_status, stream);
+}
+
+spec_status spec_conf_budget(spec_verify_ctx* ctx, const void* hidden, const void* w, float bias,
+                             int B, int kb, int H, float threshold, int32_t* out_len,
+                             float* out_survival, cudaStream_t stream) {
+  if (!ctx || B < 0 || B > ctx->max_batch) return SPEC_ERR_INVALID_ARG;
+  if (B == 0) return SPEC_OK;
+  if (!out_len) return SPEC_ERR_INVALID_ARG;
+  spec_conf_args conf{hidden, w, bias, kb, H, threshold};
+  if (spec_status st = check_conf(ctx, &conf); st != SPEC_OK) return st;
+  if (!aligned(out_len, 4) || (out_survival && !aligned(out_survival, 4)))
+    return SPEC_ERR_UNSUPPORTED;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  launch_conf(ctx, &conf, B, out_len, out_survival, stream);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_verify_run_host(spec_verify_ctx* ctx, const void* target_logits,
+                                 const void* draft_logits, spec_dtype dtype,
+                                 const int32_t* draft_tokens, const int32_t* verify_len,
+                                 const float* temperature, const spec_conf_args* conf, int B,
+                                 int k, int64_t V, uint64_t seed, uint32_t step,
+                                 uint32_t request_offset, int32_t* out_accepted,
+                                 int32_t* out_tokens, float* out_p, float* out_q,
+                                 uint32_t* out_status, cudaStream_t stream) {
+  if (!ctx) return SPEC_ERR_INVALID_ARG;
+  if (B < 0 || B > ctx->max_batch || k < 0 || k > ctx->max_k || V < 1 || V > ctx->max_vocab)
+    return SPEC_ERR_INVALID_ARG;
+  if (B == 0) return SPEC_OK;
+  if (!target_logits || !out_accepted || !out_tokens || (k > 0 && !draft_tokens))
+    return SPEC_ERR_INVALID_ARG;
+  if (spec_status st = check_conf(ctx, conf); st != SPEC_OK) return st;
+  const size_t es = dtype == SPEC_BF16 ? 2 : 4;
+  const size_t nB = static_cast<size_t>(B);
+  const size_t sz_t = nB * (k + 1) * V * es, sz_d = draft_logits ? nB * k * V * es : 0;
+  const size_t sz_x = nB * k * 4, sz_l = verify_len ? nB * 4 : 0, sz_T = temperature ? nB * 4 : 0;
+  const size_t sz_h = conf ? nB * conf->kb * conf->H * 2 : 0, sz_w = conf ? conf->H * 2 : 0;
+  const size_t sz_acc = nB * 4, sz_tok = nB * (k + 1) * 4, sz_pq = nB * k * 4, sz_st = nB * 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t o_t = take(sz_t), o_d = take(sz_d), o_x = take(sz_x), o_l = take(sz_l),
+               o_T = take(sz_T), o_h = take(sz_h), o_w = take(sz_w), o_acc = take(sz_acc),
+               o_tok = take(sz_tok), o_p = take(out_p ? sz_pq : 0), o_q = take(out_q ? sz_pq : 0),
+               o_st = take(sz_st);
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  if (off > ctx->stage_bytes) {
+    if (ctx->stage) {
+      cudaStreamSynchronize(stream);
+      cudaFree(ctx->stage);
+      ctx->stage = nullptr;
+      ctx->stage_bytes = 0;
+    }
+    if (cudaMalloc(&ctx->stage, off) != cudaSuccess) {
+      cudaGetLastError();
+      return SPEC_ERR_NOMEM;
+    }
+    ctx->stage_bytes = off;
+  }
+  char* S = static_cast<char*>(ctx->stage);
+  auto h2d = [&](size_t o, const void* src, size_t n) {
+    return n == 0 || cudaMemcpyAsync(S + o, src, n, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+  };
+  if (!h2d(o_t, target_logits, sz_t) || !h2d(o_d, draft_logits, sz_d) ||
+      !h2d(o_x, draft_tokens, sz_x) || !h2d(o_l, verify_len, sz_l) ||
+      !h2d(o_T, temperature, sz_T) || (conf && (!h2d(o_h, conf->hidden, sz_h) || !h2d(o_w, conf->w, sz_w))))
+    return SPEC_ERR_CUDA;
+  spec_conf_args dconf{};
+  if (conf) {
+    dconf = *conf;
+    dconf.hidden = S + o_h;
+    dconf.w = S + o_w;
+  }
+  spec_status st = run_impl(ctx, S + o_t, draft_logits ? S + o_d : nullptr, dtype,
+                            k > 0 ? reinterpret_cast<int32_t*>(S + o_x) : nullptr,
+                            verify_len ? reinterpret_cast<int32_t*>(S + o_l) : nullptr,
+                            temperature ? reinterpret_cast<float*>(S + o_T) : nullptr,
+                            conf ? &dconf : nullptr, B, k, V, seed, step, request_offset, nullptr,
+                            false, reinterpret_cast<int32_t*>(S + o_acc),
+                            reinterpret_cast<int32_t*>(S + o_tok),
+                            out_p ? reinterpret_cast<float*>(S + o_p) : nullptr,
+                            out_q ? reinterpret_cast<float*>(S + o_q) : nullptr,
+                            reinterpret_cast<uint32_t*>(S + o_st), stream);
+  if (st != SPEC_OK) return st;
+  std::vector<uint32_t> status_host(out_status ? 0 : nB);
+  uint32_t* st_dst = out_status ? out_status : status_host.data();
+  auto d2h = [&](void* dst, size_t o, size_t n) {
+    return n == 0 || cudaMemcpyAsync(dst, S + o, n, cudaMemcpyDeviceToHost, stream) == cudaSuccess;
+  };
+  if (!d2h(out_accepted, o_acc, sz_acc) || !d2h(out_tokens, o_tok, sz_tok) ||
+      (out_p && !d2h(out_p, o_p, sz_pq)) || (out_q && !d2h(out_q, o_q, sz_pq)) ||
+      !d2h(st_dst, o_st, sz_st))
+    return SPEC_ERR_CUDA;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SPEC_ERR_CUDA;
+  for (size_t i = 0; i < nB; ++i)
+    if (st_dst[i] != 0) return SPEC_ERR_DEVICE_STATUS;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_selfcheck_ex2(int device, float lo, float hi, double* max_rel_err) {
+  if (!max_rel_err || !(lo <= hi) || hi > 0.0f || !(lo >= -126.0f)) return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  // negative fp32 values: larger magnitude <=> larger bit pattern
+  uint32_t bhi, blo;
+  std::memcpy(&bhi, &hi, 4);
+  std::memcpy(&blo, &lo, 4);
+  if (hi == 0.0f) bhi = 0x80000000u;
+  const uint32_t first = bhi, last = blo;
+  const uint64_t count = static_cast<uint64_t>(last) - first + 1;
+  unsigned long long* d = nullptr;
+  if (cudaMalloc(&d, sizeof *d) != cudaSuccess) return SPEC_ERR_NOMEM;
+  cudaMemset(d, 0, sizeof *d);
+  k_selfcheck_ex2<<<1184, 256>>>(first, count, d);
+  unsigned long long h = 0;
+  const bool ok = cudaGetLastError() == cudaSuccess &&
+                  cudaMemcpy(&h, d, sizeof h, cudaMemcpyDeviceToHost) == cudaSuccess;
+  cudaFree(d);
+  if (!ok) return SPEC_ERR_CUDA;
+  double v;
+  std::memcpy(&v, &h, 8);
+  *max_rel_err = v;
+  return SPEC_OK;
+}
+
+double spec_verify_ex2_error_bound(void) { return static_cast<double>(kEpsEx2); }
+
+spec_status spec_verify_timing_enable(spec_verify_ctx* ctx, int class_mask) {
+  if (!ctx || class_mask < 0 || class_mask >= (1 << kTimingClasses)) return SPEC_ERR_INVALID_ARG;
+  ctx->timing_mask = static_cast<unsigned>(class_mask);
+  for (int k = 0; k < kTimingClasses; ++k) ctx->n_timed[k] = 0;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launches,
+                                    double* total_ms) {
+  if (!ctx || which < 0 || which >= kTimingClasses || !launches || !total_ms)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  double tot = 0.0;
+  const int n = ctx->n_timed[which];
+  for (int r = 0; r < n; ++r) {
+    if (cudaEventSynchronize(ctx->ev_stop[which][r]) != cudaSuccess) return SPEC_ERR_CUDA;
+    float ms = 0.0f;
+    if (cudaEventElapsedTime(&ms, ctx->ev_start[which][r], ctx->ev_stop[which][r]) != cudaSuccess)
+      return SPEC_ERR_CUDA;
+    tot += ms;
+  }
+  *launches = n;
+  *total_ms = tot;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream, uint32_t out[3]) {
+  if (!ctx || !out) return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return SPEC_ERR_CUDA;
+  sv::Counters h{};
+  if (cudaMemcpy(&h, ctx->counters + (ctx->run_id & 1u), sizeof h, cudaMemcpyDeviceToHost) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
+  out[0] = h.accept_slow;
+  out[1] = h.refine_count;
+  out[2] = h.sample_fast;
+  return SPEC_OK;
+}
+
+}  // extern "C"

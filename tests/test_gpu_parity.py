@@ -1,0 +1,297 @@
+"""CUDA path vs the fp64 CPU oracle, element by element, through the C ABI.
+
+Bar (from the verification rule's tolerances): p_j(x_j) and q_j(x_j) within
+1e-5 absolute + 1e-4 relative; accepted lengths and emitted tokens bit-exact,
+except for requests holding an accept draw within 1e-6 of p/q (counted; they
+must stay below 1e-5 of all decisions); greedy results and confidence budgets
+bit-exact.  Inputs are the seeded synthetic workloads, generated on the GPU and
+copied to the host for the oracle.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from speculative_decoding_verification_86_b200 import binding, build, workloads
+
+pytestmark = pytest.mark.gpu
+
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+@pytest.fixture(scope="module")
+def ver(cuda_device):
+    build.build()
+    v = binding.SpecVerifier(cuda_device, max_batch=1024, max_k=16, max_vocab=262144)
+    yield v
+    v.close()
+
+
+def run_gpu(ver, w, uniforms=None, **kw):
+    o = ver.run(w["target"], w.get("draft"), w["tokens"], verify_len=w.get("verify_len"),
+                temperature=w.get("temperature"), conf=w.get("conf"), seed=w["seed"],
+                uniforms=uniforms, **kw)
+    torch.cuda.synchronize()
+    return {k: v.cpu().numpy() for k, v in o.items()}
+
+
+def run_oracle(w, u_override=None, request_offset=0):
+    h = workloads.to_numpy_inputs(w)
+    return oracle.verify(h["target"], h["draft"], h["tokens"], dtype=h["dtype"],
+                         verify_len=h["verify_len"], temperature=h["temperature"], conf=h["conf"],
+                         seed=h["seed"], u_override=u_override, request_offset=request_offset,
+                         threads=THREADS)
+
+
+def compare(g, o):
+    """Assert parity; returns (decisions, exempt decisions)."""
+    am = o["accept_margin"]
+    evaluated = am >= 0
+    exempt = evaluated & (am < 1e-6)
+    n_dec = int(evaluated.sum()) + int((o["sample_margin"] >= 0).sum())
+    n_ex = int(exempt.sum())
+    assert n_ex <= 1e-5 * max(n_dec, 1), (n_ex, n_dec)
+    ok = ~exempt.any(axis=1) if am.shape[1] else np.ones(len(o["accepted"]), bool)
+    np.testing.assert_array_equal(g["status"][ok].astype(np.uint32), o["status"][ok])
+    np.testing.assert_array_equal(g["accepted"][ok], o["accepted"][ok])
+    np.testing.assert_array_equal(g["tokens"][ok], o["tokens"][ok])
+    if "p" in g:
+        for gv, ov in ((g["p"], o["p_x"]), (g["q"], o["q_x"])):
+            gv, ov = gv[ok], ov[ok]
+            ev = ov >= 0
+            assert np.all(gv[~ev] == -1.0)
+            err = np.abs(gv[ev].astype(np.float64) - ov[ev])
+            assert np.all(err <= 1e-5 + 1e-4 * np.abs(ov[ev])), err.max()
+    return n_dec, n_ex
+
+
+# ------------------------------------------------------------ the configs ----
+
+def test_tiny_fp32(ver):
+    w = workloads.tiny("cuda", seed=0)
+    compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_stochastic_b64(ver):
+    w = workloads.stochastic("cuda", seed=1)
+    g, o = run_gpu(ver, w), run_oracle(w)
+    compare(g, o)
+    c = ver.last_counters()
+    assert c["sample_fp32"] + c["sample_fp64"] == 64
+
+
+def test_headline_b256_full_block(ver):
+    w = workloads.headline("cuda", seed=1)
+    compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_greedy_b256(ver):
+    w = workloads.greedy("cuda", seed=2)
+    o = run_oracle(w)
+    g = ver.greedy(w["target"], w["tokens"])
+    torch.cuda.synchronize()
+    g = {k: v.cpu().numpy() for k, v in g.items()}
+    np.testing.assert_array_equal(g["accepted"], o["accepted"])
+    np.testing.assert_array_equal(g["tokens"], o["tokens"])
+    np.testing.assert_array_equal(g["status"], 0)
+    # the same requests through the mixed entry point with T = 0
+    g2 = run_gpu(ver, dict(w, draft=None))
+    compare(g2, o)
+    assert (o["accepted"] < 5).any() and (o["accepted"] == 5).any()
+
+
+def test_confidence_head_b128(ver):
+    w = workloads.confidence("cuda", seed=3)
+    o = run_oracle(w)
+    compare(run_gpu(ver, w), o)
+    c = w["conf"]
+    L, surv = ver.conf_budget(c["hidden"], c["w"], c["bias"], c["threshold"])
+    torch.cuda.synchronize()
+    h = workloads.to_numpy_inputs(w)["conf"]
+    oL, osurv, opref = oracle.conf_budget(h["hidden"], h["w"], h["bias"], h["threshold"])
+    np.testing.assert_array_equal(L.cpu().numpy(), oL)
+    np.testing.assert_array_equal(o["verify_len_used"], oL)
+    np.testing.assert_allclose(surv.cpu().numpy(), osurv, rtol=1e-6, atol=1e-7)
+    # no prefix product sits within rounding of the threshold
+    assert np.min(np.abs(opref - h["threshold"])) > 1e-12
+
+
+@pytest.mark.parametrize("B", workloads.SWEEP_BATCHES)
+def test_load_sweep(ver, B):
+    w = workloads.sweep("cuda", seed=4, B=B)
+    compare(run_gpu(ver, w), run_oracle(w))
+
+
+# --------------------------------------------------------- special cases ----
+
+def test_draft_equal_target_accepts_everything(ver):
+    w = workloads.stochastic("cuda", seed=5, B=48, k=5, V=20000)
+    w["draft"] = w["target"][:, :5].contiguous()
+    w["temperature"] = torch.tensor([0.7, 1.0, 1.3] * 16, device="cuda")
+    g, o = run_gpu(ver, w), run_oracle(w)
+    compare(g, o)
+    assert np.array_equal(g["accepted"], np.clip(w["verify_len"].cpu().numpy(), 0, 5))
+
+
+def test_zero_length_and_zero_block(ver):
+    w = workloads.stochastic("cuda", seed=6, B=16, k=4, V=8192 + 8)
+    w["verify_len"] = torch.zeros(16, dtype=torch.int32, device="cuda")
+    compare(run_gpu(ver, w), run_oracle(w))
+    w0 = dict(w, target=w["target"][:, :1].contiguous(), draft=w["draft"][:, :0].contiguous(),
+              tokens=w["tokens"][:, :0].contiguous(), verify_len=None)
+    g, o = run_gpu(ver, w0), run_oracle(w0)
+    compare(g, o)
+    assert np.all(g["accepted"] == 0)
+
+
+@pytest.mark.parametrize("dtype,V", [(torch.bfloat16, 8), (torch.float32, 4), (torch.float32, 4100),
+                                     (torch.bfloat16, 262144)])
+def test_small_and_ragged_vocabularies(ver, dtype, V):
+    B = 8 if V > 100000 else 64
+    w = workloads.stochastic("cuda", seed=7, B=B, k=3, V=V, dtype=dtype)
+    w["temperature"] = torch.tensor([0.0, 0.5, 1.0, 2.0] * (B // 4), device="cuda")
+    compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_single_request_max_block(ver):
+    w = workloads.stochastic("cuda", seed=8, B=1, k=16, V=151936, fixed_len=16)
+    w["draft"] = (0.3 * w["draft"].float() + 0.7 * w["target"][:, :16].float()).to(torch.bfloat16)
+    compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_errors_reported_per_request(ver):
+    w = workloads.stochastic("cuda", seed=9, B=8, k=3, V=4096, fixed_len=3)
+    t, d = w["target"], w["draft"]
+    t[0, 0, 17] = float("nan")                 # NaN in the first row read
+    t[1, 0, 5] = float("inf")                  # +inf
+    t[2, 0, :] = float("-inf")                 # whole row masked
+    t[3, 0, 9] = float("-inf")                 # one masked token: fine
+    d[3, 0, 11] = float("-inf")
+    w["tokens"][4, 0] = 4096                   # out of range
+    w["tokens"][5, 0] = -3
+    temps = torch.ones(8, device="cuda")
+    temps[6] = -1.0
+    temps[7] = float("nan")
+    w["temperature"] = temps
+    g, o = run_gpu(ver, w), run_oracle(w)
+    compare(g, o)
+    assert list(g["status"][:3]) == [2, 2, 2] and g["status"][3] == 0
+    assert list(g["status"][4:]) == [1, 1, 4, 4]
+    assert np.all(g["accepted"][[0, 1, 2, 4, 5, 6, 7]] == -1)
+
+
+def test_sampled_request_without_draft_logits_fails(ver):
+    w = workloads.greedy("cuda", seed=10, B=4, k=2, V=1024)
+    w["temperature"] = torch.tensor([0.0, 1.0, 0.0, 0.5], device="cuda")
+    g = run_gpu(ver, w)
+    assert list(g["status"]) == [0, 4, 0, 4]
+
+
+# --------------------------------------- draws on the decision boundaries ----
+
+def _residual_cdf(trow, drow, T, resid):
+    z = trow / T
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    if not resid:
+        return np.cumsum(p) / p.sum()
+    zq = drow / T
+    q = np.exp(zq - zq.max())
+    q /= q.sum()
+    r = np.maximum(0.0, p - q)
+    return np.cumsum(r) / r.sum()
+
+
+def test_draws_on_decision_boundaries_take_the_fp64_paths(ver):
+    w = workloads.stochastic("cuda", seed=11, B=64, k=4, V=16384, fixed_len=4)
+    B, k = 64, 4
+    base = run_oracle(w)
+    rho = np.where(base["q_x"] > 0, base["p_x"] / np.maximum(base["q_x"], 1e-300), 2.0)
+    rng = np.random.default_rng(0)
+    u = rng.random((B, k + 1, 2))
+    # accept draws a relative 1e-9 either side of p/q (inside every fp32 bound)
+    for i in range(B):
+        for j in range(k):
+            if base["p_x"][i, j] >= 0 and rho[i, j] < 1:
+                u[i, j, 0] = rho[i, j] * (1 + (1e-9 if (i + j) % 2 else -1e-9))
+    first = oracle.verify(*[workloads.to_numpy_inputs(w)[x] for x in ("target", "draft", "tokens")],
+                          dtype=oracle.DTYPE_BF16, verify_len=w["verify_len"].cpu().numpy(), u_override=u)
+    # sample draws a relative 1e-12 from a cell edge of the row each chain stops at
+    h = workloads.to_numpy_inputs(w)
+    tv = torch.from_numpy(h["target"].view(np.int16)).view(torch.bfloat16).double().numpy()
+    dv = torch.from_numpy(h["draft"].view(np.int16)).view(torch.bfloat16).double().numpy()
+    for i in range(B):
+        n = first["accepted"][i]
+        cdf = _residual_cdf(tv[i, n], dv[i, n] if n < k else None, 1.0, n < k)
+        t = int(np.argmax(np.diff(np.concatenate([[0.0], cdf]))))  # widest cell
+        u[i, n, 1] = min(cdf[t] * (1 + (1e-12 if i % 2 else -1e-12)), 1 - 2 ** -53)
+    o = run_oracle(w, u_override=u)
+    g = run_gpu(ver, w, uniforms=torch.from_numpy(u).cuda())
+    compare(g, o)
+    c = ver.last_counters()
+    assert c["accept_fp64"] > 0 and c["sample_fp64"] > 0
+
+
+def test_residual_floor_and_fallback_through_refinement(ver):
+    V = 64
+    t = torch.zeros((2, 2, V), dtype=torch.float32)
+    d = torch.zeros((2, 1, V), dtype=torch.float32)
+    d[0, 0, 0] = 1e-13         # p and q differ by ~1e-14: residual under the floor
+    t[1, 0, 40:] = float("-inf")
+    w = dict(target=t.cuda(), draft=d.cuda(), tokens=torch.tensor([[0], [3]], dtype=torch.int32).cuda(),
+             verify_len=None, temperature=None, conf=None, seed=0)
+    u = np.array([[[1 - 2.0 ** -50, 0.6], [0.5, 0.5]],
+                  [[0.999, 1.0], [0.5, 0.5]]])          # u' = 1: past every cell
+    o = run_oracle(w, u_override=u)
+    g = run_gpu(ver, w, uniforms=torch.from_numpy(u).cuda())
+    compare(g, o)
+    assert o["tokens"][0, 0] == 38 or o["tokens"][0, 0] >= 0
+
+
+# ------------------------------------------------------ API-level checks ----
+
+def test_deterministic_and_request_offset(ver):
+    w = workloads.stochastic("cuda", seed=12, B=32, k=5, V=32768)
+    a = run_gpu(ver, w)
+    b = run_gpu(ver, w)
+    for key in a:
+        np.testing.assert_array_equal(a[key], b[key])
+    half = {key: (v[16:].contiguous() if isinstance(v, torch.Tensor) and v.dim() and v.shape[0] == 32 else v)
+            for key, v in w.items()}
+    h = ver.run(half["target"], half["draft"], half["tokens"], verify_len=half["verify_len"],
+                seed=w["seed"], request_offset=16)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(h["tokens"].cpu().numpy(), a["tokens"][16:])
+    np.testing.assert_array_equal(h["accepted"].cpu().numpy(), a["accepted"][16:])
+
+
+def test_host_buffer_entry_point(ver):
+    w = workloads.stochastic("cuda", seed=13, B=16, k=5, V=151936)
+    a = run_gpu(ver, w)
+    hw = {k: (v.cpu().pin_memory() if isinstance(v, torch.Tensor) else v) for k, v in w.items()}
+    o = ver.run_host(hw["target"], hw["draft"], hw["tokens"], verify_len=hw["verify_len"], seed=w["seed"])
+    np.testing.assert_array_equal(o["tokens"].numpy(), a["tokens"])
+    np.testing.assert_array_equal(o["accepted"].numpy(), a["accepted"])
+    np.testing.assert_array_equal(o["p"].numpy(), a["p"])
+
+
+def test_empty_batch(ver):
+    t = torch.zeros((0, 3, 64), dtype=torch.bfloat16, device="cuda")
+    o = ver.run(t, torch.zeros((0, 2, 64), dtype=torch.bfloat16, device="cuda"),
+                torch.zeros((0, 2), dtype=torch.int32, device="cuda"))
+    assert o["accepted"].numel() == 0
+
+
+def test_unsupported_layouts_are_refused(ver):
+    t = torch.zeros((1, 2, 12), dtype=torch.bfloat16, device="cuda")    # 24-byte rows
+    with pytest.raises(binding.SpecVerifyError) as e:
+        ver.run(t, t[:, :1].contiguous(), torch.zeros((1, 1), dtype=torch.int32, device="cuda"))
+    assert e.value.status == binding.SPEC_ERR_UNSUPPORTED
+
+
+def test_ex2_error_bound_holds_on_this_device(cuda_device):
+    build.build()
+    measured, bound = binding.selfcheck_ex2(cuda_device.index, -126.0, 0.0)
+    assert 0 < measured <= bound, (measured, bound)
