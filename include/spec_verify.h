@@ -74,7 +74,8 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 /* Per-request device status bits (out_status[i]); 0 means success. */
 #define SPEC_DEV_BAD_TOKEN 1u       /* a drafted token the chain reached is outside [0, V) */
 #define SPEC_DEV_NONFINITE 2u       /* NaN/+inf in a row the chain read, or a row of all -inf */
-#define SPEC_DEV_BAD_TEMPERATURE 4u /* temperature negative, NaN, inf, or in (0, 2^-100) */
+#define SPEC_DEV_BAD_TEMPERATURE 4u /* temperature negative, NaN, inf, in (0, 2^-100), or
+                                       T > 0 with L_i > 0 but no draft logits */
 #define SPEC_DEV_INTERNAL 16u       /* internal consistency check failed (should not occur) */
 
 typedef struct spec_verify_ctx spec_verify_ctx;

@@ -224,8 +224,8 @@ __device__ __forceinline__ ReqInfo request_info(const RunParams& p, int i) {
   r.T = p.force_greedy ? 0.0f : (p.temp ? __ldg(p.temp + i) : 1.0f);
   r.bad_T = !temperature_valid(r.T);
   r.greedy = !r.bad_T && r.T == 0.0f;
-  // a sampled request needs the drafter's logits
-  if (!r.greedy && p.draft == nullptr) r.bad_T = true;
+  // a sampled request that verifies any position needs the drafter's logits
+  if (!r.bad_T && !r.greedy && r.L > 0 && p.draft == nullptr) r.bad_T = true;
   return r;
 }
 
