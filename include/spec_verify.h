@@ -142,6 +142,31 @@ spec_status spec_verify_greedy(spec_verify_ctx* ctx, const void* target_logits, 
                                int k, int64_t V, int32_t* out_accepted, int32_t* out_tokens,
                                uint32_t* out_status, cudaStream_t stream);
 
+/* Greedy verification that allocates nothing.  The verification rule has no
+ * counterpart for this entry point on the source pages: it exists for callers
+ * that must not allocate device memory -- serving engines that reserve almost
+ * all free GPU memory for their KV cache up front, plugin hosts that only lend
+ * a stream and buffers, or latency-critical paths that cannot afford
+ * cudaMalloc's implicit synchronisation.  It computes exactly what
+ * spec_verify_greedy computes, with the same arguments minus the context; the
+ * current device is used.
+ * Working space: a fixed array inside the library (about 2.3 MB per GPU that
+ * loads it, kept until the process exits).  Limits: 0 <= B <= 256, 0 <= k <= 8,
+ * and B * (2k + 1) * ceil(V / chunk) <= 139264, with chunk = 8192 (bf16) or 4096
+ * (fp32) logits -- V up to 262144 (bf16) / 131072 (fp32) at B = 256, k = 8.
+ * Larger calls return SPEC_ERR_INVALID_ARG without launching anything.
+ * No cudaMalloc/cudaFree is made.  The first call on a device looks up the
+ * array's device address (once per device; make that first call before any
+ * stream capture).  Every call zeroes the array's arrival counters on `stream`
+ * before launching; all calls share the one array, so calls that overlap on the
+ * GPU (other streams, other host threads) race and must be serialised by the
+ * caller. */
+spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dtype,
+                                       const int32_t* draft_tokens, const int32_t* verify_len,
+                                       int B, int k, int64_t V, int32_t* out_accepted,
+                                       int32_t* out_tokens, uint32_t* out_status,
+                                       cudaStream_t stream);
+
 /* Confidence-head budget alone ("What DSpark adds"): hidden [B, kb, H] bf16,
  * w [H] bf16 -> out_len [B] int32 (leading positions with prefix survival >=
  * threshold) and optionally out_survival [B, kb] fp32 (per-position sigmoid). */

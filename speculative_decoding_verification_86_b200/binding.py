@@ -73,6 +73,7 @@ def lib():
     L.spec_verify_run_with_uniforms.argtypes = run_common + [_vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_verify_run_host.argtypes = run_common + [_u64, _u32, _u32, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_verify_greedy.argtypes = [_vp, _vp, _i32, _vp, _vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp]
+    L.spec_verify_greedy_noalloc.argtypes = [_vp, _i32, _vp, _vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp]
     L.spec_conf_budget.argtypes = [_vp, _vp, _vp, ctypes.c_float, _i32, _i32, _i32,
                                    ctypes.c_float, _vp, _vp, _vp]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
@@ -84,7 +85,7 @@ def lib():
     L.spec_verify_ex2_error_bound.restype = ctypes.c_double
     for name in ("spec_verify_init", "spec_verify_destroy", "spec_verify_run",
                  "spec_verify_run_with_uniforms", "spec_verify_run_host", "spec_verify_greedy",
-                 "spec_conf_budget", "spec_verify_timing_enable", "spec_verify_timing_read",
+                 "spec_conf_budget", "spec_verify_greedy_noalloc", "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
         getattr(L, name).restype = _i32
     _lib = L
@@ -315,6 +316,28 @@ class SpecVerifier:
         _check(lib().spec_verify_last_counters(self._h, _stream_handle(stream, self.device), out),
                "spec_verify_last_counters")
         return dict(accept_fp64=out[0], sample_fp64=out[1], sample_fp32=out[2])
+
+
+def greedy_noalloc(target, tokens, verify_len=None, stream=None, out=None):
+    """spec_verify_greedy_noalloc: greedy verification for callers that may not
+    allocate device memory (the library's fixed scratch array is used; see the
+    header for the size limits).  ``out`` lets the caller pass preallocated
+    outputs (accepted [B], tokens [B, k+1], status [B], int32, on the device)."""
+    if target.dim() != 3:
+        raise ValueError("target logits must be [B, k+1, V]")
+    B, kp1, V = target.shape
+    dev = target.device
+    if out is None:
+        out = dict(accepted=torch.empty(B, dtype=torch.int32, device=dev),
+                   tokens=torch.empty((B, kp1), dtype=torch.int32, device=dev),
+                   status=torch.empty(B, dtype=torch.int32, device=dev))
+    st = lib().spec_verify_greedy_noalloc(
+        _dev_ptr(target, None, dev, "target"), _dtype_code(target),
+        _dev_ptr(tokens, torch.int32, dev, "tokens"), _dev_ptr(verify_len, torch.int32, dev, "verify_len"),
+        B, kp1 - 1, V, _dev_ptr(out["accepted"], torch.int32), _dev_ptr(out["tokens"], torch.int32),
+        _dev_ptr(out["status"]), _stream_handle(stream, dev))
+    _check(st, "spec_verify_greedy_noalloc")
+    return out
 
 
 def selfcheck_ex2(device=0, lo=-126.0, hi=0.0):

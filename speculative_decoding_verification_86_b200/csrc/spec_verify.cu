@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -47,6 +48,56 @@ struct DeviceGuard {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Scratch of spec_verify_greedy_noalloc.  Callers that may not allocate device
+// memory get their working space from this fixed array instead of a context:
+// every GPU that loads the library holds it (about 2.3 MB) until the process
+// exits.  Limits: B <= 256, k <= 8, and B * (2k + 1) * ceil(V / chunk) <=
+// 256 * 17 * 32 chunk records (chunk = 8192 bf16 or 4096 fp32 logits), i.e.
+// V <= 262144 for bf16 and V <= 131072 for fp32 at the largest B and k.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kNoAllocMaxBatch = 256;
+constexpr int kNoAllocMaxK = 8;
+constexpr size_t kNoAllocMaxRecords = size_t(kNoAllocMaxBatch) * (2 * kNoAllocMaxK + 1) * 32;
+constexpr size_t kNoAllocMetaOff = 0;
+constexpr size_t kNoAllocJobsOff = kNoAllocMetaOff + kNoAllocMaxRecords * sizeof(sv::ChunkMeta);
+constexpr size_t kNoAllocArriveOff = kNoAllocJobsOff + size_t(kNoAllocMaxBatch) * sizeof(sv::Job);
+constexpr size_t kNoAllocCountersOff = kNoAllocArriveOff + size_t(kNoAllocMaxBatch) * sizeof(unsigned);
+constexpr size_t kNoAllocBytes = kNoAllocCountersOff + 2 * sizeof(sv::Counters);
+static_assert(kNoAllocJobsOff % 16 == 0 && kNoAllocArriveOff % 16 == 0 &&
+                  kNoAllocCountersOff % 16 == 0,
+              "scratch records must stay 16-byte aligned");
+constexpr int kNoAllocMaxDevices = 64;
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices] = {};
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_greedy_scratch[kNoAllocBytes];
+
+namespace {
+// Device address of g_greedy_scratch on the current device.  In host code the
+// array's name only stands in for the symbol; the kernels must be given the
+// address the runtime reports, looked up once per device.
+spec_status noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SPEC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_greedy_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return SPEC_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return SPEC_OK;
+}
 }  // namespace
 
 struct spec_verify_ctx {
@@ -521,6 +572,62 @@ spec_status spec_verify_selfcheck_ex2(int device, float lo, float hi, double* ma
 }
 
 double spec_verify_ex2_error_bound(void) { return static_cast<double>(kEpsEx2); }
+
+spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dtype,
+                                       const int32_t* draft_tokens, const int32_t* verify_len,
+                                       int B, int k, int64_t V, int32_t* out_accepted,
+                                       int32_t* out_tokens, uint32_t* out_status,
+                                       cudaStream_t stream) {
+  if (B < 0 || B > kNoAllocMaxBatch || k < 0 || k > kNoAllocMaxK || V < 1)
+    return SPEC_ERR_INVALID_ARG;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return SPEC_ERR_INVALID_ARG;
+  const bool bf16 = dtype == SPEC_BF16;
+  const int chunk = bf16 ? sv::kChunkBf16 : sv::kChunkF32;
+  const int64_t n_chunks = (V + chunk - 1) / chunk;
+  if (static_cast<size_t>(B) * (2 * k + 1) * static_cast<size_t>(n_chunks) > kNoAllocMaxRecords)
+    return SPEC_ERR_INVALID_ARG;
+  if (B == 0) return SPEC_OK;
+  if (!target_logits || !out_accepted || !out_tokens || (k > 0 && !draft_tokens))
+    return SPEC_ERR_INVALID_ARG;
+  if ((V * (bf16 ? 2 : 4)) % 16 != 0 || !aligned(target_logits, 16)) return SPEC_ERR_UNSUPPORTED;
+  if ((draft_tokens && !aligned(draft_tokens, 4)) || (verify_len && !aligned(verify_len, 4)) ||
+      !aligned(out_accepted, 4) || !aligned(out_tokens, 4) ||
+      (out_status && !aligned(out_status, 4)))
+    return SPEC_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  if (spec_status st = noalloc_scratch(&base); st != SPEC_OK) return st;
+  char* b = static_cast<char*>(base);
+
+  sv::RunParams p{};
+  p.target = target_logits;
+  p.tokens = draft_tokens;
+  p.vlen = verify_len;
+  p.B = B;
+  p.k = k;
+  p.V = V;
+  p.n_chunks = static_cast<int>(n_chunks);
+  p.force_greedy = 1;
+  p.eps_ex2 = kEpsEx2;
+  p.out_acc = out_accepted;
+  p.out_tok = out_tokens;
+  p.out_status = out_status;
+  p.meta = reinterpret_cast<sv::ChunkMeta*>(b + kNoAllocMetaOff);
+  p.jobs = reinterpret_cast<sv::Job*>(b + kNoAllocJobsOff);
+  p.arrive_stats = reinterpret_cast<unsigned*>(b + kNoAllocArriveOff);
+  p.counters = reinterpret_cast<sv::Counters*>(b + kNoAllocCountersOff);
+  p.counters_next = p.counters + 1;
+
+  cudaGetLastError();
+  // The arrival counters must start at zero; the array keeps whatever the
+  // previous call (or an interrupted one) left there.
+  if (cudaMemsetAsync(p.arrive_stats, 0, static_cast<size_t>(B) * sizeof(unsigned), stream) !=
+      cudaSuccess)
+    return SPEC_ERR_CUDA;
+  const int64_t ctas = static_cast<int64_t>(B) * (2 * k + 1) * n_chunks;
+  if (bf16) sv::k_stats<true><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
+  else sv::k_stats<false><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
 
 spec_status spec_verify_timing_enable(spec_verify_ctx* ctx, int class_mask) {
   if (!ctx || class_mask < 0 || class_mask >= (1 << kTimingClasses)) return SPEC_ERR_INVALID_ARG;
