@@ -322,13 +322,27 @@ def run_ours(args):
     ver.timing_enable([])
     clk = clocks.stop()
     counters = ver.last_counters()
+    # per-kernel breakdown, in a separate loop so the timed region carries only
+    # the events around the statistics kernel
+    ver.timing_enable([binding.TIMING_STATS, binding.TIMING_SAMPLE, binding.TIMING_REFINE,
+                       binding.TIMING_CONF])
+    nb = min(args.steps, 200)
+    for _ in range(nb):
+        step()
+    breakdown = {}
+    for name, cls in (("stats", binding.TIMING_STATS), ("sample", binding.TIMING_SAMPLE),
+                      ("refine", binding.TIMING_REFINE), ("conf", binding.TIMING_CONF)):
+        n_c, ms_c = ver.timing_read(cls)
+        if n_c:
+            breakdown[name + "_ms"] = ms_c / n_c
+    ver.timing_enable([])
     t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total = float(t.item())
     ms_per_step = ms_total / args.steps
     value = positions * world / (ms_per_step / 1e3)
-    launches_per_step = 4 + (1 if w.get("conf") is not None else 0)
+    launches_per_step = 3 + (1 if w.get("conf") is not None else 0)
 
     # end to end: host buffers in, host results out, through the C ABI
     e2e = None
@@ -408,6 +422,7 @@ def run_ours(args):
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
         "fp64_paths": counters,
+        "kernel_ms": breakdown,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -94,7 +94,7 @@ typedef struct {
 
 /* Create a context on `device` with workspace for batches up to max_batch
  * requests, blocks up to max_k drafted tokens (max_k <= 16) and vocabularies
- * up to max_vocab.  The current device is restored on return. */
+ * up to max_vocab (<= 2097152).  The current device is restored on return. */
 spec_status spec_verify_init(spec_verify_ctx** ctx, int device, int max_batch, int max_k,
                              int64_t max_vocab);
 
@@ -200,10 +200,11 @@ spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launch
                                     double* total_ms);
 
 /* Diagnostics of the last completed run (synchronises the stream first):
- * out[0] = requests whose accept test needed the fp64 path, out[1] = samples
- * refined in fp64, out[2] = samples resolved by the fp32 filter. */
+ * out[0] = accept decisions settled by the fp64 path, out[1] = samples refined
+ * in fp64, out[2] = samples certified by the fp32 filter, out[3] = chunks the
+ * fp64 refinement recomputed outright. */
 spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
-                                      uint32_t out[3]);
+                                      uint32_t out[4]);
 
 /* Self-check of the one hardware constant the fp32 filter relies on: the
  * maximum relative error of the ex2.approx.ftz.f32 instruction against fp64

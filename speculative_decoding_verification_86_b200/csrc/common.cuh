@@ -7,25 +7,30 @@
 namespace sv {
 
 // ---------------------------------------------------------------- geometry --
-// A "chunk" is the slice of one logit row that one CTA streams: kThreads
-// threads x kUnroll 16-byte vectors each, i.e. 8192 bf16 or 4096 fp32 logits.
+// A "chunk" is the unit of the sampling passes: kThreads threads x
+// kBatchesPerChunk batches x kVecsPerBatch 16-byte vectors, i.e. 16384 bf16
+// or 8192 fp32 logits of one row.  Chunk masses are what the inverse CDF
+// prefixes before it rescans one chunk.
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
+constexpr int kVecsPerBatch = 2;
+constexpr int kBatchesPerChunk = 4;
 constexpr int kMaxK = 16;
 constexpr int kMaxRows = 2 * kMaxK + 1;  // k+1 target rows + k draft rows
 
 template <bool BF16>
 struct Geo {
-  static constexpr int kPerVec = BF16 ? 8 : 4;                  // logits per 16-byte vector
-  static constexpr int kChunkVecs = kThreads * kUnroll;          // vectors per chunk
-  static constexpr int kChunk = kChunkVecs * kPerVec;            // logits per chunk
-  static constexpr int kPerThread = kUnroll * kPerVec;           // logits per thread
-  static constexpr int kSumLevels = BF16 ? 5 : 4;                // pairwise-sum depth per thread
+  static constexpr int kPerVec = BF16 ? 8 : 4;                                  // logits per vector
+  static constexpr int kChunkVecs = kThreads * kVecsPerBatch * kBatchesPerChunk; // 2048 vectors
+  static constexpr int kChunk = kChunkVecs * kPerVec;                            // logits per chunk
+  static constexpr int kBatchElems = kVecsPerBatch * kPerVec;                    // per thread and batch
+  static constexpr int kPerThread = kBatchElems * kBatchesPerChunk;              // per thread and chunk
+  static constexpr int kSumLevels = BF16 ? 4 : 3;                                // pairwise depth of a batch sum
 };
 
-constexpr int kChunkBf16 = Geo<true>::kChunk;   // 8192
-constexpr int kChunkF32 = Geo<false>::kChunk;   // 4096
+constexpr int kChunkBf16 = Geo<true>::kChunk;   // 16384
+constexpr int kChunkF32 = Geo<false>::kChunk;   // 8192
+constexpr int kMaxChunksPerRow = 1024;  // block-wide prefixes cover 4 records per thread
 
 // ------------------------------------------------------------ status bits --
 constexpr uint32_t kDevBadToken = 1u;
@@ -34,12 +39,16 @@ constexpr uint32_t kDevBadTemperature = 4u;
 constexpr uint32_t kDevInternal = 16u;
 
 // ------------------------------------------------------- workspace records --
-// Statistics of one chunk of one row.
-//   stochastic row: K = fl(mraw * c) (reference of the exponent sums),
+// Statistics of one segment of one row.
+//   stochastic row: K = integer exponent reference (NaN if the segment holds
+//                   NaN or +inf, -inf if it holds only masked logits),
 //                   mraw = NaN-propagating max of the raw logits,
-//                   err = sum_t e_t * |a_t| (argument-rounding weight), arg unused;
+//                   err = sum_t e_t |a_t| (a_t the rounded exponent in the frame
+//                   it was computed in: bounds the exponent rounding),
+//                   arg = bits of sum_t e_t (K - K_t) (frame offsets, fp32);
 //                   the sum of e_t = 2^(l_t c - K) is stored separately in fp64.
-//   greedy row:     mraw = NaN-propagating max, arg = lowest index attaining it.
+//   greedy row:     mraw = NaN-propagating max (NaN if any logit is NaN),
+//                   arg = lowest index attaining it.
 struct ChunkMeta {
   float K;
   float mraw;
@@ -62,13 +71,16 @@ struct Job {
   float Kb;     // exponent reference of the draft row
   float A;      // fp32 1 / Za   (1 for bonus jobs)
   float Bq;     // fp32 1 / Zb
-  float kappa;  // ln2 * (2^-24 + |eta|): relative error per unit |argument|
+  float kappa;  // ln2 * (2^-24 + |eta|): relative error per unit |argument| in a frame
   float mraw_a; // raw max of the target row (fp64 refinement)
   float mraw_b; // raw max of the draft row
   double eps0a; // argument-independent relative error bound of p terms
   double eps0b; // ... of q terms
   double u2;    // the sample's uniform draw
   double T;     // temperature
+  double eta_ln2; // ln2 * |relative error of fp32 log2(e)/T|
+  double rho_lo;  // refinement: Z_a / Z_b (max-relative frames) lies in [rho_lo, rho_hi]
+  double rho_hi;
 };
 
 struct SampleChunk {
@@ -80,7 +92,7 @@ struct Counters {
   unsigned refine_count;   // samples queued for fp64 refinement
   unsigned accept_slow;    // accept decisions resolved in fp64
   unsigned sample_fast;    // samples certified by the fp32 filter
-  unsigned pad;
+  unsigned chunks_redone;  // refinement chunks recomputed outright (support unsettled)
 };
 
 // -------------------------------------------------------------- run params --
@@ -95,7 +107,8 @@ struct RunParams {
   int B;
   int k;
   int64_t V;
-  int n_chunks;
+  int n_chunks;            // 8192 / 4096-logit chunks (sampling and refinement passes)
+  int n_segs;              // 32768 / 16384-logit segments (statistics pass)
   uint64_t seed;
   uint32_t step;
   uint32_t req_off;
@@ -117,9 +130,10 @@ struct RunParams {
   int* refine_list;        // [B]
   unsigned* arrive_r1;     // [B]
   unsigned* arrive_r2;     // [B]
-  double2* rz;             // [B, n_chunks] fp64 Z partials (target, draft)
-  double2* rZ;             // [B] merged fp64 Z
-  double2* rm;             // [B, n_chunks] fp64 masses (residual, target)
+  double2* rz;             // [B, 4 n_chunks] fp64 normaliser partials per sub-chunk
+  double2* rZ;             // [B] (unused)
+  double2* rm;             // [B, 4 n_chunks] fp64 support masses (target, draft)
+  int* runc;               // [B, 4 n_chunks] sub-chunks holding unsettled logits
   Counters* counters;      // this run's counters
   Counters* counters_next; // the other run's counters, reset here
 };
@@ -188,10 +202,77 @@ __device__ __forceinline__ void unpack(const uint4& v, float (&x)[Geo<BF16>::kPe
   }
 }
 
+// NaN-propagating maximum of kUnroll vectors.
+template <bool BF16>
+__device__ __forceinline__ float vec_max(const uint4 (&v)[kVecsPerBatch]) {
+  if constexpr (BF16) {
+    uint32_t m2 = hmax2_nan(v[0].x, v[0].y);
+    m2 = hmax2_nan(m2, v[0].z);
+    m2 = hmax2_nan(m2, v[0].w);
+#pragma unroll
+    for (int u = 1; u < kVecsPerBatch; ++u) {
+      m2 = hmax2_nan(m2, v[u].x);
+      m2 = hmax2_nan(m2, v[u].y);
+      m2 = hmax2_nan(m2, v[u].z);
+      m2 = hmax2_nan(m2, v[u].w);
+    }
+    return fmax_nan(bf16_lo(m2), bf16_hi(m2));
+  } else {
+    float m = fmax_nan(__uint_as_float(v[0].x), __uint_as_float(v[0].y));
+    m = fmax_nan(m, __uint_as_float(v[0].z));
+    m = fmax_nan(m, __uint_as_float(v[0].w));
+#pragma unroll
+    for (int u = 1; u < kVecsPerBatch; ++u) {
+      m = fmax_nan(m, __uint_as_float(v[u].x));
+      m = fmax_nan(m, __uint_as_float(v[u].y));
+      m = fmax_nan(m, __uint_as_float(v[u].z));
+      m = fmax_nan(m, __uint_as_float(v[u].w));
+    }
+    return m;
+  }
+}
+
 template <bool BF16>
 __device__ __forceinline__ uint4 neg_inf_vec() {
   const uint32_t w = BF16 ? 0xFF80FF80u : 0xFF800000u;
   return make_uint4(w, w, w, w);
+}
+
+// Batch b of chunk c of a row, coalesced layout: thread t holds vectors
+// t + (b * kVecsPerBatch + u) * kThreads of the chunk, so each load
+// instruction of a warp covers 512 contiguous bytes.  Vectors past the row end
+// read as -inf (weight 0).
+template <bool BF16>
+__device__ __forceinline__ void load_batch_coalesced(const void* row, int64_t V, int c, int b,
+                                                     uint4 (&v)[kVecsPerBatch]) {
+  using G = Geo<BF16>;
+  const int64_t nvec = V / G::kPerVec;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads;
+    v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
+  }
+}
+
+// Batch b of chunk c, contiguous layout: thread t holds the kPerThread logits
+// starting at chunk offset t * kPerThread, batch b being its b-th run of
+// kBatchElems -- index order, for scans.  Returns the chunk offset of the batch.
+template <bool BF16>
+__device__ __forceinline__ int load_batch_contiguous(const void* row, int64_t V, int c, int b,
+                                                     uint4 (&v)[kVecsPerBatch]) {
+  using G = Geo<BF16>;
+  const int64_t nvec = V / G::kPerVec;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int off = threadIdx.x * G::kPerThread + b * G::kBatchElems;
+  const int64_t base = (static_cast<int64_t>(c) * G::kChunk + off) / G::kPerVec;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = base + u;
+    v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
+  }
+  return off;
 }
 
 __device__ __forceinline__ bool temperature_valid(float T) {
@@ -229,11 +310,11 @@ __device__ __forceinline__ ReqInfo request_info(const RunParams& p, int i) {
   return r;
 }
 
-// Number of (row, chunk) CTAs the statistics pass runs for request i.
-__device__ __forceinline__ int stats_expected(const ReqInfo& r, int n_chunks) {
+// Number of (row, segment) CTAs the statistics pass runs for request i.
+__device__ __forceinline__ int stats_expected(const ReqInfo& r, int n_segs) {
   if (r.bad_T) return 1;
-  if (r.greedy) return (r.L + 1) * n_chunks;
-  return (2 * r.L + 1) * n_chunks;
+  if (r.greedy) return (r.L + 1) * n_segs;
+  return (2 * r.L + 1) * n_segs;
 }
 
 // ------------------------------------------------------- block reductions --
@@ -325,6 +406,20 @@ __device__ __forceinline__ double block_exclusive_scan_d(double x, double* sh, d
   }
   total = all;
   return warp_base + incl - x;
+}
+
+// Block-wide exclusive prefix of per-chunk values v[c], c < n (n <= 4 *
+// kThreads): thread t owns chunks 4t .. 4t+3.  Fills pre[4] (prefix before each
+// owned chunk) and returns the total.
+__device__ __forceinline__ double chunk_prefix(const double (&v)[4], double (&pre)[4], double* sh) {
+  const double local = (v[0] + v[1]) + (v[2] + v[3]);
+  double total;
+  const double base = block_exclusive_scan_d(local, sh, total);
+  pre[0] = base;
+  pre[1] = base + v[0];
+  pre[2] = pre[1] + v[1];
+  pre[3] = pre[2] + v[2];
+  return total;
 }
 
 // Arrival on a per-request counter: returns true in exactly one CTA, the last

@@ -5,202 +5,314 @@
 // under the 1e-12 floor), inverse CDF in index order with the smallest-index
 // rule and the largest-positive-index fallback.
 //
-// Two launches, each a grid-stride loop over (queued request, chunk):
-//   k_refine_z    : fp64 normalisers of the row pair, merged in chunk order;
-//   k_refine_pick : fp64 chunk masses, then the last CTA of the request
-//                   prefixes them and scans the one chunk holding u * total.
-// Both read the queue length written by the sampling pass and exit at once
-// when nothing was queued.
+// One launch, a grid-stride loop over (queued request, sub-chunk of 4096 bf16 /
+// 2048 fp32 logits: one batch of the chunk layout), one fp64 pass over the row
+// pair.  The exact normalisers Z_a, Z_b are only known once every
+// chunk is done, but the residual's support {t : p_t > q_t} = {alpha_t > rho
+// beta_t} (alpha = exp(a/T - m_a), beta likewise, rho = Z_a / Z_b) can be
+// settled early: the fp32 pass bounds rho in [rho_lo, rho_hi], so a chunk adds
+// alpha and beta of every logit with alpha > rho_hi beta to its support sums
+// and only counts the few with rho_lo beta <= alpha <= rho_hi beta.  The
+// request's last CTA then has each chunk's residual mass as A_c/Z_a - B_c/Z_b,
+// recomputes outright the rare chunks holding unsettled logits (or all of
+// them if rho missed its bracket), prefixes the masses block-wide and scans the
+// one chunk holding u * total.  Weights are exp2_fast (fp64.cuh) of
+// l * (log2(e)/T) - m * log2(e).
 #pragma once
 #include "common.cuh"
+#include "fp64.cuh"
 #include "stats.cuh"
 
 namespace sv {
 
 struct RefineShared {
+  double tab[kExp2Table];
   double d[kWarps];
   int i[kWarps];
   int flag;
   int cstar;
-  double base, total, target;
+  int redo_all;
   int use_resid;
   int found;
+  double base, target, Za, Zb;
 };
 
-__device__ __forceinline__ double exact_weight_p(const void* ra, int64_t t, bool bf16, double T,
-                                                 double ma) {
-  return exp(static_cast<double>(load_logit(ra, t, bf16)) / T - ma);
+struct RefineRow {
+  double s, ma2, mb2;  // log2(e)/T and the row maxima times it (exponents in base 2)
+};
+
+__device__ __forceinline__ RefineRow refine_row(const Job& jb) {
+  RefineRow r;
+  r.s = kLog2E / jb.T;
+  r.ma2 = static_cast<double>(jb.mraw_a) * r.s;
+  r.mb2 = static_cast<double>(jb.mraw_b) * r.s;
+  return r;
 }
 
+constexpr int kSubsPerChunk = kBatchesPerChunk;  // a sub-chunk is one batch of a chunk
+
+// One pass over sub-chunk (c, bt): alpha/beta sums and, for residual jobs, the
+// support sums A, B and the count of unsettled logits (alpha > 0 only: where
+// alpha = 0, p_t = 0 and the weight is 0 whatever rho is).
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) k_refine_z(RunParams p) {
-  __shared__ RefineShared sh;
+__device__ __forceinline__ void refine_sub_pass(const RunParams& p, int i, const Job& jb,
+                                                const RefineRow& rr, int c, int bt, bool residual,
+                                                const double* tab, double& za, double& zb,
+                                                double& A, double& Bm, int& unc) {
   using G = Geo<BF16>;
-  const unsigned count = __ldcg(&p.counters->refine_count);
-  const int64_t work = static_cast<int64_t>(count) * p.n_chunks;
-  for (int64_t wi = blockIdx.x; wi < work; wi += gridDim.x) {
-    const int slot = static_cast<int>(wi / p.n_chunks);
-    const int c = static_cast<int>(wi % p.n_chunks);
-    const int i = __ldcg(p.refine_list + slot);
-    const Job jb = p.jobs[i];
-    const double T = jb.T;
-    const double ma = static_cast<double>(jb.mraw_a) / T;
-    const double mb = static_cast<double>(jb.mraw_b) / T;
-    const void* ra = target_row(p, i, jb.row, BF16);
-    const void* rb = jb.kind == kJobResidual ? draft_row(p, i, jb.row, BF16) : nullptr;
-    const int64_t t0 = static_cast<int64_t>(c) * G::kChunk;
-    const int64_t t1 = min(p.V, t0 + G::kChunk);
-    double za = 0.0, zb = 0.0;
-    for (int64_t t = t0 + threadIdx.x; t < t1; t += kThreads) {
-      za += exact_weight_p(ra, t, BF16, T, ma);
-      if (rb) zb += exact_weight_p(rb, t, BF16, T, mb);
-    }
-    za = block_sum_d(za, sh.d);
-    __syncthreads();
-    zb = block_sum_d(zb, sh.d);
-    if (threadIdx.x == 0) p.rz[static_cast<int64_t>(slot) * p.n_chunks + c] = make_double2(za, zb);
-    if (arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(p.n_chunks), &sh.flag)) {
-      __threadfence();
-      if (threadIdx.x == 0) {
-        double A = 0.0, Bz = 0.0;
-        for (int cc = 0; cc < p.n_chunks; ++cc) {
-          const double2 r = __ldcg(p.rz + static_cast<int64_t>(slot) * p.n_chunks + cc);
-          A += r.x;
-          Bz += r.y;
+  const void* ra = target_row(p, i, jb.row, BF16);
+  const void* rb = residual ? draft_row(p, i, jb.row, BF16) : nullptr;
+  uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+  load_batch_coalesced<BF16>(ra, p.V, c, bt, va);
+  if (residual) load_batch_coalesced<BF16>(rb, p.V, c, bt, vb);
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    float xa[G::kPerVec], xb[G::kPerVec];
+    unpack<BF16>(va[u], xa);
+    if (residual) unpack<BF16>(vb[u], xb);
+#pragma unroll
+    for (int q = 0; q < G::kPerVec; ++q) {
+      const double al = exp_weight(xa[q], rr.s, rr.ma2, tab);
+      za += al;
+      if (residual) {
+        const double be = exp_weight(xb[q], rr.s, rr.mb2, tab);
+        zb += be;
+        if (al > be * jb.rho_hi) {
+          A += al;
+          Bm += be;
+        } else if (al > 0.0 && al >= be * jb.rho_lo) {
+          ++unc;
         }
-        p.rZ[slot] = make_double2(A, Bz);
       }
     }
-    __syncthreads();
   }
 }
 
+// Exact weight of the logit at chunk offset (bt, u, q) of the contiguous layout.
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) k_refine_pick(RunParams p) {
+__device__ __forceinline__ double exact_weight(float a, float b, bool use_resid,
+                                               const RefineRow& rr, double iza, double izb,
+                                               const double* tab) {
+  const double pe = exp_weight(a, rr.s, rr.ma2, tab);
+  if (!use_resid) return pe;
+  const double r = pe * iza - exp_weight(b, rr.s, rr.mb2, tab) * izb;
+  return r > 0.0 ? r : 0.0;
+}
+
+// Exact residual mass of sub-chunk (c, bt), block-reduced in a fixed order.
+template <bool BF16>
+__device__ double exact_sub_mass(const RunParams& p, int i, const Job& jb, const RefineRow& rr,
+                                 int c, int bt, double iza, double izb, RefineShared& sh) {
+  using G = Geo<BF16>;
+  uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+  load_batch_coalesced<BF16>(target_row(p, i, jb.row, BF16), p.V, c, bt, va);
+  load_batch_coalesced<BF16>(draft_row(p, i, jb.row, BF16), p.V, c, bt, vb);
+  double m = 0.0;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    float xa[G::kPerVec], xb[G::kPerVec];
+    unpack<BF16>(va[u], xa);
+    unpack<BF16>(vb[u], xb);
+#pragma unroll
+    for (int q = 0; q < G::kPerVec; ++q) m += exact_weight<BF16>(xa[q], xb[q], true, rr, iza, izb, sh.tab);
+  }
+  __syncthreads();
+  return block_sum_d(m, sh.d);
+}
+
+// Sub-chunk (c, bt) is the contiguous logit range [c*kChunk + bt*4096 (bf16),
+// +4096); in index order thread t holds its kVecsPerBatch vectors t*2, t*2+1.
+template <bool BF16>
+__device__ __forceinline__ int load_sub_contiguous(const void* row, int64_t V, int c, int bt,
+                                                   uint4 (&v)[kVecsPerBatch]) {
+  using G = Geo<BF16>;
+  const int64_t nvec = V / G::kPerVec;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs +
+                       static_cast<int64_t>(bt) * (kVecsPerBatch * kThreads) +
+                       threadIdx.x * kVecsPerBatch;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = base + u;
+    v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
+  }
+  return bt * G::kBatchElems * kThreads + threadIdx.x * G::kBatchElems;  // offset in the chunk
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads, 2) k_refine(RunParams p) {
   __shared__ RefineShared sh;
   using G = Geo<BF16>;
   const unsigned count = __ldcg(&p.counters->refine_count);
-  const int64_t work = static_cast<int64_t>(count) * p.n_chunks;
+  const int n_subs = p.n_chunks * kSubsPerChunk;
+  const int64_t work = static_cast<int64_t>(count) * n_subs;
+  if (blockIdx.x >= work) return;
+  exp2_table_init(sh.tab);
+#pragma unroll 1
   for (int64_t wi = blockIdx.x; wi < work; wi += gridDim.x) {
-    const int slot = static_cast<int>(wi / p.n_chunks);
-    const int c = static_cast<int>(wi % p.n_chunks);
+    const int slot = static_cast<int>(wi / n_subs);
+    const int sub = static_cast<int>(wi % n_subs);
     const int i = __ldcg(p.refine_list + slot);
     const Job jb = p.jobs[i];
+    const RefineRow rr = refine_row(jb);
     const bool residual = jb.kind == kJobResidual;
-    const double T = jb.T;
-    const double ma = static_cast<double>(jb.mraw_a) / T;
-    const double mb = static_cast<double>(jb.mraw_b) / T;
-    const double2 Z = __ldcg(p.rZ + slot);
-    const void* ra = target_row(p, i, jb.row, BF16);
-    const void* rb = residual ? draft_row(p, i, jb.row, BF16) : nullptr;
-    const int64_t t0 = static_cast<int64_t>(c) * G::kChunk;
-    const int64_t t1 = min(p.V, t0 + G::kChunk);
-    double mr = 0.0, mp = 0.0;
-    for (int64_t t = t0 + threadIdx.x; t < t1; t += kThreads) {
-      const double pe = exact_weight_p(ra, t, BF16, T, ma);
-      mp += pe;
-      if (rb) {
-        const double r = pe / Z.x - exact_weight_p(rb, t, BF16, T, mb) / Z.y;
-        mr += r > 0.0 ? r : 0.0;
-      }
-    }
-    mr = block_sum_d(mr, sh.d);
+    double za = 0.0, zb = 0.0, A = 0.0, Bm = 0.0;
+    int unc = 0;
+    refine_sub_pass<BF16>(p, i, jb, rr, sub / kSubsPerChunk, sub % kSubsPerChunk, residual, sh.tab,
+                          za, zb, A, Bm, unc);
+    za = block_sum_d(za, sh.d);
     __syncthreads();
-    mp = block_sum_d(mp, sh.d);
-    if (threadIdx.x == 0) p.rm[static_cast<int64_t>(slot) * p.n_chunks + c] = make_double2(mr, mp);
-    if (!arrive_last(p.arrive_r2 + slot, static_cast<unsigned>(p.n_chunks), &sh.flag)) continue;
+    zb = block_sum_d(zb, sh.d);
+    __syncthreads();
+    A = block_sum_d(A, sh.d);
+    __syncthreads();
+    Bm = block_sum_d(Bm, sh.d);
+    unc = __syncthreads_or(unc);
+    const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
+    if (threadIdx.x == 0) {
+      p.rz[rec0 + sub] = make_double2(za, zb);
+      p.rm[rec0 + sub] = make_double2(A, Bm);
+      p.runc[rec0 + sub] = unc;
+    }
+    if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(n_subs), &sh.flag)) continue;
     __threadfence();
 
-    // ---- last CTA of this request: locate the token in fp64 ----
-    const double2* rm = p.rm + static_cast<int64_t>(slot) * p.n_chunks;
+    // ---- last CTA of this request: exact sub-chunk masses, then the token ----
+    // thread t owns sub-chunks 4t .. 4t+3
+    double zav[4], zbv[4], pz[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int ss = 4 * threadIdx.x + q;
+      const double2 z = ss < n_subs ? __ldcg(p.rz + rec0 + ss) : make_double2(0.0, 0.0);
+      zav[q] = z.x;
+      zbv[q] = z.y;
+    }
+    const double Za = chunk_prefix(zav, pz, sh.d);
+    const double Zb = chunk_prefix(zbv, pz, sh.d);
+    const double iza = 1.0 / Za, izb = residual ? 1.0 / Zb : 0.0;
+    const double rho = residual ? Za / Zb : 0.0;
+    const bool redo_all = residual && !(rho >= jb.rho_lo && rho <= jb.rho_hi);
+    double mv[4];
+    int flagged = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int ss = 4 * threadIdx.x + q;
+      mv[q] = 0.0;
+      if (ss < n_subs) {
+        if (residual) {
+          const double2 ab = __ldcg(p.rm + rec0 + ss);
+          const double r = ab.x * iza - ab.y * izb;
+          mv[q] = r > 0.0 ? r : 0.0;
+          if (redo_all || __ldcg(p.runc + rec0 + ss)) flagged |= 1 << q;
+        } else {
+          mv[q] = zav[q];
+        }
+      }
+    }
+    // sub-chunks whose support was not settled: recompute outright (rare)
+    if (__syncthreads_or(flagged)) {
+#pragma unroll 1
+      for (int ss = 0; ss < n_subs; ++ss) {
+        const int owner = ss / 4;
+        if (threadIdx.x == owner) sh.found = (flagged >> (ss % 4)) & 1;
+        __syncthreads();
+        if (sh.found) {
+          if (threadIdx.x == 0) atomicAdd(&p.counters->chunks_redone, 1u);
+          const double m = exact_sub_mass<BF16>(p, i, jb, rr, ss / kSubsPerChunk,
+                                                ss % kSubsPerChunk, iza, izb, sh);
+          if (threadIdx.x == owner) mv[ss % 4] = m;
+        }
+        __syncthreads();
+      }
+    }
+    double pm[4];
+    const double R = chunk_prefix(mv, pm, sh.d);
+    const bool use_resid = residual && R >= 1e-12;
+    if (!use_resid && residual) {  // floor: target weights exp(a/T - m_a)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mv[q] = zav[q];
+      chunk_prefix(mv, pm, sh.d);
+    }
+    const double W = use_resid ? R : Za;
+    const double target = jb.u2 * W;
     if (threadIdx.x == 0) {
-      double R = 0.0, P = 0.0;
-      for (int cc = 0; cc < p.n_chunks; ++cc) {
-        const double2 r = __ldcg(rm + cc);
-        R += r.x;
-        P += r.y;
-      }
-      const int use_resid = residual && R >= 1e-12;
-      const double W = use_resid ? R : P;
-      const double target = jb.u2 * W;
-      double run = 0.0;
-      int cstar = -1;
-      for (int cc = 0; cc < p.n_chunks; ++cc) {
-        const double2 r = __ldcg(rm + cc);
-        const double m = use_resid ? r.x : r.y;
-        if (run + m > target) {
-          cstar = cc;
-          break;
-        }
-        run += m;
-      }
-      sh.use_resid = use_resid;
-      sh.cstar = cstar;
-      sh.base = run;
-      sh.target = target;
+      sh.cstar = -1;
       sh.found = -1;
-      if (cstar < 0) {
-        // rounding left no cell above target: the last chunk with positive weight
-        for (int cc = p.n_chunks - 1; cc >= 0; --cc) {
-          const double2 r = __ldcg(rm + cc);
-          if ((use_resid ? r.x : r.y) > 0.0) {
-            sh.cstar = cc;
-            break;
-          }
-        }
-        sh.found = -2;  // marks the fallback
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int ss = 4 * threadIdx.x + q;
+      if (ss < n_subs && pm[q] <= target && pm[q] + mv[q] > target) {
+        sh.cstar = ss;
+        sh.base = pm[q];
       }
     }
     __syncthreads();
-    const int cstar = sh.cstar;
-    const bool fallback = sh.found == -2;
-    const bool use_resid = sh.use_resid != 0;
+    bool fallback = false;
+    if (sh.cstar < 0) {
+      // rounding left no cell above target: the last sub-chunk with positive weight
+      int last = -1;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int ss = 4 * threadIdx.x + q;
+        if (ss < n_subs && mv[q] > 0.0) last = ss;
+      }
+      last = -block_min_i(last >= 0 ? -last : 1, sh.i);
+      if (threadIdx.x == 0) sh.cstar = last >= 0 ? last : -1;
+      __syncthreads();
+      fallback = true;
+    }
+    const int sstar = sh.cstar;
     int token = -1;
-    if (cstar >= 0) {
-      const int64_t chunk0 = static_cast<int64_t>(cstar) * G::kChunk;
-      const int64_t seg0 = chunk0 + static_cast<int64_t>(threadIdx.x) * G::kPerThread;
-      double wv[G::kPerThread];
+    if (sstar >= 0) {
+      const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
+      const void* ra = target_row(p, i, jb.row, BF16);
+      const void* rb = use_resid ? draft_row(p, i, jb.row, BF16) : nullptr;
+      uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+      const int off = load_sub_contiguous<BF16>(ra, p.V, c, bt, va);
+      if (use_resid) load_sub_contiguous<BF16>(rb, p.V, c, bt, vb);
+      double wv[G::kBatchElems];
       double tsum = 0.0;
       int last_pos = -1;
-      for (int e = 0; e < G::kPerThread; ++e) {
-        const int64_t t = seg0 + e;
-        double wt = 0.0;
-        if (t < p.V) {
-          const double pe = exact_weight_p(ra, t, BF16, T, ma);
-          if (use_resid) {
-            const double r = pe / Z.x - exact_weight_p(rb, t, BF16, T, mb) / Z.y;
-            wt = r > 0.0 ? r : 0.0;
-          } else {
-            wt = pe;
-          }
+#pragma unroll
+      for (int u = 0; u < kVecsPerBatch; ++u) {
+        float xa[G::kPerVec], xb[G::kPerVec];
+        unpack<BF16>(va[u], xa);
+        if (use_resid) unpack<BF16>(vb[u], xb);
+#pragma unroll
+        for (int q = 0; q < G::kPerVec; ++q) {
+          const double wt = exact_weight<BF16>(xa[q], use_resid ? xb[q] : 0.0f, use_resid, rr,
+                                               iza, izb, sh.tab);
+          wv[u * G::kPerVec + q] = wt;
+          tsum += wt;
+          if (wt > 0.0) last_pos = off + u * G::kPerVec + q;
         }
-        wv[e] = wt;
-        tsum += wt;
-        if (wt > 0.0) last_pos = static_cast<int>(t - chunk0);
       }
-      if (fallback) {
-        // largest index with positive weight in this chunk
-        int neg = last_pos >= 0 ? -last_pos : INT_MAX;
-        neg = block_min_i(neg, sh.i);
-        token = neg == INT_MAX ? -1 : static_cast<int>(chunk0 - neg);
-      } else {
+      int found = -1;
+      if (!fallback) {
         double all;
         const double pre = block_exclusive_scan_d(tsum, sh.d, all);
         const double start = sh.base + pre;
-        const double target = sh.target;
         if (start <= target && start + tsum > target) {
           double run = start;
-          for (int e = 0; e < G::kPerThread; ++e) {
+#pragma unroll
+          for (int e = 0; e < G::kBatchElems; ++e) {
             run += wv[e];
-            if (run > target) {
-              sh.found = static_cast<int>(seg0 - chunk0) + e;
-              break;
-            }
+            if (run > target && sh.found < 0) sh.found = off + e;
           }
         }
         __syncthreads();
-        token = sh.found >= 0 ? static_cast<int>(chunk0 + sh.found) : -1;
+        found = sh.found;
       }
+      if (found < 0) {
+        // fallback, or the sub-chunk's scanned total fell a rounding short of
+        // target: the last logit of the sub-chunk with positive weight
+        int neg = last_pos >= 0 ? -last_pos : INT_MAX;
+        neg = block_min_i(neg, sh.i);
+        found = neg == INT_MAX ? -1 : -neg;
+      }
+      token = found >= 0 ? static_cast<int>(static_cast<int64_t>(c) * G::kChunk + found) : -1;
     }
     if (threadIdx.x == 0) {
       p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;

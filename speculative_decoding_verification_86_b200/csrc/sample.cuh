@@ -5,112 +5,213 @@
 // draft-and-verify does not change the output").
 //
 // Inverse-CDF sampling in index order: the token is the smallest t whose
-// running weight exceeds u * (total weight).  One CTA per (request, chunk)
-// computes the chunk's weight mass in fp32 (fp64 accumulation) together with
-// a certified bound on its error; the request's last CTA prefixes the chunk
-// masses, rescans the one chunk holding u * total and checks that the chosen
-// cell's edges sit farther from u * total than the accumulated bound.  When
-// they do not, the request is queued for the fp64 refinement (refine.cuh),
-// which recomputes the weights exactly as the fp64 rule defines them.
+// running weight exceeds u * (total weight).  One CTA per (request, segment of
+// kChunksPerSeg chunks) computes each chunk's weight mass in fp32 (fp64
+// accumulation) together with a certified bound on its error; the request's
+// last CTA prefixes the chunk masses block-wide, rescans the one chunk holding
+// u * total and checks that the chosen cell's edges sit farther from u * total
+// than the accumulated bound.  When they do not, the request is queued for the
+// fp64 refinement (refine.cuh), which recomputes the weights exactly as the
+// fp64 rule defines them.
 #pragma once
 #include "common.cuh"
 #include "stats.cuh"
 
 namespace sv {
 
-// Weight of one logit pair and its error bound (fp32 path).
-//   residual: w = max(0, p~ - q~) with p~ = 2^(a c - Ka) / Za, q~ likewise;
-//   bonus:    w = 2^(a c - Ka)  (unnormalised; sampling is scale free).
+// Weight of one logit pair and its error bound (fp32 path), in a frame:
+//   residual: w = max(0, p~ - q~) with p~ = 2^(a c - Fa) * Aeff, Aeff = 2^(Fa - Ka) / Za;
+//   bonus:    w = 2^(a c - Fa) * Aeff, Aeff = 2^(Fa - Ka)  (unnormalised; sampling is scale free).
+// Fa, Fb are integer frames at or above the logits they serve (a batch's own
+// maximum), so the exponent argument, and with it its rounding, stays small.
+// Bound per term: p~ (epsa + kappa |xa|) + q~ (epsb + kappa |xb|) where eps
+// carries the ex2 error, the products' rounding, the normaliser's bound and the
+// frame's share of the temperature-rounding term.
 struct WeightCtx {
-  float cc, Ka, Kb, A, Bq, kappa, eps0a, eps0b;
+  float cc, Fa, Fb, Aeff, Beff, kappa, epsa, epsb;
   bool residual;
 };
 
 __device__ __forceinline__ void weight_and_bound(const WeightCtx& w, float a, float b, float& wt,
                                                  float& bd) {
-  const float xa = fmaxf(fmaf(a, w.cc, -w.Ka), -1024.0f);
-  const float pa = ex2_approx(xa) * w.A;
+  const float xa = fmaxf(fmaf(a, w.cc, -w.Fa), -1024.0f);
+  const float pa = ex2_approx(xa) * w.Aeff;
   if (!w.residual) {
     wt = pa;
-    bd = pa * fmaf(w.kappa, fabsf(xa), w.eps0a);
+    bd = pa * fmaf(w.kappa, -xa, w.epsa);
     return;
   }
-  const float xb = fmaxf(fmaf(b, w.cc, -w.Kb), -1024.0f);
-  const float qb = ex2_approx(xb) * w.Bq;
+  const float xb = fmaxf(fmaf(b, w.cc, -w.Fb), -1024.0f);
+  const float qb = ex2_approx(xb) * w.Beff;
   wt = fmaxf(pa - qb, 0.0f);
   // Only cells where p >= q is possible can carry weight (errors are < 1e-4).
   const bool near = pa * 1.0001f >= qb;
-  bd = near ? fmaf(pa, fmaf(w.kappa, fabsf(xa), w.eps0a), qb * fmaf(w.kappa, fabsf(xb), w.eps0b))
-            : 0.0f;
+  bd = near ? fmaf(pa, fmaf(w.kappa, -xa, w.epsa), qb * fmaf(w.kappa, -xb, w.epsb)) : 0.0f;
 }
 
-__device__ __forceinline__ WeightCtx weight_ctx(const Job& jb) {
+// 2^d for an integer d in [-126, 0], exactly.
+__device__ __forceinline__ float pow2i(int d) { return __int_as_float((127 + d) << 23); }
+
+// Frame of a set of logits whose maximum is `m`: the integer ceil(m c) (capped
+// at the row's frame K), the matching scale 2^(F - K) * zinv and the bound's
+// constant eps0 + eta_ln2 (K - F).  All-masked sets (or ones 2^-126 below the
+// row's maximum) get scale 0: their weights are below 2^-126 of the maximum's.
+__device__ __forceinline__ void make_frame(float m, float cc, float K, float zinv, float eps0,
+                                           float eta_ln2, float& F, float& scale, float& eps) {
+  F = fminf(ceilf(m * cc), K);
+  const float d = F - K;  // <= 0, integer; -inf if all masked
+  if (!(d >= -126.0f)) {
+    scale = 0.0f;
+    eps = 0.0f;
+    F = K;
+    return;
+  }
+  scale = zinv * pow2i(static_cast<int>(d));
+  eps = fmaf(eta_ln2, -d, eps0);
+}
+
+struct JobF32 {  // the job's constants in the precision the fp32 pass uses
+  float cc, Ka, Kb, A, Bq, kappa, eps0a, eps0b, eta_ln2;
+  bool residual;
+};
+
+__device__ __forceinline__ JobF32 job_f32(const Job& jb) {
+  JobF32 j;
+  j.cc = jb.cc;
+  j.Ka = jb.Ka;
+  j.Kb = jb.Kb;
+  j.A = jb.A;
+  j.Bq = jb.Bq;
+  j.kappa = jb.kappa;
+  j.eps0a = static_cast<float>(jb.eps0a) * 1.0001f;
+  j.eps0b = static_cast<float>(jb.eps0b) * 1.0001f;
+  j.eta_ln2 = static_cast<float>(jb.eta_ln2) * 1.001f;
+  j.residual = jb.kind == kJobResidual;
+  return j;
+}
+
+__device__ __forceinline__ WeightCtx weight_ctx(const JobF32& j, float ma, float mb) {
   WeightCtx w;
-  w.cc = jb.cc;
-  w.Ka = jb.Ka;
-  w.Kb = jb.Kb;
-  w.A = jb.A;
-  w.Bq = jb.Bq;
-  w.kappa = jb.kappa;
-  w.eps0a = static_cast<float>(jb.eps0a);
-  w.eps0b = static_cast<float>(jb.eps0b);
-  w.residual = jb.kind == kJobResidual;
+  w.cc = j.cc;
+  w.kappa = j.kappa;
+  w.residual = j.residual;
+  make_frame(ma, j.cc, j.Ka, j.A, j.eps0a, j.eta_ln2, w.Fa, w.Aeff, w.epsa);
+  if (j.residual) make_frame(mb, j.cc, j.Kb, j.Bq, j.eps0b, j.eta_ln2, w.Fb, w.Beff, w.epsb);
+  else { w.Fb = 0.0f; w.Beff = 0.0f; w.epsb = 0.0f; }
   return w;
 }
 
+// Weights of one batch (kBatchElems logits per thread), reduced two ways:
+// `sum` is their pairwise fp32 sum (the mass pass), `exact` the fp64 sum of the
+// same fp32 weights (the rescans); `bound` sums their error bounds in fp32.
+template <bool BF16, bool EXACT>
+__device__ __forceinline__ void batch_weights(const JobF32& j, const uint4 (&va)[kVecsPerBatch],
+                                              const uint4 (&vb)[kVecsPerBatch], float& sum,
+                                              double& exact, float& bound) {
+  using G = Geo<BF16>;
+  const WeightCtx w = weight_ctx(j, vec_max<BF16>(va), j.residual ? vec_max<BF16>(vb) : 0.0f);
+  float vs[kVecsPerBatch];
+  float bd_sum = 0.0f;
+  double ex = 0.0;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    float xa[G::kPerVec], xb[G::kPerVec], wt[G::kPerVec];
+    unpack<BF16>(va[u], xa);
+    if (j.residual) unpack<BF16>(vb[u], xb);
+#pragma unroll
+    for (int q = 0; q < G::kPerVec; ++q) {
+      float bd;
+      weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt[q], bd);
+      bd_sum += bd;
+      if (EXACT) ex += static_cast<double>(wt[q]);
+    }
+    if constexpr (BF16) {
+      vs[u] = ((wt[0] + wt[1]) + (wt[2] + wt[3])) + ((wt[4] + wt[5]) + (wt[6] + wt[7]));
+    } else {
+      vs[u] = (wt[0] + wt[1]) + (wt[2] + wt[3]);
+    }
+  }
+  sum = vs[0] + vs[1];
+  exact = ex;
+  bound = bd_sum;
+}
+
+constexpr int kChunksPerSeg = SegGeo<true>::kSegVecs / Geo<true>::kChunkVecs;  // 2
+static_assert(SegGeo<false>::kSegVecs / Geo<false>::kChunkVecs == kChunksPerSeg, "geometry");
+
 struct SampleShared {
   double d[kWarps];
-  float f[kWarps];
+  double cm[kChunksPerSeg][kWarps];   // per chunk masses of each warp
+  double cb[kChunksPerSeg][kWarps];   // ... and bounds
   int flag;
   // locate
   int cstar;
   double base;        // weight before chunk cstar
-  double base_bound;  // bound before chunk cstar (incl. accumulation slack)
-  double total;       // total weight
-  double total_bound;
+  double base_bound;  // bound before chunk cstar
   int found;          // local index of the crossing in cstar, or -1
   double lo_gap, hi_gap, cell_bound;
 };
 
-// Chunk-ordered vectors again: thread t holds vectors t, t + 256, ... so the
-// loads coalesce, exactly as in the statistics pass.
+// One CTA per (request, segment of kChunksPerSeg chunks), coalesced loads, the
+// next batch's vectors in flight while the current one is reduced.
 template <bool BF16>
-__device__ __forceinline__ void chunk_mass(const RunParams& p, int i, const Job& jb, int c,
-                                           SampleShared& sh) {
-  using G = Geo<BF16>;
-  const WeightCtx w = weight_ctx(jb);
-  uint4 va[kUnroll], vb[kUnroll];
-  load_chunk<BF16>(target_row(p, i, jb.row, BF16), p.V, c, va);
-  if (w.residual) load_chunk<BF16>(draft_row(p, i, jb.row, BF16), p.V, c, vb);
-  float vsum[kUnroll];
-  float bound = 0.0f;
-#pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    float xa[G::kPerVec], xb[G::kPerVec], wt[G::kPerVec];
-    unpack<BF16>(va[u], xa);
-    if (w.residual) unpack<BF16>(vb[u], xb);
-#pragma unroll
-    for (int q = 0; q < G::kPerVec; ++q) {
-      float bd;
-      weight_and_bound(w, xa[q], w.residual ? xb[q] : 0.0f, wt[q], bd);
-      bound += bd;
+__device__ __forceinline__ void segment_masses(const RunParams& p, int i, const Job& jb, int seg,
+                                               SampleShared& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const JobF32 j = job_f32(jb);
+  const void* ra = target_row(p, i, jb.row, BF16);
+  const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
+  constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
+  const int c0 = seg * kChunksPerSeg;
+  uint4 va[kVecsPerBatch], vb[kVecsPerBatch], na[kVecsPerBatch], nb[kVecsPerBatch];
+  load_batch_coalesced<BF16>(ra, p.V, c0, 0, va);
+  if (j.residual) load_batch_coalesced<BF16>(rb, p.V, c0, 0, vb);
+  double cmass = 0.0, cbound = 0.0;
+#pragma unroll 1
+  for (int s = 0; s < kSteps; ++s) {
+    if (s + 1 < kSteps) {
+      const int c = c0 + (s + 1) / kBatchesPerChunk, b = (s + 1) % kBatchesPerChunk;
+      load_batch_coalesced<BF16>(ra, p.V, c, b, na);
+      if (j.residual) load_batch_coalesced<BF16>(rb, p.V, c, b, nb);
     }
-    if constexpr (BF16) {
-      vsum[u] = ((wt[0] + wt[1]) + (wt[2] + wt[3])) + ((wt[4] + wt[5]) + (wt[6] + wt[7]));
-    } else {
-      vsum[u] = (wt[0] + wt[1]) + (wt[2] + wt[3]);
+    float sum, bound;
+    double unused;
+    batch_weights<BF16, false>(j, va, vb, sum, unused, bound);
+    cmass += static_cast<double>(sum);
+    cbound += static_cast<double>(bound);
+    if ((s + 1) % kBatchesPerChunk == 0) {
+      const double m = warp_sum_d(cmass);
+      const double bb = warp_sum_d(cbound);
+      if (lane == 0) {
+        sh.cm[s / kBatchesPerChunk][warp] = m;
+        sh.cb[s / kBatchesPerChunk][warp] = bb;
+      }
+      cmass = 0.0;
+      cbound = 0.0;
+    }
+#pragma unroll
+    for (int u = 0; u < kVecsPerBatch; ++u) {
+      va[u] = na[u];
+      if (j.residual) vb[u] = nb[u];
     }
   }
-  const float tsum = (vsum[0] + vsum[1]) + (vsum[2] + vsum[3]);
-  const double mass = block_sum_d(static_cast<double>(tsum), sh.d);
-  // bound accumulated in fp32: inflate for its own rounding
-  const double bsum = static_cast<double>(block_sum_f(bound, sh.f)) * 1.001;
-  if (threadIdx.x == 0) {
-    SampleChunk r;
-    r.mass = mass;
-    // pairwise-sum rounding of the fp32 groups
-    r.bound = bsum + (G::kSumLevels + 1) * kU24 * mass;
-    p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
+  __syncthreads();
+  if (threadIdx.x < kChunksPerSeg) {
+    const int b = threadIdx.x;
+    const int c = c0 + b;
+    if (c < p.n_chunks) {
+      double m = 0.0, bb = 0.0;
+      for (int w2 = 0; w2 < kWarps; ++w2) {
+        m += sh.cm[b][w2];
+        bb += sh.cb[b][w2];
+      }
+      SampleChunk r;
+      r.mass = m;
+      // the bound was accumulated in fp32 per batch (inflate for its own
+      // rounding), plus the pairwise rounding of the fp32 batch sums
+      r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
+      p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
+    }
   }
 }
 
@@ -120,89 +221,104 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
   using G = Geo<BF16>;
   const int tid = threadIdx.x;
   const SampleChunk* sc = p.smass + static_cast<int64_t>(i) * p.n_chunks;
-  if (tid == 0) {
-    double total = 0.0, tb = 0.0;
-    for (int c = 0; c < p.n_chunks; ++c) {
+  // 1. block-wide prefix of the chunk masses and bounds (thread t: chunks 4t..4t+3)
+  double m[4], b[4], pm[4], pb[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = 4 * tid + q;
+    if (c < p.n_chunks) {
       const double2 r = __ldcg(reinterpret_cast<const double2*>(sc + c));
-      total += r.x;
-      tb += r.y;
+      m[q] = r.x;
+      b[q] = r.y;
+    } else {
+      m[q] = 0.0;
+      b[q] = 0.0;
     }
-    tb += 1e-15 * total;
-    const double target = jb.u2 * total;
-    double run = 0.0, runb = 0.0;
-    int cstar = -1;
-    for (int c = 0; c < p.n_chunks; ++c) {
-      const double2 r = __ldcg(reinterpret_cast<const double2*>(sc + c));
-      if (run + r.x > target) {
-        cstar = c;
-        break;
-      }
-      run += r.x;
-      runb += r.y;
+  }
+  if (tid == 0) sh.cstar = -1;
+  const double total = chunk_prefix(m, pm, sh.d);
+  __syncthreads();
+  const double tb = chunk_prefix(b, pb, sh.d) + 1e-15 * total;
+  const double target = jb.u2 * total;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int c = 4 * tid + q;
+    if (c < p.n_chunks && pm[q] <= target && pm[q] + m[q] > target) {
+      sh.cstar = c;
+      sh.base = pm[q];
+      sh.base_bound = pb[q] + 1e-15 * pm[q];
     }
-    sh.cstar = cstar;
-    sh.base = run;
-    sh.base_bound = runb + 1e-15 * run;
-    sh.total = total;
-    sh.total_bound = tb;
-    sh.found = -1;
-    // residual mass must clear the 1e-12 floor with certainty
-    if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) sh.cstar = -1;
   }
   __syncthreads();
-  const int cstar = sh.cstar;
+  int cstar = sh.cstar;
+  // residual mass must clear the 1e-12 floor with certainty
+  if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) cstar = -1;
   bool certain = false;
   int token = -1;
   if (cstar >= 0) {
-    // Rescan chunk cstar with contiguous per-thread segments (index order).
-    const WeightCtx w = weight_ctx(jb);
-    const int64_t chunk0 = static_cast<int64_t>(cstar) * G::kChunk;
-    const int64_t seg0 = chunk0 + static_cast<int64_t>(tid) * G::kPerThread;
+    // 2. rescan chunk cstar in index order (contiguous runs per thread): exact
+    //    fp64 sums of the fp32 weights and their bounds
+    const JobF32 j = job_f32(jb);
     const void* ra = target_row(p, i, jb.row, BF16);
-    const void* rb = w.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
-    float wt[G::kPerThread], bd[G::kPerThread];
+    const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
     double tsum = 0.0, tbound = 0.0;
-#pragma unroll 4
-    for (int e = 0; e < G::kPerThread; ++e) {
-      const int64_t t = seg0 + e;
-      if (t < p.V) {
-        const float a = load_logit(ra, t, BF16);
-        const float b = w.residual ? load_logit(rb, t, BF16) : 0.0f;
-        weight_and_bound(w, a, b, wt[e], bd[e]);
-      } else {
-        wt[e] = 0.0f;
-        bd[e] = 0.0f;
-      }
-      tsum += static_cast<double>(wt[e]);
-      tbound += static_cast<double>(bd[e]);
+#pragma unroll 1
+    for (int bt = 0; bt < kBatchesPerChunk; ++bt) {
+      uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+      load_batch_contiguous<BF16>(ra, p.V, cstar, bt, va);
+      if (j.residual) load_batch_contiguous<BF16>(rb, p.V, cstar, bt, vb);
+      else for (int u = 0; u < kVecsPerBatch; ++u) vb[u] = va[u];
+      float s, bd;
+      double ex;
+      batch_weights<BF16, true>(j, va, vb, s, ex, bd);
+      tsum += ex;
+      tbound += static_cast<double>(bd);
     }
     double all, allb;
     const double pre = block_exclusive_scan_d(tsum, sh.d, all);
     __syncthreads();
     const double preb = block_exclusive_scan_d(tbound, sh.d, allb);
-    const double target = jb.u2 * sh.total;
     const double start = sh.base + pre;
+    if (tid == 0) sh.found = -1;
+    __syncthreads();
     if (start <= target && start + tsum > target) {
-      double run = start, runb = sh.base_bound + preb;
-      for (int e = 0; e < G::kPerThread; ++e) {
-        const double before = run;
-        run += static_cast<double>(wt[e]);
-        runb += static_cast<double>(bd[e]);
-        if (run > target) {
-          sh.found = static_cast<int>(seg0 - chunk0) + e;
-          sh.lo_gap = target - before;
-          sh.hi_gap = run - target;
-          sh.cell_bound = runb;
-          break;
+      // the one thread holding the crossing walks its logits again (same values)
+      double run = start, runb = sh.base_bound + preb * 1.001;
+      bool done = false;
+      for (int bt = 0; bt < kBatchesPerChunk && !done; ++bt) {
+        uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+        const int off = load_batch_contiguous<BF16>(ra, p.V, cstar, bt, va);
+        if (j.residual) load_batch_contiguous<BF16>(rb, p.V, cstar, bt, vb);
+        else for (int u = 0; u < kVecsPerBatch; ++u) vb[u] = va[u];
+        const WeightCtx w = weight_ctx(j, vec_max<BF16>(va), j.residual ? vec_max<BF16>(vb) : 0.0f);
+        for (int u = 0; u < kVecsPerBatch && !done; ++u) {
+          float xa[G::kPerVec], xb[G::kPerVec];
+          unpack<BF16>(va[u], xa);
+          if (j.residual) unpack<BF16>(vb[u], xb);
+          for (int q = 0; q < G::kPerVec; ++q) {
+            float wt, bq;
+            weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt, bq);
+            const double before = run;
+            run += static_cast<double>(wt);
+            runb += static_cast<double>(bq) * 1.001;
+            if (run > target) {
+              sh.found = off + u * G::kPerVec + q;
+              sh.lo_gap = target - before;
+              sh.hi_gap = run - target;
+              sh.cell_bound = runb;
+              done = true;
+              break;
+            }
+          }
         }
       }
     }
     __syncthreads();
     if (tid == 0 && sh.found >= 0) {
-      const double slack = jb.u2 * sh.total_bound + 1e-14 * sh.total;
+      const double slack = jb.u2 * tb + 1e-14 * total;
       const double need = sh.cell_bound + slack;
       certain = sh.lo_gap > need && sh.hi_gap > need;
-      token = static_cast<int>(chunk0 + sh.found);
+      token = static_cast<int>(static_cast<int64_t>(cstar) * G::kChunk + sh.found);
     }
   }
   if (tid == 0) {
@@ -217,15 +333,15 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads) k_sample(RunParams p) {
+__global__ void __launch_bounds__(kThreads, 3) k_sample(RunParams p) {
   __shared__ SampleShared sh;
   const int64_t b = blockIdx.x;
-  const int i = static_cast<int>(b / p.n_chunks);
-  const int c = static_cast<int>(b % p.n_chunks);
+  const int i = static_cast<int>(b / p.n_segs);
+  const int seg = static_cast<int>(b % p.n_segs);
   const Job jb = p.jobs[i];
   if (jb.kind == kJobNone) return;
-  chunk_mass<BF16>(p, i, jb, c, sh);
-  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_chunks), &sh.flag)) return;
+  segment_masses<BF16>(p, i, jb, seg, sh);
+  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_segs), &sh.flag)) return;
   __threadfence();
   locate_sample<BF16>(p, i, jb, sh);
 }

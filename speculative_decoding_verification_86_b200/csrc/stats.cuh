@@ -23,28 +23,50 @@
 namespace sv {
 
 // ---------------------------------------------------------------------------
-// Chunk statistics of one row.
+// Streaming statistics of one row segment.
+//
+// A segment is kThreads x kSegVecsPerThread 16-byte vectors (32768 bf16 or
+// 16384 fp32 logits); thread t owns vectors t, t + 256, ... so every load
+// instruction of a warp covers 512 contiguous bytes.  The vectors arrive in
+// batches of kBatchVecs, the next batch's loads issued before the current one
+// is reduced.  Each thread keeps its own exponent reference K_t: an integer,
+// raised to ceil(max * c) whenever a batch brings a larger logit, so the
+// rescaling of its running sums is an exact power of two and no block-wide
+// maximum is needed before the exponentials.  One barrier per segment merges
+// the threads.
 // ---------------------------------------------------------------------------
+constexpr int kSegVecsPerThread = 16;
+constexpr int kBatchVecs = 4;
+constexpr int kBatches = kSegVecsPerThread / kBatchVecs;
+
 template <bool BF16>
-__device__ __forceinline__ void load_chunk(const void* row, int64_t V, int c,
-                                           uint4 (&v)[kUnroll]) {
-  using G = Geo<BF16>;
-  const int64_t nvec = V / G::kPerVec;
-  const uint4* rv = static_cast<const uint4*>(row);
-  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
+struct SegGeo {
+  static constexpr int kPerVec = BF16 ? 8 : 4;
+  static constexpr int kSegVecs = kThreads * kSegVecsPerThread;   // 4096 vectors
+  static constexpr int kSeg = kSegVecs * kPerVec;                 // logits per segment
+  static constexpr int kBatchElems = kBatchVecs * kPerVec;        // per thread per batch
+  static constexpr int kSumLevels = BF16 ? 5 : 4;                 // pairwise depth of a batch sum
+};
+
+template <bool BF16>
+__device__ __forceinline__ void load_batch(const uint4* rv, int64_t nvec, int64_t seg0, int b,
+                                           uint4 (&v)[kBatchVecs]) {
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
-    const int64_t idx = base + u * kThreads;
+  for (int u = 0; u < kBatchVecs; ++u) {
+    const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
     v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
   }
 }
 
+// NaN-propagating maximum of one batch.
 template <bool BF16>
-__device__ __forceinline__ float chunk_local_max(const uint4 (&v)[kUnroll]) {
+__device__ __forceinline__ float batch_max(const uint4 (&v)[kBatchVecs]) {
   if constexpr (BF16) {
-    uint32_t m2 = v[0].x;
+    uint32_t m2 = hmax2_nan(v[0].x, v[0].y);
+    m2 = hmax2_nan(m2, v[0].z);
+    m2 = hmax2_nan(m2, v[0].w);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 1; u < kBatchVecs; ++u) {
       m2 = hmax2_nan(m2, v[u].x);
       m2 = hmax2_nan(m2, v[u].y);
       m2 = hmax2_nan(m2, v[u].z);
@@ -52,9 +74,11 @@ __device__ __forceinline__ float chunk_local_max(const uint4 (&v)[kUnroll]) {
     }
     return fmax_nan(bf16_lo(m2), bf16_hi(m2));
   } else {
-    float m = __uint_as_float(v[0].x);
+    float m = fmax_nan(__uint_as_float(v[0].x), __uint_as_float(v[0].y));
+    m = fmax_nan(m, __uint_as_float(v[0].z));
+    m = fmax_nan(m, __uint_as_float(v[0].w));
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int u = 1; u < kBatchVecs; ++u) {
       m = fmax_nan(m, __uint_as_float(v[u].x));
       m = fmax_nan(m, __uint_as_float(v[u].y));
       m = fmax_nan(m, __uint_as_float(v[u].z));
@@ -64,96 +88,236 @@ __device__ __forceinline__ float chunk_local_max(const uint4 (&v)[kUnroll]) {
   }
 }
 
+// Exact 2^d for an integer-valued d <= 0 (0 below the double range).
+__device__ __forceinline__ double pow2_exact(float d) {
+  return d < -1074.0f ? 0.0 : ldexp(1.0, static_cast<int>(d));
+}
+
 struct StatsShared {
-  float f[kWarps];
-  double d[kWarps];
-  int i[kWarps];
+  float K[kWarps];
+  double s[kWarps];
+  float er[kWarps];
+  float om[kWarps];
+  float mraw[kWarps];
+  int bad[kWarps];
+  int arg[kWarps];
   int flag;
 };
 
-// Softmax statistics of chunk c of a stochastic row.
-template <bool BF16>
-__device__ __forceinline__ void stochastic_chunk(const void* row, int64_t V, int c, float cc,
-                                                 ChunkMeta* meta_out, double* sum_out,
-                                                 StatsShared& sh) {
-  using G = Geo<BF16>;
-  uint4 v[kUnroll];
-  load_chunk<BF16>(row, V, c, v);
-  const float m = block_max_nan(chunk_local_max<BF16>(v), sh.f);
-  // NaN or +inf anywhere in the chunk, or nothing but -inf: no exponentials.
-  if (!(m > -INFINITY) || isinf(m) || isnan(m)) {
-    if (threadIdx.x == 0) {
-      ChunkMeta r;
-      r.K = (isnan(m) || m > 0.0f) ? (isnan(m) ? m : INFINITY) : -INFINITY;
-      r.mraw = m;
-      r.err = 0.0f;
-      r.arg = 0;
-      *meta_out = r;
-      *sum_out = (isnan(m) || m > 0.0f) ? __longlong_as_double(0x7ff8000000000000LL) : 0.0;
+// Running softmax statistics of one thread, in the thread's frame K (integer).
+//   s  = sum of e_t = 2^(fl(l_t c - K)),
+//   er = sum of e_t |a_t| with a_t the rounded exponent at the time the term
+//        was computed (bounds the exponent rounding, relative per term),
+//   om = sum of e_t (K - K_then): how far the term's own frame lay below K.
+struct SoftAcc {
+  float K = -INFINITY;
+  double s = 0.0;
+  float er = 0.0f;
+  float om = 0.0f;
+  float mraw = -INFINITY;
+  int bad = 0;
+
+  __device__ __forceinline__ void rebase(float Knew) {  // Knew > K
+    if (K == -INFINITY) {
+      s = 0.0;
+      er = 0.0f;
+      om = 0.0f;
+    } else {
+      const double f = pow2_exact(K - Knew);
+      const float ff = static_cast<float>(f);
+      om = (om + (Knew - K) * static_cast<float>(s)) * ff;
+      s *= f;
+      er *= ff;
     }
-    return;
+    K = Knew;
   }
-  const float K = m * cc;
-  float vsum[kUnroll];
-  float err = 0.0f;
+};
+
+template <bool BF16>
+__device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatchVecs], float cc) {
+  using G = SegGeo<BF16>;
+  const float bm = batch_max<BF16>(v);
+  acc.mraw = fmax_nan(acc.mraw, bm);
+  if (isnan(bm) || bm == INFINITY) acc.bad = 1;
+  const float Kb = ceilf(bm * cc);
+  if (Kb > acc.K) acc.rebase(Kb);
+  if (!(acc.K > -INFINITY) || acc.K == INFINITY) return;  // nothing finite yet, or +inf seen
+  const float K = acc.K;
+  float vs[kBatchVecs];
+  float er = acc.er;
 #pragma unroll
-  for (int u = 0; u < kUnroll; ++u) {
+  for (int u = 0; u < kBatchVecs; ++u) {
     float x[G::kPerVec];
     unpack<BF16>(v[u], x);
     float e[G::kPerVec];
 #pragma unroll
     for (int q = 0; q < G::kPerVec; ++q) {
-      const float a = fmaxf(fmaf(x[q], cc, -K), -1024.0f);
+      const float a = fmaxf(fmaf(x[q], cc, -K), -1024.0f);  // <= 0; -inf (masked) -> -1024
       e[q] = ex2_approx(a);
-      err = fmaf(e[q], fabsf(a), err);
+      er = fmaf(e[q], -a, er);
     }
     if constexpr (BF16) {
-      vsum[u] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
+      vs[u] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
     } else {
-      vsum[u] = (e[0] + e[1]) + (e[2] + e[3]);
+      vs[u] = (e[0] + e[1]) + (e[2] + e[3]);
     }
   }
-  const float tsum = (vsum[0] + vsum[1]) + (vsum[2] + vsum[3]);
-  const double s = block_sum_d(static_cast<double>(tsum), sh.d);
-  const float errs = block_sum_f(err, sh.f);
-  if (threadIdx.x == 0) {
-    ChunkMeta r;
-    r.K = K;
-    r.mraw = m;
-    r.err = errs;
-    r.arg = 0;
-    *meta_out = r;
-    *sum_out = s;
+  acc.er = er;
+  acc.s += static_cast<double>((vs[0] + vs[1]) + (vs[2] + vs[3]));
+}
+
+// Merge `acc` of all threads of the CTA into one record (called by every thread).
+__device__ __forceinline__ void soft_merge_block(SoftAcc acc, StatsShared& sh, ChunkMeta* meta_out,
+                                                 double* sum_out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int level = 0; level < 2; ++level) {
+    int bad = __any_sync(0xffffffffu, acc.bad);
+    float Kw = acc.K;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) Kw = fmaxf(Kw, __shfl_xor_sync(0xffffffffu, Kw, off));
+    double s = 0.0;
+    float er = 0.0f, om = 0.0f;
+    if (!bad && acc.K > -INFINITY) {
+      const double f = pow2_exact(acc.K - Kw);
+      const float ff = static_cast<float>(f);
+      s = acc.s * f;
+      er = acc.er * ff;
+      om = (acc.om + (Kw - acc.K) * static_cast<float>(acc.s)) * ff;
+    }
+    s = warp_sum_d(s);
+    er = warp_sum_f(er);
+    om = warp_sum_f(om);
+    const float mraw = warp_max_nan(acc.mraw);
+    if (level == 0) {
+      if (lane == 0) {
+        sh.K[warp] = Kw;
+        sh.s[warp] = s;
+        sh.er[warp] = er;
+        sh.om[warp] = om;
+        sh.mraw[warp] = mraw;
+        sh.bad[warp] = bad;
+      }
+      __syncthreads();
+      if (warp != 0) return;
+      const bool have = lane < kWarps;
+      acc.K = have ? sh.K[lane] : -INFINITY;
+      acc.s = have ? sh.s[lane] : 0.0;
+      acc.er = have ? sh.er[lane] : 0.0f;
+      acc.om = have ? sh.om[lane] : 0.0f;
+      acc.mraw = have ? sh.mraw[lane] : -INFINITY;
+      acc.bad = have ? sh.bad[lane] : 0;
+    } else if (lane == 0) {
+      ChunkMeta r;
+      if (bad || isnan(mraw) || mraw == INFINITY) {
+        r.K = __int_as_float(0x7fc00000);  // NaN marks a row the chain must not use
+        *sum_out = __longlong_as_double(0x7ff8000000000000LL);
+      } else {
+        r.K = Kw;  // -inf if the segment held only masked logits
+        *sum_out = Kw == -INFINITY ? 0.0 : s;
+      }
+      r.mraw = mraw;
+      r.err = er;
+      r.arg = __float_as_int(om);
+      *meta_out = r;
+    }
   }
 }
 
-// Max and lowest arg-max of chunk c of a greedy row.
 template <bool BF16>
-__device__ __forceinline__ void greedy_chunk(const void* row, int64_t V, int c, ChunkMeta* meta_out,
-                                             StatsShared& sh) {
-  using G = Geo<BF16>;
-  uint4 v[kUnroll];
-  load_chunk<BF16>(row, V, c, v);
-  const float m = block_max_nan(chunk_local_max<BF16>(v), sh.f);
-  int first = INT_MAX;
-  const int64_t chunk0 = static_cast<int64_t>(c) * G::kChunk;
+__device__ __forceinline__ void stochastic_segment(const void* row, int64_t V, int seg, float cc,
+                                                   ChunkMeta* meta_out, double* sum_out,
+                                                   StatsShared& sh) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  SoftAcc acc;
+  uint4 va[kBatchVecs], vb[kBatchVecs];
+  load_batch<BF16>(rv, nvec, seg0, 0, va);
 #pragma unroll
-  for (int u = kUnroll - 1; u >= 0; --u) {  // later vectors first, so the lowest index wins
-    float x[G::kPerVec];
-    unpack<BF16>(v[u], x);
-#pragma unroll
-    for (int q = G::kPerVec - 1; q >= 0; --q) {
-      if (x[q] == m) first = (u * kThreads + threadIdx.x) * G::kPerVec + q;
-    }
+  for (int b = 0; b < kBatches; b += 2) {
+    if (b + 1 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 1, vb);
+    soft_batch<BF16>(acc, va, cc);
+    if (b + 2 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 2, va);
+    if (b + 1 < kBatches) soft_batch<BF16>(acc, vb, cc);
   }
-  first = block_min_i(first, sh.i);
-  if (threadIdx.x == 0) {
-    ChunkMeta r;
-    r.K = 0.0f;
-    r.mraw = m;
-    r.err = 0.0f;
-    r.arg = first == INT_MAX ? -1 : static_cast<int>(chunk0 + first);
-    *meta_out = r;
+  soft_merge_block(acc, sh, meta_out, sum_out);
+}
+
+// Max and lowest arg-max of one segment of a greedy row.
+template <bool BF16>
+__device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int seg,
+                                               ChunkMeta* meta_out, StatsShared& sh) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  float best = -INFINITY;
+  int64_t best_idx = INT64_MAX;
+  int bad = 0;
+  uint4 va[kBatchVecs], vb[kBatchVecs];
+  auto scan = [&](const uint4 (&v)[kBatchVecs], int b) {
+    const float bm = batch_max<BF16>(v);
+    if (isnan(bm)) bad = 1;
+    if (!(bm > best) && best_idx != INT64_MAX) return;  // earlier batches hold lower indices
+    if (!(bm >= best)) return;
+    // first element of this batch equal to its max, in index order
+    int64_t first = INT64_MAX;
+#pragma unroll
+    for (int u = kBatchVecs - 1; u >= 0; --u) {
+      float x[G::kPerVec];
+      unpack<BF16>(v[u], x);
+#pragma unroll
+      for (int q = G::kPerVec - 1; q >= 0; --q) {
+        if (x[q] == bm)
+          first = (seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x) *
+                      G::kPerVec + q;
+      }
+    }
+    best = bm;
+    best_idx = first;
+  };
+  load_batch<BF16>(rv, nvec, seg0, 0, va);
+#pragma unroll
+  for (int b = 0; b < kBatches; b += 2) {
+    if (b + 1 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 1, vb);
+    scan(va, b);
+    if (b + 2 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 2, va);
+    if (b + 1 < kBatches) scan(vb, b + 1);
+  }
+  // block reduction: larger value wins, ties go to the lower index
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int idx = best_idx == INT64_MAX ? INT_MAX : static_cast<int>(best_idx);
+  for (int level = 0; level < 2; ++level) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+      if (ob > best || (ob == best && oi < idx)) {
+        best = ob;
+        idx = oi;
+      }
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (level == 0) {
+      if (lane == 0) {
+        sh.mraw[warp] = best;
+        sh.arg[warp] = idx;
+        sh.bad[warp] = bad;
+      }
+      __syncthreads();
+      if (warp != 0) return;
+      best = lane < kWarps ? sh.mraw[lane] : -INFINITY;
+      idx = lane < kWarps ? sh.arg[lane] : INT_MAX;
+      bad = lane < kWarps ? sh.bad[lane] : 0;
+    } else if (lane == 0) {
+      ChunkMeta r;
+      r.K = 0.0f;
+      r.mraw = bad ? __int_as_float(0x7fc00000) : best;
+      r.err = 0.0f;
+      r.arg = idx == INT_MAX ? -1 : idx;
+      *meta_out = r;
+    }
   }
 }
 
@@ -161,9 +325,10 @@ __device__ __forceinline__ void greedy_chunk(const void* row, int64_t V, int c, 
 // Merged row records, built by the deciding CTA in shared memory.
 // ---------------------------------------------------------------------------
 struct RowMerged {
-  double Z;      // sum of 2^(l c - K) over the row (fp32 terms)
-  double E;      // bound on sum e |a| in the row's frame
-  float K;       // exponent reference (max over chunks)
+  double Z;      // sum of 2^(fl(l c - K_then)) 2^(K_then - K) over the row (fp32 terms)
+  double ER;     // sum of e |a_then| in the row's frame: exponent-rounding weight
+  double EA;     // sum of e |a| with a measured from K: Z times minus the mean exponent
+  float K;       // exponent reference of the row (integer)
   float mraw;    // raw max
   int arg;       // greedy: lowest arg-max
   int bad;       // NaN / +inf / all -inf
@@ -178,43 +343,47 @@ struct DecideShared {
   double exact_Za, exact_Zb;
 };
 
-// Merge the chunk records of stochastic row `slot` with one warp.
+// Merge the segment records of stochastic row `slot` with one warp.
 __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, int slot,
                                                      RowMerged& out) {
   const int lane = threadIdx.x & 31;
-  const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_chunks;
+  const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
   float K = -INFINITY, mraw = -INFINITY;
   int bad = 0;
-  for (int c = lane; c < p.n_chunks; c += 32) {
+  for (int c = lane; c < p.n_segs; c += 32) {
     const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
-    const float Kc = m4.x;
-    if (isnan(Kc) || Kc == INFINITY) bad = 1;
-    K = fmaxf(K, Kc);
+    if (isnan(m4.x) || m4.x == INFINITY) bad = 1;
+    K = fmaxf(K, m4.x);
     mraw = fmax_nan(mraw, m4.y);
   }
   K = warp_max_nan(K);
   mraw = warp_max_nan(mraw);
   bad = __any_sync(0xffffffffu, bad);
   if (!(K > -INFINITY)) bad = 1;
-  double Z = 0.0, E = 0.0;
+  double Z = 0.0, ER = 0.0, EA = 0.0;
   if (!bad) {
-    for (int c = lane; c < p.n_chunks; c += 32) {
+    for (int c = lane; c < p.n_segs; c += 32) {
       const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
       if (m4.x == -INFINITY) continue;
       const double s = __ldcg(p.ssum + base + c);
-      const double d = static_cast<double>(m4.x) - static_cast<double>(K);  // <= 0, exact
-      const double f = exp2(d);
+      const double d = static_cast<double>(K) - static_cast<double>(m4.x);  // integer >= 0
+      const double f = pow2_exact(static_cast<float>(-d));
       Z += s * f;
-      // |a| measured against K_c; against K it grows by at most (K - K_c) per unit mass.
-      E += (static_cast<double>(m4.z) + (-d) * s) * f;
+      ER += static_cast<double>(m4.z) * f;
+      // |a| from K = |a_then| + (K_then's distance below K): the rounding weight,
+      // plus the offsets recorded inside the segment, plus the segment's own offset.
+      EA += (static_cast<double>(m4.z) + static_cast<double>(m4.w) +
+             d * s) * f;
     }
   }
   Z = warp_sum_d(Z);
-  E = warp_sum_d(E);
+  ER = warp_sum_d(ER);
+  EA = warp_sum_d(EA);
   if (!(Z > 0.0) || isinf(Z) || isnan(Z)) bad = 1;
   if (lane == 0) {
     out.Z = Z;
-    out.E = E;
+    out.ER = ER;
+    out.EA = EA;
     out.K = K;
     out.mraw = mraw;
     out.arg = -1;
@@ -225,11 +394,11 @@ __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, 
 __device__ __forceinline__ void merge_greedy_row(const RunParams& p, int i, int slot,
                                                  RowMerged& out) {
   const int lane = threadIdx.x & 31;
-  const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_chunks;
+  const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
   float best = -INFINITY;
   int arg = INT_MAX;
   int bad = 0;
-  for (int c = lane; c < p.n_chunks; c += 32) {
+  for (int c = lane; c < p.n_segs; c += 32) {
     const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
     const float m = m4.y;
     const int a = __float_as_int(m4.w);
@@ -252,7 +421,8 @@ __device__ __forceinline__ void merge_greedy_row(const RunParams& p, int i, int 
   if (isinf(best)) bad = 1;  // +inf, or -inf everywhere
   if (lane == 0) {
     out.Z = 0.0;
-    out.E = 0.0;
+    out.ER = 0.0;
+    out.EA = 0.0;
     out.K = 0.0f;
     out.mraw = best;
     out.arg = arg;
@@ -350,8 +520,14 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   const float cc = static_cast<float>(1.4426950408889634 / T);
   const double c_exact = 1.4426950408889634 / T;
   const double eta = fabs((c_exact - static_cast<double>(cc)) / static_cast<double>(cc));
+  // Relative error of a row's fp32 normaliser Z~: one ex2 error per term, the
+  // pairwise rounding of the batch sums, and the exponent rounding (weighted by
+  // sum e|a|).  Rounding log2(e)/T to fp32 (relative eta) reshapes p itself:
+  // log p/p~ moves by at most ln2 * eta * |a_x - mean(a)|.
   const double kappa = kLn2 * (kU24 + eta) * 1.0001;
-  const double eps_base = static_cast<double>(p.eps_ex2) + (Geo<BF16>::kSumLevels + 1) * kU24 + 1e-14;
+  const double eps_base =
+      static_cast<double>(p.eps_ex2) + SegGeo<BF16>::kSumLevels * kU24 + 1e-14;
+  auto dZ = [&](const RowMerged& r) { return eps_base + kLn2 * kU24 * 1.0001 * r.ER / r.Z; };
 
   // thread 0 carries the chain; other threads join the fp64 slow path.
   int n = L;
@@ -382,9 +558,9 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
         if (qb == 0.0) {
           decision = pa > 0.0 ? 1 : 0;
         } else {
-          const double dp = eps_base + kappa * ra.E / ra.Z + kLn2 * eta * fabs(arg_a);
-          const double dq = eps_base + kappa * rb.E / rb.Z + kLn2 * eta * fabs(arg_b);
-          const double delta = (dp + dq) * 1.01;
+          const double dp = dZ(ra) + kLn2 * eta * (fabs(arg_a + ra.EA / ra.Z) + 1e-3);
+          const double dq = dZ(rb) + kLn2 * eta * (fabs(arg_b + rb.EA / rb.Z) + 1e-3);
+          const double delta = (dp + dq) * 1.01 + 1e-13;
           const double rho = pa / qb;
           if (u < rho * (1.0 - delta)) decision = 1;
           else if (u >= rho * (1.0 + delta)) decision = 0;
@@ -454,6 +630,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     jb.pad0 = 0;
     jb.cc = cc;
     jb.kappa = static_cast<float>(kappa);
+    jb.eta_ln2 = kLn2 * eta;
     jb.T = T;
     jb.u2 = draw(p, i, n, 1);
     const RowMerged& ra = sh.rows[n];
@@ -469,8 +646,23 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
       jb.Bq = static_cast<float>(1.0 / rb.Z);
       // per-term constant: ex2 error, rounding of 1/Z and of the products,
       // the normaliser's own bound (incl. the temperature-rounding term).
-      jb.eps0a = eps_base + 3 * kU24 + kappa * ra.E / ra.Z;
-      jb.eps0b = eps_base + 3 * kU24 + kappa * rb.E / rb.Z;
+      // per term: ex2 error, rounding of 1/Z, of the scaled product and of the
+      // difference, the normaliser's own bound, and |mean exponent| of the
+      // temperature-rounding term (the frame adds its offset, the term its |a|).
+      jb.eps0a = static_cast<double>(p.eps_ex2) + 4 * kU24 + dZ(ra) + kLn2 * eta * ra.EA / ra.Z;
+      jb.eps0b = static_cast<double>(p.eps_ex2) + 4 * kU24 + dZ(rb) + kLn2 * eta * rb.EA / rb.Z;
+      // Bracket of rho = Z_a / Z_b in the refinement's frames (each row relative
+      // to its own max at the true temperature): the fp32 sums' bounds, the
+      // reshaping by the rounded temperature factor, and a factor 3 of margin.
+      const double cex = c_exact;
+      const double rho = (ra.Z / rb.Z) *
+          exp2((static_cast<double>(ra.K) - static_cast<double>(rb.K)) -
+               (static_cast<double>(ra.mraw) - static_cast<double>(rb.mraw)) * cex);
+      const double band = 3.0 * (dZ(ra) + dZ(rb) +
+          kLn2 * eta * (fabs(static_cast<double>(ra.mraw) - static_cast<double>(rb.mraw)) * cex +
+                        ra.EA / ra.Z + rb.EA / rb.Z + 1.0)) + 1e-12;
+      jb.rho_lo = rho * (1.0 - band);
+      jb.rho_hi = rho * (1.0 + band);
     } else {
       jb.kind = kJobBonus;
       jb.Kb = 0.0f;
@@ -479,13 +671,15 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
       jb.Bq = 0.0f;
       jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + 1e-14;
       jb.eps0b = 0.0;
+      jb.rho_lo = 0.0;
+      jb.rho_hi = 0.0;
     }
     *job = jb;
   }
 }
 
 // ---------------------------------------------------------------------------
-// The kernel: one CTA per (request, row slot, chunk).
+// The kernel: one CTA per (request, row slot, segment).
 // ---------------------------------------------------------------------------
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) k_stats(RunParams p) {
@@ -493,8 +687,8 @@ __global__ void __launch_bounds__(kThreads) k_stats(RunParams p) {
   __shared__ DecideShared dsh;
   const int rows_per_req = 2 * p.k + 1;
   const int64_t b = blockIdx.x;
-  const int c = static_cast<int>(b % p.n_chunks);
-  const int64_t slot_global = b / p.n_chunks;
+  const int seg = static_cast<int>(b % p.n_segs);
+  const int64_t slot_global = b / p.n_segs;
   const int i = static_cast<int>(slot_global / rows_per_req);
   const int slot = static_cast<int>(slot_global - static_cast<int64_t>(i) * rows_per_req);
   if (b == 0 && threadIdx.x == 0) *p.counters_next = Counters{0u, 0u, 0u, 0u};
@@ -503,24 +697,25 @@ __global__ void __launch_bounds__(kThreads) k_stats(RunParams p) {
   const bool is_draft = slot > p.k;
   const int j = is_draft ? slot - (p.k + 1) : slot;
   bool needed;
-  if (ri.bad_T) needed = (slot == 0 && c == 0);
+  if (ri.bad_T) needed = (slot == 0 && seg == 0);
   else if (ri.greedy) needed = !is_draft && j <= ri.L;
   else needed = is_draft ? (j < ri.L) : (j <= ri.L);
   if (!needed) return;
 
   if (!ri.bad_T) {
-    const int64_t rec = slot_global * p.n_chunks + c;
+    const int64_t rec = slot_global * p.n_segs + seg;
     const void* row = is_draft ? draft_row(p, i, j, BF16) : target_row(p, i, j, BF16);
     if (ri.greedy) {
-      greedy_chunk<BF16>(row, p.V, c, p.meta + rec, sh);
+      greedy_segment<BF16>(row, p.V, seg, p.meta + rec, sh);
     } else {
       const float cc = static_cast<float>(1.4426950408889634 / static_cast<double>(ri.T));
-      stochastic_chunk<BF16>(row, p.V, c, cc, p.meta + rec, p.ssum + rec, sh);
+      stochastic_segment<BF16>(row, p.V, seg, cc, p.meta + rec, p.ssum + rec, sh);
     }
   }
-  if (!arrive_last(p.arrive_stats + i, static_cast<unsigned>(stats_expected(ri, p.n_chunks)),
+  if (!arrive_last(p.arrive_stats + i, static_cast<unsigned>(stats_expected(ri, p.n_segs)),
                    &sh.flag))
     return;
+  __threadfence();
   decide_request<BF16>(p, i, ri, dsh);
 }
 
