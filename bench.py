@@ -50,6 +50,7 @@ def parse_args():
     ap.add_argument("--workload", default="headline")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="prefix", choices=["prefix", "dense"])
     return ap.parse_args()
 
 
@@ -91,6 +92,20 @@ def dense_row_bytes(w, L):
     T = w.get("temperature")
     sampled = (T > 0) if T is not None else torch.ones_like(L, dtype=torch.bool)
     rows = (L + 1) + torch.where(sampled, L, torch.zeros_like(L))
+    return int(rows.sum().item()) * V * es
+
+
+def prefix_row_bytes(w, L, accepted):
+    """Algorithmic bytes in prefix order: rows up to and including the first
+    rejection (or the bonus row): n_i + 1 target rows and, for sampled
+    requests, min(n_i + 1, L_i) draft rows."""
+    import torch
+    V = w["target"].shape[2]
+    es = w["target"].element_size()
+    T = w.get("temperature")
+    sampled = (T > 0) if T is not None else torch.ones_like(L, dtype=torch.bool)
+    n = accepted.clamp(min=0)
+    rows = (n + 1) + torch.where(sampled, torch.minimum(n + 1, L), torch.zeros_like(L))
     return int(rows.sum().item()) * V * es
 
 
@@ -285,7 +300,7 @@ def run_ours(args):
     L = effective_lengths(w)
     positions = int(L.sum().item())
     step_bytes = dense_row_bytes(w, L)
-    ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V)
+    ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V, mode=args.mode)
     out = ver._outputs(B, k, True)
     stream = torch.cuda.current_stream(dev)
 
@@ -322,27 +337,34 @@ def run_ours(args):
     ver.timing_enable([])
     clk = clocks.stop()
     counters = ver.last_counters()
-    # per-kernel breakdown, in a separate loop so the timed region carries only
-    # the events around the statistics kernel
-    ver.timing_enable([binding.TIMING_STATS, binding.TIMING_SAMPLE, binding.TIMING_REFINE,
-                       binding.TIMING_CONF])
-    nb = min(args.steps, 200)
+    # the other statistics order, timed the same way on the same batch
+    other = "dense" if ver.mode == "prefix" else "prefix"
+    ver.set_mode(other)
+    for _ in range(3):
+        step()
+    nb = min(args.steps, 500)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    o0 = torch.cuda.Event(enable_timing=True)
+    o1 = torch.cuda.Event(enable_timing=True)
+    o0.record(stream)
     for _ in range(nb):
         step()
-    breakdown = {}
-    for name, cls in (("stats", binding.TIMING_STATS), ("sample", binding.TIMING_SAMPLE),
-                      ("refine", binding.TIMING_REFINE), ("conf", binding.TIMING_CONF)):
-        n_c, ms_c = ver.timing_read(cls)
-        if n_c:
-            breakdown[name + "_ms"] = ms_c / n_c
-    ver.timing_enable([])
+    o1.record(stream)
+    torch.cuda.synchronize(dev)
+    other_ms = o0.elapsed_time(o1) / nb
+    other_line = {"mode": other, "ms_per_step": other_ms,
+                  "value": positions * world / (other_ms / 1e3),
+                  "hbm_gbs": dense_row_bytes(w, L) / (other_ms * 1e-3) / 1e9 if other == "dense" else None}
+    ver.set_mode(args.mode)
     t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms_total = float(t.item())
     ms_per_step = ms_total / args.steps
     value = positions * world / (ms_per_step / 1e3)
-    launches_per_step = 3 + (1 if w.get("conf") is not None else 0)
+    launches_per_step = 1 + (1 if w.get("conf") is not None else 0)
 
     # end to end: host buffers in, host results out, through the C ABI
     e2e = None
@@ -405,24 +427,27 @@ def run_ours(args):
     else:
         peak, peak_src = FALLBACK_HBM_GBS, "fallback"
     ms_stats_avg = ms_stats / max(n_stats, 1)
-    achieved = step_bytes / (ms_stats_avg * 1e-3) / 1e9 if n_stats else None
-    traffic = profiled_traffic("k_stats", args.workload.replace(":", ""))
-    step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
+    algo_bytes = step_bytes if args.mode == "dense" else prefix_row_bytes(w, L, out["accepted"])
+    achieved = algo_bytes / (ms_stats_avg * 1e-3) / 1e9 if n_stats else None
+    traffic = profiled_traffic("k_engine", "%s_%s" % (args.workload.replace(":", ""), args.mode))
+    step_gbs = algo_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
         "data": "synthetic", "config": config_dict(w, args.workload, world, L),
         "hbm_gbs": step_gbs, "hbm_frac_measured": step_gbs / peak, "hbm_frac_nominal_8tbs": step_gbs / NOMINAL_HBM_GBS,
-        "roofline": {"bound": "hbm", "kernel": "k_stats", "achieved": achieved, "peak": peak,
+        "roofline": {"bound": "hbm", "kernel": "k_engine", "achieved": achieved, "peak": peak,
                      "peak_source": peak_src, "unit": "GB/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": step_bytes,
+                     "algorithmic_bytes_per_launch": algo_bytes,
+                     "algorithmic_bytes_dense": step_bytes,
                      "launch_ms": ms_stats_avg, "launches_timed": n_stats},
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
         "fp64_paths": counters,
-        "kernel_ms": breakdown,
+        "mode": args.mode,
+        "other_mode": other_line,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -71,6 +71,15 @@ typedef enum {
 
 typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
+/* Order in which the statistics pass reads a request's rows.  Both give the
+ * same outputs, bit for bit:
+ *   SPEC_MODE_PREFIX (default): position j+1's rows are read only once position
+ *     j was accepted ("at the first disagreement ... throw away the rest of
+ *     the draft"), so rows past the first rejection are never touched;
+ *   SPEC_MODE_DENSE: every verified position's target and draft rows are
+ *     reduced, then the chain is walked. */
+typedef enum { SPEC_MODE_DENSE = 0, SPEC_MODE_PREFIX = 1 } spec_mode;
+
 /* Per-request device status bits (out_status[i]); 0 means success. */
 #define SPEC_DEV_BAD_TOKEN 1u       /* a drafted token the chain reached is outside [0, V) */
 #define SPEC_DEV_NONFINITE 2u       /* NaN/+inf in a row the chain read, or a row of all -inf */
@@ -93,13 +102,16 @@ typedef struct {
 } spec_conf_args;
 
 /* Create a context on `device` with workspace for batches up to max_batch
- * requests, blocks up to max_k drafted tokens (max_k <= 16) and vocabularies
+ * (<= 65535) requests, blocks up to max_k drafted tokens (max_k <= 16) and vocabularies
  * up to max_vocab (<= 2097152).  The current device is restored on return. */
 spec_status spec_verify_init(spec_verify_ctx** ctx, int device, int max_batch, int max_k,
                              int64_t max_vocab);
 
 /* Free the context and its workspace (synchronises its device first). NULL is a no-op. */
 spec_status spec_verify_destroy(spec_verify_ctx* ctx);
+
+/* Select the statistics order for later runs on this context (spec_mode). */
+spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode);
 
 /* Stochastic/mixed verification of B requests.
  *   target_logits [B, k+1, V]: row j scores drafted position j; row k is the bonus row.
@@ -189,8 +201,9 @@ spec_status spec_verify_run_host(spec_verify_ctx* ctx, const void* target_logits
                                  uint32_t* out_status, cudaStream_t stream);
 
 /* Per-kernel timing: launches of the kernel classes selected by `class_mask`
- * (bit c selects class c: 0 = row statistics + accept chain, 1 = residual/bonus
- * sampling, 2 = fp64 refinement, 3 = confidence head; 0 turns timing off) are
+ * (bit c selects class c: 0 = the verification engine (statistics, chain,
+ * sampling and fp64 refinement in one launch), 1 and 2 = unused, 3 =
+ * confidence head; 0 turns timing off) are
  * bracketed by CUDA events on the caller's stream.  spec_verify_timing_read
  * synchronises on those events and returns, for class `which`, the number of
  * launches and their total milliseconds since timing was last enabled (enabling

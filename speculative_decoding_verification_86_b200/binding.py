@@ -28,12 +28,17 @@ SPEC_ERR_TIMEOUT = 6
 SPEC_F32 = 0
 SPEC_BF16 = 1
 
+SPEC_MODE_DENSE = 0
+SPEC_MODE_PREFIX = 1
+MODES = {"dense": SPEC_MODE_DENSE, "prefix": SPEC_MODE_PREFIX}
+
 DEV_BAD_TOKEN = 1
 DEV_NONFINITE = 2
 DEV_BAD_TEMPERATURE = 4
 DEV_INTERNAL = 16
 
-TIMING_STATS, TIMING_SAMPLE, TIMING_REFINE, TIMING_CONF = 0, 1, 2, 3
+TIMING_ENGINE, TIMING_CONF = 0, 3
+TIMING_STATS = TIMING_ENGINE
 
 
 class SpecVerifyError(RuntimeError):
@@ -76,6 +81,7 @@ def lib():
     L.spec_verify_greedy_noalloc.argtypes = [_vp, _i32, _vp, _vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp]
     L.spec_conf_budget.argtypes = [_vp, _vp, _vp, ctypes.c_float, _i32, _i32, _i32,
                                    ctypes.c_float, _vp, _vp, _vp]
+    L.spec_verify_set_mode.argtypes = [_vp, _i32]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
     L.spec_verify_last_counters.argtypes = [_vp, _vp, ctypes.POINTER(_u32)]
@@ -85,7 +91,8 @@ def lib():
     L.spec_verify_ex2_error_bound.restype = ctypes.c_double
     for name in ("spec_verify_init", "spec_verify_destroy", "spec_verify_run",
                  "spec_verify_run_with_uniforms", "spec_verify_run_host", "spec_verify_greedy",
-                 "spec_conf_budget", "spec_verify_greedy_noalloc", "spec_verify_timing_enable", "spec_verify_timing_read",
+                 "spec_conf_budget", "spec_verify_greedy_noalloc", "spec_verify_set_mode",
+                 "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
         getattr(L, name).restype = _i32
     _lib = L
@@ -144,7 +151,7 @@ class SpecVerifier:
     (default: current) torch stream and return output tensors.
     """
 
-    def __init__(self, device=None, max_batch=1024, max_k=8, max_vocab=262144):
+    def __init__(self, device=None, max_batch=1024, max_k=8, max_vocab=262144, mode="prefix"):
         dev = torch.device("cuda") if device is None else torch.device(device)
         if dev.type != "cuda":
             raise ValueError("SpecVerifier needs a CUDA device, got %s" % dev)
@@ -156,6 +163,13 @@ class SpecVerifier:
         _check(lib().spec_verify_init(ctypes.byref(h), self.device.index, max_batch, max_k,
                                       max_vocab), "spec_verify_init")
         self._h = h
+        self.set_mode(mode)
+
+    def set_mode(self, mode):
+        """Statistics order: "prefix" (default: rows past the first rejection
+        are never read) or "dense" (every verified position's rows)."""
+        _check(lib().spec_verify_set_mode(self._h, MODES[mode]), "spec_verify_set_mode")
+        self.mode = mode
 
     # -- lifecycle ------------------------------------------------------------
     def close(self):

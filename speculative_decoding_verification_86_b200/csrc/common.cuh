@@ -93,7 +93,15 @@ struct Counters {
   unsigned accept_slow;    // accept decisions resolved in fp64
   unsigned sample_fast;    // samples certified by the fp32 filter
   unsigned chunks_redone;  // refinement chunks recomputed outright (support unsettled)
+  unsigned queue_error;    // engine: 1 a wait gave up, 2 the queue overflowed
+  unsigned pad[3];
 };
+
+// Engine: orders of the statistics pass, and the queue's control words.
+constexpr int kModeDense = 0;
+constexpr int kModePrefix = 1;
+constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQWords = 8;
+constexpr int kEngineMinBlocks = 3;
 
 // -------------------------------------------------------------- run params --
 struct RunParams {
@@ -136,6 +144,14 @@ struct RunParams {
   int* runc;               // [B, 4 n_chunks] sub-chunks holding unsettled logits
   Counters* counters;      // this run's counters
   Counters* counters_next; // the other run's counters, reset here
+
+  // engine
+  int mode;                        // kModeDense / kModePrefix
+  unsigned long long* q_slots;     // queue: (epoch << 32) | payload
+  unsigned q_capacity;
+  unsigned q_epoch;                // this run's epoch, never 0
+  unsigned* q_ctl;                 // head, tail, done, exits
+  unsigned n_init;                 // implicit initial tickets
 };
 
 struct ConfParams {

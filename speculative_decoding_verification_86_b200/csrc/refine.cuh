@@ -5,9 +5,9 @@
 // under the 1e-12 floor), inverse CDF in index order with the smallest-index
 // rule and the largest-positive-index fallback.
 //
-// One launch, a grid-stride loop over (queued request, sub-chunk of 4096 bf16 /
-// 2048 fp32 logits: one batch of the chunk layout), one fp64 pass over the row
-// pair.  The exact normalisers Z_a, Z_b are only known once every
+// Work items are (queued request, sub-chunk of 4096 bf16 / 2048 fp32 logits:
+// one batch of the chunk layout); together they make one fp64 pass over the
+// row pair.  The exact normalisers Z_a, Z_b are only known once every
 // chunk is done, but the residual's support {t : p_t > q_t} = {alpha_t > rho
 // beta_t} (alpha = exp(a/T - m_a), beta likewise, rho = Z_a / Z_b) can be
 // settled early: the fp32 pass bounds rho in [rho_lo, rho_hi], so a chunk adds
@@ -139,190 +139,189 @@ __device__ __forceinline__ int load_sub_contiguous(const void* row, int64_t V, i
   return bt * G::kBatchElems * kThreads + threadIdx.x * G::kBatchElems;  // offset in the chunk
 }
 
+// One fp64 work item: sub-chunk `sub` of refinement slot `slot`.  Returns true
+// in the CTA that completes the slot (all its sub-chunks are in).
 template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 2) k_refine(RunParams p) {
-  __shared__ RefineShared sh;
-  using G = Geo<BF16>;
-  const unsigned count = __ldcg(&p.counters->refine_count);
+__device__ bool refine_item(const RunParams& p, int slot, int sub, RefineShared& sh) {
   const int n_subs = p.n_chunks * kSubsPerChunk;
-  const int64_t work = static_cast<int64_t>(count) * n_subs;
-  if (blockIdx.x >= work) return;
-  exp2_table_init(sh.tab);
-#pragma unroll 1
-  for (int64_t wi = blockIdx.x; wi < work; wi += gridDim.x) {
-    const int slot = static_cast<int>(wi / n_subs);
-    const int sub = static_cast<int>(wi % n_subs);
-    const int i = __ldcg(p.refine_list + slot);
-    const Job jb = p.jobs[i];
-    const RefineRow rr = refine_row(jb);
-    const bool residual = jb.kind == kJobResidual;
-    double za = 0.0, zb = 0.0, A = 0.0, Bm = 0.0;
-    int unc = 0;
-    refine_sub_pass<BF16>(p, i, jb, rr, sub / kSubsPerChunk, sub % kSubsPerChunk, residual, sh.tab,
-                          za, zb, A, Bm, unc);
-    za = block_sum_d(za, sh.d);
-    __syncthreads();
-    zb = block_sum_d(zb, sh.d);
-    __syncthreads();
-    A = block_sum_d(A, sh.d);
-    __syncthreads();
-    Bm = block_sum_d(Bm, sh.d);
-    unc = __syncthreads_or(unc);
-    const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
-    if (threadIdx.x == 0) {
-      p.rz[rec0 + sub] = make_double2(za, zb);
-      p.rm[rec0 + sub] = make_double2(A, Bm);
-      p.runc[rec0 + sub] = unc;
-    }
-    if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(n_subs), &sh.flag)) continue;
-    __threadfence();
-
-    // ---- last CTA of this request: exact sub-chunk masses, then the token ----
-    // thread t owns sub-chunks 4t .. 4t+3
-    double zav[4], zbv[4], pz[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int ss = 4 * threadIdx.x + q;
-      const double2 z = ss < n_subs ? __ldcg(p.rz + rec0 + ss) : make_double2(0.0, 0.0);
-      zav[q] = z.x;
-      zbv[q] = z.y;
-    }
-    const double Za = chunk_prefix(zav, pz, sh.d);
-    const double Zb = chunk_prefix(zbv, pz, sh.d);
-    const double iza = 1.0 / Za, izb = residual ? 1.0 / Zb : 0.0;
-    const double rho = residual ? Za / Zb : 0.0;
-    const bool redo_all = residual && !(rho >= jb.rho_lo && rho <= jb.rho_hi);
-    double mv[4];
-    int flagged = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int ss = 4 * threadIdx.x + q;
-      mv[q] = 0.0;
-      if (ss < n_subs) {
-        if (residual) {
-          const double2 ab = __ldcg(p.rm + rec0 + ss);
-          const double r = ab.x * iza - ab.y * izb;
-          mv[q] = r > 0.0 ? r : 0.0;
-          if (redo_all || __ldcg(p.runc + rec0 + ss)) flagged |= 1 << q;
-        } else {
-          mv[q] = zav[q];
-        }
-      }
-    }
-    // sub-chunks whose support was not settled: recompute outright (rare)
-    if (__syncthreads_or(flagged)) {
-#pragma unroll 1
-      for (int ss = 0; ss < n_subs; ++ss) {
-        const int owner = ss / 4;
-        if (threadIdx.x == owner) sh.found = (flagged >> (ss % 4)) & 1;
-        __syncthreads();
-        if (sh.found) {
-          if (threadIdx.x == 0) atomicAdd(&p.counters->chunks_redone, 1u);
-          const double m = exact_sub_mass<BF16>(p, i, jb, rr, ss / kSubsPerChunk,
-                                                ss % kSubsPerChunk, iza, izb, sh);
-          if (threadIdx.x == owner) mv[ss % 4] = m;
-        }
-        __syncthreads();
-      }
-    }
-    double pm[4];
-    const double R = chunk_prefix(mv, pm, sh.d);
-    const bool use_resid = residual && R >= 1e-12;
-    if (!use_resid && residual) {  // floor: target weights exp(a/T - m_a)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) mv[q] = zav[q];
-      chunk_prefix(mv, pm, sh.d);
-    }
-    const double W = use_resid ? R : Za;
-    const double target = jb.u2 * W;
-    if (threadIdx.x == 0) {
-      sh.cstar = -1;
-      sh.found = -1;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int ss = 4 * threadIdx.x + q;
-      if (ss < n_subs && pm[q] <= target && pm[q] + mv[q] > target) {
-        sh.cstar = ss;
-        sh.base = pm[q];
-      }
-    }
-    __syncthreads();
-    bool fallback = false;
-    if (sh.cstar < 0) {
-      // rounding left no cell above target: the last sub-chunk with positive weight
-      int last = -1;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int ss = 4 * threadIdx.x + q;
-        if (ss < n_subs && mv[q] > 0.0) last = ss;
-      }
-      last = -block_min_i(last >= 0 ? -last : 1, sh.i);
-      if (threadIdx.x == 0) sh.cstar = last >= 0 ? last : -1;
-      __syncthreads();
-      fallback = true;
-    }
-    const int sstar = sh.cstar;
-    int token = -1;
-    if (sstar >= 0) {
-      const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
-      const void* ra = target_row(p, i, jb.row, BF16);
-      const void* rb = use_resid ? draft_row(p, i, jb.row, BF16) : nullptr;
-      uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
-      const int off = load_sub_contiguous<BF16>(ra, p.V, c, bt, va);
-      if (use_resid) load_sub_contiguous<BF16>(rb, p.V, c, bt, vb);
-      double wv[G::kBatchElems];
-      double tsum = 0.0;
-      int last_pos = -1;
-#pragma unroll
-      for (int u = 0; u < kVecsPerBatch; ++u) {
-        float xa[G::kPerVec], xb[G::kPerVec];
-        unpack<BF16>(va[u], xa);
-        if (use_resid) unpack<BF16>(vb[u], xb);
-#pragma unroll
-        for (int q = 0; q < G::kPerVec; ++q) {
-          const double wt = exact_weight<BF16>(xa[q], use_resid ? xb[q] : 0.0f, use_resid, rr,
-                                               iza, izb, sh.tab);
-          wv[u * G::kPerVec + q] = wt;
-          tsum += wt;
-          if (wt > 0.0) last_pos = off + u * G::kPerVec + q;
-        }
-      }
-      int found = -1;
-      if (!fallback) {
-        double all;
-        const double pre = block_exclusive_scan_d(tsum, sh.d, all);
-        const double start = sh.base + pre;
-        if (start <= target && start + tsum > target) {
-          double run = start;
-#pragma unroll
-          for (int e = 0; e < G::kBatchElems; ++e) {
-            run += wv[e];
-            if (run > target && sh.found < 0) sh.found = off + e;
-          }
-        }
-        __syncthreads();
-        found = sh.found;
-      }
-      if (found < 0) {
-        // fallback, or the sub-chunk's scanned total fell a rounding short of
-        // target: the last logit of the sub-chunk with positive weight
-        int neg = last_pos >= 0 ? -last_pos : INT_MAX;
-        neg = block_min_i(neg, sh.i);
-        found = neg == INT_MAX ? -1 : -neg;
-      }
-      token = found >= 0 ? static_cast<int>(static_cast<int64_t>(c) * G::kChunk + found) : -1;
-    }
-    if (threadIdx.x == 0) {
-      p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;
-      if (token < 0) {
-        p.out_acc[i] = -1;
-        if (p.out_status) p.out_status[i] |= kDevInternal;
-      }
-    }
-    __syncthreads();
+  const int i = __ldcg(p.refine_list + slot);
+  const Job jb = p.jobs[i];
+  const RefineRow rr = refine_row(jb);
+  const bool residual = jb.kind == kJobResidual;
+  double za = 0.0, zb = 0.0, A = 0.0, Bm = 0.0;
+  int unc = 0;
+  refine_sub_pass<BF16>(p, i, jb, rr, sub / kSubsPerChunk, sub % kSubsPerChunk, residual, sh.tab,
+                        za, zb, A, Bm, unc);
+  za = block_sum_d(za, sh.d);
+  zb = block_sum_d(zb, sh.d);
+  A = block_sum_d(A, sh.d);
+  Bm = block_sum_d(Bm, sh.d);
+  unc = __syncthreads_or(unc);
+  const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
+  if (threadIdx.x == 0) {
+    p.rz[rec0 + sub] = make_double2(za, zb);
+    p.rm[rec0 + sub] = make_double2(A, Bm);
+    p.runc[rec0 + sub] = unc;
   }
+  if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(n_subs), &sh.flag)) return false;
+  __threadfence();
+  return true;
+}
+
+// The last CTA of refinement slot `slot`: exact sub-chunk masses, the token.
+template <bool BF16>
+__device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) {
+  using G = Geo<BF16>;
+  const int n_subs = p.n_chunks * kSubsPerChunk;
+  const int i = __ldcg(p.refine_list + slot);
+  const Job jb = p.jobs[i];
+  const RefineRow rr = refine_row(jb);
+  const bool residual = jb.kind == kJobResidual;
+  const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
+  // thread t owns sub-chunks 4t .. 4t+3
+  double zav[4], zbv[4], pz[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int ss = 4 * threadIdx.x + q;
+    const double2 z = ss < n_subs ? __ldcg(p.rz + rec0 + ss) : make_double2(0.0, 0.0);
+    zav[q] = z.x;
+    zbv[q] = z.y;
+  }
+  const double Za = chunk_prefix(zav, pz, sh.d);
+  const double Zb = chunk_prefix(zbv, pz, sh.d);
+  const double iza = 1.0 / Za, izb = residual ? 1.0 / Zb : 0.0;
+  const double rho = residual ? Za / Zb : 0.0;
+  const bool redo_all = residual && !(rho >= jb.rho_lo && rho <= jb.rho_hi);
+  double mv[4];
+  int flagged = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int ss = 4 * threadIdx.x + q;
+    mv[q] = 0.0;
+    if (ss < n_subs) {
+      if (residual) {
+        const double2 ab = __ldcg(p.rm + rec0 + ss);
+        const double r = ab.x * iza - ab.y * izb;
+        mv[q] = r > 0.0 ? r : 0.0;
+        if (redo_all || __ldcg(p.runc + rec0 + ss)) flagged |= 1 << q;
+      } else {
+        mv[q] = zav[q];
+      }
+    }
+  }
+  // sub-chunks whose support was not settled: recompute outright (rare)
+  if (__syncthreads_or(flagged)) {
+#pragma unroll 1
+    for (int ss = 0; ss < n_subs; ++ss) {
+      const int owner = ss / 4;
+      if (threadIdx.x == owner) sh.found = (flagged >> (ss % 4)) & 1;
+      __syncthreads();
+      if (sh.found) {
+        if (threadIdx.x == 0) atomicAdd(&p.counters->chunks_redone, 1u);
+        const double m = exact_sub_mass<BF16>(p, i, jb, rr, ss / kSubsPerChunk,
+                                              ss % kSubsPerChunk, iza, izb, sh);
+        if (threadIdx.x == owner) mv[ss % 4] = m;
+      }
+      __syncthreads();
+    }
+  }
+  double pm[4];
+  const double R = chunk_prefix(mv, pm, sh.d);
+  const bool use_resid = residual && R >= 1e-12;
+  if (!use_resid && residual) {  // floor: target weights exp(a/T - m_a)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mv[q] = zav[q];
+    chunk_prefix(mv, pm, sh.d);
+  }
+  const double W = use_resid ? R : Za;
+  const double target = jb.u2 * W;
+  if (threadIdx.x == 0) {
+    sh.cstar = -1;
+    sh.found = -1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int ss = 4 * threadIdx.x + q;
+    if (ss < n_subs && pm[q] <= target && pm[q] + mv[q] > target) {
+      sh.cstar = ss;
+      sh.base = pm[q];
+    }
+  }
+  __syncthreads();
+  bool fallback = false;
+  if (sh.cstar < 0) {
+    // rounding left no cell above target: the last sub-chunk with positive weight
+    int last = -1;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int ss = 4 * threadIdx.x + q;
+      if (ss < n_subs && mv[q] > 0.0) last = ss;
+    }
+    last = -block_min_i(last >= 0 ? -last : 1, sh.i);
+    if (threadIdx.x == 0) sh.cstar = last >= 0 ? last : -1;
+    __syncthreads();
+    fallback = true;
+  }
+  const int sstar = sh.cstar;
+  int token = -1;
+  if (sstar >= 0) {
+    const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
+    const void* ra = target_row(p, i, jb.row, BF16);
+    const void* rb = use_resid ? draft_row(p, i, jb.row, BF16) : nullptr;
+    uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+    const int off = load_sub_contiguous<BF16>(ra, p.V, c, bt, va);
+    if (use_resid) load_sub_contiguous<BF16>(rb, p.V, c, bt, vb);
+    double wv[G::kBatchElems];
+    double tsum = 0.0;
+    int last_pos = -1;
+#pragma unroll
+    for (int u = 0; u < kVecsPerBatch; ++u) {
+      float xa[G::kPerVec], xb[G::kPerVec];
+      unpack<BF16>(va[u], xa);
+      if (use_resid) unpack<BF16>(vb[u], xb);
+#pragma unroll
+      for (int q = 0; q < G::kPerVec; ++q) {
+        const double wt = exact_weight<BF16>(xa[q], use_resid ? xb[q] : 0.0f, use_resid, rr,
+                                             iza, izb, sh.tab);
+        wv[u * G::kPerVec + q] = wt;
+        tsum += wt;
+        if (wt > 0.0) last_pos = off + u * G::kPerVec + q;
+      }
+    }
+    int found = -1;
+    if (!fallback) {
+      double all;
+      const double pre = block_exclusive_scan_d(tsum, sh.d, all);
+      const double start = sh.base + pre;
+      if (start <= target && start + tsum > target) {
+        double run = start;
+#pragma unroll
+        for (int e = 0; e < G::kBatchElems; ++e) {
+          run += wv[e];
+          if (run > target && sh.found < 0) sh.found = off + e;
+        }
+      }
+      __syncthreads();
+      found = sh.found;
+    }
+    if (found < 0) {
+      // fallback, or the sub-chunk's scanned total fell a rounding short of
+      // target: the last logit of the sub-chunk with positive weight
+      int neg = last_pos >= 0 ? -last_pos : INT_MAX;
+      neg = block_min_i(neg, sh.i);
+      found = neg == INT_MAX ? -1 : -neg;
+    }
+    token = found >= 0 ? static_cast<int>(static_cast<int64_t>(c) * G::kChunk + found) : -1;
+  }
+  if (threadIdx.x == 0) {
+    p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;
+    if (token < 0) {
+      p.out_acc[i] = -1;
+      if (p.out_status) p.out_status[i] |= kDevInternal;
+    }
+  }
+  __syncthreads();
 }
 
 }  // namespace sv

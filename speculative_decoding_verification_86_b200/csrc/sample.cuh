@@ -149,6 +149,7 @@ struct SampleShared {
   double base;        // weight before chunk cstar
   double base_bound;  // bound before chunk cstar
   int found;          // local index of the crossing in cstar, or -1
+  int refine_slot;    // locate's outcome: -1 certain, else the refinement slot
   double lo_gap, hi_gap, cell_bound;
 };
 
@@ -325,25 +326,14 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
     if (certain) {
       p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;
       atomicAdd(&p.counters->sample_fast, 1u);
+      sh.refine_slot = -1;
     } else {
       const unsigned slot = atomicAdd(&p.counters->refine_count, 1u);
       p.refine_list[slot] = i;
+      sh.refine_slot = static_cast<int>(slot);
     }
   }
-}
-
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, 3) k_sample(RunParams p) {
-  __shared__ SampleShared sh;
-  const int64_t b = blockIdx.x;
-  const int i = static_cast<int>(b / p.n_segs);
-  const int seg = static_cast<int>(b % p.n_segs);
-  const Job jb = p.jobs[i];
-  if (jb.kind == kJobNone) return;
-  segment_masses<BF16>(p, i, jb, seg, sh);
-  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_segs), &sh.flag)) return;
-  __threadfence();
-  locate_sample<BF16>(p, i, jb, sh);
+  __syncthreads();
 }
 
 }  // namespace sv

@@ -1,21 +1,21 @@
 // Host side of the C ABI declared in include/spec_verify.h: argument checks,
-// the context's device workspace, and the launch sequence
-//   [k_conf] -> k_stats (row statistics + accept chain)
-//            -> k_sample (residual / bonus sampling, fp32 filter)
-//            -> k_refine (fp64, only queued samples).
-// Every launch goes to the caller's stream; nothing here synchronises except
-// the host-buffer entry point, the diagnostics and the timing read-out.
+// the context's device workspace, and the launches: [k_conf] then one
+// persistent k_engine (engine.cuh) per run.  Every launch goes to the caller's
+// stream; nothing here synchronises except the host-buffer entry point, the
+// diagnostics and the timing read-out.
 #include "spec_verify.h"
 
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <new>
 #include <vector>
 
 #include "common.cuh"
 #include "conf.cuh"
+#include "engine.cuh"
 #include "philox.cuh"
 #include "refine.cuh"
 #include "sample.cuh"
@@ -30,7 +30,7 @@ namespace {
 // require it to stay at or below this bound.
 constexpr float kEpsEx2 = 1.5e-7f;
 
-constexpr int kClassStats = 0, kClassSample = 1, kClassRefine = 2, kClassConf = 3;
+constexpr int kClassStats = 0, kClassConf = 3;  // timing classes (1, 2: unused)
 constexpr int kTimingClasses = 4;
 constexpr int kMaxTimed = 4096;
 
@@ -126,6 +126,11 @@ struct spec_verify_ctx {
   int* runc = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
   int32_t* conf_len = nullptr;
+  unsigned long long* q_slots = nullptr;
+  unsigned q_capacity = 0;
+  unsigned* q_ctl = nullptr;
+  int engine_grid = 0;
+  int mode = sv::kModePrefix;
   unsigned run_id = 0;
 
   unsigned timing_mask = 0;  // bit c set: bracket launches of class c with events
@@ -178,6 +183,17 @@ spec_status carve(spec_verify_ctx* c) {
   const size_t o_runc = take(per_req_subs * sizeof(int));
   const size_t o_cnt = take(2 * sizeof(sv::Counters));
   const size_t o_conf = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
+  // queue: every row segment, sample segment and refinement sub-chunk of a
+  // batch, plus one exit ticket per CTA
+  const size_t max_segs = static_cast<size_t>((c->max_vocab + sv::SegGeo<false>::kSeg - 1) /
+                                              sv::SegGeo<false>::kSeg);
+  const size_t max_subs = static_cast<size_t>(c->max_chunks) * sv::kBatchesPerChunk;
+  const size_t cap = static_cast<size_t>(c->max_batch) *
+                         ((2 * c->max_k + 1) * max_segs + max_segs + max_subs) + 8192;
+  if (cap > 0xFFFFFFF0ull) return SPEC_ERR_INVALID_ARG;
+  c->q_capacity = static_cast<unsigned>(cap);
+  const size_t o_qs = take(cap * sizeof(unsigned long long));
+  const size_t o_qc = take(sv::kQWords * sizeof(unsigned));
   if (cudaMalloc(&c->ws, off) != cudaSuccess) {
     cudaGetLastError();
     return SPEC_ERR_NOMEM;
@@ -200,6 +216,8 @@ spec_status carve(spec_verify_ctx* c) {
   c->runc = reinterpret_cast<int*>(b + o_runc);
   c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
   c->conf_len = reinterpret_cast<int32_t*>(b + o_conf);
+  c->q_slots = reinterpret_cast<unsigned long long*>(b + o_qs);
+  c->q_ctl = reinterpret_cast<unsigned*>(b + o_qc);
   if (cudaMemset(c->ws, 0, off) != cudaSuccess) return SPEC_ERR_CUDA;
   return SPEC_OK;
 }
@@ -316,7 +334,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.rZ = c->rZ;
   p.rm = c->rm;
   p.runc = c->runc;
-  c->run_id++;
+  if (++c->run_id == 0) c->run_id = 1;
   p.counters = c->counters + (c->run_id & 1u);
   p.counters_next = c->counters + ((c->run_id + 1u) & 1u);
 
@@ -325,23 +343,19 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     launch_conf(c, conf, B, c->conf_len, nullptr, s);
     p.conf_len = c->conf_len;
   }
-  const int64_t stats_ctas = static_cast<int64_t>(B) * (2 * k + 1) * n_segs;
+  p.mode = force_greedy ? sv::kModePrefix : c->mode;
+  p.q_slots = c->q_slots;
+  p.q_capacity = c->q_capacity;
+  p.q_ctl = c->q_ctl;
+  p.q_epoch = c->run_id;  // >= 1: slots left by earlier runs carry older epochs
+  const uint64_t n_init = static_cast<uint64_t>(B) *
+                          (p.mode == sv::kModeDense ? (2 * k + 1) : 2) * n_segs;
+  if (n_init > 0xFFFF0000ull) return SPEC_ERR_INVALID_ARG;
+  p.n_init = static_cast<unsigned>(n_init);
   timing_mark(c, kClassStats, true, s);
-  if (bf16) sv::k_stats<true><<<static_cast<unsigned>(stats_ctas), sv::kThreads, 0, s>>>(p);
-  else sv::k_stats<false><<<static_cast<unsigned>(stats_ctas), sv::kThreads, 0, s>>>(p);
+  if (bf16) sv::k_engine<true><<<c->engine_grid, sv::kThreads, 0, s>>>(p);
+  else sv::k_engine<false><<<c->engine_grid, sv::kThreads, 0, s>>>(p);
   timing_mark(c, kClassStats, false, s);
-  if (!force_greedy) {
-    const unsigned sample_ctas = static_cast<unsigned>(static_cast<int64_t>(B) * n_segs);
-    const unsigned refine_ctas = static_cast<unsigned>(4 * c->num_sms);
-    timing_mark(c, kClassSample, true, s);
-    if (bf16) sv::k_sample<true><<<sample_ctas, sv::kThreads, 0, s>>>(p);
-    else sv::k_sample<false><<<sample_ctas, sv::kThreads, 0, s>>>(p);
-    timing_mark(c, kClassSample, false, s);
-    timing_mark(c, kClassRefine, true, s);
-    if (bf16) sv::k_refine<true><<<refine_ctas, sv::kThreads, 0, s>>>(p);
-    else sv::k_refine<false><<<refine_ctas, sv::kThreads, 0, s>>>(p);
-    timing_mark(c, kClassRefine, false, s);
-  }
   if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
   return SPEC_OK;
 }
@@ -367,7 +381,7 @@ spec_status spec_verify_init(spec_verify_ctx** out, int device, int max_batch, i
                              int64_t max_vocab) {
   if (!out) return SPEC_ERR_INVALID_ARG;
   *out = nullptr;
-  if (max_batch < 1 || max_k < 0 || max_k > sv::kMaxK || max_vocab < 1 ||
+  if (max_batch < 1 || max_batch > 65535 || max_k < 0 || max_k > sv::kMaxK || max_vocab < 1 ||
       max_vocab > static_cast<int64_t>(sv::kMaxChunksPerRow) * (sv::kChunkF32 / sv::kBatchesPerChunk))
     return SPEC_ERR_INVALID_ARG;
   int ndev = 0;
@@ -395,6 +409,16 @@ spec_status spec_verify_init(spec_verify_ctx** out, int device, int max_batch, i
     delete c;
     return st;
   }
+  int occ_a = 0, occ_b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, sv::k_engine<true>, sv::kThreads, 0) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, sv::k_engine<false>, sv::kThreads, 0) !=
+          cudaSuccess) {
+    cudaFree(c->ws);
+    delete c;
+    return SPEC_ERR_CUDA;
+  }
+  c->engine_grid = c->num_sms * std::max(1, std::min(occ_a, occ_b));
   *out = c;
   return SPEC_OK;
 }
@@ -635,6 +659,12 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
   if (bf16) sv::k_stats<true><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
   else sv::k_stats<false><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode) {
+  if (!ctx || (mode != SPEC_MODE_DENSE && mode != SPEC_MODE_PREFIX)) return SPEC_ERR_INVALID_ARG;
+  ctx->mode = mode == SPEC_MODE_DENSE ? sv::kModeDense : sv::kModePrefix;
+  return SPEC_OK;
 }
 
 spec_status spec_verify_timing_enable(spec_verify_ctx* ctx, int class_mask) {

@@ -450,7 +450,164 @@ __device__ __forceinline__ double draw(const RunParams& p, int i, int j, int d) 
 constexpr double kU24 = 0x1p-24;
 constexpr double kLn2 = 0.69314718055994530942;
 
-// Resolve request i after all its chunk statistics are in.
+// Constants of a request's temperature for the fp32 path and its bounds.
+struct TempConsts {
+  double T;         // temperature
+  double c_exact;   // log2(e) / T in fp64
+  double eta;       // |relative error| of cc
+  double kappa;     // ln2 (2^-24 + eta): bound per unit |exponent argument|
+  double eps_base;  // ex2 error + pairwise-sum rounding + slack
+  float cc;         // fp32 log2(e) / T used by the fp32 path
+};
+
+template <bool BF16>
+__device__ __forceinline__ TempConsts temp_consts(const RunParams& p, float Tf) {
+  TempConsts t;
+  t.T = static_cast<double>(Tf);
+  t.cc = static_cast<float>(1.4426950408889634 / t.T);
+  t.c_exact = 1.4426950408889634 / t.T;
+  t.eta = fabs((t.c_exact - static_cast<double>(t.cc)) / static_cast<double>(t.cc));
+  t.kappa = kLn2 * (kU24 + t.eta) * 1.0001;
+  t.eps_base = static_cast<double>(p.eps_ex2) + SegGeo<BF16>::kSumLevels * kU24 + 1e-14;
+  return t;
+}
+
+// Relative error bound of a row's fp32 normaliser Z~: one ex2 error per term,
+// the pairwise rounding of the batch sums, and the exponent rounding (weighted
+// by sum e|a|).  Rounding log2(e)/T to fp32 (relative eta) reshapes p itself:
+// log p/p~ moves by at most ln2 * eta * |a_x - mean(a)|; that part is added
+// where p(x) is formed.
+__device__ __forceinline__ double row_dZ(const TempConsts& t, const RowMerged& r) {
+  return t.eps_base + kLn2 * kU24 * 1.0001 * r.ER / r.Z;
+}
+
+// Accept test of drafted token xj at position j from the fp32 statistics of
+// target row ra and draft row rb: 1 accept, 0 reject, -1 inside the bound.
+// Also returns p~(x), q~(x).  (Thread-local; any one thread may call it.)
+template <bool BF16>
+__device__ __forceinline__ int accept_eval(const RunParams& p, int i, int j, int xj,
+                                          const RowMerged& ra, const RowMerged& rb,
+                                          const TempConsts& t, double& pa, double& qb) {
+  const float la = load_logit(target_row(p, i, j, BF16), xj, BF16);
+  const float lb = load_logit(draft_row(p, i, j, BF16), xj, BF16);
+  const double arg_a = static_cast<double>(la) * t.cc - static_cast<double>(ra.K);
+  const double arg_b = static_cast<double>(lb) * t.cc - static_cast<double>(rb.K);
+  pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) / ra.Z;
+  qb = (lb == -INFINITY) ? 0.0 : exp2(arg_b) / rb.Z;
+  const double u = draw(p, i, j, 0);
+  if (qb == 0.0) return pa > 0.0 ? 1 : 0;
+  const double dp = row_dZ(t, ra) + kLn2 * t.eta * (fabs(arg_a + ra.EA / ra.Z) + 1e-3);
+  const double dq = row_dZ(t, rb) + kLn2 * t.eta * (fabs(arg_b + rb.EA / rb.Z) + 1e-3);
+  const double delta = (dp + dq) * 1.01 + 1e-13;
+  const double rho = pa / qb;
+  if (u < rho * (1.0 - delta)) return 1;
+  if (u >= rho * (1.0 + delta)) return 0;
+  return -1;
+}
+
+// Slow path of an accept decision inside its bound: both normalisers in fp64
+// at the true temperature (all threads of the block).  Returns the exact
+// decision in *accept (thread 0) and p(x), q(x).
+template <bool BF16>
+__device__ void accept_exact(const RunParams& p, int i, int j, int xj, const RowMerged& ra,
+                             const RowMerged& rb, const TempConsts& t, double* red, bool& accept,
+                             double& pa, double& qb) {
+  const double ma = static_cast<double>(ra.mraw) / t.T;
+  const double mb = static_cast<double>(rb.mraw) / t.T;
+  const double Za = exact_row_sum(target_row(p, i, j, BF16), p.V, BF16, t.T, ma, red);
+  __syncthreads();
+  const double Zb = exact_row_sum(draft_row(p, i, j, BF16), p.V, BF16, t.T, mb, red);
+  if (threadIdx.x == 0) {
+    const double la = load_logit(target_row(p, i, j, BF16), xj, BF16);
+    const double lb = load_logit(draft_row(p, i, j, BF16), xj, BF16);
+    pa = exp(la / t.T - ma) / Za;
+    qb = exp(lb / t.T - mb) / Zb;
+    const double u = draw(p, i, j, 0);
+    atomicAdd(&p.counters->accept_slow, 1u);
+    accept = u * qb < pa;
+  }
+}
+
+// The job that samples position n of request i: the residual of row pair n
+// (n < L) or the bonus row L.  (Thread 0.)
+template <bool BF16>
+__device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerged& ra,
+                          const RowMerged* rb, const TempConsts& t) {
+  Job jb;
+  jb.n = n;
+  jb.pad0 = 0;
+  jb.cc = t.cc;
+  jb.kappa = static_cast<float>(t.kappa);
+  jb.eta_ln2 = kLn2 * t.eta;
+  jb.T = t.T;
+  jb.u2 = draw(p, i, n, 1);
+  jb.row = n;
+  jb.Ka = ra.K;
+  jb.mraw_a = ra.mraw;
+  if (n < L) {
+    jb.kind = kJobResidual;
+    jb.Kb = rb->K;
+    jb.mraw_b = rb->mraw;
+    jb.A = static_cast<float>(1.0 / ra.Z);
+    jb.Bq = static_cast<float>(1.0 / rb->Z);
+    // per term: ex2 error, rounding of 1/Z, of the scaled product and of the
+    // difference, the normaliser's own bound, and |mean exponent| of the
+    // temperature-rounding term (the frame adds its offset, the term its |a|).
+    jb.eps0a = static_cast<double>(p.eps_ex2) + 4 * kU24 + row_dZ(t, ra) + kLn2 * t.eta * ra.EA / ra.Z;
+    jb.eps0b = static_cast<double>(p.eps_ex2) + 4 * kU24 + row_dZ(t, *rb) + kLn2 * t.eta * rb->EA / rb->Z;
+    // Bracket of rho = Z_a / Z_b in the refinement's frames (each row relative
+    // to its own max at the true temperature): the fp32 sums' bounds, the
+    // reshaping by the rounded temperature factor, and a factor 3 of margin.
+    const double rho = (ra.Z / rb->Z) *
+        exp2((static_cast<double>(ra.K) - static_cast<double>(rb->K)) -
+             (static_cast<double>(ra.mraw) - static_cast<double>(rb->mraw)) * t.c_exact);
+    const double band = 3.0 * (row_dZ(t, ra) + row_dZ(t, *rb) +
+        kLn2 * t.eta * (fabs(static_cast<double>(ra.mraw) - static_cast<double>(rb->mraw)) * t.c_exact +
+                        ra.EA / ra.Z + rb->EA / rb->Z + 1.0)) + 1e-12;
+    jb.rho_lo = rho * (1.0 - band);
+    jb.rho_hi = rho * (1.0 + band);
+  } else {
+    jb.kind = kJobBonus;
+    jb.Kb = 0.0f;
+    jb.mraw_b = 0.0f;
+    jb.A = 1.0f;
+    jb.Bq = 0.0f;
+    jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + 1e-14;
+    jb.eps0b = 0.0;
+    jb.rho_lo = 0.0;
+    jb.rho_hi = 0.0;
+  }
+  p.jobs[i] = jb;
+}
+
+// All outputs of request i at their "nothing decided" values (every thread).
+__device__ __forceinline__ void write_defaults(const RunParams& p, int i) {
+  const int k = p.k;
+  int32_t* tok = p.out_tok + static_cast<int64_t>(i) * (k + 1);
+  for (int j = threadIdx.x; j <= k; j += kThreads) tok[j] = -1;
+  for (int j = threadIdx.x; j < k; j += kThreads) {
+    if (p.out_p) p.out_p[static_cast<int64_t>(i) * k + j] = -1.0f;
+    if (p.out_q) p.out_q[static_cast<int64_t>(i) * k + j] = -1.0f;
+  }
+}
+
+// Request i failed with `status` (thread 0): outputs back to -1, n = -1.
+__device__ __forceinline__ void fail_request(const RunParams& p, int i, uint32_t status) {
+  const int k = p.k;
+  int32_t* tok = p.out_tok + static_cast<int64_t>(i) * (k + 1);
+  for (int jj = 0; jj <= k; ++jj) tok[jj] = -1;
+  for (int jj = 0; jj < k; ++jj) {
+    if (p.out_p) p.out_p[static_cast<int64_t>(i) * k + jj] = -1.0f;
+    if (p.out_q) p.out_q[static_cast<int64_t>(i) * k + jj] = -1.0f;
+  }
+  p.out_acc[i] = -1;
+  if (p.out_status) p.out_status[i] = status;
+  p.jobs[i].kind = kJobNone;
+}
+
+// Resolve request i after all its rows' statistics are in (dense order: every
+// verified position's rows were read).  Leaves p.jobs[i] describing the sample
+// still to draw (kind kJobNone when the request is finished).
 template <bool BF16>
 __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, DecideShared& sh) {
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -459,21 +616,11 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   float* op = p.out_p ? p.out_p + static_cast<int64_t>(i) * k : nullptr;
   float* oq = p.out_q ? p.out_q + static_cast<int64_t>(i) * k : nullptr;
   const int32_t* x = p.tokens + static_cast<int64_t>(i) * k;
-  Job* job = p.jobs + i;
 
-  // Defaults: nothing accepted yet, every slot -1.
-  for (int j = tid; j <= k; j += kThreads) tok[j] = -1;
-  for (int j = tid; j < k; j += kThreads) {
-    if (op) op[j] = -1.0f;
-    if (oq) oq[j] = -1.0f;
-  }
-
+  write_defaults(p, i);
   if (ri.bad_T) {
-    if (tid == 0) {
-      p.out_acc[i] = -1;
-      if (p.out_status) p.out_status[i] = kDevBadTemperature;
-      job->kind = kJobNone;
-    }
+    __syncthreads();
+    if (tid == 0) fail_request(p, i, kDevBadTemperature);
     return;
   }
 
@@ -481,9 +628,8 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   const int nrows = ri.greedy ? L + 1 : 2 * L + 1;
   for (int r = warp; r < nrows; r += kWarps) {
     const int slot = r <= L ? r : (k + 1) + (r - (L + 1));
-    const int dst = r <= L ? r : (k + 1) + (r - (L + 1));
-    if (ri.greedy) merge_greedy_row(p, i, slot, sh.rows[dst]);
-    else merge_stochastic_row(p, i, slot, sh.rows[dst]);
+    if (ri.greedy) merge_greedy_row(p, i, slot, sh.rows[slot]);
+    else merge_stochastic_row(p, i, slot, sh.rows[slot]);
   }
   __syncthreads();
 
@@ -506,38 +652,26 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
         else tok[L] = sh.rows[L].arg;
       }
       if (status) {
-        for (int j = 0; j <= k; ++j) tok[j] = -1;
+        fail_request(p, i, status);
+      } else {
+        p.out_acc[i] = n;
+        if (p.out_status) p.out_status[i] = 0;
+        p.jobs[i].kind = kJobNone;
       }
-      p.out_acc[i] = status ? -1 : n;
-      if (p.out_status) p.out_status[i] = status;
-      job->kind = kJobNone;
     }
     return;
   }
 
-  // Stochastic chain.
-  const double T = static_cast<double>(ri.T);
-  const float cc = static_cast<float>(1.4426950408889634 / T);
-  const double c_exact = 1.4426950408889634 / T;
-  const double eta = fabs((c_exact - static_cast<double>(cc)) / static_cast<double>(cc));
-  // Relative error of a row's fp32 normaliser Z~: one ex2 error per term, the
-  // pairwise rounding of the batch sums, and the exponent rounding (weighted by
-  // sum e|a|).  Rounding log2(e)/T to fp32 (relative eta) reshapes p itself:
-  // log p/p~ moves by at most ln2 * eta * |a_x - mean(a)|.
-  const double kappa = kLn2 * (kU24 + eta) * 1.0001;
-  const double eps_base =
-      static_cast<double>(p.eps_ex2) + SegGeo<BF16>::kSumLevels * kU24 + 1e-14;
-  auto dZ = [&](const RowMerged& r) { return eps_base + kLn2 * kU24 * 1.0001 * r.ER / r.Z; };
-
-  // thread 0 carries the chain; other threads join the fp64 slow path.
+  // Stochastic chain: thread 0 carries it; the block joins the fp64 slow path.
+  const TempConsts t = temp_consts<BF16>(p, ri.T);
   int n = L;
   uint32_t status = 0;
-  int j = 0;
-  for (; j < L; ++j) {
+  for (int j = 0; j < L; ++j) {
+    int xj = 0;
     if (tid == 0) {
       sh.state = 0;
       sh.need_exact = -1;
-      const int xj = __ldg(x + j);
+      xj = __ldg(x + j);
       const RowMerged& ra = sh.rows[j];
       const RowMerged& rb = sh.rows[k + 1 + j];
       if (xj < 0 || static_cast<int64_t>(xj) >= p.V) {
@@ -547,25 +681,8 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
         status = kDevNonfinite;
         sh.state = 1;
       } else {
-        const float la = load_logit(target_row(p, i, j, BF16), xj, BF16);
-        const float lb = load_logit(draft_row(p, i, j, BF16), xj, BF16);
-        const double arg_a = static_cast<double>(la) * cc - static_cast<double>(ra.K);
-        const double arg_b = static_cast<double>(lb) * cc - static_cast<double>(rb.K);
-        const double pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) / ra.Z;
-        const double qb = (lb == -INFINITY) ? 0.0 : exp2(arg_b) / rb.Z;
-        const double u = draw(p, i, j, 0);
-        int decision;  // 1 accept, 0 reject, -1 inside the error bound
-        if (qb == 0.0) {
-          decision = pa > 0.0 ? 1 : 0;
-        } else {
-          const double dp = dZ(ra) + kLn2 * eta * (fabs(arg_a + ra.EA / ra.Z) + 1e-3);
-          const double dq = dZ(rb) + kLn2 * eta * (fabs(arg_b + rb.EA / rb.Z) + 1e-3);
-          const double delta = (dp + dq) * 1.01 + 1e-13;
-          const double rho = pa / qb;
-          if (u < rho * (1.0 - delta)) decision = 1;
-          else if (u >= rho * (1.0 + delta)) decision = 0;
-          else decision = -1;
-        }
+        double pa, qb;
+        const int decision = accept_eval<BF16>(p, i, j, xj, ra, rb, t, pa, qb);
         if (op) op[j] = static_cast<float>(pa);
         if (oq) oq[j] = static_cast<float>(qb);
         if (decision < 0) {
@@ -580,25 +697,15 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     }
     __syncthreads();
     if (sh.need_exact >= 0) {
-      // fp64 at the true temperature: recompute both normalisers exactly.
-      const RowMerged& ra = sh.rows[j];
-      const RowMerged& rb = sh.rows[k + 1 + j];
-      const double ma = static_cast<double>(ra.mraw) / T;
-      const double mb = static_cast<double>(rb.mraw) / T;
-      const double Za = exact_row_sum(target_row(p, i, j, BF16), p.V, BF16, T, ma, sh.red);
-      const double Zb = exact_row_sum(draft_row(p, i, j, BF16), p.V, BF16, T, mb, sh.red);
+      bool accept = false;
+      double pa = 0.0, qb = 0.0;
+      const int xs = __ldg(x + j);
+      accept_exact<BF16>(p, i, j, xs, sh.rows[j], sh.rows[k + 1 + j], t, sh.red, accept, pa, qb);
       if (tid == 0) {
-        const int xj = __ldg(x + j);
-        const double la = load_logit(target_row(p, i, j, BF16), xj, BF16);
-        const double lb = load_logit(draft_row(p, i, j, BF16), xj, BF16);
-        const double pa = exp(la / T - ma) / Za;
-        const double qb = exp(lb / T - mb) / Zb;
-        const double u = draw(p, i, j, 0);
         if (op) op[j] = static_cast<float>(pa);
         if (oq) oq[j] = static_cast<float>(qb);
-        atomicAdd(&p.counters->accept_slow, 1u);
-        if (u * qb < pa) {
-          tok[j] = xj;
+        if (accept) {
+          tok[j] = xs;
         } else {
           n = j;
           sh.state = 1;
@@ -615,67 +722,122 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   if (tid == 0) {
     if (!status && n == L && sh.rows[L].bad) status = kDevNonfinite;
     if (status) {
-      for (int jj = 0; jj <= k; ++jj) tok[jj] = -1;
-      if (op) for (int jj = 0; jj < k; ++jj) op[jj] = -1.0f;
-      if (oq) for (int jj = 0; jj < k; ++jj) oq[jj] = -1.0f;
-      p.out_acc[i] = -1;
-      if (p.out_status) p.out_status[i] = status;
-      job->kind = kJobNone;
+      fail_request(p, i, status);
       return;
     }
     p.out_acc[i] = n;
     if (p.out_status) p.out_status[i] = 0;
-    Job jb;
-    jb.n = n;
-    jb.pad0 = 0;
-    jb.cc = cc;
-    jb.kappa = static_cast<float>(kappa);
-    jb.eta_ln2 = kLn2 * eta;
-    jb.T = T;
-    jb.u2 = draw(p, i, n, 1);
-    const RowMerged& ra = sh.rows[n];
-    jb.row = n;
-    jb.Ka = ra.K;
-    jb.mraw_a = ra.mraw;
-    if (n < L) {
-      const RowMerged& rb = sh.rows[k + 1 + n];
-      jb.kind = kJobResidual;
-      jb.Kb = rb.K;
-      jb.mraw_b = rb.mraw;
-      jb.A = static_cast<float>(1.0 / ra.Z);
-      jb.Bq = static_cast<float>(1.0 / rb.Z);
-      // per-term constant: ex2 error, rounding of 1/Z and of the products,
-      // the normaliser's own bound (incl. the temperature-rounding term).
-      // per term: ex2 error, rounding of 1/Z, of the scaled product and of the
-      // difference, the normaliser's own bound, and |mean exponent| of the
-      // temperature-rounding term (the frame adds its offset, the term its |a|).
-      jb.eps0a = static_cast<double>(p.eps_ex2) + 4 * kU24 + dZ(ra) + kLn2 * eta * ra.EA / ra.Z;
-      jb.eps0b = static_cast<double>(p.eps_ex2) + 4 * kU24 + dZ(rb) + kLn2 * eta * rb.EA / rb.Z;
-      // Bracket of rho = Z_a / Z_b in the refinement's frames (each row relative
-      // to its own max at the true temperature): the fp32 sums' bounds, the
-      // reshaping by the rounded temperature factor, and a factor 3 of margin.
-      const double cex = c_exact;
-      const double rho = (ra.Z / rb.Z) *
-          exp2((static_cast<double>(ra.K) - static_cast<double>(rb.K)) -
-               (static_cast<double>(ra.mraw) - static_cast<double>(rb.mraw)) * cex);
-      const double band = 3.0 * (dZ(ra) + dZ(rb) +
-          kLn2 * eta * (fabs(static_cast<double>(ra.mraw) - static_cast<double>(rb.mraw)) * cex +
-                        ra.EA / ra.Z + rb.EA / rb.Z + 1.0)) + 1e-12;
-      jb.rho_lo = rho * (1.0 - band);
-      jb.rho_hi = rho * (1.0 + band);
-    } else {
-      jb.kind = kJobBonus;
-      jb.Kb = 0.0f;
-      jb.mraw_b = 0.0f;
-      jb.A = 1.0f;
-      jb.Bq = 0.0f;
-      jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + 1e-14;
-      jb.eps0b = 0.0;
-      jb.rho_lo = 0.0;
-      jb.rho_hi = 0.0;
-    }
-    *job = jb;
+    write_job<BF16>(p, i, n, L, sh.rows[n], n < L ? &sh.rows[k + 1 + n] : nullptr, t);
   }
+}
+
+// Prefix order: resolve position j of request i once its rows (target j, and
+// draft j for a sampled position before L) are in.  Outcome in sh.state:
+//   0 finished (outputs final, no job), 1 rows of position j+1 needed,
+//   2 a sample job was written (p.jobs[i]).
+template <bool BF16>
+__device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, int j,
+                                DecideShared& sh) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int k = p.k, L = ri.L;
+  int32_t* tok = p.out_tok + static_cast<int64_t>(i) * (k + 1);
+  float* op = p.out_p ? p.out_p + static_cast<int64_t>(i) * k : nullptr;
+  float* oq = p.out_q ? p.out_q + static_cast<int64_t>(i) * k : nullptr;
+  const int32_t* x = p.tokens + static_cast<int64_t>(i) * k;
+  if (j == 0) write_defaults(p, i);
+  if (ri.bad_T) {
+    __syncthreads();
+    if (tid == 0) {
+      fail_request(p, i, kDevBadTemperature);
+      sh.state = 0;
+    }
+    __syncthreads();
+    return;
+  }
+  const bool pair = !ri.greedy && j < L;
+  if (warp == 0) {
+    if (ri.greedy) merge_greedy_row(p, i, j, sh.rows[0]);
+    else merge_stochastic_row(p, i, j, sh.rows[0]);
+  } else if (warp == 1 && pair) {
+    merge_stochastic_row(p, i, k + 1 + j, sh.rows[1]);
+  }
+  __syncthreads();
+  const RowMerged& ra = sh.rows[0];
+  const RowMerged& rb = sh.rows[1];
+  const TempConsts t = temp_consts<BF16>(p, ri.T);
+  if (tid == 0) {
+    sh.need_exact = -1;
+    sh.state = 0;
+    uint32_t status = 0;
+    if (j == L) {  // the bonus row
+      if (ra.bad) status = kDevNonfinite;
+      else if (ri.greedy) tok[L] = ra.arg;
+      if (!status) {
+        p.out_acc[i] = L;
+        if (p.out_status) p.out_status[i] = 0;
+        if (ri.greedy) {
+          p.jobs[i].kind = kJobNone;
+        } else {
+          write_job<BF16>(p, i, L, L, ra, nullptr, t);
+          sh.state = 2;
+        }
+      }
+    } else {
+      const int xj = __ldg(x + j);
+      if (xj < 0 || static_cast<int64_t>(xj) >= p.V) {
+        status = kDevBadToken;
+      } else if (ra.bad || (pair && rb.bad)) {
+        status = kDevNonfinite;
+      } else if (ri.greedy) {
+        if (xj == ra.arg) {
+          tok[j] = xj;
+          sh.state = 1;
+        } else {
+          tok[j] = ra.arg;
+          p.out_acc[i] = j;
+          if (p.out_status) p.out_status[i] = 0;
+          p.jobs[i].kind = kJobNone;
+        }
+      } else {
+        double pa, qb;
+        const int decision = accept_eval<BF16>(p, i, j, xj, ra, rb, t, pa, qb);
+        if (op) op[j] = static_cast<float>(pa);
+        if (oq) oq[j] = static_cast<float>(qb);
+        if (decision < 0) sh.need_exact = 1;
+        else if (decision == 1) {
+          tok[j] = xj;
+          sh.state = 1;
+        } else {
+          p.out_acc[i] = j;
+          if (p.out_status) p.out_status[i] = 0;
+          write_job<BF16>(p, i, j, L, ra, &rb, t);
+          sh.state = 2;
+        }
+      }
+    }
+    if (status) fail_request(p, i, status);
+  }
+  __syncthreads();
+  if (sh.need_exact > 0) {
+    bool accept = false;
+    double pa = 0.0, qb = 0.0;
+    const int xj = __ldg(x + j);
+    accept_exact<BF16>(p, i, j, xj, ra, rb, t, sh.red, accept, pa, qb);
+    if (tid == 0) {
+      if (op) op[j] = static_cast<float>(pa);
+      if (oq) oq[j] = static_cast<float>(qb);
+      if (accept) {
+        tok[j] = xj;
+        sh.state = 1;
+      } else {
+        p.out_acc[i] = j;
+        if (p.out_status) p.out_status[i] = 0;
+        write_job<BF16>(p, i, j, L, ra, &rb, t);
+        sh.state = 2;
+      }
+    }
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------

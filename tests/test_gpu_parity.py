@@ -21,10 +21,11 @@ pytestmark = pytest.mark.gpu
 THREADS = max(1, min(32, os.cpu_count() or 1))
 
 
-@pytest.fixture(scope="module")
-def ver(cuda_device):
+@pytest.fixture(scope="module", params=["prefix", "dense"])
+def ver(cuda_device, request):
     build.build()
-    v = binding.SpecVerifier(cuda_device, max_batch=1024, max_k=16, max_vocab=262144)
+    v = binding.SpecVerifier(cuda_device, max_batch=1024, max_k=16, max_vocab=262144,
+                             mode=request.param)
     yield v
     v.close()
 
