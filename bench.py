@@ -281,7 +281,7 @@ def run_reference(args):
 def run_ours(args):
     import torch
     import torch.distributed as dist
-    from speculative_decoding_verification_86_b200 import binding, build
+    from speculative_decoding_verification_86_b200 import binding, build, ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -307,7 +307,7 @@ def run_ours(args):
     def step():
         ver.run(w["target"], w.get("draft"), w["tokens"], verify_len=w.get("verify_len"),
                 temperature=w.get("temperature"), conf=w.get("conf"), seed=w["seed"],
-                request_offset=rank * B, out=out)
+                request_offset=ranks.weak_offset(B, rank), out=out)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -353,15 +353,12 @@ def run_ours(args):
         step()
     o1.record(stream)
     torch.cuda.synchronize(dev)
-    other_ms = o0.elapsed_time(o1) / nb
+    other_ms = ranks.max_over_ranks(o0.elapsed_time(o1), dev) / nb
     other_line = {"mode": other, "ms_per_step": other_ms,
                   "value": positions * world / (other_ms / 1e3),
                   "hbm_gbs": dense_row_bytes(w, L) / (other_ms * 1e-3) / 1e9 if other == "dense" else None}
     ver.set_mode(args.mode)
-    t = torch.tensor([ms_local], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = ranks.max_over_ranks(ms_local, dev)
     ms_per_step = ms_total / args.steps
     value = positions * world / (ms_per_step / 1e3)
     launches_per_step = 1 + (1 if w.get("conf") is not None else 0)
@@ -384,7 +381,7 @@ def run_ours(args):
         def hstep():
             ver.run_host(host["target"], host.get("draft"), host["tokens"], verify_len=host.get("verify_len"),
                          temperature=host.get("temperature"), conf=hconf, seed=w["seed"],
-                         request_offset=rank * B, out=hout)
+                         request_offset=ranks.weak_offset(B, rank), out=hout)
 
         hstep()
         if world > 1:
@@ -397,10 +394,7 @@ def run_ours(args):
             hstep()
         a1.record(stream)
         torch.cuda.synchronize(dev)
-        te = torch.tensor([a0.elapsed_time(a1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item()) / args.e2e_steps
+        e2e_ms = ranks.max_over_ranks(a0.elapsed_time(a1), dev) / args.e2e_steps
         h2d = sum(v.numel() * v.element_size() for key, v in host.items()
                   if isinstance(v, torch.Tensor) and key in ("target", "draft", "tokens", "verify_len", "temperature"))
         if hconf is not None:

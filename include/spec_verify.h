@@ -91,7 +91,14 @@ typedef struct spec_verify_ctx spec_verify_ctx;
 
 /* Confidence-head arguments ("What DSpark adds"): survival s_j =
  * sigmoid(w . hidden[i, j, :] + bias) for j < kb; the budget of request i is the
- * number of leading positions whose prefix product prod_{j'<=j} s_j' >= threshold. */
+ * number of leading positions whose prefix product P_ij = prod_{j'<=j} s_ij' >=
+ * threshold.
+ * total_budget > 0 adds the batch-wide, load-aware limit (same section: how much
+ * is verified follows the predicted survival and the load): of the positions
+ * left by verify_len and the threshold, only the total_budget ones with the
+ * largest P_ij are verified, ties going to the lower request index and then to
+ * the lower position; P_ij never grows with j, so each request keeps a leading
+ * run.  sum_i L_i = min(total_budget, positions left).  <= 0: no such limit. */
 typedef struct {
     const void* hidden; /* device, [B, kb, H] bf16 drafter hidden states */
     const void* w;      /* device, [H] bf16 projection */
@@ -99,6 +106,7 @@ typedef struct {
     int kb;             /* positions scored by the head (1..16) */
     int H;              /* hidden width (1..65536) */
     float threshold;
+    int64_t total_budget; /* batch-wide verify budget (positions); <= 0: none */
 } spec_conf_args;
 
 /* Create a context on `device` with workspace for batches up to max_batch
@@ -119,7 +127,8 @@ spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode);
  *   draft_tokens  [B, k] int32.
  *   verify_len    [B] int32 positions to verify per request (clamped to [0, k]), or NULL => k.
  *   temperature   [B] fp32 per request (0 => greedy), or NULL => 1.0 for all.
- *   conf          NULL, or a confidence head; then L_i = min(verify_len_i, budget_i).
+ *   conf          NULL, or a confidence head; then L_i = min(verify_len_i, budget_i),
+ *                 further limited by conf->total_budget (see spec_verify_lengths).
  *   seed, step, request_offset select the random draws (see counter layout above).
  * Outputs:
  *   out_accepted [B] int32: n_i = accepted drafted tokens (-1 if the request failed).
@@ -185,6 +194,16 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
 spec_status spec_conf_budget(spec_verify_ctx* ctx, const void* hidden, const void* w,
                              float bias, int B, int kb, int H, float threshold,
                              int32_t* out_len, float* out_survival, cudaStream_t stream);
+
+/* Verified lengths alone, as spec_verify_run would use them: L_i = verify_len_i
+ * (NULL => k) clamped to [0, k], limited by the confidence head's per-request
+ * budget and then by conf->total_budget (see spec_conf_args).  A serving loop
+ * calls this before the target's forward pass to decide how many positions of
+ * each request to score.  out_len [B] int32; out_survival [B, kb] fp32 or NULL.
+ * Limits: 0 <= B <= max_batch, 0 <= k <= max_k; `conf` is required. */
+spec_status spec_verify_lengths(spec_verify_ctx* ctx, const spec_conf_args* conf,
+                                const int32_t* verify_len, int B, int k, int32_t* out_len,
+                                float* out_survival, cudaStream_t stream);
 
 /* spec_verify_run on HOST buffers: copies the inputs (pinned or pageable host
  * memory) to device staging owned by the context, verifies, copies the outputs

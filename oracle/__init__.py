@@ -56,6 +56,7 @@ class _Inputs(ctypes.Structure):
         ("conf_threshold", ctypes.c_float),
         ("conf_kb", ctypes.c_int),
         ("conf_H", ctypes.c_int),
+        ("conf_total", ctypes.c_int64),
         ("B", ctypes.c_int),
         ("k", ctypes.c_int),
         ("V", ctypes.c_int64),
@@ -95,6 +96,11 @@ def lib():
             _lib.oracle_uniform_fill.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
                                                  ctypes.c_uint32, ctypes.c_uint32, ctypes.c_void_p]
             _lib.oracle_uniform_fill.restype = None
+            _lib.oracle_budget_topn.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                                ctypes.c_int, ctypes.c_int64, ctypes.c_void_p]
+            _lib.oracle_budget_topn.restype = ctypes.c_int
+            _lib.oracle_verify_lengths.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+            _lib.oracle_verify_lengths.restype = ctypes.c_int
             _lib.oracle_conf_budget.argtypes = [
                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int, ctypes.c_int,
                 ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
@@ -186,6 +192,7 @@ def _verify_slice(d, lo, hi, res):
     inp.conf_threshold = d["conf_threshold"]
     inp.conf_kb = d["conf_kb"]
     inp.conf_H = d["conf_H"]
+    inp.conf_total = d.get("conf_total", 0)
     inp.B = B
     inp.k = k
     inp.V = d["V"]
@@ -206,6 +213,41 @@ def _verify_slice(d, lo, hi, res):
     assert rc == 0, rc
 
 
+def _verify_lengths(d, B):
+    keep = []
+    def keepref(a):
+        keep.append(a)
+        return _ptr(a)
+    inp = _Inputs()
+    inp.verify_len = keepref(d["verify_len"])
+    inp.conf_hidden = keepref(d["conf_hidden"])
+    inp.conf_w = keepref(d["conf_w"])
+    inp.conf_bias = d["conf_bias"]
+    inp.conf_threshold = d["conf_threshold"]
+    inp.conf_kb = d["conf_kb"]
+    inp.conf_H = d["conf_H"]
+    inp.conf_total = d["conf_total"]
+    inp.B = B
+    inp.k = d["k"]
+    out = np.zeros(B, dtype=np.int32)
+    rc = lib().oracle_verify_lengths(ctypes.byref(inp), _ptr(out))
+    assert rc == 0, rc
+    return out
+
+
+def budget_topn(prefix: np.ndarray, cap: np.ndarray, total: int) -> np.ndarray:
+    """Batch-wide verify budget: prefix [B, kb] fp64 survival products, cap [B]
+    candidate positions per request, total budget -> L [B] int32."""
+    prefix = np.ascontiguousarray(prefix, dtype=np.float64)
+    B, kb = prefix.shape
+    cap = np.ascontiguousarray(cap, dtype=np.int32)
+    out = np.zeros(B, dtype=np.int32)
+    rc = lib().oracle_budget_topn(_ptr(prefix), _ptr(cap), B, kb, int(total), _ptr(out))
+    if rc:
+        raise ValueError("oracle_budget_topn rejected its arguments (%d)" % rc)
+    return out
+
+
 def verify(target, draft, draft_tokens, *, dtype, verify_len=None, temperature=None,
            conf=None, seed=0, step=0, request_offset=0, u_override=None, threads=1):
     """Run the oracle over a batch.
@@ -213,7 +255,8 @@ def verify(target, draft, draft_tokens, *, dtype, verify_len=None, temperature=N
     target: [B, k+1, V] float32 or uint16 (bf16 bits); draft: [B, k, V] same
     dtype or None; draft_tokens: [B, k] int32; verify_len: [B] int32 or None;
     temperature: [B] float32 or None; conf: dict(hidden=[B,kb,H] uint16,
-    w=[H] uint16, bias=float, threshold=float) or None; u_override:
+    w=[H] uint16, bias=float, threshold=float[, total=int batch-wide verify
+    budget]) or None; u_override:
     [B, k+1, 2] float64 or None.  ``threads`` > 1 runs contiguous request
     groups concurrently (each request is independent; the global request index
     keeps the random draws identical).
@@ -233,6 +276,7 @@ def verify(target, draft, draft_tokens, *, dtype, verify_len=None, temperature=N
         conf_threshold=0.0 if conf is None else float(conf["threshold"]),
         conf_kb=0 if conf is None else int(conf["hidden"].shape[1]),
         conf_H=0 if conf is None else int(conf["hidden"].shape[2]),
+        conf_total=0 if conf is None else int(conf.get("total", 0)),
         k=k, V=V, seed=int(seed), step=int(step), request_offset=int(request_offset),
         u_override=None if u_override is None else np.ascontiguousarray(u_override, dtype=np.float64),
     )
@@ -253,6 +297,11 @@ def verify(target, draft, draft_tokens, *, dtype, verify_len=None, temperature=N
     if B == 0:
         return res
     threads = max(1, min(int(threads), B))
+    if threads > 1 and d["conf_total"] > 0:
+        # the batch-wide budget couples the requests: fix every L_i on the
+        # whole batch first, then verify slices with those lengths
+        lengths = _verify_lengths(d, B)
+        d = dict(d, verify_len=lengths, conf_hidden=None, conf_total=0)
     if threads == 1:
         _verify_slice(d, 0, B, res)
     else:

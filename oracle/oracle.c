@@ -41,6 +41,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define ORC_DTYPE_F32 0
@@ -157,6 +158,7 @@ typedef struct {
     float conf_threshold;
     int conf_kb;
     int conf_H;
+    int64_t conf_total;           /* batch-wide verify budget; <= 0: none */
     int B;
     int k;
     int64_t V;
@@ -176,6 +178,86 @@ typedef struct {
     int32_t* verify_len_used; /* [B]: L_i after clamping and the confidence budget */
     uint32_t* status;         /* [B]: error bits */
 } oracle_outputs;
+
+/* ------------------------------------------------------------------------ */
+/* Batch-wide verify budget (the load-aware form of the confidence rule:     */
+/* "Speculative decoding becomes standard: DSpark and multi-token drafters", */
+/* section "What DSpark adds" -- the verified length follows the predicted   */
+/* survival and the load of the batch).  Among the candidate positions       */
+/* (request i, position j < cap_i) keep the `total` ones with the largest    */
+/* prefix survival P_ij, ties going to the lower request index, then to the  */
+/* lower position; L_i = how many of request i's positions were kept.        */
+/* Because P_ij does not increase with j, the kept positions of a request    */
+/* are always a leading run.  total >= number of candidates keeps them all.  */
+/* Written as its definition: list the candidates, sort them, take a prefix. */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    double P;
+    int i;
+    int j;
+} orc_candidate;
+
+static int candidate_order(const void* a, const void* b) {
+    const orc_candidate* x = (const orc_candidate*)a;
+    const orc_candidate* y = (const orc_candidate*)b;
+    if (x->P != y->P) return x->P > y->P ? -1 : 1;  /* larger survival first */
+    if (x->i != y->i) return x->i < y->i ? -1 : 1;  /* then lower request */
+    return (x->j > y->j) - (x->j < y->j);           /* then lower position */
+}
+
+int oracle_budget_topn(const double* prefix, const int32_t* cap, int B, int kb,
+                       int64_t total, int32_t* out_len) {
+    if (B < 0 || kb < 0 || total < 0) return 1;
+    int64_t n = 0;
+    for (int i = 0; i < B; ++i) {
+        if (cap[i] < 0 || cap[i] > kb) return 1;
+        n += cap[i];
+    }
+    orc_candidate* c = (orc_candidate*)malloc((size_t)(n > 0 ? n : 1) * sizeof *c);
+    if (!c) return 2;
+    int64_t m = 0;
+    for (int i = 0; i < B; ++i) {
+        for (int j = 0; j < cap[i]; ++j) {
+            c[m].P = prefix[(int64_t)i * kb + j];
+            c[m].i = i;
+            c[m].j = j;
+            ++m;
+        }
+    }
+    qsort(c, (size_t)n, sizeof *c, candidate_order);
+    for (int i = 0; i < B; ++i) out_len[i] = 0;  /* after the last read of cap */
+    for (int64_t r = 0; r < n && r < total; ++r) out_len[c[r].i]++;
+    free(c);
+    return 0;
+}
+
+/* Verified length of every request: verify_len clamped to [0, k], then the
+ * confidence head's per-request budget, then (if conf_total > 0) the batch-wide
+ * budget over the positions that survive the first two limits. */
+int oracle_verify_lengths(const oracle_inputs* in, int32_t* out_len) {
+    const int B = in->B, k = in->k;
+    if (B < 0 || k < 0) return 1;
+    for (int i = 0; i < B; ++i) {
+        int L = in->verify_len ? in->verify_len[i] : k;
+        if (L < 0) L = 0;
+        if (L > k) L = k;
+        out_len[i] = L;
+    }
+    if (!in->conf_hidden || B == 0) return 0;
+    const int kb = in->conf_kb;
+    int32_t* budget = (int32_t*)malloc((size_t)B * sizeof *budget);
+    double* prefix = (double*)malloc((size_t)B * (size_t)(kb > 0 ? kb : 1) * sizeof *prefix);
+    if (!budget || !prefix) { free(budget); free(prefix); return 2; }
+    oracle_conf_budget(in->conf_hidden, in->conf_w, in->conf_bias, B, kb, in->conf_H,
+                       in->conf_threshold, budget, NULL, prefix);
+    for (int i = 0; i < B; ++i)
+        if (budget[i] < out_len[i]) out_len[i] = budget[i];
+    int rc = 0;
+    if (in->conf_total > 0) rc = oracle_budget_topn(prefix, out_len, B, kb, in->conf_total, out_len);
+    free(budget);
+    free(prefix);
+    return rc;
+}
 
 static double draw_uniform(const oracle_inputs* in, int i, int position, int draw) {
     if (in->u_override) return in->u_override[((int64_t)i * (in->k + 1) + position) * 2 + draw];
@@ -304,7 +386,10 @@ int oracle_verify(const oracle_inputs* in, const oracle_outputs* out) {
     const int B = in->B, k = in->k;
     const int64_t V = in->V;
     if (B < 0 || k < 0 || V <= 0) return 1;
-    int32_t* budget = NULL;
+    {
+        const int rc = oracle_verify_lengths(in, out->verify_len_used);
+        if (rc) return rc;
+    }
     for (int i = 0; i < B; ++i) {
         out->status[i] = 0;
         out->sample_margin[i] = -1.0;
@@ -315,20 +400,8 @@ int oracle_verify(const oracle_inputs* in, const oracle_outputs* out) {
             out->accept_margin[(int64_t)i * k + j] = -1.0;
         }
 
-        /* 1. verification length: verify_len clamped to [0, k], then the
-         *    confidence budget (if a head is given). */
-        int L = in->verify_len ? in->verify_len[i] : k;
-        if (L < 0) L = 0;
-        if (L > k) L = k;
-        if (in->conf_hidden) {
-            int32_t b = 0;
-            oracle_conf_budget(in->conf_hidden + (int64_t)i * in->conf_kb * in->conf_H,
-                               in->conf_w, in->conf_bias, 1, in->conf_kb, in->conf_H,
-                               in->conf_threshold, &b, NULL, NULL);
-            if (b < L) L = b;
-        }
-        out->verify_len_used[i] = L;
-        (void)budget;
+        /* 1. verification length (computed for the whole batch above). */
+        const int L = out->verify_len_used[i];
 
         float Tf = in->temperature ? in->temperature[i] : 1.0f;
         if (!temperature_valid(Tf)) { fail_request(in, out, i, ORC_ERR_BAD_TEMPERATURE); continue; }

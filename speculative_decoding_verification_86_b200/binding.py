@@ -49,7 +49,8 @@ class SpecVerifyError(RuntimeError):
 
 class ConfArgs(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_void_p), ("w", ctypes.c_void_p), ("bias", ctypes.c_float),
-                ("kb", ctypes.c_int), ("H", ctypes.c_int), ("threshold", ctypes.c_float)]
+                ("kb", ctypes.c_int), ("H", ctypes.c_int), ("threshold", ctypes.c_float),
+                ("total_budget", ctypes.c_int64)]
 
 
 _lib = None
@@ -81,6 +82,7 @@ def lib():
     L.spec_verify_greedy_noalloc.argtypes = [_vp, _i32, _vp, _vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp]
     L.spec_conf_budget.argtypes = [_vp, _vp, _vp, ctypes.c_float, _i32, _i32, _i32,
                                    ctypes.c_float, _vp, _vp, _vp]
+    L.spec_verify_lengths.argtypes = [_vp, ctypes.POINTER(ConfArgs), _vp, _i32, _i32, _vp, _vp, _vp]
     L.spec_verify_set_mode.argtypes = [_vp, _i32]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
@@ -91,7 +93,8 @@ def lib():
     L.spec_verify_ex2_error_bound.restype = ctypes.c_double
     for name in ("spec_verify_init", "spec_verify_destroy", "spec_verify_run",
                  "spec_verify_run_with_uniforms", "spec_verify_run_host", "spec_verify_greedy",
-                 "spec_conf_budget", "spec_verify_greedy_noalloc", "spec_verify_set_mode",
+                 "spec_conf_budget", "spec_verify_lengths", "spec_verify_greedy_noalloc",
+                 "spec_verify_set_mode",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
         getattr(L, name).restype = _i32
@@ -208,7 +211,8 @@ class SpecVerifier:
         hidden, w = conf["hidden"], conf["w"]
         c = ConfArgs(_dev_ptr(hidden, torch.bfloat16, self.device, "conf.hidden"),
                      _dev_ptr(w, torch.bfloat16, self.device, "conf.w"), float(conf["bias"]),
-                     int(hidden.shape[1]), int(hidden.shape[2]), float(conf["threshold"]))
+                     int(hidden.shape[1]), int(hidden.shape[2]), float(conf["threshold"]),
+                     int(conf.get("total", 0)))
         return ctypes.byref(c), c
 
     def _shape(self, target, draft, tokens):
@@ -276,6 +280,23 @@ class SpecVerifier:
         _check(st, "spec_conf_budget")
         return out_len, surv
 
+    def lengths(self, conf, k, verify_len=None, stream=None, with_survival=False):
+        """spec_verify_lengths: the verified lengths L [B] int32 that
+        spec_verify_run would use (verify_len, threshold, conf["total"]), and
+        optionally the survival [B, kb] fp32."""
+        B, kb, _ = conf["hidden"].shape
+        if verify_len is not None and tuple(verify_len.shape) != (B,):
+            raise ValueError("verify_len must be [B]")
+        cref, keep = self._conf(conf)
+        out_len = torch.empty(B, dtype=torch.int32, device=self.device)
+        surv = torch.empty((B, kb), dtype=torch.float32, device=self.device) if with_survival else None
+        st = lib().spec_verify_lengths(
+            self._h, cref, _dev_ptr(verify_len, torch.int32, self.device, "verify_len"), B, int(k),
+            _dev_ptr(out_len, torch.int32), _dev_ptr(surv), _stream_handle(stream, self.device))
+        del keep
+        _check(st, "spec_verify_lengths")
+        return out_len, surv
+
     def run_host(self, target, draft, tokens, verify_len=None, temperature=None, conf=None,
                  seed=0, step=0, request_offset=0, stream=None, out=None, allow_failed=True):
         """spec_verify_run_host: CPU tensors in (pinned for speed), CPU tensors out."""
@@ -299,7 +320,7 @@ class SpecVerifier:
         if conf is not None:
             keep = ConfArgs(hp(conf["hidden"]), hp(conf["w"]), float(conf["bias"]),
                             int(conf["hidden"].shape[1]), int(conf["hidden"].shape[2]),
-                            float(conf["threshold"]))
+                            float(conf["threshold"]), int(conf.get("total", 0)))
             cref = ctypes.byref(keep)
         st = lib().spec_verify_run_host(
             self._h, hp(target), hp(draft), dt, hp(tokens), hp(verify_len), hp(temperature), cref,

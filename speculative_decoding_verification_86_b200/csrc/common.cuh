@@ -100,7 +100,7 @@ struct Counters {
 // Engine: orders of the statistics pass, and the queue's control words.
 constexpr int kModeDense = 0;
 constexpr int kModePrefix = 1;
-constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQWords = 8;
+constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQInit = 4, kQWords = 8;
 constexpr int kEngineMinBlocks = 3;
 
 // -------------------------------------------------------------- run params --
@@ -162,6 +162,12 @@ struct ConfParams {
   int B;
   int kb;
   int H;
+  int k;                   // verify_len cap applies when >= 0 (clamp to [0, k])
+  const int32_t* vlen;     // [B] or nullptr (=> k)
+  long long total;         // batch-wide verify budget; <= 0: none
+  double* prefix;          // [B, kb] workspace: prefix survival (total > 0)
+  int32_t* cap;            // [B] workspace: per-request limit before the batch budget
+  unsigned* arrive;        // arrival counter (self-resetting)
   int32_t* out_len;        // [B]
   float* out_survival;     // [B, kb] or nullptr
 };
@@ -179,6 +185,26 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed fp32 pairs (sm_100): two independent round-to-nearest operations per
+// instruction, each rounded exactly as its scalar counterpart.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)),
+        "l"(reinterpret_cast<const unsigned long long&>(b)),
+        "l"(reinterpret_cast<const unsigned long long&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)),
+        "l"(reinterpret_cast<const unsigned long long&>(b)));
+  return d;
 }
 
 __device__ __forceinline__ float fmax_nan(float a, float b) {

@@ -6,16 +6,102 @@
 // budget is the number of leading positions whose prefix product stays at or
 // above the threshold.
 //
+// The same section ties how much is verified to the load of the batch.  With a
+// batch-wide budget N > 0, the positions left by the per-request rule (and by
+// verify_len) are candidates, and only the N with the largest prefix survival
+// are verified -- ties to the lower request, then the lower position.  The
+// prefix product never grows along a request, so the kept positions of each
+// request are a leading run and its verified length is their count.
+//
 // One CTA per request, one warp per position: the bf16 x bf16 products are
-// exact in fp32 and are summed in fp64, so the budget decision is made on an
-// fp64 prefix product.
+// exact in fp32 and are summed in fp64, so every decision is made on an fp64
+// prefix product.  With a batch budget the last CTA to finish selects: a
+// radix select (8 passes of 8 bits over the fp64 bit patterns, which order
+// like the non-negative values) finds the N-th largest survival t and how many
+// of the candidates equal to t are kept; a scan over the requests in index
+// order hands those ties out.
 #pragma once
 #include "common.cuh"
 
 namespace sv {
 
+// Last CTA of k_conf: the batch-wide selection.  Reads the prefix products and
+// per-request limits every CTA published, writes out_len.
+__device__ void conf_select(const ConfParams& cp) {
+  __shared__ unsigned hist[256];
+  __shared__ double sh_d[kWarps];
+  __shared__ unsigned long long s_key;
+  __shared__ long long s_rank;
+  const int B = cp.B, kb = cp.kb;
+  const long long n = static_cast<long long>(B) * kb;
+
+  double m_local = 0.0;
+  for (int i = threadIdx.x; i < B; i += kThreads) m_local += __ldcg(cp.cap + i);
+  const long long M = static_cast<long long>(block_sum_d(m_local, sh_d));
+  if (cp.total >= M) {
+    for (int i = threadIdx.x; i < B; i += kThreads) cp.out_len[i] = __ldcg(cp.cap + i);
+    return;
+  }
+
+  // t = the total-th largest candidate key (1-based rank from the top).
+  if (threadIdx.x == 0) {
+    s_key = 0ull;
+    s_rank = cp.total;
+  }
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int d = threadIdx.x; d < 256; d += kThreads) hist[d] = 0u;
+    __syncthreads();
+    const unsigned long long want = s_key;
+    const unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+    for (long long e = threadIdx.x; e < n; e += kThreads) {
+      const int i = static_cast<int>(e / kb), j = static_cast<int>(e - static_cast<long long>(i) * kb);
+      if (j >= __ldcg(cp.cap + i)) continue;
+      const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(__ldcg(cp.prefix + e)));
+      if ((key & hi_mask) == want) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      long long above = 0;
+      int d = 255;
+      for (; d > 0; --d) {
+        if (above + hist[d] >= s_rank) break;
+        above += hist[d];
+      }
+      s_rank -= above;  // rank among the keys with this digit
+      s_key = want | (static_cast<unsigned long long>(d) << shift);
+    }
+    __syncthreads();
+  }
+  const unsigned long long t = s_key;
+  const long long take_eq = s_rank;  // how many candidates equal to t are kept
+  double carry = 0.0;
+  for (int base = 0; base < B; base += kThreads) {
+    const int i = base + threadIdx.x;
+    int gt = 0, eq = 0;
+    if (i < B) {
+      const int c = __ldcg(cp.cap + i);
+      for (int j = 0; j < c; ++j) {
+        const unsigned long long key =
+            static_cast<unsigned long long>(__double_as_longlong(__ldcg(cp.prefix + static_cast<long long>(i) * kb + j)));
+        gt += key > t;
+        eq += key == t;
+      }
+    }
+    double tot;
+    const double before = carry + block_exclusive_scan_d(static_cast<double>(eq), sh_d, tot);
+    if (i < B) {
+      const long long left = take_eq - static_cast<long long>(before);
+      const long long take = left <= 0 ? 0 : (left < eq ? left : eq);
+      cp.out_len[i] = gt + static_cast<int>(take);
+    }
+    carry += tot;
+    __syncthreads();
+  }
+}
+
 __global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
   __shared__ double s_surv[kMaxK];
+  __shared__ int s_last;
   const int i = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int j = warp; j < cp.kb; j += kWarps) {
@@ -39,9 +125,20 @@ __global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
       if (counting && prefix >= static_cast<double>(cp.threshold)) ++budget;
       else counting = false;
       if (cp.out_survival) cp.out_survival[static_cast<int64_t>(i) * cp.kb + j] = static_cast<float>(s_surv[j]);
+      if (cp.total > 0) cp.prefix[static_cast<int64_t>(i) * cp.kb + j] = prefix;
     }
-    cp.out_len[i] = budget;
+    if (cp.k >= 0) {
+      int L = cp.vlen ? cp.vlen[i] : cp.k;
+      L = L < 0 ? 0 : (L > cp.k ? cp.k : L);
+      budget = budget < L ? budget : L;
+    }
+    if (cp.total > 0) cp.cap[i] = budget;
+    else cp.out_len[i] = budget;
   }
+  if (cp.total <= 0) return;
+  if (!arrive_last(cp.arrive, static_cast<unsigned>(cp.B), &s_last)) return;
+  __threadfence();
+  conf_select(cp);
 }
 
 }  // namespace sv

@@ -126,6 +126,9 @@ struct spec_verify_ctx {
   int* runc = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
   int32_t* conf_len = nullptr;
+  double* conf_prefix = nullptr;  // [max_batch, kMaxK]
+  int32_t* conf_cap = nullptr;    // [max_batch]
+  unsigned* conf_arrive = nullptr;
   unsigned long long* q_slots = nullptr;
   unsigned q_capacity = 0;
   unsigned* q_ctl = nullptr;
@@ -183,6 +186,9 @@ spec_status carve(spec_verify_ctx* c) {
   const size_t o_runc = take(per_req_subs * sizeof(int));
   const size_t o_cnt = take(2 * sizeof(sv::Counters));
   const size_t o_conf = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
+  const size_t o_cpre = take(static_cast<size_t>(c->max_batch) * sv::kMaxK * sizeof(double));
+  const size_t o_ccap = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
+  const size_t o_carr = take(sizeof(unsigned));
   // queue: every row segment, sample segment and refinement sub-chunk of a
   // batch, plus one exit ticket per CTA
   const size_t max_segs = static_cast<size_t>((c->max_vocab + sv::SegGeo<false>::kSeg - 1) /
@@ -216,6 +222,9 @@ spec_status carve(spec_verify_ctx* c) {
   c->runc = reinterpret_cast<int*>(b + o_runc);
   c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
   c->conf_len = reinterpret_cast<int32_t*>(b + o_conf);
+  c->conf_prefix = reinterpret_cast<double*>(b + o_cpre);
+  c->conf_cap = reinterpret_cast<int32_t*>(b + o_ccap);
+  c->conf_arrive = reinterpret_cast<unsigned*>(b + o_carr);
   c->q_slots = reinterpret_cast<unsigned long long*>(b + o_qs);
   c->q_ctl = reinterpret_cast<unsigned*>(b + o_qc);
   if (cudaMemset(c->ws, 0, off) != cudaSuccess) return SPEC_ERR_CUDA;
@@ -248,8 +257,10 @@ spec_status check_conf(const spec_verify_ctx* c, const spec_conf_args* conf) {
   return SPEC_OK;
 }
 
-spec_status launch_conf(spec_verify_ctx* c, const spec_conf_args* conf, int B, int32_t* out_len,
-                        float* out_surv, cudaStream_t s) {
+// k_conf: per-request budgets, capped by verify_len when k >= 0, then the
+// batch-wide budget when conf->total_budget > 0.
+spec_status launch_conf(spec_verify_ctx* c, const spec_conf_args* conf, int B, int k,
+                        const int32_t* vlen, int32_t* out_len, float* out_surv, cudaStream_t s) {
   sv::ConfParams cp;
   cp.hidden = static_cast<const uint16_t*>(conf->hidden);
   cp.w = static_cast<const uint16_t*>(conf->w);
@@ -258,6 +269,12 @@ spec_status launch_conf(spec_verify_ctx* c, const spec_conf_args* conf, int B, i
   cp.B = B;
   cp.kb = conf->kb;
   cp.H = conf->H;
+  cp.k = k;
+  cp.vlen = vlen;
+  cp.total = conf->total_budget > 0 ? conf->total_budget : 0;
+  cp.prefix = c->conf_prefix;
+  cp.cap = c->conf_cap;
+  cp.arrive = c->conf_arrive;
   cp.out_len = out_len;
   cp.out_survival = out_surv;
   timing_mark(c, kClassConf, true, s);
@@ -340,7 +357,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
 
   cudaGetLastError();  // clear stale errors so the check below is ours
   if (conf) {
-    launch_conf(c, conf, B, c->conf_len, nullptr, s);
+    launch_conf(c, conf, B, k, vlen, c->conf_len, nullptr, s);
     p.conf_len = c->conf_len;
   }
   p.mode = force_greedy ? sv::kModePrefix : c->mode;
@@ -476,14 +493,32 @@ spec_status spec_conf_budget(spec_verify_ctx* ctx, const void* hidden, const voi
   if (!ctx || B < 0 || B > ctx->max_batch) return SPEC_ERR_INVALID_ARG;
   if (B == 0) return SPEC_OK;
   if (!out_len) return SPEC_ERR_INVALID_ARG;
-  spec_conf_args conf{hidden, w, bias, kb, H, threshold};
+  spec_conf_args conf{hidden, w, bias, kb, H, threshold, 0};
   if (spec_status st = check_conf(ctx, &conf); st != SPEC_OK) return st;
   if (!aligned(out_len, 4) || (out_survival && !aligned(out_survival, 4)))
     return SPEC_ERR_UNSUPPORTED;
   DeviceGuard g(ctx->device);
   if (!g.ok) return SPEC_ERR_CUDA;
   cudaGetLastError();
-  launch_conf(ctx, &conf, B, out_len, out_survival, stream);
+  launch_conf(ctx, &conf, B, -1, nullptr, out_len, out_survival, stream);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_verify_lengths(spec_verify_ctx* ctx, const spec_conf_args* conf,
+                                const int32_t* verify_len, int B, int k, int32_t* out_len,
+                                float* out_survival, cudaStream_t stream) {
+  if (!ctx || !conf || B < 0 || B > ctx->max_batch || k < 0 || k > ctx->max_k)
+    return SPEC_ERR_INVALID_ARG;
+  if (B == 0) return SPEC_OK;
+  if (!out_len) return SPEC_ERR_INVALID_ARG;
+  if (spec_status st = check_conf(ctx, conf); st != SPEC_OK) return st;
+  if (!aligned(out_len, 4) || (out_survival && !aligned(out_survival, 4)) ||
+      (verify_len && !aligned(verify_len, 4)))
+    return SPEC_ERR_UNSUPPORTED;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  launch_conf(ctx, conf, B, k, verify_len, out_len, out_survival, stream);
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
 

@@ -133,37 +133,59 @@ struct SoftAcc {
   }
 };
 
+// One batch of a thread's logits into its running statistics.  Logits are
+// taken in pairs (the two halves of a bf16x2 word, or two fp32 words) so the
+// exponent arguments, the bound terms and the sums use packed fp32x2
+// instructions; every lane is rounded as the scalar operation would be.  The
+// argument is formed negated, n = K - l c = -(l c - K) (the same rounding,
+// negated), clamped at 1024 so masked (-inf) logits give e = 0 and a finite
+// bound term.  The batch sum is a balanced pairwise tree: across the batch's
+// vectors, then across the pairs of a vector, then the two lanes.
 template <bool BF16>
 __device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatchVecs], float cc) {
-  using G = SegGeo<BF16>;
   const float bm = batch_max<BF16>(v);
   acc.mraw = fmax_nan(acc.mraw, bm);
   if (isnan(bm) || bm == INFINITY) acc.bad = 1;
   const float Kb = ceilf(bm * cc);
   if (Kb > acc.K) acc.rebase(Kb);
   if (!(acc.K > -INFINITY) || acc.K == INFINITY) return;  // nothing finite yet, or +inf seen
-  const float K = acc.K;
-  float vs[kBatchVecs];
-  float er = acc.er;
+  const float2 ncc = make_float2(-cc, -cc);
+  const float2 K2 = make_float2(acc.K, acc.K);
+  float2 er2 = make_float2(acc.er, 0.0f);
+  constexpr int kPairs = BF16 ? 4 : 2;  // logit pairs per 16-byte vector
+  float2 ps[kBatchVecs][kPairs];
 #pragma unroll
   for (int u = 0; u < kBatchVecs; ++u) {
-    float x[G::kPerVec];
-    unpack<BF16>(v[u], x);
-    float e[G::kPerVec];
+    const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-    for (int q = 0; q < G::kPerVec; ++q) {
-      const float a = fmaxf(fmaf(x[q], cc, -K), -1024.0f);  // <= 0; -inf (masked) -> -1024
-      e[q] = ex2_approx(a);
-      er = fmaf(e[q], -a, er);
-    }
-    if constexpr (BF16) {
-      vs[u] = ((e[0] + e[1]) + (e[2] + e[3])) + ((e[4] + e[5]) + (e[6] + e[7]));
-    } else {
-      vs[u] = (e[0] + e[1]) + (e[2] + e[3]);
+    for (int q = 0; q < kPairs; ++q) {
+      float2 x;
+      if constexpr (BF16) {
+        x = make_float2(bf16_lo(wd[q]), bf16_hi(wd[q]));
+      } else {
+        x = make_float2(__uint_as_float(wd[2 * q]), __uint_as_float(wd[2 * q + 1]));
+      }
+      float2 n = ffma2(x, ncc, K2);  // K - l c >= 0
+      n.x = fminf(n.x, 1024.0f);
+      n.y = fminf(n.y, 1024.0f);
+      const float2 e = make_float2(ex2_approx(-n.x), ex2_approx(-n.y));
+      er2 = ffma2(e, n, er2);
+      ps[u][q] = e;
     }
   }
-  acc.er = er;
-  acc.s += static_cast<double>((vs[0] + vs[1]) + (vs[2] + vs[3]));
+  // across vectors (kBatchVecs = 4: two levels)
+#pragma unroll
+  for (int q = 0; q < kPairs; ++q) {
+    ps[0][q] = fadd2(fadd2(ps[0][q], ps[1][q]), fadd2(ps[2][q], ps[3][q]));
+  }
+  float2 t;
+  if constexpr (BF16) {
+    t = fadd2(fadd2(ps[0][0], ps[0][1]), fadd2(ps[0][2], ps[0][3]));
+  } else {
+    t = fadd2(ps[0][0], ps[0][1]);
+  }
+  acc.er = er2.x + er2.y;
+  acc.s += static_cast<double>(t.x + t.y);
 }
 
 // Merge `acc` of all threads of the CTA into one record (called by every thread).

@@ -143,6 +143,18 @@ def confidence(device="cpu", seed=3, B=128, k=8, V=VOCAB_GEMMA, H=2560):
                 conf=conf, seed=seed, name="verify + confidence head B=%d k=%d V=%d" % (B, k, V))
 
 
+def confidence_batch_budget(device="cpu", seed=3, B=128, k=8, V=VOCAB_GEMMA, H=2560,
+                            threshold=0.05, total=None):
+    """The confidence workload under a batch-wide verify budget: the same
+    logits and head, a low per-request threshold (0.05) and a budget of
+    ``total`` positions for the whole batch (default 2 per request)."""
+    w = confidence(device, seed, B, k, V, H)
+    w["conf"] = dict(w["conf"], threshold=threshold, total=2 * B if total is None else int(total))
+    w["name"] = "verify + confidence head, batch budget %d, B=%d k=%d V=%d" % (
+        w["conf"]["total"], B, k, V)
+    return w
+
+
 def sweep(device="cpu", seed=4, B=128, k=5, V=VOCAB_QWEN):
     """Load sweep point: correlated bf16 logits, T_i drawn from {0, 0.7, 1.0},
     L_i ~ U{1..5}."""
@@ -179,7 +191,8 @@ def to_numpy_inputs(w):
         c = w["conf"]
         conf = dict(hidden=c["hidden"].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16),
                     w=c["w"].detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16),
-                    bias=float(c["bias"]), threshold=float(c["threshold"]))
+                    bias=float(c["bias"]), threshold=float(c["threshold"]),
+                    total=int(c.get("total", 0)))
     return dict(target=logits(w["target"]), draft=logits(w.get("draft")),
                 tokens=opt(w["tokens"]), verify_len=opt(w.get("verify_len")),
                 temperature=opt(w.get("temperature")), conf=conf,

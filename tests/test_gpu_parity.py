@@ -298,3 +298,112 @@ def test_ex2_error_bound_holds_on_this_device(cuda_device):
     build.build()
     measured, bound = binding.selfcheck_ex2(cuda_device.index, -126.0, 0.0)
     assert 0 < measured <= bound, (measured, bound)
+
+
+# ------------------------------------------------------ batch-wide budget ----
+
+def _conf_case(B, kb, H, seed, bias=0.5, same_rows=False):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    hidden = torch.randn(B, kb, H, generator=g, device="cuda").to(torch.bfloat16)
+    if same_rows:
+        hidden[:] = hidden[0]
+    w = (torch.randn(H, generator=g, device="cuda") * (2.0 / H ** 0.5)).to(torch.bfloat16)
+    return hidden, w
+
+
+def _oracle_lengths(hidden, w, bias, tau, vlen, k, total):
+    hb = hidden.cpu().view(torch.int16).numpy().view(np.uint16)
+    wb = w.cpu().view(torch.int16).numpy().view(np.uint16)
+    static, _, pref = oracle.conf_budget(hb, wb, bias, tau)
+    lim = np.full(len(static), k) if vlen is None else np.clip(vlen.cpu().numpy(), 0, k)
+    cap = np.minimum(lim, static).astype(np.int32)
+    if total <= 0:
+        return cap, pref, cap
+    return oracle.budget_topn(pref, cap, total), pref, cap
+
+
+def _assert_decidable(L, pref, cap):
+    """Kept and dropped survivals are apart by more than rounding (so the
+    fp64 values of the two sides cannot order them differently)."""
+    kept = [pref[i, j] for i in range(len(L)) for j in range(L[i])]
+    drop = [pref[i, j] for i in range(len(L)) for j in range(L[i], cap[i])]
+    if kept and drop:
+        assert min(kept) - max(drop) > 1e-12 * max(drop)
+
+
+@pytest.mark.parametrize("B,kb,H,with_vlen", [(128, 8, 2560, False), (77, 5, 300, True),
+                                              (1000, 16, 64, True)])
+def test_batch_budget_lengths(ver, B, kb, H, with_vlen):
+    hidden, w = _conf_case(B, kb, H, seed=B)
+    k = kb
+    g = torch.Generator(device="cuda").manual_seed(B + 1)
+    vlen = torch.randint(-1, k + 2, (B,), generator=g, device="cuda", dtype=torch.int32) if with_vlen else None
+    bias, tau = 0.5, 0.02
+    _, pref0, cap0 = _oracle_lengths(hidden, w, bias, tau, vlen, k, 0)
+    M = int(cap0.sum())
+    assert M > 2
+    for total in (0, 1, 2, M // 3, M - 1, M, M + 5, 10 ** 9):
+        conf = dict(hidden=hidden, w=w, bias=bias, threshold=tau, total=total)
+        L, surv = ver.lengths(conf, k, verify_len=vlen, with_survival=True)
+        torch.cuda.synchronize()
+        oL, pref, cap = _oracle_lengths(hidden, w, bias, tau, vlen, k, total)
+        np.testing.assert_array_equal(L.cpu().numpy(), oL, err_msg="total=%d" % total)
+        assert int(oL.sum()) == (M if total <= 0 else min(total, M))
+        _assert_decidable(oL, pref, cap)
+
+
+def test_batch_budget_ties_go_to_lower_request_then_position(ver):
+    B, kb, H = 40, 6, 128
+    # identical requests: equal survivals across requests
+    hidden, w = _conf_case(B, kb, H, seed=5, same_rows=True)
+    for total in (1, 7, 59, 100, 239):
+        conf = dict(hidden=hidden, w=w, bias=0.5, threshold=0.0, total=total)
+        L, _ = ver.lengths(conf, kb)
+        torch.cuda.synchronize()
+        oL, _, _ = _oracle_lengths(hidden, w, 0.5, 0.0, None, kb, total)
+        np.testing.assert_array_equal(L.cpu().numpy(), oL, err_msg="total=%d" % total)
+    # survival exactly 1 everywhere: every position ties; requests fill in order
+    for total in (1, 13, 100):
+        conf = dict(hidden=hidden, w=w, bias=100.0, threshold=0.5, total=total)
+        L, _ = ver.lengths(conf, kb)
+        torch.cuda.synchronize()
+        expect = np.clip(total - kb * np.arange(B), 0, kb)
+        np.testing.assert_array_equal(L.cpu().numpy(), expect)
+
+
+def test_batch_budget_through_verification(ver):
+    w = workloads.confidence_batch_budget("cuda", seed=3)
+    o = run_oracle(w)
+    g = run_gpu(ver, w)
+    compare(g, o)
+    total = w["conf"]["total"]
+    assert int(o["verify_len_used"].sum()) == total
+    L, _ = ver.lengths(w["conf"], w["tokens"].shape[1])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(L.cpu().numpy(), o["verify_len_used"])
+    # the host-buffer entry point carries the budget too
+    h = {key: (v.cpu() if isinstance(v, torch.Tensor) else v) for key, v in w.items()}
+    hc = dict(w["conf"], hidden=w["conf"]["hidden"].cpu(), w=w["conf"]["w"].cpu())
+    gh = ver.run_host(h["target"], h["draft"], h["tokens"], conf=hc, seed=w["seed"])
+    np.testing.assert_array_equal(gh["accepted"].numpy(), g["accepted"])
+    np.testing.assert_array_equal(gh["tokens"].numpy(), g["tokens"])
+
+
+# ------------------------------------------------------ hand-worked cases ----
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_hand_worked_golden_cases(ver, dtype):
+    """The hand-derived cases (several with a draw exactly on a decision edge)
+    through the C ABI, in both logit formats."""
+    import golden_cases
+    for c in golden_cases.load():
+        dev = ver.device
+        w = dict(target=torch.from_numpy(c["target"]).to(dev, dtype),
+                 draft=torch.from_numpy(c["draft"]).to(dev, dtype),
+                 tokens=torch.from_numpy(c["tokens"]).to(dev),
+                 verify_len=torch.from_numpy(c["verify_len"]).to(dev),
+                 temperature=torch.from_numpy(c["temperature"]).to(dev), seed=0)
+        g = run_gpu(ver, w, uniforms=torch.from_numpy(c["u"]).to(dev))
+        assert g["status"][0] == 0, c["name"]
+        assert g["accepted"][0] == c["n"], c["name"]
+        assert g["tokens"][0].tolist() == c["out_tokens"].tolist(), c["name"]

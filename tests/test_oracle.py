@@ -398,3 +398,18 @@ def test_empty_batch(oracle_lib):
     res = oracle.verify(np.zeros((0, 3, 8), dtype=np.float32), np.zeros((0, 2, 8), dtype=np.float32),
                         np.zeros((0, 2), dtype=np.int32), dtype=F32)
     assert res["accepted"].shape == (0,)
+
+
+# ------------------------------------------------------ hand-worked cases ----
+
+def test_hand_worked_golden_cases(oracle_lib):
+    import golden_cases
+    cases = golden_cases.load()
+    assert len(cases) >= 8
+    for c in cases:
+        res = oracle.verify(c["target"], c["draft"], c["tokens"], dtype=F32,
+                            verify_len=c["verify_len"], temperature=c["temperature"],
+                            u_override=c["u"])
+        assert res["status"][0] == 0, c["name"]
+        assert res["accepted"][0] == c["n"], c["name"]
+        assert res["tokens"][0].tolist() == c["out_tokens"].tolist(), c["name"]
