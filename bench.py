@@ -12,7 +12,7 @@ per second (sum of L_i over the batch / step time), plus the HBM bandwidth
 the step sustains.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload headline|stochastic|greedy|conf|sweep:B]
+                  [--workload headline|stochastic|greedy|conf|conf_budget|sweep:B]
 
 With N > 1 (launched by torch.distributed.run) every rank verifies its own
 batch of the same shape (weak scaling, no collective on the data path); the
@@ -66,6 +66,8 @@ def make_workload(name, device, rank):
         w = W.greedy(device, seed=2)
     elif name == "conf":
         w = W.confidence(device, seed=3)
+    elif name == "conf_budget":
+        w = W.confidence_batch_budget(device, seed=3)
     elif name.startswith("sweep:"):
         w = W.sweep(device, seed=4, B=int(name.split(":")[1]))
     else:
@@ -73,11 +75,17 @@ def make_workload(name, device, rank):
     return w
 
 
-def effective_lengths(w):
-    """L_i after clamping (and after the confidence budget, if any), on the host."""
+def effective_lengths(w, ver=None):
+    """L_i after clamping and, with a confidence head, after its budgets: the
+    lengths the run verifies (computed by the library when a verifier is
+    given, else from verify_len alone)."""
     import torch
     B, kp1, _ = w["target"].shape
     k = kp1 - 1
+    if w.get("conf") is not None and ver is not None:
+        L, _ = ver.lengths(w["conf"], k, verify_len=w.get("verify_len"))
+        torch.cuda.synchronize()
+        return L
     L = (w["verify_len"].clamp(0, k) if w.get("verify_len") is not None
          else torch.full((B,), k, dtype=torch.int32, device=w["target"].device))
     return L
@@ -297,10 +305,10 @@ def run_ours(args):
     w = make_workload(args.workload, dev, rank)
     B, kp1, V = w["target"].shape
     k = kp1 - 1
-    L = effective_lengths(w)
+    ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V, mode=args.mode)
+    L = effective_lengths(w, ver)
     positions = int(L.sum().item())
     step_bytes = dense_row_bytes(w, L)
-    ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V, mode=args.mode)
     out = ver._outputs(B, k, True)
     stream = torch.cuda.current_stream(dev)
 
@@ -317,7 +325,7 @@ def run_ours(args):
     clocks = ClockSampler(phys)
     clocks.start()
     time.sleep(0.2)
-    ver.timing_enable([binding.TIMING_STATS])
+    ver.timing_enable([binding.TIMING_STATS, binding.TIMING_CONF])
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -334,6 +342,7 @@ def run_ours(args):
         dist.barrier()
     ms_local = e0.elapsed_time(e1)
     n_stats, ms_stats = ver.timing_read(binding.TIMING_STATS)
+    n_conf, ms_conf = ver.timing_read(binding.TIMING_CONF)
     ver.timing_enable([])
     clk = clocks.stop()
     counters = ver.last_counters()
@@ -440,6 +449,7 @@ def run_ours(args):
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
         "fp64_paths": counters,
+        "conf_launch_ms": (ms_conf / n_conf) if n_conf else None,
         "mode": args.mode,
         "other_mode": other_line,
     }

@@ -234,9 +234,11 @@ spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launch
 /* Diagnostics of the last completed run (synchronises the stream first):
  * out[0] = accept decisions settled by the fp64 path, out[1] = samples refined
  * in fp64, out[2] = samples certified by the fp32 filter, out[3] = chunks the
- * fp64 refinement recomputed outright. */
+ * fp64 refinement recomputed outright, out[4] = engine error bits (0 on a good
+ * run; 1 a wait for work timed out, 2 the work queue overflowed -- the run's
+ * outputs are then not to be used). */
 spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
-                                      uint32_t out[4]);
+                                      uint32_t out[5]);
 
 /* Self-check of the one hardware constant the fp32 filter relies on: the
  * maximum relative error of the ex2.approx.ftz.f32 instruction against fp64

@@ -347,10 +347,11 @@ class SpecVerifier:
         return n.value, ms.value
 
     def last_counters(self, stream=None):
-        out = (_u32 * 4)()
+        out = (_u32 * 5)()
         _check(lib().spec_verify_last_counters(self._h, _stream_handle(stream, self.device), out),
                "spec_verify_last_counters")
-        return dict(accept_fp64=out[0], sample_fp64=out[1], sample_fp32=out[2], chunks_fp64=out[3])
+        return dict(accept_fp64=out[0], sample_fp64=out[1], sample_fp32=out[2], chunks_fp64=out[3],
+                    engine_error=out[4])
 
 
 def greedy_noalloc(target, tokens, verify_len=None, stream=None, out=None):

@@ -83,6 +83,21 @@ struct Job {
   double rho_hi;
 };
 
+static_assert(sizeof(Job) % 8 == 0 && alignof(Job) == 8, "Job is read as 64-bit words");
+
+// A job is written by the CTA that decides and read by others after they
+// acquired the queue slot that announced it.  Jobs of neighbouring requests
+// share cache lines, so a plain (L1-cached) load could return a line this SM
+// cached earlier for a neighbour; read from L2 instead.
+__device__ __forceinline__ Job load_job(const Job* src) {
+  Job j;
+  const unsigned long long* s = reinterpret_cast<const unsigned long long*>(src);
+  unsigned long long* d = reinterpret_cast<unsigned long long*>(&j);
+#pragma unroll
+  for (int q = 0; q < static_cast<int>(sizeof(Job) / 8); ++q) d[q] = __ldcg(s + q);
+  return j;
+}
+
 struct SampleChunk {
   double mass;   // sum of fp32 weights over the chunk (fp64 accumulation of pairwise groups)
   double bound;  // certified bound on |mass - exact mass|
@@ -93,15 +108,14 @@ struct Counters {
   unsigned accept_slow;    // accept decisions resolved in fp64
   unsigned sample_fast;    // samples certified by the fp32 filter
   unsigned chunks_redone;  // refinement chunks recomputed outright (support unsettled)
-  unsigned queue_error;    // engine: 1 a wait gave up, 2 the queue overflowed
+  unsigned queue_error;    // engine: 1 a wait for work gave up, 2 the queue overflowed
   unsigned pad[3];
 };
 
 // Engine: orders of the statistics pass, and the queue's control words.
 constexpr int kModeDense = 0;
 constexpr int kModePrefix = 1;
-constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQInit = 4, kQWords = 8;
-constexpr int kEngineMinBlocks = 3;
+constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQWords = 8;
 
 // -------------------------------------------------------------- run params --
 struct RunParams {
@@ -187,6 +201,23 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Barrier over the kThreads threads of a CTA (named barrier 1, so that code
+// shared by several kernels never depends on which barrier the caller uses).
+__device__ __forceinline__ void sync_compute() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory");
+}
+// The same barrier, returning whether any compute thread passed x != 0.
+__device__ __forceinline__ int sync_compute_or(int x) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.s32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, 1, %2, pi;\n\tselp.s32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(x), "n"(kThreads)
+      : "memory");
+  return r;
+}
+
 // Packed fp32 pairs (sm_100): two independent round-to-nearest operations per
 // instruction, each rounded exactly as its scalar counterpart.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
@@ -196,6 +227,14 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
       : "l"(reinterpret_cast<const unsigned long long&>(a)),
         "l"(reinterpret_cast<const unsigned long long&>(b)),
         "l"(reinterpret_cast<const unsigned long long&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<unsigned long long&>(d))
+      : "l"(reinterpret_cast<const unsigned long long&>(a)),
+        "l"(reinterpret_cast<const unsigned long long&>(b)));
   return d;
 }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
@@ -390,9 +429,9 @@ __device__ __forceinline__ int warp_min_i(int x) {
 __device__ __forceinline__ float block_max_nan(float x, float* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   x = warp_max_nan(x);
-  __syncthreads();
+  sync_compute();
   if (lane == 0) sh[warp] = x;
-  __syncthreads();
+  sync_compute();
   float y = lane < kWarps ? sh[lane] : -INFINITY;
   return warp_max_nan(y);
 }
@@ -400,9 +439,9 @@ __device__ __forceinline__ float block_max_nan(float x, float* sh) {
 __device__ __forceinline__ double block_sum_d(double x, double* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   x = warp_sum_d(x);
-  __syncthreads();
+  sync_compute();
   if (lane == 0) sh[warp] = x;
-  __syncthreads();
+  sync_compute();
   double y = lane < kWarps ? sh[lane] : 0.0;
   return warp_sum_d(y);
 }
@@ -410,9 +449,9 @@ __device__ __forceinline__ double block_sum_d(double x, double* sh) {
 __device__ __forceinline__ float block_sum_f(float x, float* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   x = warp_sum_f(x);
-  __syncthreads();
+  sync_compute();
   if (lane == 0) sh[warp] = x;
-  __syncthreads();
+  sync_compute();
   float y = lane < kWarps ? sh[lane] : 0.0f;
   return warp_sum_f(y);
 }
@@ -420,9 +459,9 @@ __device__ __forceinline__ float block_sum_f(float x, float* sh) {
 __device__ __forceinline__ int block_min_i(int x, int* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   x = warp_min_i(x);
-  __syncthreads();
+  sync_compute();
   if (lane == 0) sh[warp] = x;
-  __syncthreads();
+  sync_compute();
   int y = lane < kWarps ? sh[lane] : INT_MAX;
   return warp_min_i(y);
 }
@@ -437,9 +476,9 @@ __device__ __forceinline__ double block_exclusive_scan_d(double x, double* sh, d
     const double y = __shfl_up_sync(0xffffffffu, incl, off);
     if (lane >= off) incl += y;
   }
-  __syncthreads();
+  sync_compute();
   if (lane == 31) sh[warp] = incl;
-  __syncthreads();
+  sync_compute();
   double warp_base = 0.0, all = 0.0;
   for (int w = 0; w < kWarps; ++w) {
     const double s = sh[w];
@@ -468,7 +507,7 @@ __device__ __forceinline__ double chunk_prefix(const double (&v)[4], double (&pr
 // of `expected` arrivals, and resets the counter for the next launch.  Writes
 // this CTA made before the call are visible to the last arriver afterwards.
 __device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* sh_flag) {
-  __syncthreads();
+  sync_compute();
   if (threadIdx.x == 0) {
     __threadfence();
     const unsigned old = atomicAdd(counter, 1u);
@@ -479,7 +518,7 @@ __device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected
     }
     *sh_flag = last ? 1 : 0;
   }
-  __syncthreads();
+  sync_compute();
   return *sh_flag != 0;
 }
 

@@ -20,11 +20,10 @@
 //   prefix : a request's position j+1 rows are read only after position j was
 //            accepted.  The outputs are identical; prefix reads fewer bytes.
 //
-// The initial items are implicit: the rows of position 0 (prefix) or of every
-// position (dense), decoded from a ticket number 0 .. n_init-1.  Items generated
-// during the run go to the queue, whose slots carry the run's epoch in their
-// upper 32 bits so a slot left by an earlier run is never taken for a new item;
-// they are served before the remaining initial items.  A CTA waiting
+// The first tickets (0 .. n_init-1) are implicit: the rows of position 0 (prefix)
+// or of every position (dense), decoded from the ticket number.  Later tickets
+// index the queue, whose slots carry the run's epoch in their upper 32 bits so
+// a slot left by an earlier run is never taken for a new item.  A CTA waiting
 // for a slot sleeps between polls and gives up after a bounded time (setting
 // the queue error), as does the whole kernel once every request is finished.
 // The last CTA to leave resets the queue counters for the next run.
@@ -38,7 +37,10 @@ namespace sv {
 
 constexpr uint32_t kItemStats = 0u, kItemSample = 1u, kItemRefine = 2u;
 constexpr uint32_t kItemExit = 0xFFFFFFFFu;
-constexpr unsigned kSpinLimit = 1u << 24;  // ~ seconds of polling at the sleep below
+constexpr unsigned kSpinLimit = 1u << 24;
+constexpr int kEngineMinBlocks = 3;
+constexpr int kEngineThreads = kThreads;
+constexpr size_t kEngineDynSmem = 0;  // ~ seconds of polling at the sleep below
 
 __device__ __forceinline__ uint32_t item_stats(int i, int slot, int seg) {
   return (kItemStats << 30) | (static_cast<uint32_t>(i) << 14) |
@@ -84,50 +86,22 @@ __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h
   return item_stats(static_cast<int>(i), slot, static_cast<int>(r % p.n_segs));
 }
 
-__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* a) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
-  return v;
-}
-
-// Thread 0: wait for queue slot g (a ticket already taken) and return its item,
-// or kItemExit once every request is finished (or the wait limit is reached).
-__device__ uint32_t wait_slot(const RunParams& p, unsigned g) {
-  if (g >= p.q_capacity) {
-    atomicOr(&p.counters->queue_error, 2u);
-    return kItemExit;
-  }
+// Thread 0: the next item (or kItemExit).
+__device__ uint32_t fetch_item(const RunParams& p) {
+  const unsigned h = atomicAdd(p.q_ctl + kQHead, 1u);
+  if (h < p.n_init) return implicit_item(p, h);
+  const unsigned d = h - p.n_init;
   for (unsigned spin = 0;; ++spin) {
-    const unsigned long long v = ld_acquire_u64(p.q_slots + g);
-    if (static_cast<unsigned>(v >> 32) == p.q_epoch) return static_cast<uint32_t>(v);
-    if ((spin & 7u) == 7u && ld_relaxed_u32(p.q_ctl + kQDone) >= static_cast<unsigned>(p.B))
-      return kItemExit;
+    if (d < p.q_capacity) {
+      const unsigned long long v = ld_acquire_u64(p.q_slots + d);
+      if (static_cast<unsigned>(v >> 32) == p.q_epoch) return static_cast<uint32_t>(v);
+    }
+    if (ld_acquire_u32(p.q_ctl + kQDone) >= static_cast<unsigned>(p.B)) return kItemExit;
     if (spin >= kSpinLimit) {
       atomicOr(&p.counters->queue_error, 1u);
       return kItemExit;
     }
-    __nanosleep(spin < 16 ? 32 : 256);
-  }
-}
-
-// Thread 0: the next item (or kItemExit).  Two ticket counters, both taken
-// with a plain atomicAdd: one over the implicit initial items, one over the
-// queue of items generated during the run.  A CTA takes a queue ticket when
-// the queue looks non-empty (head < tail) or the initial items are all taken,
-// so generated items -- the next position of a chain, a sample whose rows are
-// still in L2, a refinement -- are served ahead of the remaining initial
-// items.  A queue ticket may be taken just before its slot is written; the
-// CTA then waits on that slot alone, so no control word is polled by many
-// CTAs at once.
-__device__ uint32_t fetch_item(const RunParams& p, bool& init_done) {
-  for (;;) {
-    if (init_done ||
-        ld_relaxed_u32(p.q_ctl + kQHead) < ld_relaxed_u32(p.q_ctl + kQTail)) {
-      return wait_slot(p, atomicAdd(p.q_ctl + kQHead, 1u));
-    }
-    const unsigned g = atomicAdd(p.q_ctl + kQInit, 1u);
-    if (g < p.n_init) return implicit_item(p, g);
-    init_done = true;
+    __nanosleep(spin < 32 ? 64 : 512);
   }
 }
 
@@ -192,7 +166,7 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
   if (p.mode == kModeDense) {
     decide_request<BF16>(p, i, ri, dec);
     __syncthreads();
-    if (p.jobs[i].kind != kJobNone) enqueue_sample<BF16>(p, i, s_base);
+    if (__ldcg(&p.jobs[i].kind) != kJobNone) enqueue_sample<BF16>(p, i, s_base);
     else finish_request(p);
     return;
   }
@@ -215,7 +189,7 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
 template <bool BF16>
 __device__ void engine_sample(const RunParams& p, int i, int seg, SampleShared& sa,
                               unsigned* s_base) {
-  const Job jb = p.jobs[i];
+  const Job jb = load_job(p.jobs + i);
   segment_masses<BF16>(p, i, jb, seg, sa);
   if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_segs), &sa.flag)) return;
   __threadfence();
@@ -231,7 +205,9 @@ __device__ void engine_sample(const RunParams& p, int i, int seg, SampleShared& 
 
 template <bool BF16>
 __device__ void engine_refine(const RunParams& p, int slot, int sub, RefineShared& rf) {
-  if (!refine_item<BF16>(p, slot, sub, rf)) return;
+  refine_item<BF16>(p, slot, sub, rf);
+  if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(p.n_chunks * kSubsPerChunk), &rf.flag)) return;
+  __threadfence();
   refine_finalize<BF16>(p, slot, rf);
   finish_request(p);
 }
@@ -245,10 +221,9 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
   __shared__ uint32_t s_item;
   __shared__ unsigned s_base;
   exp2_table_init(rf.tab);
-  bool init_done = false;  // thread 0's view: every initial item is taken
 #pragma unroll 1
   for (;;) {
-    if (threadIdx.x == 0) s_item = fetch_item(p, init_done);
+    if (threadIdx.x == 0) s_item = fetch_item(p);
     __syncthreads();
     const uint32_t it = s_item;
     if (it == kItemExit) break;
@@ -268,7 +243,6 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
     if (atomicAdd(p.q_ctl + kQExits, 1u) == gridDim.x - 1) {
       p.q_ctl[kQHead] = 0u;
       p.q_ctl[kQTail] = 0u;
-      p.q_ctl[kQInit] = 0u;
       p.q_ctl[kQDone] = 0u;
       p.q_ctl[kQExits] = 0u;
       *p.counters_next = Counters{};

@@ -10,6 +10,7 @@
 // it with exp2() over the whole argument range.
 #pragma once
 #include <cuda_runtime.h>
+#include "common.cuh"
 
 namespace sv {
 
@@ -17,10 +18,11 @@ constexpr int kExp2Table = 32;
 constexpr double kLog2E = 1.4426950408889634074;
 constexpr double kLn2d = 0.69314718055994530942;
 
-// Every thread of the CTA must call this before the first exp2_fast.
+// Every compute thread (warps 0 .. kWarps-1) must call this before the first
+// exp2_fast.
 __device__ __forceinline__ void exp2_table_init(double* tab) {
-  for (int j = threadIdx.x; j < kExp2Table; j += blockDim.x) tab[j] = exp2(j / 32.0);
-  __syncthreads();
+  for (int j = threadIdx.x; j < kExp2Table; j += kThreads) tab[j] = exp2(j / 32.0);
+  sync_compute();
 }
 
 __device__ __forceinline__ double exp2_fast(double x, const double* tab) {

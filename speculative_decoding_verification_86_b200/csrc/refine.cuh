@@ -116,7 +116,7 @@ __device__ double exact_sub_mass(const RunParams& p, int i, const Job& jb, const
 #pragma unroll
     for (int q = 0; q < G::kPerVec; ++q) m += exact_weight<BF16>(xa[q], xb[q], true, rr, iza, izb, sh.tab);
   }
-  __syncthreads();
+  sync_compute();
   return block_sum_d(m, sh.d);
 }
 
@@ -142,10 +142,10 @@ __device__ __forceinline__ int load_sub_contiguous(const void* row, int64_t V, i
 // One fp64 work item: sub-chunk `sub` of refinement slot `slot`.  Returns true
 // in the CTA that completes the slot (all its sub-chunks are in).
 template <bool BF16>
-__device__ bool refine_item(const RunParams& p, int slot, int sub, RefineShared& sh) {
+__device__ void refine_item(const RunParams& p, int slot, int sub, RefineShared& sh) {
   const int n_subs = p.n_chunks * kSubsPerChunk;
   const int i = __ldcg(p.refine_list + slot);
-  const Job jb = p.jobs[i];
+  const Job jb = load_job(p.jobs + i);
   const RefineRow rr = refine_row(jb);
   const bool residual = jb.kind == kJobResidual;
   double za = 0.0, zb = 0.0, A = 0.0, Bm = 0.0;
@@ -156,16 +156,13 @@ __device__ bool refine_item(const RunParams& p, int slot, int sub, RefineShared&
   zb = block_sum_d(zb, sh.d);
   A = block_sum_d(A, sh.d);
   Bm = block_sum_d(Bm, sh.d);
-  unc = __syncthreads_or(unc);
+  unc = sync_compute_or(unc);
   const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
   if (threadIdx.x == 0) {
     p.rz[rec0 + sub] = make_double2(za, zb);
     p.rm[rec0 + sub] = make_double2(A, Bm);
     p.runc[rec0 + sub] = unc;
   }
-  if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(n_subs), &sh.flag)) return false;
-  __threadfence();
-  return true;
 }
 
 // The last CTA of refinement slot `slot`: exact sub-chunk masses, the token.
@@ -174,7 +171,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
   using G = Geo<BF16>;
   const int n_subs = p.n_chunks * kSubsPerChunk;
   const int i = __ldcg(p.refine_list + slot);
-  const Job jb = p.jobs[i];
+  const Job jb = load_job(p.jobs + i);
   const RefineRow rr = refine_row(jb);
   const bool residual = jb.kind == kJobResidual;
   const int64_t rec0 = static_cast<int64_t>(slot) * n_subs;
@@ -210,19 +207,19 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     }
   }
   // sub-chunks whose support was not settled: recompute outright (rare)
-  if (__syncthreads_or(flagged)) {
+  if (sync_compute_or(flagged)) {
 #pragma unroll 1
     for (int ss = 0; ss < n_subs; ++ss) {
       const int owner = ss / 4;
       if (threadIdx.x == owner) sh.found = (flagged >> (ss % 4)) & 1;
-      __syncthreads();
+      sync_compute();
       if (sh.found) {
         if (threadIdx.x == 0) atomicAdd(&p.counters->chunks_redone, 1u);
         const double m = exact_sub_mass<BF16>(p, i, jb, rr, ss / kSubsPerChunk,
                                               ss % kSubsPerChunk, iza, izb, sh);
         if (threadIdx.x == owner) mv[ss % 4] = m;
       }
-      __syncthreads();
+      sync_compute();
     }
   }
   double pm[4];
@@ -239,7 +236,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     sh.cstar = -1;
     sh.found = -1;
   }
-  __syncthreads();
+  sync_compute();
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int ss = 4 * threadIdx.x + q;
@@ -248,7 +245,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
       sh.base = pm[q];
     }
   }
-  __syncthreads();
+  sync_compute();
   bool fallback = false;
   if (sh.cstar < 0) {
     // rounding left no cell above target: the last sub-chunk with positive weight
@@ -260,7 +257,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     }
     last = -block_min_i(last >= 0 ? -last : 1, sh.i);
     if (threadIdx.x == 0) sh.cstar = last >= 0 ? last : -1;
-    __syncthreads();
+    sync_compute();
     fallback = true;
   }
   const int sstar = sh.cstar;
@@ -302,7 +299,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
           if (run > target && sh.found < 0) sh.found = off + e;
         }
       }
-      __syncthreads();
+      sync_compute();
       found = sh.found;
     }
     if (found < 0) {
@@ -321,7 +318,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
       if (p.out_status) p.out_status[i] |= kDevInternal;
     }
   }
-  __syncthreads();
+  sync_compute();
 }
 
 }  // namespace sv

@@ -101,39 +101,99 @@ __device__ __forceinline__ WeightCtx weight_ctx(const JobF32& j, float ma, float
   return w;
 }
 
+// The weights and bounds of two logit pairs at once with packed fp32x2
+// instructions.  Every weight is bit-identical to weight_and_bound's: the
+// exponent argument is formed negated (F - x c, the same rounding), the draft
+// term is carried negated (-q~), so p~ - q~ is one packed add.  The bound uses
+// the same terms; its "near" test is taken on the exact value of
+// 1.0001 p~ - q~, an equally valid criterion.
+struct WeightCtx2 {
+  float2 ncc, Fa, Fb, Aeff, nBeff, kappa, nkappa, epsa, nepsb;
+  bool residual;
+};
+
+__device__ __forceinline__ WeightCtx2 pack_ctx(const WeightCtx& w) {
+  WeightCtx2 v;
+  v.ncc = make_float2(-w.cc, -w.cc);
+  v.Fa = make_float2(w.Fa, w.Fa);
+  v.Fb = make_float2(w.Fb, w.Fb);
+  v.Aeff = make_float2(w.Aeff, w.Aeff);
+  v.nBeff = make_float2(-w.Beff, -w.Beff);
+  v.kappa = make_float2(w.kappa, w.kappa);
+  v.nkappa = make_float2(-w.kappa, -w.kappa);
+  v.epsa = make_float2(w.epsa, w.epsa);
+  v.nepsb = make_float2(-w.epsb, -w.epsb);
+  v.residual = w.residual;
+  return v;
+}
+
+__device__ __forceinline__ void weight_and_bound2(const WeightCtx2& w, float2 a, float2 b,
+                                                  float2& wt, float2& bd) {
+  float2 na = ffma2(a, w.ncc, w.Fa);  // -(a c - Fa)
+  na.x = fminf(na.x, 1024.0f);
+  na.y = fminf(na.y, 1024.0f);
+  const float2 pa = fmul2(make_float2(ex2_approx(-na.x), ex2_approx(-na.y)), w.Aeff);
+  const float2 ta = ffma2(w.kappa, na, w.epsa);  // epsa + kappa |xa|
+  if (!w.residual) {
+    wt = pa;
+    bd = fmul2(pa, ta);
+    return;
+  }
+  float2 nb = ffma2(b, w.ncc, w.Fb);
+  nb.x = fminf(nb.x, 1024.0f);
+  nb.y = fminf(nb.y, 1024.0f);
+  const float2 nqb = fmul2(make_float2(ex2_approx(-nb.x), ex2_approx(-nb.y)), w.nBeff);  // -q~
+  const float2 diff = fadd2(pa, nqb);
+  wt = make_float2(fmaxf(diff.x, 0.0f), fmaxf(diff.y, 0.0f));
+  const float2 near = ffma2(pa, make_float2(1.0001f, 1.0001f), nqb);
+  const float2 ntb = ffma2(w.nkappa, nb, w.nepsb);  // -(epsb + kappa |xb|)
+  const float2 full = ffma2(pa, ta, fmul2(nqb, ntb));
+  bd = make_float2(near.x >= 0.0f ? full.x : 0.0f, near.y >= 0.0f ? full.y : 0.0f);
+}
+
 // Weights of one batch (kBatchElems logits per thread), reduced two ways:
 // `sum` is their pairwise fp32 sum (the mass pass), `exact` the fp64 sum of the
 // same fp32 weights (the rescans); `bound` sums their error bounds in fp32.
+// The pairwise tree has depth log2(kBatchElems) = Geo::kSumLevels.
 template <bool BF16, bool EXACT>
 __device__ __forceinline__ void batch_weights(const JobF32& j, const uint4 (&va)[kVecsPerBatch],
                                               const uint4 (&vb)[kVecsPerBatch], float& sum,
                                               double& exact, float& bound) {
-  using G = Geo<BF16>;
-  const WeightCtx w = weight_ctx(j, vec_max<BF16>(va), j.residual ? vec_max<BF16>(vb) : 0.0f);
-  float vs[kVecsPerBatch];
-  float bd_sum = 0.0f;
+  constexpr int kPairs = BF16 ? 4 : 2;  // logit pairs per vector
+  const WeightCtx2 w = pack_ctx(weight_ctx(j, vec_max<BF16>(va), j.residual ? vec_max<BF16>(vb) : 0.0f));
+  float2 bd_sum = make_float2(0.0f, 0.0f);
+  float2 vs[kVecsPerBatch];
   double ex = 0.0;
 #pragma unroll
   for (int u = 0; u < kVecsPerBatch; ++u) {
-    float xa[G::kPerVec], xb[G::kPerVec], wt[G::kPerVec];
-    unpack<BF16>(va[u], xa);
-    if (j.residual) unpack<BF16>(vb[u], xb);
+    const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
+    const uint32_t wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+    float2 wt[kPairs];
 #pragma unroll
-    for (int q = 0; q < G::kPerVec; ++q) {
-      float bd;
-      weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt[q], bd);
-      bd_sum += bd;
-      if (EXACT) ex += static_cast<double>(wt[q]);
+    for (int q = 0; q < kPairs; ++q) {
+      float2 xa, xb;
+      if constexpr (BF16) {
+        xa = make_float2(bf16_lo(wa[q]), bf16_hi(wa[q]));
+        xb = make_float2(bf16_lo(wb[q]), bf16_hi(wb[q]));
+      } else {
+        xa = make_float2(__uint_as_float(wa[2 * q]), __uint_as_float(wa[2 * q + 1]));
+        xb = make_float2(__uint_as_float(wb[2 * q]), __uint_as_float(wb[2 * q + 1]));
+      }
+      float2 bd;
+      weight_and_bound2(w, xa, xb, wt[q], bd);
+      bd_sum = fadd2(bd_sum, bd);
+      if (EXACT) ex += static_cast<double>(wt[q].x) + static_cast<double>(wt[q].y);
     }
     if constexpr (BF16) {
-      vs[u] = ((wt[0] + wt[1]) + (wt[2] + wt[3])) + ((wt[4] + wt[5]) + (wt[6] + wt[7]));
+      vs[u] = fadd2(fadd2(wt[0], wt[1]), fadd2(wt[2], wt[3]));
     } else {
-      vs[u] = (wt[0] + wt[1]) + (wt[2] + wt[3]);
+      vs[u] = fadd2(wt[0], wt[1]);
     }
   }
-  sum = vs[0] + vs[1];
+  const float2 t = fadd2(vs[0], vs[1]);
+  sum = t.x + t.y;
   exact = ex;
-  bound = bd_sum;
+  bound = bd_sum.x + bd_sum.y;
 }
 
 constexpr int kChunksPerSeg = SegGeo<true>::kSegVecs / Geo<true>::kChunkVecs;  // 2
@@ -196,7 +256,7 @@ __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const 
       if (j.residual) vb[u] = nb[u];
     }
   }
-  __syncthreads();
+  sync_compute();
   if (threadIdx.x < kChunksPerSeg) {
     const int b = threadIdx.x;
     const int c = c0 + b;
@@ -238,7 +298,7 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
   }
   if (tid == 0) sh.cstar = -1;
   const double total = chunk_prefix(m, pm, sh.d);
-  __syncthreads();
+  sync_compute();
   const double tb = chunk_prefix(b, pb, sh.d) + 1e-15 * total;
   const double target = jb.u2 * total;
 #pragma unroll
@@ -250,7 +310,7 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
       sh.base_bound = pb[q] + 1e-15 * pm[q];
     }
   }
-  __syncthreads();
+  sync_compute();
   int cstar = sh.cstar;
   // residual mass must clear the 1e-12 floor with certainty
   if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) cstar = -1;
@@ -277,11 +337,11 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
     }
     double all, allb;
     const double pre = block_exclusive_scan_d(tsum, sh.d, all);
-    __syncthreads();
+    sync_compute();
     const double preb = block_exclusive_scan_d(tbound, sh.d, allb);
     const double start = sh.base + pre;
     if (tid == 0) sh.found = -1;
-    __syncthreads();
+    sync_compute();
     if (start <= target && start + tsum > target) {
       // the one thread holding the crossing walks its logits again (same values)
       double run = start, runb = sh.base_bound + preb * 1.001;
@@ -314,7 +374,7 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
         }
       }
     }
-    __syncthreads();
+    sync_compute();
     if (tid == 0 && sh.found >= 0) {
       const double slack = jb.u2 * tb + 1e-14 * total;
       const double need = sh.cell_bound + slack;
@@ -333,7 +393,7 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
       sh.refine_slot = static_cast<int>(slot);
     }
   }
-  __syncthreads();
+  sync_compute();
 }
 
 }  // namespace sv

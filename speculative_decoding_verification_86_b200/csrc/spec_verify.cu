@@ -728,7 +728,7 @@ spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launch
   return SPEC_OK;
 }
 
-spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream, uint32_t out[4]) {
+spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream, uint32_t out[5]) {
   if (!ctx || !out) return SPEC_ERR_INVALID_ARG;
   DeviceGuard g(ctx->device);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SPEC_ERR_CUDA;
@@ -740,6 +740,7 @@ spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
   out[1] = h.refine_count;
   out[2] = h.sample_fast;
   out[3] = h.chunks_redone;
+  out[4] = h.queue_error;
   return SPEC_OK;
 }
 

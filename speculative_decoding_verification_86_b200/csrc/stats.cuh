@@ -219,7 +219,7 @@ __device__ __forceinline__ void soft_merge_block(SoftAcc acc, StatsShared& sh, C
         sh.mraw[warp] = mraw;
         sh.bad[warp] = bad;
       }
-      __syncthreads();
+      sync_compute();
       if (warp != 0) return;
       const bool have = lane < kWarps;
       acc.K = have ? sh.K[lane] : -INFINITY;
@@ -266,19 +266,18 @@ __device__ __forceinline__ void stochastic_segment(const void* row, int64_t V, i
   soft_merge_block(acc, sh, meta_out, sum_out);
 }
 
-// Max and lowest arg-max of one segment of a greedy row.
+// Max and lowest arg-max of one segment of a greedy row: each thread keeps its
+// running maximum and the lowest index attaining it (batches arrive in index
+// order per thread), then the CTA reduces (larger value wins, ties go to the
+// lower index).
 template <bool BF16>
-__device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int seg,
-                                               ChunkMeta* meta_out, StatsShared& sh) {
-  using G = SegGeo<BF16>;
-  const uint4* rv = static_cast<const uint4*>(row);
-  const int64_t nvec = V / G::kPerVec;
-  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+struct GreedyScan {
   float best = -INFINITY;
   int64_t best_idx = INT64_MAX;
   int bad = 0;
-  uint4 va[kBatchVecs], vb[kBatchVecs];
-  auto scan = [&](const uint4 (&v)[kBatchVecs], int b) {
+
+  __device__ __forceinline__ void scan(const uint4 (&v)[kBatchVecs], int64_t seg0, int b) {
+    using G = SegGeo<BF16>;
     const float bm = batch_max<BF16>(v);
     if (isnan(bm)) bad = 1;
     if (!(bm > best) && best_idx != INT64_MAX) return;  // earlier batches hold lower indices
@@ -298,49 +297,63 @@ __device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int s
     }
     best = bm;
     best_idx = first;
-  };
+  }
+
+  __device__ __forceinline__ void finish(ChunkMeta* meta_out, StatsShared& sh) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int idx = best_idx == INT64_MAX ? INT_MAX : static_cast<int>(best_idx);
+    for (int level = 0; level < 2; ++level) {
+#pragma unroll
+      for (int off = 16; off; off >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
+        if (ob > best || (ob == best && oi < idx)) {
+          best = ob;
+          idx = oi;
+        }
+      }
+      bad = __any_sync(0xffffffffu, bad);
+      if (level == 0) {
+        if (lane == 0) {
+          sh.mraw[warp] = best;
+          sh.arg[warp] = idx;
+          sh.bad[warp] = bad;
+        }
+        sync_compute();
+        if (warp != 0) return;
+        best = lane < kWarps ? sh.mraw[lane] : -INFINITY;
+        idx = lane < kWarps ? sh.arg[lane] : INT_MAX;
+        bad = lane < kWarps ? sh.bad[lane] : 0;
+      } else if (lane == 0) {
+        ChunkMeta r;
+        r.K = 0.0f;
+        r.mraw = bad ? __int_as_float(0x7fc00000) : best;
+        r.err = 0.0f;
+        r.arg = idx == INT_MAX ? -1 : idx;
+        *meta_out = r;
+      }
+    }
+  }
+};
+
+template <bool BF16>
+__device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int seg,
+                                               ChunkMeta* meta_out, StatsShared& sh) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  GreedyScan<BF16> g;
+  uint4 va[kBatchVecs], vb[kBatchVecs];
   load_batch<BF16>(rv, nvec, seg0, 0, va);
 #pragma unroll
   for (int b = 0; b < kBatches; b += 2) {
     if (b + 1 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 1, vb);
-    scan(va, b);
+    g.scan(va, seg0, b);
     if (b + 2 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 2, va);
-    if (b + 1 < kBatches) scan(vb, b + 1);
+    if (b + 1 < kBatches) g.scan(vb, seg0, b + 1);
   }
-  // block reduction: larger value wins, ties go to the lower index
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int idx = best_idx == INT64_MAX ? INT_MAX : static_cast<int>(best_idx);
-  for (int level = 0; level < 2; ++level) {
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, idx, off);
-      if (ob > best || (ob == best && oi < idx)) {
-        best = ob;
-        idx = oi;
-      }
-    }
-    bad = __any_sync(0xffffffffu, bad);
-    if (level == 0) {
-      if (lane == 0) {
-        sh.mraw[warp] = best;
-        sh.arg[warp] = idx;
-        sh.bad[warp] = bad;
-      }
-      __syncthreads();
-      if (warp != 0) return;
-      best = lane < kWarps ? sh.mraw[lane] : -INFINITY;
-      idx = lane < kWarps ? sh.arg[lane] : INT_MAX;
-      bad = lane < kWarps ? sh.bad[lane] : 0;
-    } else if (lane == 0) {
-      ChunkMeta r;
-      r.K = 0.0f;
-      r.mraw = bad ? __int_as_float(0x7fc00000) : best;
-      r.err = 0.0f;
-      r.arg = idx == INT_MAX ? -1 : idx;
-      *meta_out = r;
-    }
-  }
+  g.finish(meta_out, sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -537,7 +550,7 @@ __device__ void accept_exact(const RunParams& p, int i, int j, int xj, const Row
   const double ma = static_cast<double>(ra.mraw) / t.T;
   const double mb = static_cast<double>(rb.mraw) / t.T;
   const double Za = exact_row_sum(target_row(p, i, j, BF16), p.V, BF16, t.T, ma, red);
-  __syncthreads();
+  sync_compute();
   const double Zb = exact_row_sum(draft_row(p, i, j, BF16), p.V, BF16, t.T, mb, red);
   if (threadIdx.x == 0) {
     const double la = load_logit(target_row(p, i, j, BF16), xj, BF16);
@@ -641,7 +654,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
 
   write_defaults(p, i);
   if (ri.bad_T) {
-    __syncthreads();
+    sync_compute();
     if (tid == 0) fail_request(p, i, kDevBadTemperature);
     return;
   }
@@ -653,7 +666,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     if (ri.greedy) merge_greedy_row(p, i, slot, sh.rows[slot]);
     else merge_stochastic_row(p, i, slot, sh.rows[slot]);
   }
-  __syncthreads();
+  sync_compute();
 
   if (ri.greedy) {
     if (tid == 0) {
@@ -717,7 +730,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
         }
       }
     }
-    __syncthreads();
+    sync_compute();
     if (sh.need_exact >= 0) {
       bool accept = false;
       double pa = 0.0, qb = 0.0;
@@ -734,10 +747,10 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
         }
         sh.need_exact = -1;
       }
-      __syncthreads();
+      sync_compute();
     }
     const int stop = sh.state;
-    __syncthreads();
+    sync_compute();
     if (stop) break;
   }
 
@@ -768,12 +781,12 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
   const int32_t* x = p.tokens + static_cast<int64_t>(i) * k;
   if (j == 0) write_defaults(p, i);
   if (ri.bad_T) {
-    __syncthreads();
+    sync_compute();
     if (tid == 0) {
       fail_request(p, i, kDevBadTemperature);
       sh.state = 0;
     }
-    __syncthreads();
+    sync_compute();
     return;
   }
   const bool pair = !ri.greedy && j < L;
@@ -783,7 +796,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
   } else if (warp == 1 && pair) {
     merge_stochastic_row(p, i, k + 1 + j, sh.rows[1]);
   }
-  __syncthreads();
+  sync_compute();
   const RowMerged& ra = sh.rows[0];
   const RowMerged& rb = sh.rows[1];
   const TempConsts t = temp_consts<BF16>(p, ri.T);
@@ -839,7 +852,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
     }
     if (status) fail_request(p, i, status);
   }
-  __syncthreads();
+  sync_compute();
   if (sh.need_exact > 0) {
     bool accept = false;
     double pa = 0.0, qb = 0.0;
@@ -859,7 +872,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
       }
     }
   }
-  __syncthreads();
+  sync_compute();
 }
 
 // ---------------------------------------------------------------------------

@@ -35,6 +35,7 @@ def run_gpu(ver, w, uniforms=None, **kw):
                 temperature=w.get("temperature"), conf=w.get("conf"), seed=w["seed"],
                 uniforms=uniforms, **kw)
     torch.cuda.synchronize()
+    assert ver.last_counters()["engine_error"] == 0
     return {k: v.cpu().numpy() for k, v in o.items()}
 
 
