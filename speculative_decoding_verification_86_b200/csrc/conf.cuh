@@ -26,51 +26,69 @@
 namespace sv {
 
 // Last CTA of k_conf: the batch-wide selection.  Reads the prefix products and
-// per-request limits every CTA published, writes out_len.
+// per-request limits every CTA published, writes out_len.  Batches of up to
+// kSelCache candidate slots are first copied to shared memory (one pass of
+// independent loads), so the eight radix passes and the final count run on
+// shared memory; larger batches stream the candidates from L2 in every pass.
+constexpr int kSelCache = 4096;
+constexpr unsigned long long kNoKey = ~0ull;  // not a candidate (valid keys are <= bits of 1.0)
+static_assert(kThreads == 256, "one radix bin per thread");
+
 __device__ void conf_select(const ConfParams& cp) {
+  __shared__ unsigned long long s_keys[kSelCache];
   __shared__ unsigned hist[256];
   __shared__ double sh_d[kWarps];
   __shared__ unsigned long long s_key;
   __shared__ long long s_rank;
   const int B = cp.B, kb = cp.kb;
   const long long n = static_cast<long long>(B) * kb;
-
+  const bool cached = n <= kSelCache;
+  auto load_key = [&](long long e) -> unsigned long long {
+    const int i = static_cast<int>(e / kb), j = static_cast<int>(e - static_cast<long long>(i) * kb);
+    if (j >= __ldcg(cp.cap + i)) return kNoKey;
+    return static_cast<unsigned long long>(__double_as_longlong(__ldcg(cp.prefix + e)));
+  };
+  if (cached) {
+    for (long long e = threadIdx.x; e < n; e += kThreads) s_keys[e] = load_key(e);
+  }
   double m_local = 0.0;
   for (int i = threadIdx.x; i < B; i += kThreads) m_local += __ldcg(cp.cap + i);
-  const long long M = static_cast<long long>(block_sum_d(m_local, sh_d));
+  const long long M = static_cast<long long>(block_sum_d(m_local, sh_d));  // (also a barrier)
   if (cp.total >= M) {
     for (int i = threadIdx.x; i < B; i += kThreads) cp.out_len[i] = __ldcg(cp.cap + i);
     return;
   }
+  auto key_at = [&](long long e) -> unsigned long long { return cached ? s_keys[e] : load_key(e); };
 
-  // t = the total-th largest candidate key (1-based rank from the top).
+  // t = the total-th largest candidate key (rank 1 = the largest).
   if (threadIdx.x == 0) {
     s_key = 0ull;
     s_rank = cp.total;
   }
   for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int d = threadIdx.x; d < 256; d += kThreads) hist[d] = 0u;
-    __syncthreads();
+    hist[threadIdx.x] = 0u;  // kThreads == 256 bins
+    sync_compute();
     const unsigned long long want = s_key;
+    const long long rank = s_rank;
     const unsigned long long hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
     for (long long e = threadIdx.x; e < n; e += kThreads) {
-      const int i = static_cast<int>(e / kb), j = static_cast<int>(e - static_cast<long long>(i) * kb);
-      if (j >= __ldcg(cp.cap + i)) continue;
-      const unsigned long long key = static_cast<unsigned long long>(__double_as_longlong(__ldcg(cp.prefix + e)));
-      if ((key & hi_mask) == want) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      const unsigned long long key = key_at(e);
+      if (key != kNoKey && (key & hi_mask) == want) atomicAdd(&hist[(key >> shift) & 255u], 1u);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      long long above = 0;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (above + hist[d] >= s_rank) break;
-        above += hist[d];
-      }
-      s_rank -= above;  // rank among the keys with this digit
-      s_key = want | (static_cast<unsigned long long>(d) << shift);
+    sync_compute();
+    // thread t looks after digit 255 - t: the keys above it are the exclusive
+    // prefix in that order; exactly one digit holds the rank
+    const int digit = 255 - static_cast<int>(threadIdx.x);
+    const unsigned c = hist[digit];
+    double tot;
+    const long long above =
+        static_cast<long long>(block_exclusive_scan_d(static_cast<double>(c), sh_d, tot));
+    sync_compute();  // every thread has read s_key and s_rank
+    if (c > 0 && above < rank && above + static_cast<long long>(c) >= rank) {
+      s_rank = rank - above;  // rank among the keys with this digit
+      s_key = want | (static_cast<unsigned long long>(digit) << shift);
     }
-    __syncthreads();
+    sync_compute();
   }
   const unsigned long long t = s_key;
   const long long take_eq = s_rank;  // how many candidates equal to t are kept
@@ -79,10 +97,9 @@ __device__ void conf_select(const ConfParams& cp) {
     const int i = base + threadIdx.x;
     int gt = 0, eq = 0;
     if (i < B) {
-      const int c = __ldcg(cp.cap + i);
-      for (int j = 0; j < c; ++j) {
-        const unsigned long long key =
-            static_cast<unsigned long long>(__double_as_longlong(__ldcg(cp.prefix + static_cast<long long>(i) * kb + j)));
+      for (int j = 0; j < kb; ++j) {
+        const unsigned long long key = key_at(static_cast<long long>(i) * kb + j);
+        if (key == kNoKey) break;  // candidates are a leading run of the request
         gt += key > t;
         eq += key == t;
       }
@@ -95,7 +112,7 @@ __device__ void conf_select(const ConfParams& cp) {
       cp.out_len[i] = gt + static_cast<int>(take);
     }
     carry += tot;
-    __syncthreads();
+    sync_compute();
   }
 }
 

@@ -38,7 +38,7 @@ namespace sv {
 constexpr uint32_t kItemStats = 0u, kItemSample = 1u, kItemRefine = 2u;
 constexpr uint32_t kItemExit = 0xFFFFFFFFu;
 constexpr unsigned kSpinLimit = 1u << 24;
-constexpr int kEngineMinBlocks = 3;
+constexpr int kEngineMinBlocks = 4;  // 64 registers: four CTAs per SM (measured best)
 constexpr int kEngineThreads = kThreads;
 constexpr size_t kEngineDynSmem = 0;  // ~ seconds of polling at the sleep below
 
