@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", default="prefix", choices=["prefix", "dense"])
+    ap.add_argument("--vocab-shards", type=int, default=1,
+                    help="N > 1: time the vocabulary-parallel protocol with N ranks emulated "
+                         "on this one GPU (one rank per context, exchanges as copies)")
     return ap.parse_args()
 
 
@@ -460,10 +463,94 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_vocab_parallel(args):
+    """The vocabulary-parallel protocol with N ranks emulated on one GPU.  Every
+    rank's phases are timed with events on the stream; a step on N GPUs would
+    take the slowest rank's phases plus three small collectives (not timed
+    here: no run of this build has more than one GPU)."""
+    import torch
+    from speculative_decoding_verification_86_b200 import binding, build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = make_workload(args.workload, dev, 0)
+    B, kp1, V = w["target"].shape
+    k = kp1 - 1
+    n = args.vocab_shards
+    bounds, b1, b2 = binding.shard_layout(B, k, V, w["target"].dtype, n)
+    ranks = [binding.ShardRank(dev, r, n, max_batch=B, max_k=max(k, 1), max_vocab=V) for r in range(n)]
+    shards = [(w["target"][:, :, bounds[r]:bounds[r + 1]].contiguous(),
+               None if w.get("draft") is None else w["draft"][:, :, bounds[r]:bounds[r + 1]].contiguous())
+              for r in range(n)]
+    kw = dict(verify_len=w.get("verify_len"), temperature=w.get("temperature"), conf=w.get("conf"))
+    all1 = torch.empty(n * b1, dtype=torch.uint8, device=dev)
+    all2 = torch.empty(n * b2, dtype=torch.uint8, device=dev)
+    votes = torch.empty((n, B), dtype=torch.int32, device=dev)
+    outs = [rk.ver._outputs(B, k, True) for rk in ranks]
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    phase_ms = [[0.0, 0.0, 0.0] for _ in range(n)]
+    redo_counts = []
+
+    def step(timed):
+        marks = []
+        for r, rk in enumerate(ranks):
+            e0, e1 = ev(), ev()
+            e0.record()
+            rk.stats(shards[r][0], shards[r][1], w["tokens"], V, all1[r * b1:(r + 1) * b1], **kw)
+            e1.record()
+            marks.append((r, 0, e0, e1))
+        for r, rk in enumerate(ranks):
+            e0, e1 = ev(), ev()
+            e0.record()
+            rk.decide(all1, shards[r][0], shards[r][1], w["tokens"], V, outs[r],
+                      all2[r * b2:(r + 1) * b2], seed=w["seed"], **kw)
+            e1.record()
+            marks.append((r, 1, e0, e1))
+        for r, rk in enumerate(ranks):
+            e0, e1 = ev(), ev()
+            e0.record()
+            rk.locate(all2, shards[r][0], shards[r][1], w["tokens"], V, votes[r], **kw)
+            vmax = votes.max(dim=0).values.contiguous()
+            redo = rk.finish(vmax, outs[r])
+            e1.record()
+            marks.append((r, 2, e0, e1))
+        torch.cuda.synchronize()
+        if timed:
+            for r, ph, e0, e1 in marks:
+                phase_ms[r][ph] += e0.elapsed_time(e1)
+            redo_counts.append(int(redo.sum().item()))
+
+    for _ in range(max(args.warmup, 3)):
+        step(False)
+    steps = min(args.steps, 200)
+    for _ in range(steps):
+        step(True)
+    per_rank = [[x / steps for x in ph] for ph in phase_ms]
+    slowest = max(sum(ph) for ph in per_rank)
+    L = effective_lengths(w, ranks[0].ver)
+    positions = int(L.sum().item())
+    line = {
+        "metric": "vocabulary-parallel verification, %d ranks emulated on one GPU" % n,
+        "value": positions / (slowest * 1e-3), "unit": "positions/s (slowest rank's phases)",
+        "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step_slowest_rank": slowest,
+        "higher_is_better": True, "data": "synthetic", "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
+        "config": {"workload": w["name"], "vocab_bounds": bounds},
+        "per_rank_ms": [{"stats": a, "decide_and_masses": b, "locate": c} for a, b, c in per_rank],
+        "exchange_bytes_per_rank": {"block1": b1, "block2": b2, "votes": 4 * B},
+        "requests_redone_per_step": sum(redo_counts) / max(len(redo_counts), 1),
+        "note": "excludes the three collectives and the redo of flagged requests",
+    }
+    print(json.dumps(line), flush=True)
+    for rk in ranks:
+        rk.close()
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.vocab_shards > 1:
+        run_vocab_parallel(args)
     else:
         run_ours(args)
 

@@ -205,6 +205,53 @@ spec_status spec_verify_lengths(spec_verify_ctx* ctx, const spec_conf_args* conf
                                 const int32_t* verify_len, int B, int k, int32_t* out_len,
                                 float* out_survival, cudaStream_t stream);
 
+/* ---- Vocabulary-parallel verification (the LM heads split by vocabulary) ----
+ * Rank r of n_shards holds the logits of tokens [bounds[r], bounds[r+1]) of
+ * every row: target [B, k+1, w] and draft [B, k, w], w = bounds[r+1] -
+ * bounds[r] (whole 32768-logit bf16 / 16384-logit fp32 segments, split as
+ * evenly as their count allows; 1 <= n_shards <= 16 and n_shards <= the
+ * segment count).  Same rule, readings and random draws as spec_verify_run
+ * (dense statistics order); the caller moves the small exchange blocks:
+ *   1. spec_shard_stats  -> this rank's block 1 (block1_bytes, 256-byte aligned);
+ *      all-gather the blocks of ranks 0..n-1 into one contiguous buffer;
+ *   2. spec_shard_decide(all blocks 1) -> outputs of every request (identical on
+ *      every rank) except the sample token, and this rank's block 2;
+ *      all-gather blocks 2;
+ *   3. spec_shard_locate(all blocks 2) -> token_votes [B] int32 (device): the
+ *      token, -1 (redo), or -2 (not this rank); element-wise MAX over ranks;
+ *   4. spec_shard_finish(max votes) -> writes the sample tokens into
+ *      out_tokens and out_redo [B] int32: 1 marks a request that needs an fp64
+ *      path (an accept draw inside its certified bound, or a sample the fp32
+ *      filter cannot certify).  Redo such a request whole with spec_verify_run
+ *      on its gathered rows (B = 1, request_offset = request_offset + i), which
+ *      gives exactly the single-rank result.
+ * All four calls of one verification use the same context, stream, arguments
+ * and outputs.  Merged statistics are the whole-vocabulary run's record for
+ * record, so decisions, probabilities and tokens equal spec_verify_run's. */
+spec_status spec_shard_layout(int B, int k, int64_t V, spec_dtype dtype, int n_shards,
+                              int64_t* bounds /* host [n_shards + 1] or NULL */,
+                              size_t* block1_bytes, size_t* block2_bytes);
+spec_status spec_shard_stats(spec_verify_ctx* ctx, int rank, int n_shards, const void* target_shard,
+                             const void* draft_shard, spec_dtype dtype, const int32_t* draft_tokens,
+                             const int32_t* verify_len, const float* temperature,
+                             const spec_conf_args* conf, int B, int k, int64_t V, void* block1,
+                             cudaStream_t stream);
+spec_status spec_shard_decide(spec_verify_ctx* ctx, int rank, int n_shards, const void* blocks1,
+                              const void* target_shard, const void* draft_shard, spec_dtype dtype,
+                              const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* temperature, const spec_conf_args* conf, int B, int k,
+                              int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                              int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                              float* out_q, uint32_t* out_status, void* block2,
+                              cudaStream_t stream);
+spec_status spec_shard_locate(spec_verify_ctx* ctx, int rank, int n_shards, const void* blocks2,
+                              const void* target_shard, const void* draft_shard, spec_dtype dtype,
+                              const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* temperature, const spec_conf_args* conf, int B, int k,
+                              int64_t V, int32_t* token_votes, cudaStream_t stream);
+spec_status spec_shard_finish(spec_verify_ctx* ctx, const int32_t* token_votes_max, int B, int k,
+                              int32_t* out_tokens, int32_t* out_redo, cudaStream_t stream);
+
 /* spec_verify_run on HOST buffers: copies the inputs (pinned or pageable host
  * memory) to device staging owned by the context, verifies, copies the outputs
  * back and synchronises `stream`.  Staging grows on demand and is freed with the

@@ -83,6 +83,14 @@ def lib():
     L.spec_conf_budget.argtypes = [_vp, _vp, _vp, ctypes.c_float, _i32, _i32, _i32,
                                    ctypes.c_float, _vp, _vp, _vp]
     L.spec_verify_lengths.argtypes = [_vp, ctypes.POINTER(ConfArgs), _vp, _i32, _i32, _vp, _vp, _vp]
+    shard_common = [_vp, _i32, _i32]
+    shard_inputs = [_vp, _vp, _i32, _vp, _vp, _vp, ctypes.POINTER(ConfArgs), _i32, _i32, _i64]
+    L.spec_shard_layout.argtypes = [_i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp]
+    L.spec_shard_stats.argtypes = shard_common + shard_inputs + [_vp, _vp]
+    L.spec_shard_decide.argtypes = shard_common + [_vp] + shard_inputs + [
+        _u64, _u32, _u32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    L.spec_shard_locate.argtypes = shard_common + [_vp] + shard_inputs + [_vp, _vp]
+    L.spec_shard_finish.argtypes = [_vp, _vp, _i32, _i32, _vp, _vp, _vp]
     L.spec_verify_set_mode.argtypes = [_vp, _i32]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
@@ -94,6 +102,8 @@ def lib():
     for name in ("spec_verify_init", "spec_verify_destroy", "spec_verify_run",
                  "spec_verify_run_with_uniforms", "spec_verify_run_host", "spec_verify_greedy",
                  "spec_conf_budget", "spec_verify_lengths", "spec_verify_greedy_noalloc",
+                 "spec_shard_layout", "spec_shard_stats", "spec_shard_decide", "spec_shard_locate",
+                 "spec_shard_finish",
                  "spec_verify_set_mode",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
@@ -407,3 +417,184 @@ def spec_conf_budget(ctx: SpecVerifier, *a, **kw):
 
 def spec_verify_run_host(ctx: SpecVerifier, *a, **kw):
     return ctx.run_host(*a, **kw)
+
+
+# ----------------------------------------------------- vocabulary-parallel --
+
+def shard_layout(B, k, V, dtype, n_shards):
+    """Vocabulary split and exchange-block sizes: (bounds [n+1], block1 bytes,
+    block2 bytes).  Rank r holds tokens [bounds[r], bounds[r+1])."""
+    bounds = (_i64 * (n_shards + 1))()
+    b1, b2 = ctypes.c_size_t(), ctypes.c_size_t()
+    code = SPEC_BF16 if dtype == torch.bfloat16 else SPEC_F32
+    _check(lib().spec_shard_layout(B, k, int(V), code, n_shards, bounds, ctypes.byref(b1),
+                                   ctypes.byref(b2)), "spec_shard_layout")
+    return list(bounds), b1.value, b2.value
+
+
+class ShardRank:
+    """One rank of a vocabulary-parallel verification (its own context).  The
+    phases follow include/spec_verify.h; `verify_vocab_parallel` runs them with
+    torch.distributed collectives, `emulate_vocab_parallel` on one device."""
+
+    def __init__(self, device, rank, n_shards, max_batch, max_k, max_vocab):
+        self.ver = SpecVerifier(device, max_batch=max_batch, max_k=max_k, max_vocab=max_vocab,
+                                mode="dense")
+        self.device = self.ver.device
+        self.rank, self.n = int(rank), int(n_shards)
+
+    def _inputs(self, target, draft, tokens, verify_len, temperature, conf, V):
+        B, kp1, _ = target.shape
+        k = kp1 - 1
+        cref, keep = self.ver._conf(conf)
+        args = [_dev_ptr(target, None, self.device, "target shard"),
+                _dev_ptr(draft, None, self.device, "draft shard"), _dtype_code(target),
+                _dev_ptr(tokens, torch.int32, self.device, "tokens"),
+                _dev_ptr(verify_len, torch.int32, self.device, "verify_len"),
+                _dev_ptr(temperature, torch.float32, self.device, "temperature"), cref, B, k, int(V)]
+        return args, keep
+
+    def stats(self, target, draft, tokens, V, block1, verify_len=None, temperature=None, conf=None,
+              stream=None):
+        args, keep = self._inputs(target, draft, tokens, verify_len, temperature, conf, V)
+        _check(lib().spec_shard_stats(self.ver._h, self.rank, self.n, *args, _dev_ptr(block1),
+                                      _stream_handle(stream, self.device)), "spec_shard_stats")
+        del keep
+
+    def decide(self, blocks1, target, draft, tokens, V, out, block2, verify_len=None,
+               temperature=None, conf=None, seed=0, step=0, request_offset=0, stream=None):
+        args, keep = self._inputs(target, draft, tokens, verify_len, temperature, conf, V)
+        _check(lib().spec_shard_decide(
+            self.ver._h, self.rank, self.n, _dev_ptr(blocks1), *args, int(seed), int(step),
+            int(request_offset), _dev_ptr(out["accepted"]), _dev_ptr(out["tokens"]),
+            _dev_ptr(out.get("p")), _dev_ptr(out.get("q")), _dev_ptr(out["status"]),
+            _dev_ptr(block2), _stream_handle(stream, self.device)), "spec_shard_decide")
+        del keep
+
+    def locate(self, blocks2, target, draft, tokens, V, votes, verify_len=None, temperature=None,
+               conf=None, stream=None):
+        args, keep = self._inputs(target, draft, tokens, verify_len, temperature, conf, V)
+        _check(lib().spec_shard_locate(self.ver._h, self.rank, self.n, _dev_ptr(blocks2), *args,
+                                       _dev_ptr(votes), _stream_handle(stream, self.device)),
+               "spec_shard_locate")
+        del keep
+
+    def finish(self, votes_max, out, stream=None):
+        B, kp1 = out["tokens"].shape
+        redo = torch.empty(B, dtype=torch.int32, device=self.device)
+        _check(lib().spec_shard_finish(self.ver._h, _dev_ptr(votes_max), B, kp1 - 1,
+                                       _dev_ptr(out["tokens"]), _dev_ptr(redo),
+                                       _stream_handle(stream, self.device)), "spec_shard_finish")
+        return redo
+
+    def close(self):
+        self.ver.close()
+
+
+def _redo_requests(ver, redo, rows_of, tokens, verify_len, temperature, conf, seed, step,
+                   request_offset, out):
+    """Requests flagged for an fp64 path: verified whole on their gathered rows
+    (the single-rank path, same global request index and draws)."""
+    idx = torch.nonzero(redo.cpu()).flatten().tolist()
+    for i in idx:
+        t_full, d_full = rows_of(i)
+        sl = slice(i, i + 1)
+        c = None
+        if conf is not None:
+            c = dict(conf, hidden=conf["hidden"][sl])
+        o = ver.run(t_full, d_full, tokens[sl].contiguous(),
+                    verify_len=None if verify_len is None else verify_len[sl].contiguous(),
+                    temperature=None if temperature is None else temperature[sl].contiguous(),
+                    conf=c, seed=seed, step=step, request_offset=request_offset + i)
+        for key in out:
+            out[key][sl] = o[key]
+    return idx
+
+
+def verify_vocab_parallel(rank_obj, target, draft, tokens, V, verify_len=None, temperature=None,
+                          conf=None, seed=0, step=0, request_offset=0, group=None):
+    """Vocabulary-parallel verification on this rank's shard with
+    torch.distributed collectives (all ranks call it with the same arguments
+    apart from their shards).  Returns the outputs (identical on every rank)."""
+    import torch.distributed as dist
+    n, r = rank_obj.n, rank_obj.rank
+    B, kp1, _ = target.shape
+    k = kp1 - 1
+    bounds, b1, b2 = shard_layout(B, k, V, target.dtype, n)
+    dev = rank_obj.device
+    blk1 = torch.empty(b1, dtype=torch.uint8, device=dev)
+    all1 = torch.empty(n * b1, dtype=torch.uint8, device=dev)
+    blk2 = torch.empty(b2, dtype=torch.uint8, device=dev)
+    all2 = torch.empty(n * b2, dtype=torch.uint8, device=dev)
+    out = rank_obj.ver._outputs(B, k, True)
+    votes = torch.empty(B, dtype=torch.int32, device=dev)
+    kw = dict(verify_len=verify_len, temperature=temperature, conf=conf)
+    rank_obj.stats(target, draft, tokens, V, blk1, **kw)
+    dist.all_gather_into_tensor(all1, blk1, group=group)
+    rank_obj.decide(all1, target, draft, tokens, V, out, blk2, seed=seed, step=step,
+                    request_offset=request_offset, **kw)
+    dist.all_gather_into_tensor(all2, blk2, group=group)
+    rank_obj.locate(all2, target, draft, tokens, V, votes, **kw)
+    dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
+    redo = rank_obj.finish(votes, out)
+
+    widths = [bounds[q + 1] - bounds[q] for q in range(n)]
+    wmax = max(widths)
+
+    def gather_rows(x):  # [1, rows, w_r] on every rank -> [1, rows, V]
+        pad = torch.zeros((1, x.shape[1], wmax), dtype=x.dtype, device=dev)
+        pad[:, :, :x.shape[2]] = x
+        parts = [torch.empty_like(pad) for _ in range(n)]
+        dist.all_gather(parts, pad, group=group)
+        return torch.cat([parts[q][:, :, :widths[q]] for q in range(n)], dim=2).contiguous()
+
+    def rows_of(i):
+        t_full = gather_rows(target[i:i + 1])
+        d_full = gather_rows(draft[i:i + 1]) if draft is not None else None
+        return t_full, d_full
+
+    _redo_requests(rank_obj.ver, redo, rows_of, tokens, verify_len, temperature, conf, seed, step,
+                   request_offset, out)
+    return out
+
+
+def emulate_vocab_parallel(ranks, target, draft, tokens, verify_len=None, temperature=None,
+                           conf=None, seed=0, step=0, request_offset=0):
+    """The vocabulary-parallel protocol on ONE device: `ranks` are ShardRank
+    objects (their own contexts), each given its slice of the full logits; the
+    all-gathers become concatenations and the max a torch.max.  Returns
+    (outputs of every rank, final outputs, requests redone)."""
+    n = len(ranks)
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    bounds, b1, b2 = shard_layout(B, k, V, target.dtype, n)
+    dev = ranks[0].device
+    shards = [(target[:, :, bounds[r]:bounds[r + 1]].contiguous(),
+               None if draft is None else draft[:, :, bounds[r]:bounds[r + 1]].contiguous())
+              for r in range(n)]
+    kw = dict(verify_len=verify_len, temperature=temperature, conf=conf)
+    all1 = torch.empty(n * b1, dtype=torch.uint8, device=dev)
+    for r, rk in enumerate(ranks):
+        rk.stats(shards[r][0], shards[r][1], tokens, V, all1[r * b1:(r + 1) * b1], **kw)
+    all2 = torch.empty(n * b2, dtype=torch.uint8, device=dev)
+    outs = []
+    for r, rk in enumerate(ranks):
+        o = rk.ver._outputs(B, k, True)
+        rk.decide(all1, shards[r][0], shards[r][1], tokens, V, o, all2[r * b2:(r + 1) * b2],
+                  seed=seed, step=step, request_offset=request_offset, **kw)
+        outs.append(o)
+    votes = torch.empty((n, B), dtype=torch.int32, device=dev)
+    for r, rk in enumerate(ranks):
+        rk.locate(all2, shards[r][0], shards[r][1], tokens, V, votes[r], **kw)
+    vmax = votes.max(dim=0).values.contiguous()
+    redo = None
+    for r, rk in enumerate(ranks):
+        redo = rk.finish(vmax, outs[r])
+    final = {key: v.clone() for key, v in outs[0].items()}
+
+    def rows_of(i):
+        return (target[i:i + 1].contiguous(), None if draft is None else draft[i:i + 1].contiguous())
+
+    redone = _redo_requests(ranks[0].ver, redo, rows_of, tokens, verify_len, temperature, conf,
+                            seed, step, request_offset, final)
+    return outs, final, redone, votes

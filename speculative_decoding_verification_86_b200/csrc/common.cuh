@@ -128,7 +128,9 @@ struct RunParams {
   const double* uniforms;  // [B, k+1, 2] test override or nullptr
   int B;
   int k;
-  int64_t V;
+  int64_t V;               // vocabulary size (token indices are global)
+  int64_t row_stride;      // logits per row in the buffers: V, or a shard's width
+  int64_t v_lo;            // first token the buffers hold (0, or a shard's start)
   int n_chunks;            // 8192 / 4096-logit chunks (sampling and refinement passes)
   int n_segs;              // 32768 / 16384-logit segments (statistics pass)
   uint64_t seed;
@@ -158,6 +160,12 @@ struct RunParams {
   int* runc;               // [B, 4 n_chunks] sub-chunks holding unsettled logits
   Counters* counters;      // this run's counters
   Counters* counters_next; // the other run's counters, reset here
+
+  // vocabulary-parallel runs (nullptr / 0 otherwise)
+  const float* tok_logits; // [B, k, 2]: target and draft logit of each drafted token
+  int32_t* fallback;       // [B]: set when a decision needs rows held by other ranks
+  int32_t* shard_tok;      // [B]: located token, -1 to redo the request whole, -2 not here
+  int c_lo, c_hi;          // chunks whose logits the buffers hold (c_hi = 0: all)
 
   // engine
   int mode;                        // kModeDense / kModePrefix
@@ -360,14 +368,21 @@ __device__ __forceinline__ bool temperature_valid(float T) {
   return (T >= 0.0f) && !isinf(T) && !(T > 0.0f && T < 0x1p-100f);
 }
 
-// Row pointers.
+// Row pointers, indexed by global token index: element t of the returned row
+// is token t.  A vocabulary shard holds tokens [v_lo, v_lo + row_stride), and
+// only those are ever read through its rows.
+__device__ __forceinline__ const void* row_at(const void* base, int64_t row, const RunParams& p,
+                                              bool bf16) {
+  const int64_t es = bf16 ? 2 : 4;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(base) +
+                      static_cast<uintptr_t>((row * p.row_stride - p.v_lo) * es);
+  return reinterpret_cast<const void*>(a);
+}
 __device__ __forceinline__ const void* target_row(const RunParams& p, int i, int j, bool bf16) {
-  const int64_t idx = (static_cast<int64_t>(i) * (p.k + 1) + j) * p.V;
-  return static_cast<const char*>(p.target) + idx * (bf16 ? 2 : 4);
+  return row_at(p.target, static_cast<int64_t>(i) * (p.k + 1) + j, p, bf16);
 }
 __device__ __forceinline__ const void* draft_row(const RunParams& p, int i, int j, bool bf16) {
-  const int64_t idx = (static_cast<int64_t>(i) * p.k + j) * p.V;
-  return static_cast<const char*>(p.draft) + idx * (bf16 ? 2 : 4);
+  return row_at(p.draft, static_cast<int64_t>(i) * p.k + j, p, bf16);
 }
 
 struct ReqInfo {

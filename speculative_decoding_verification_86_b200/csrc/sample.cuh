@@ -314,6 +314,16 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
   int cstar = sh.cstar;
   // residual mass must clear the 1e-12 floor with certainty
   if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) cstar = -1;
+  // vocabulary-parallel: only the rank holding chunk cstar rescans it
+  const bool sharded = p.c_hi > 0;
+  if (sharded && cstar >= 0 && (cstar < p.c_lo || cstar >= p.c_hi)) {
+    if (tid == 0) {
+      p.shard_tok[i] = -2;
+      sh.refine_slot = -1;
+    }
+    sync_compute();
+    return;
+  }
   bool certain = false;
   int token = -1;
   if (cstar >= 0) {
@@ -383,7 +393,12 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
     }
   }
   if (tid == 0) {
-    if (certain) {
+    if (sharded) {
+      // the fp64 refinement would need every rank's logits: redo the request whole
+      p.shard_tok[i] = certain ? token : -1;
+      if (certain) atomicAdd(&p.counters->sample_fast, 1u);
+      sh.refine_slot = -1;
+    } else if (certain) {
       p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;
       atomicAdd(&p.counters->sample_fast, 1u);
       sh.refine_slot = -1;

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "conf.cuh"
 #include "engine.cuh"
+#include "shard.cuh"
 #include "philox.cuh"
 #include "refine.cuh"
 #include "sample.cuh"
@@ -126,6 +127,8 @@ struct spec_verify_ctx {
   int* runc = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
   int32_t* conf_len = nullptr;
+  float* tok_logits = nullptr;    // [max_batch, max_k, 2] (vocabulary-parallel runs)
+  int32_t* fallback = nullptr;    // [max_batch]
   double* conf_prefix = nullptr;  // [max_batch, kMaxK]
   int32_t* conf_cap = nullptr;    // [max_batch]
   unsigned* conf_arrive = nullptr;
@@ -186,6 +189,8 @@ spec_status carve(spec_verify_ctx* c) {
   const size_t o_runc = take(per_req_subs * sizeof(int));
   const size_t o_cnt = take(2 * sizeof(sv::Counters));
   const size_t o_conf = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
+  const size_t o_tokl = take(static_cast<size_t>(c->max_batch) * c->max_k * 2 * sizeof(float));
+  const size_t o_fall = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
   const size_t o_cpre = take(static_cast<size_t>(c->max_batch) * sv::kMaxK * sizeof(double));
   const size_t o_ccap = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
   const size_t o_carr = take(sizeof(unsigned));
@@ -222,6 +227,8 @@ spec_status carve(spec_verify_ctx* c) {
   c->runc = reinterpret_cast<int*>(b + o_runc);
   c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
   c->conf_len = reinterpret_cast<int32_t*>(b + o_conf);
+  c->tok_logits = reinterpret_cast<float*>(b + o_tokl);
+  c->fallback = reinterpret_cast<int32_t*>(b + o_fall);
   c->conf_prefix = reinterpret_cast<double*>(b + o_cpre);
   c->conf_cap = reinterpret_cast<int32_t*>(b + o_ccap);
   c->conf_arrive = reinterpret_cast<unsigned*>(b + o_carr);
@@ -326,6 +333,13 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.B = B;
   p.k = k;
   p.V = V;
+  p.row_stride = V;
+  p.v_lo = 0;
+  p.tok_logits = nullptr;
+  p.fallback = nullptr;
+  p.shard_tok = nullptr;
+  p.c_lo = 0;
+  p.c_hi = 0;
   p.n_chunks = n_chunks;
   p.n_segs = n_segs;
   p.seed = seed;
@@ -377,6 +391,92 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   return SPEC_OK;
 }
 
+
+// ---------------------------------------------------- vocabulary-parallel --
+// Shards are whole statistics segments, split as evenly as the segment count
+// allows; the exchange blocks have the widest rank's size on every rank.
+spec_status shard_geometry(int64_t V, bool bf16, int n_shards, sv::ShardBounds* sb,
+                           int64_t* seg_len_out) {
+  const int64_t segl = bf16 ? sv::SegGeo<true>::kSeg : sv::SegGeo<false>::kSeg;
+  if (V < 1 || n_shards < 1 || n_shards > sv::kMaxShards) return SPEC_ERR_INVALID_ARG;
+  const int64_t n_segs = (V + segl - 1) / segl;
+  if (n_segs < n_shards) return SPEC_ERR_INVALID_ARG;
+  sb->n = n_shards;
+  sb->nls_max = 0;
+  for (int r = 0; r <= n_shards; ++r) sb->seg_lo[r] = static_cast<int>(n_segs * r / n_shards);
+  for (int r = 0; r < n_shards; ++r) sb->nls_max = std::max(sb->nls_max, sb->seg_lo[r + 1] - sb->seg_lo[r]);
+  *seg_len_out = segl;
+  return SPEC_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct ShardSizes {
+  size_t rec_bytes, tok_off, block1, block2;
+  int nlc_max;
+};
+
+ShardSizes shard_sizes(int B, int k, const sv::ShardBounds& sb) {
+  ShardSizes z;
+  z.rec_bytes = static_cast<size_t>(B) * (2 * k + 1) * sb.nls_max * sizeof(sv::ShardRec);
+  z.tok_off = align256(z.rec_bytes);
+  z.block1 = z.tok_off + align256(static_cast<size_t>(B) * k * 2 * sizeof(float));
+  z.nlc_max = sb.nls_max * sv::kChunksPerSeg;
+  z.block2 = static_cast<size_t>(B) * z.nlc_max * sizeof(sv::SampleChunk);
+  return z;
+}
+
+// Common checks and parameters of the per-rank phases: the rank's logits are
+// [B, k+1, width] / [B, k, width] for tokens [v_lo, v_lo + width).
+spec_status shard_params(spec_verify_ctx* c, int rank, int n_shards, const void* target,
+                         const void* draft, spec_dtype dtype, const int32_t* tokens,
+                         const int32_t* vlen, const float* temp, const spec_conf_args* conf,
+                         int B, int k, int64_t V, sv::RunParams* pp, sv::ShardBounds* sb,
+                         int64_t* seg_len) {
+  if (!c || B < 1 || B > c->max_batch || k < 0 || k > c->max_k || V < 1 || V > c->max_vocab)
+    return SPEC_ERR_INVALID_ARG;
+  if (dtype != SPEC_F32 && dtype != SPEC_BF16) return SPEC_ERR_INVALID_ARG;
+  const bool bf16 = dtype == SPEC_BF16;
+  if (spec_status st = shard_geometry(V, bf16, n_shards, sb, seg_len); st != SPEC_OK) return st;
+  if (rank < 0 || rank >= n_shards) return SPEC_ERR_INVALID_ARG;
+  if (!target || (k > 0 && !tokens)) return SPEC_ERR_INVALID_ARG;
+  if (spec_status st = check_conf(c, conf); st != SPEC_OK) return st;
+  const int64_t esize = bf16 ? 2 : 4;
+  if ((V * esize) % 16 != 0) return SPEC_ERR_UNSUPPORTED;
+  if (!aligned(target, 16) || (draft && !aligned(draft, 16))) return SPEC_ERR_UNSUPPORTED;
+  const int64_t v_lo = std::min<int64_t>(static_cast<int64_t>(sb->seg_lo[rank]) * *seg_len, V);
+  const int64_t v_hi = std::min<int64_t>(static_cast<int64_t>(sb->seg_lo[rank + 1]) * *seg_len, V);
+  sv::RunParams p{};
+  p.target = target;
+  p.draft = draft;
+  p.tokens = tokens;
+  p.vlen = vlen;
+  p.temp = temp;
+  p.conf_len = conf ? c->conf_len : nullptr;
+  p.B = B;
+  p.k = k;
+  p.V = V;
+  p.row_stride = v_hi - v_lo;
+  p.v_lo = v_lo;
+  const int chunk = bf16 ? sv::kChunkBf16 : sv::kChunkF32;
+  p.n_chunks = static_cast<int>((V + chunk - 1) / chunk);
+  p.n_segs = sb->seg_lo[n_shards];
+  p.c_lo = sb->seg_lo[rank] * sv::kChunksPerSeg;
+  p.c_hi = std::min(sb->seg_lo[rank + 1] * sv::kChunksPerSeg, p.n_chunks);
+  p.eps_ex2 = kEpsEx2;
+  p.meta = c->meta;
+  p.ssum = c->ssum;
+  p.jobs = c->jobs;
+  p.smass = c->smass;
+  p.tok_logits = c->tok_logits;
+  p.fallback = c->fallback;
+  p.counters = c->counters + (c->run_id & 1u);
+  p.counters_next = c->counters + ((c->run_id + 1u) & 1u);
+  *pp = p;
+  return SPEC_OK;
+}
+
+int grid_for(int64_t n) { return static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)); }
 }  // namespace
 
 extern "C" {
@@ -670,6 +770,7 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
   p.B = B;
   p.k = k;
   p.V = V;
+  p.row_stride = V;
   p.n_chunks = static_cast<int>((V + (bf16 ? sv::kChunkBf16 : sv::kChunkF32) - 1) /
                                 (bf16 ? sv::kChunkBf16 : sv::kChunkF32));
   p.n_segs = static_cast<int>(n_segs);
@@ -744,4 +845,153 @@ spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
   return SPEC_OK;
 }
 
+
+spec_status spec_shard_layout(int B, int k, int64_t V, spec_dtype dtype, int n_shards,
+                              int64_t* bounds, size_t* block1_bytes, size_t* block2_bytes) {
+  if (B < 1 || k < 0 || (dtype != SPEC_F32 && dtype != SPEC_BF16)) return SPEC_ERR_INVALID_ARG;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_geometry(V, dtype == SPEC_BF16, n_shards, &sb, &segl); st != SPEC_OK)
+    return st;
+  const ShardSizes z = shard_sizes(B, k, sb);
+  if (bounds)
+    for (int r = 0; r <= n_shards; ++r) bounds[r] = std::min<int64_t>(sb.seg_lo[r] * segl, V);
+  if (block1_bytes) *block1_bytes = z.block1;
+  if (block2_bytes) *block2_bytes = z.block2;
+  return SPEC_OK;
+}
+
+spec_status spec_shard_stats(spec_verify_ctx* ctx, int rank, int n_shards, const void* target_shard,
+                             const void* draft_shard, spec_dtype dtype, const int32_t* draft_tokens,
+                             const int32_t* verify_len, const float* temperature,
+                             const spec_conf_args* conf, int B, int k, int64_t V, void* block1,
+                             cudaStream_t stream) {
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, rank, n_shards, target_shard, draft_shard, dtype,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  if (!block1 || !aligned(block1, 256)) return SPEC_ERR_UNSUPPORTED;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  if (conf) launch_conf(ctx, conf, B, k, verify_len, ctx->conf_len, nullptr, stream);
+  const ShardSizes z = shard_sizes(B, k, sb);
+  const int nls = sb.seg_lo[rank + 1] - sb.seg_lo[rank];
+  const int64_t ctas = static_cast<int64_t>(B) * (2 * k + 1) * nls;
+  auto* recs = static_cast<sv::ShardRec*>(block1);
+  const bool bf16 = dtype == SPEC_BF16;
+  if (ctas > 0) {
+    if (bf16) sv::k_shard_stats<true><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls, recs);
+    else sv::k_shard_stats<false><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls, recs);
+  }
+  if (k > 0) {
+    float* tl = reinterpret_cast<float*>(static_cast<char*>(block1) + z.tok_off);
+    const int grid = grid_for(static_cast<int64_t>(B) * k);
+    if (bf16) sv::k_shard_token_logits<true><<<grid, 256, 0, stream>>>(p, tl);
+    else sv::k_shard_token_logits<false><<<grid, 256, 0, stream>>>(p, tl);
+  }
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_decide(spec_verify_ctx* ctx, int rank, int n_shards, const void* blocks1,
+                              const void* target_shard, const void* draft_shard, spec_dtype dtype,
+                              const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* temperature, const spec_conf_args* conf, int B, int k,
+                              int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                              int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                              float* out_q, uint32_t* out_status, void* block2,
+                              cudaStream_t stream) {
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, rank, n_shards, target_shard, draft_shard, dtype,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  if (!blocks1 || !block2 || !out_accepted || !out_tokens || !aligned(blocks1, 256) ||
+      !aligned(block2, 16))
+    return SPEC_ERR_INVALID_ARG;
+  const int rows = 2 * k + 1;
+  if (static_cast<int64_t>(B) * rows * p.n_segs >
+      static_cast<int64_t>(ctx->max_batch) * (2 * ctx->max_k + 1) * ctx->max_chunks)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  p.seed = seed;
+  p.step = step;
+  p.req_off = request_offset;
+  p.out_acc = out_accepted;
+  p.out_tok = out_tokens;
+  p.out_p = out_p;
+  p.out_q = out_q;
+  p.out_status = out_status;
+  const ShardSizes z = shard_sizes(B, k, sb);
+  const bool bf16 = dtype == SPEC_BF16;
+  sv::k_shard_gather_stats<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
+      p, sb, static_cast<const char*>(blocks1), z.block1, z.tok_off, segl);
+  if (bf16) sv::k_shard_decide<true><<<B, sv::kThreads, 0, stream>>>(p);
+  else sv::k_shard_decide<false><<<B, sv::kThreads, 0, stream>>>(p);
+  const int nls = sb.seg_lo[rank + 1] - sb.seg_lo[rank];
+  if (nls > 0) {
+    if (bf16) sv::k_shard_masses<true><<<B * nls, sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls);
+    else sv::k_shard_masses<false><<<B * nls, sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls);
+  }
+  sv::k_shard_pack_masses<<<grid_for(static_cast<int64_t>(B) * z.nlc_max), 256, 0, stream>>>(
+      p, p.c_lo, p.c_hi - p.c_lo, z.nlc_max, static_cast<sv::SampleChunk*>(block2));
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_locate(spec_verify_ctx* ctx, int rank, int n_shards, const void* blocks2,
+                              const void* target_shard, const void* draft_shard, spec_dtype dtype,
+                              const int32_t* draft_tokens, const int32_t* verify_len,
+                              const float* temperature, const spec_conf_args* conf, int B, int k,
+                              int64_t V, int32_t* out_token_votes, cudaStream_t stream) {
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, rank, n_shards, target_shard, draft_shard, dtype,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  if (!blocks2 || !out_token_votes || !aligned(blocks2, 16) || !aligned(out_token_votes, 4))
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  const ShardSizes z = shard_sizes(B, k, sb);
+  p.shard_tok = out_token_votes;
+  sv::k_shard_unpack_masses<<<grid_for(static_cast<int64_t>(B) * p.n_chunks), 256, 0, stream>>>(
+      p, sb, static_cast<const sv::SampleChunk*>(blocks2), z.nlc_max);
+  if (dtype == SPEC_BF16) sv::k_shard_locate<true><<<B, sv::kThreads, 0, stream>>>(p);
+  else sv::k_shard_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_finish(spec_verify_ctx* ctx, const int32_t* token_votes_max, int B, int k,
+                              int32_t* out_tokens, int32_t* out_redo, cudaStream_t stream) {
+  if (!ctx || B < 1 || B > ctx->max_batch || k < 0 || k > ctx->max_k || !token_votes_max ||
+      !out_tokens || !out_redo)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  sv::RunParams p{};
+  p.B = B;
+  p.k = k;
+  p.jobs = ctx->jobs;
+  p.fallback = ctx->fallback;
+  p.out_tok = out_tokens;
+  sv::k_shard_finish<<<grid_for(B), 256, 0, stream>>>(p, token_votes_max);
+  if (cudaMemcpyAsync(out_redo, ctx->fallback, static_cast<size_t>(B) * sizeof(int32_t),
+                      cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
 }  // extern "C"

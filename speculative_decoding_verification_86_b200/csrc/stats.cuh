@@ -523,8 +523,9 @@ template <bool BF16>
 __device__ __forceinline__ int accept_eval(const RunParams& p, int i, int j, int xj,
                                           const RowMerged& ra, const RowMerged& rb,
                                           const TempConsts& t, double& pa, double& qb) {
-  const float la = load_logit(target_row(p, i, j, BF16), xj, BF16);
-  const float lb = load_logit(draft_row(p, i, j, BF16), xj, BF16);
+  const int64_t tl = (static_cast<int64_t>(i) * p.k + j) * 2;
+  const float la = p.tok_logits ? __ldcg(p.tok_logits + tl) : load_logit(target_row(p, i, j, BF16), xj, BF16);
+  const float lb = p.tok_logits ? __ldcg(p.tok_logits + tl + 1) : load_logit(draft_row(p, i, j, BF16), xj, BF16);
   const double arg_a = static_cast<double>(la) * t.cc - static_cast<double>(ra.K);
   const double arg_b = static_cast<double>(lb) * t.cc - static_cast<double>(rb.K);
   pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) / ra.Z;
@@ -731,6 +732,14 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
       }
     }
     sync_compute();
+    if (sh.need_exact >= 0 && p.fallback) {
+      // the fp64 row sums need every rank's logits: the request is redone whole
+      if (tid == 0) {
+        p.fallback[i] = 1;
+        p.jobs[i].kind = kJobNone;
+      }
+      return;
+    }
     if (sh.need_exact >= 0) {
       bool accept = false;
       double pa = 0.0, qb = 0.0;
