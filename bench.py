@@ -477,7 +477,7 @@ def run_vocab_parallel(args):
     B, kp1, V = w["target"].shape
     k = kp1 - 1
     n = args.vocab_shards
-    bounds, b1, b2 = binding.shard_layout(B, k, V, w["target"].dtype, n)
+    bounds, b1, b2, b3 = binding.shard_layout(B, k, V, w["target"].dtype, n)
     ranks = [binding.ShardRank(dev, r, n, max_batch=B, max_k=max(k, 1), max_vocab=V) for r in range(n)]
     shards = [(w["target"][:, :, bounds[r]:bounds[r + 1]].contiguous(),
                None if w.get("draft") is None else w["draft"][:, :, bounds[r]:bounds[r + 1]].contiguous())
@@ -485,10 +485,11 @@ def run_vocab_parallel(args):
     kw = dict(verify_len=w.get("verify_len"), temperature=w.get("temperature"), conf=w.get("conf"))
     all1 = torch.empty(n * b1, dtype=torch.uint8, device=dev)
     all2 = torch.empty(n * b2, dtype=torch.uint8, device=dev)
+    all3 = torch.empty(n * b3, dtype=torch.uint8, device=dev)
     votes = torch.empty((n, B), dtype=torch.int32, device=dev)
     outs = [rk.ver._outputs(B, k, True) for rk in ranks]
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    phase_ms = [[0.0, 0.0, 0.0] for _ in range(n)]
+    phase_ms = [[0.0, 0.0, 0.0, 0.0] for _ in range(n)]
     redo_counts = []
 
     def step(timed):
@@ -510,15 +511,26 @@ def run_vocab_parallel(args):
             e0, e1 = ev(), ev()
             e0.record()
             rk.locate(all2, shards[r][0], shards[r][1], w["tokens"], V, votes[r], **kw)
-            vmax = votes.max(dim=0).values.contiguous()
-            redo = rk.finish(vmax, outs[r])
             e1.record()
             marks.append((r, 2, e0, e1))
+        vmax = votes.max(dim=0).values.contiguous()
+        redo = [rk.finish(vmax, outs[r]) for r, rk in enumerate(ranks)][0]
+        if bool((redo == 2).any()):
+            for r, rk in enumerate(ranks):
+                e0, e1 = ev(), ev()
+                e0.record()
+                rk.refine_partials(shards[r][0], shards[r][1], w["tokens"], V,
+                                   all3[r * b3:(r + 1) * b3], **kw)
+                rk.refine_locate(all3, shards[r][0], shards[r][1], w["tokens"], V, votes[r], **kw)
+                e1.record()
+                marks.append((r, 3, e0, e1))
+            vmax = votes.max(dim=0).values.contiguous()
+            redo = [rk.refine_finish(vmax, outs[r]) for r, rk in enumerate(ranks)][0]
         torch.cuda.synchronize()
         if timed:
             for r, ph, e0, e1 in marks:
                 phase_ms[r][ph] += e0.elapsed_time(e1)
-            redo_counts.append(int(redo.sum().item()))
+            redo_counts.append(int((redo == 1).sum().item()))
 
     for _ in range(max(args.warmup, 3)):
         step(False)
@@ -535,10 +547,11 @@ def run_vocab_parallel(args):
         "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step_slowest_rank": slowest,
         "higher_is_better": True, "data": "synthetic", "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
         "config": {"workload": w["name"], "vocab_bounds": bounds},
-        "per_rank_ms": [{"stats": a, "decide_and_masses": b, "locate": c} for a, b, c in per_rank],
-        "exchange_bytes_per_rank": {"block1": b1, "block2": b2, "votes": 4 * B},
+        "per_rank_ms": [{"stats": a, "decide_and_masses": b, "locate": c, "fp64_refinement": d}
+                        for a, b, c, d in per_rank],
+        "exchange_bytes_per_rank": {"block1": b1, "block2": b2, "block3": b3, "votes": 4 * B},
         "requests_redone_per_step": sum(redo_counts) / max(len(redo_counts), 1),
-        "note": "excludes the three collectives and the redo of flagged requests",
+        "note": "excludes the collectives (3, or 5 with a refinement) and whole redos",
     }
     print(json.dumps(line), flush=True)
     for rk in ranks:

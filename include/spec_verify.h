@@ -219,18 +219,24 @@ spec_status spec_verify_lengths(spec_verify_ctx* ctx, const spec_conf_args* conf
  *      all-gather blocks 2;
  *   3. spec_shard_locate(all blocks 2) -> token_votes [B] int32 (device): the
  *      token, -1 (redo), or -2 (not this rank); element-wise MAX over ranks;
- *   4. spec_shard_finish(max votes) -> writes the sample tokens into
- *      out_tokens and out_redo [B] int32: 1 marks a request that needs an fp64
- *      path (an accept draw inside its certified bound, or a sample the fp32
- *      filter cannot certify).  Redo such a request whole with spec_verify_run
- *      on its gathered rows (B = 1, request_offset = request_offset + i), which
- *      gives exactly the single-rank result.
+ *   4. spec_shard_finish(max votes) -> writes the certified sample tokens into
+ *      out_tokens and out_redo [B] int32: 2 marks a sample the fp32 filter
+ *      could not certify, 1 a request whose accept draw fell inside its
+ *      certified bound.
+ *   5. only if some out_redo == 2: spec_shard_refine_partials -> block 3
+ *      (fp64 partial sums of this rank's sub-chunks); all-gather;
+ *      spec_shard_refine_locate(all blocks 3) -> votes; MAX over ranks;
+ *      spec_shard_refine_finish(max votes) -> the exact tokens, and out_redo
+ *      with 1 left only where the refinement itself needed other ranks' rows.
+ *   6. redo every request with out_redo == 1 whole: spec_verify_run on its
+ *      gathered rows (B = 1, request_offset = request_offset + i) gives
+ *      exactly the single-rank result.
  * All four calls of one verification use the same context, stream, arguments
  * and outputs.  Merged statistics are the whole-vocabulary run's record for
  * record, so decisions, probabilities and tokens equal spec_verify_run's. */
 spec_status spec_shard_layout(int B, int k, int64_t V, spec_dtype dtype, int n_shards,
                               int64_t* bounds /* host [n_shards + 1] or NULL */,
-                              size_t* block1_bytes, size_t* block2_bytes);
+                              size_t* block1_bytes, size_t* block2_bytes, size_t* block3_bytes);
 spec_status spec_shard_stats(spec_verify_ctx* ctx, int rank, int n_shards, const void* target_shard,
                              const void* draft_shard, spec_dtype dtype, const int32_t* draft_tokens,
                              const int32_t* verify_len, const float* temperature,
@@ -251,6 +257,21 @@ spec_status spec_shard_locate(spec_verify_ctx* ctx, int rank, int n_shards, cons
                               int64_t V, int32_t* token_votes, cudaStream_t stream);
 spec_status spec_shard_finish(spec_verify_ctx* ctx, const int32_t* token_votes_max, int B, int k,
                               int32_t* out_tokens, int32_t* out_redo, cudaStream_t stream);
+spec_status spec_shard_refine_partials(spec_verify_ctx* ctx, int rank, int n_shards,
+                                       const void* target_shard, const void* draft_shard,
+                                       spec_dtype dtype, const int32_t* draft_tokens,
+                                       const int32_t* verify_len, const float* temperature,
+                                       const spec_conf_args* conf, int B, int k, int64_t V,
+                                       void* block3, cudaStream_t stream);
+spec_status spec_shard_refine_locate(spec_verify_ctx* ctx, int rank, int n_shards,
+                                     const void* blocks3, const void* target_shard,
+                                     const void* draft_shard, spec_dtype dtype,
+                                     const int32_t* draft_tokens, const int32_t* verify_len,
+                                     const float* temperature, const spec_conf_args* conf, int B,
+                                     int k, int64_t V, int32_t* token_votes, cudaStream_t stream);
+spec_status spec_shard_refine_finish(spec_verify_ctx* ctx, const int32_t* token_votes_max, int B,
+                                     int k, int32_t* out_tokens, int32_t* out_redo,
+                                     cudaStream_t stream);
 
 /* spec_verify_run on HOST buffers: copies the inputs (pinned or pageable host
  * memory) to device staging owned by the context, verifies, copies the outputs

@@ -85,7 +85,10 @@ def lib():
     L.spec_verify_lengths.argtypes = [_vp, ctypes.POINTER(ConfArgs), _vp, _i32, _i32, _vp, _vp, _vp]
     shard_common = [_vp, _i32, _i32]
     shard_inputs = [_vp, _vp, _i32, _vp, _vp, _vp, ctypes.POINTER(ConfArgs), _i32, _i32, _i64]
-    L.spec_shard_layout.argtypes = [_i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp]
+    L.spec_shard_layout.argtypes = [_i32, _i32, _i64, _i32, _i32, _vp, _vp, _vp, _vp]
+    L.spec_shard_refine_partials.argtypes = shard_common + shard_inputs + [_vp, _vp]
+    L.spec_shard_refine_locate.argtypes = shard_common + [_vp] + shard_inputs + [_vp, _vp]
+    L.spec_shard_refine_finish.argtypes = [_vp, _vp, _i32, _i32, _vp, _vp, _vp]
     L.spec_shard_stats.argtypes = shard_common + shard_inputs + [_vp, _vp]
     L.spec_shard_decide.argtypes = shard_common + [_vp] + shard_inputs + [
         _u64, _u32, _u32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
@@ -103,7 +106,8 @@ def lib():
                  "spec_verify_run_with_uniforms", "spec_verify_run_host", "spec_verify_greedy",
                  "spec_conf_budget", "spec_verify_lengths", "spec_verify_greedy_noalloc",
                  "spec_shard_layout", "spec_shard_stats", "spec_shard_decide", "spec_shard_locate",
-                 "spec_shard_finish",
+                 "spec_shard_finish", "spec_shard_refine_partials", "spec_shard_refine_locate",
+                 "spec_shard_refine_finish",
                  "spec_verify_set_mode",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
@@ -422,14 +426,14 @@ def spec_verify_run_host(ctx: SpecVerifier, *a, **kw):
 # ----------------------------------------------------- vocabulary-parallel --
 
 def shard_layout(B, k, V, dtype, n_shards):
-    """Vocabulary split and exchange-block sizes: (bounds [n+1], block1 bytes,
-    block2 bytes).  Rank r holds tokens [bounds[r], bounds[r+1])."""
+    """Vocabulary split and exchange-block sizes: (bounds [n+1], block1, block2,
+    block3 bytes).  Rank r holds tokens [bounds[r], bounds[r+1])."""
     bounds = (_i64 * (n_shards + 1))()
-    b1, b2 = ctypes.c_size_t(), ctypes.c_size_t()
+    b1, b2, b3 = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     code = SPEC_BF16 if dtype == torch.bfloat16 else SPEC_F32
     _check(lib().spec_shard_layout(B, k, int(V), code, n_shards, bounds, ctypes.byref(b1),
-                                   ctypes.byref(b2)), "spec_shard_layout")
-    return list(bounds), b1.value, b2.value
+                                   ctypes.byref(b2), ctypes.byref(b3)), "spec_shard_layout")
+    return list(bounds), b1.value, b2.value, b3.value
 
 
 class ShardRank:
@@ -479,6 +483,32 @@ class ShardRank:
                "spec_shard_locate")
         del keep
 
+    def refine_partials(self, target, draft, tokens, V, block3, verify_len=None, temperature=None,
+                        conf=None, stream=None):
+        args, keep = self._inputs(target, draft, tokens, verify_len, temperature, conf, V)
+        _check(lib().spec_shard_refine_partials(self.ver._h, self.rank, self.n, *args, _dev_ptr(block3),
+                                                _stream_handle(stream, self.device)),
+               "spec_shard_refine_partials")
+        del keep
+
+    def refine_locate(self, blocks3, target, draft, tokens, V, votes, verify_len=None,
+                      temperature=None, conf=None, stream=None):
+        args, keep = self._inputs(target, draft, tokens, verify_len, temperature, conf, V)
+        _check(lib().spec_shard_refine_locate(self.ver._h, self.rank, self.n, _dev_ptr(blocks3),
+                                              *args, _dev_ptr(votes),
+                                              _stream_handle(stream, self.device)),
+               "spec_shard_refine_locate")
+        del keep
+
+    def refine_finish(self, votes_max, out, stream=None):
+        B, kp1 = out["tokens"].shape
+        redo = torch.empty(B, dtype=torch.int32, device=self.device)
+        _check(lib().spec_shard_refine_finish(self.ver._h, _dev_ptr(votes_max), B, kp1 - 1,
+                                              _dev_ptr(out["tokens"]), _dev_ptr(redo),
+                                              _stream_handle(stream, self.device)),
+               "spec_shard_refine_finish")
+        return redo
+
     def finish(self, votes_max, out, stream=None):
         B, kp1 = out["tokens"].shape
         redo = torch.empty(B, dtype=torch.int32, device=self.device)
@@ -495,7 +525,7 @@ def _redo_requests(ver, redo, rows_of, tokens, verify_len, temperature, conf, se
                    request_offset, out):
     """Requests flagged for an fp64 path: verified whole on their gathered rows
     (the single-rank path, same global request index and draws)."""
-    idx = torch.nonzero(redo.cpu()).flatten().tolist()
+    idx = torch.nonzero(redo.cpu() == 1).flatten().tolist()
     for i in idx:
         t_full, d_full = rows_of(i)
         sl = slice(i, i + 1)
@@ -520,7 +550,7 @@ def verify_vocab_parallel(rank_obj, target, draft, tokens, V, verify_len=None, t
     n, r = rank_obj.n, rank_obj.rank
     B, kp1, _ = target.shape
     k = kp1 - 1
-    bounds, b1, b2 = shard_layout(B, k, V, target.dtype, n)
+    bounds, b1, b2, b3 = shard_layout(B, k, V, target.dtype, n)
     dev = rank_obj.device
     blk1 = torch.empty(b1, dtype=torch.uint8, device=dev)
     all1 = torch.empty(n * b1, dtype=torch.uint8, device=dev)
@@ -537,6 +567,14 @@ def verify_vocab_parallel(rank_obj, target, draft, tokens, V, verify_len=None, t
     rank_obj.locate(all2, target, draft, tokens, V, votes, **kw)
     dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
     redo = rank_obj.finish(votes, out)
+    if bool((redo == 2).any()):  # the same on every rank: the decisions are replicated
+        blk3 = torch.empty(b3, dtype=torch.uint8, device=dev)
+        all3 = torch.empty(n * b3, dtype=torch.uint8, device=dev)
+        rank_obj.refine_partials(target, draft, tokens, V, blk3, **kw)
+        dist.all_gather_into_tensor(all3, blk3, group=group)
+        rank_obj.refine_locate(all3, target, draft, tokens, V, votes, **kw)
+        dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
+        redo = rank_obj.refine_finish(votes, out)
 
     widths = [bounds[q + 1] - bounds[q] for q in range(n)]
     wmax = max(widths)
@@ -563,11 +601,12 @@ def emulate_vocab_parallel(ranks, target, draft, tokens, verify_len=None, temper
     """The vocabulary-parallel protocol on ONE device: `ranks` are ShardRank
     objects (their own contexts), each given its slice of the full logits; the
     all-gathers become concatenations and the max a torch.max.  Returns
-    (outputs of every rank, final outputs, requests redone)."""
+    (outputs of every rank, final outputs, {"redone", "refined"} request lists,
+    the phase-3 votes)."""
     n = len(ranks)
     B, kp1, V = target.shape
     k = kp1 - 1
-    bounds, b1, b2 = shard_layout(B, k, V, target.dtype, n)
+    bounds, b1, b2, b3 = shard_layout(B, k, V, target.dtype, n)
     dev = ranks[0].device
     shards = [(target[:, :, bounds[r]:bounds[r + 1]].contiguous(),
                None if draft is None else draft[:, :, bounds[r]:bounds[r + 1]].contiguous())
@@ -587,9 +626,22 @@ def emulate_vocab_parallel(ranks, target, draft, tokens, verify_len=None, temper
     for r, rk in enumerate(ranks):
         rk.locate(all2, shards[r][0], shards[r][1], tokens, V, votes[r], **kw)
     vmax = votes.max(dim=0).values.contiguous()
-    redo = None
-    for r, rk in enumerate(ranks):
-        redo = rk.finish(vmax, outs[r])
+    redos = [rk.finish(vmax, outs[r]) for r, rk in enumerate(ranks)]
+    redo = redos[0]
+    refined = []
+    if bool((redo == 2).any()):
+        refined = torch.nonzero(redo == 2).flatten().tolist()
+        all3 = torch.empty(n * b3, dtype=torch.uint8, device=dev)
+        for r, rk in enumerate(ranks):
+            rk.refine_partials(shards[r][0], shards[r][1], tokens, V, all3[r * b3:(r + 1) * b3], **kw)
+        votes3 = torch.empty((n, B), dtype=torch.int32, device=dev)
+        for r, rk in enumerate(ranks):
+            rk.refine_locate(all3, shards[r][0], shards[r][1], tokens, V, votes3[r], **kw)
+        vmax3 = votes3.max(dim=0).values.contiguous()
+        redos = [rk.refine_finish(vmax3, outs[r]) for r, rk in enumerate(ranks)]
+        redo = redos[0]
+    for other in redos[1:]:
+        assert torch.equal(other, redo), "ranks disagree on the requests to redo"
     final = {key: v.clone() for key, v in outs[0].items()}
 
     def rows_of(i):
@@ -597,4 +649,4 @@ def emulate_vocab_parallel(ranks, target, draft, tokens, verify_len=None, temper
 
     redone = _redo_requests(ranks[0].ver, redo, rows_of, tokens, verify_len, temperature, conf,
                             seed, step, request_offset, final)
-    return outs, final, redone, votes
+    return outs, final, dict(redone=redone, refined=refined), votes

@@ -206,8 +206,16 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
       }
     }
   }
-  // sub-chunks whose support was not settled: recompute outright (rare)
-  if (sync_compute_or(flagged)) {
+  // sub-chunks whose support was not settled: recompute outright (rare).  A
+  // vocabulary shard holds only its own sub-chunks: the request is redone whole.
+  const bool sharded = p.c_hi > 0;
+  if (sharded) {
+    if (sync_compute_or(flagged)) {
+      if (threadIdx.x == 0) p.shard_tok[i] = -1;
+      sync_compute();
+      return;
+    }
+  } else if (sync_compute_or(flagged)) {
 #pragma unroll 1
     for (int ss = 0; ss < n_subs; ++ss) {
       const int owner = ss / 4;
@@ -261,6 +269,12 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     fallback = true;
   }
   const int sstar = sh.cstar;
+  if (sharded && sstar >= 0 &&
+      (sstar / kSubsPerChunk < p.c_lo || sstar / kSubsPerChunk >= p.c_hi)) {
+    if (threadIdx.x == 0) p.shard_tok[i] = -2;  // another rank holds the sub-chunk
+    sync_compute();
+    return;
+  }
   int token = -1;
   if (sstar >= 0) {
     const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
@@ -311,7 +325,9 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     }
     token = found >= 0 ? static_cast<int>(static_cast<int64_t>(c) * G::kChunk + found) : -1;
   }
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && sharded) {
+    p.shard_tok[i] = token >= 0 ? token : -1;
+  } else if (threadIdx.x == 0) {
     p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + jb.n] = token;
     if (token < 0) {
       p.out_acc[i] = -1;

@@ -17,11 +17,15 @@
 //
 // Shards are whole statistics segments, so the merged records are exactly the
 // whole-vocabulary run's: every decision, probability and token is identical.
-// The two fp64 paths (an accept draw inside its certified bound, a sample the
-// fp32 filter cannot certify) need every rank's logits; such a request is
-// flagged and redone whole after its rows are gathered.
+// A sample the fp32 filter cannot certify goes to the fp64 refinement, also
+// split by vocabulary (4. refine: every rank's fp64 partial sums over its own
+// sub-chunks -> exchange block 3; the rank holding the drawn sub-chunk scans
+// it).  The rare cases that need rows of other ranks -- an accept draw inside
+// its certified bound, a refinement whose support is not settled -- flag the
+// request, which is redone whole after its rows are gathered.
 #pragma once
 #include "common.cuh"
+#include "refine.cuh"
 #include "sample.cuh"
 #include "stats.cuh"
 
@@ -195,16 +199,106 @@ __global__ void __launch_bounds__(kThreads) k_shard_locate(RunParams p) {
   locate_sample<BF16>(p, i, jb, sa);
 }
 
+// Request states after each phase (p.fallback): 0 done or in progress, 1 redo
+// whole, 2 the sample needs the fp64 refinement.
+constexpr int32_t kShardRedo = 1, kShardRefine = 2;
+
 // Phase 3: the token agreed by the ranks (element-wise max of their answers:
-// the token, -1 to redo the request whole, -2 for "not here").
+// the token, -1 = not certified, -2 = not here).
 __global__ void k_shard_finish(RunParams p, const int32_t* tok_max) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x) {
     if (p.fallback[i]) continue;
     const int kind = __ldcg(&p.jobs[i].kind);
     if (kind == kJobNone) continue;
     const int32_t t = tok_max[i];
-    if (t >= 0) p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + __ldcg(&p.jobs[i].n)] = t;
-    else p.fallback[i] = 1;
+    if (t >= 0) {
+      p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + __ldcg(&p.jobs[i].n)] = t;
+    } else {
+      p.fallback[i] = kShardRefine;
+      p.refine_list[i] = i;  // refinement slot = request index
+    }
+  }
+}
+
+// Phase 4: fp64 partial sums of this rank's sub-chunks for the requests whose
+// sample needs the refinement (refinement slot = request index).
+struct alignas(16) RefRec {
+  double2 z;  // alpha, beta sums
+  double2 m;  // support masses A, B
+  int unc;    // logits of unsettled support
+  int pad[3];
+};
+static_assert(sizeof(RefRec) == 48, "exchange record layout");
+
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads) k_shard_refine_partials(RunParams p, int sub_lo, int nsub) {
+  __shared__ RefineShared rf;
+  exp2_table_init(rf.tab);
+  const int i = static_cast<int>(blockIdx.x / nsub);
+  const int ls = static_cast<int>(blockIdx.x % nsub);
+  if (__ldcg(p.fallback + i) != kShardRefine) return;
+  refine_item<BF16>(p, i, sub_lo + ls, rf);
+}
+
+__global__ void k_shard_pack_refine(RunParams p, int sub_lo, int nsub, int nsub_max, RefRec* out) {
+  const int n_subs = p.n_chunks * kSubsPerChunk;
+  const int64_t n = static_cast<int64_t>(p.B) * nsub_max;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(e / nsub_max), ls = static_cast<int>(e % nsub_max);
+    RefRec r{};
+    if (ls < nsub && p.fallback[i] == kShardRefine) {
+      const int64_t g = static_cast<int64_t>(i) * n_subs + sub_lo + ls;
+      r.z = p.rz[g];
+      r.m = p.rm[g];
+      r.unc = p.runc[g];
+    }
+    out[e] = r;
+  }
+}
+
+__global__ void k_shard_unpack_refine(RunParams p, ShardBounds sb, const RefRec* blocks, int nsub_max) {
+  const int n_subs = p.n_chunks * kSubsPerChunk;
+  const int64_t n = static_cast<int64_t>(p.B) * n_subs;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int i = static_cast<int>(e / n_subs), ss = static_cast<int>(e % n_subs);
+    if (p.fallback[i] != kShardRefine) continue;
+    const int seg = ss / (kSubsPerChunk * kChunksPerSeg);
+    int r = 0;
+    while (r + 1 < sb.n && seg >= sb.seg_lo[r + 1]) ++r;
+    const int ls = ss - sb.seg_lo[r] * kChunksPerSeg * kSubsPerChunk;
+    const RefRec* src = blocks + (static_cast<int64_t>(r) * p.B + i) * nsub_max + ls;
+    p.rz[e] = make_double2(__ldcg(&src->z.x), __ldcg(&src->z.y));
+    p.rm[e] = make_double2(__ldcg(&src->m.x), __ldcg(&src->m.y));
+    p.runc[e] = __ldcg(&src->unc);
+  }
+}
+
+// Phase 4: exact token of each refined request; the rank holding the drawn
+// sub-chunk scans it (votes as in phase 3, -1 = redo the request whole).
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads) k_shard_refine_locate(RunParams p) {
+  __shared__ RefineShared rf;
+  exp2_table_init(rf.tab);
+  const int i = blockIdx.x;
+  if (__ldcg(p.fallback + i) != kShardRefine) {
+    if (threadIdx.x == 0) p.shard_tok[i] = -2;
+    return;
+  }
+  refine_finalize<BF16>(p, i, rf);
+}
+
+__global__ void k_shard_refine_finish(RunParams p, const int32_t* tok_max) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x) {
+    if (p.fallback[i] != kShardRefine) continue;
+    const int32_t t = tok_max[i];
+    if (t >= 0) {
+      p.out_tok[static_cast<int64_t>(i) * (p.k + 1) + __ldcg(&p.jobs[i].n)] = t;
+      p.fallback[i] = 0;
+    } else {
+      p.fallback[i] = kShardRedo;
+    }
   }
 }
 

@@ -412,8 +412,8 @@ spec_status shard_geometry(int64_t V, bool bf16, int n_shards, sv::ShardBounds* 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct ShardSizes {
-  size_t rec_bytes, tok_off, block1, block2;
-  int nlc_max;
+  size_t rec_bytes, tok_off, block1, block2, block3;
+  int nlc_max, nsub_max;
 };
 
 ShardSizes shard_sizes(int B, int k, const sv::ShardBounds& sb) {
@@ -423,6 +423,8 @@ ShardSizes shard_sizes(int B, int k, const sv::ShardBounds& sb) {
   z.block1 = z.tok_off + align256(static_cast<size_t>(B) * k * 2 * sizeof(float));
   z.nlc_max = sb.nls_max * sv::kChunksPerSeg;
   z.block2 = static_cast<size_t>(B) * z.nlc_max * sizeof(sv::SampleChunk);
+  z.nsub_max = z.nlc_max * sv::kSubsPerChunk;
+  z.block3 = static_cast<size_t>(B) * z.nsub_max * sizeof(sv::RefRec);
   return z;
 }
 
@@ -470,6 +472,10 @@ spec_status shard_params(spec_verify_ctx* c, int rank, int n_shards, const void*
   p.smass = c->smass;
   p.tok_logits = c->tok_logits;
   p.fallback = c->fallback;
+  p.refine_list = c->refine_list;
+  p.rz = c->rz;
+  p.rm = c->rm;
+  p.runc = c->runc;
   p.counters = c->counters + (c->run_id & 1u);
   p.counters_next = c->counters + ((c->run_id + 1u) & 1u);
   *pp = p;
@@ -847,7 +853,8 @@ spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
 
 
 spec_status spec_shard_layout(int B, int k, int64_t V, spec_dtype dtype, int n_shards,
-                              int64_t* bounds, size_t* block1_bytes, size_t* block2_bytes) {
+                              int64_t* bounds, size_t* block1_bytes, size_t* block2_bytes,
+                              size_t* block3_bytes) {
   if (B < 1 || k < 0 || (dtype != SPEC_F32 && dtype != SPEC_BF16)) return SPEC_ERR_INVALID_ARG;
   sv::ShardBounds sb;
   int64_t segl = 0;
@@ -858,6 +865,7 @@ spec_status spec_shard_layout(int B, int k, int64_t V, spec_dtype dtype, int n_s
     for (int r = 0; r <= n_shards; ++r) bounds[r] = std::min<int64_t>(sb.seg_lo[r] * segl, V);
   if (block1_bytes) *block1_bytes = z.block1;
   if (block2_bytes) *block2_bytes = z.block2;
+  if (block3_bytes) *block3_bytes = z.block3;
   return SPEC_OK;
 }
 
@@ -987,8 +995,89 @@ spec_status spec_shard_finish(spec_verify_ctx* ctx, const int32_t* token_votes_m
   p.k = k;
   p.jobs = ctx->jobs;
   p.fallback = ctx->fallback;
+  p.refine_list = ctx->refine_list;
   p.out_tok = out_tokens;
   sv::k_shard_finish<<<grid_for(B), 256, 0, stream>>>(p, token_votes_max);
+  if (cudaMemcpyAsync(out_redo, ctx->fallback, static_cast<size_t>(B) * sizeof(int32_t),
+                      cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_refine_partials(spec_verify_ctx* ctx, int rank, int n_shards,
+                                       const void* target_shard, const void* draft_shard,
+                                       spec_dtype dtype, const int32_t* draft_tokens,
+                                       const int32_t* verify_len, const float* temperature,
+                                       const spec_conf_args* conf, int B, int k, int64_t V,
+                                       void* block3, cudaStream_t stream) {
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, rank, n_shards, target_shard, draft_shard, dtype,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  if (!block3 || !aligned(block3, 16)) return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  const ShardSizes z = shard_sizes(B, k, sb);
+  const int sub_lo = p.c_lo * sv::kSubsPerChunk;
+  const int nsub = (p.c_hi - p.c_lo) * sv::kSubsPerChunk;
+  if (nsub > 0) {
+    if (dtype == SPEC_BF16) sv::k_shard_refine_partials<true><<<B * nsub, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
+    else sv::k_shard_refine_partials<false><<<B * nsub, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
+  }
+  sv::k_shard_pack_refine<<<grid_for(static_cast<int64_t>(B) * z.nsub_max), 256, 0, stream>>>(
+      p, sub_lo, nsub, z.nsub_max, static_cast<sv::RefRec*>(block3));
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_refine_locate(spec_verify_ctx* ctx, int rank, int n_shards,
+                                     const void* blocks3, const void* target_shard,
+                                     const void* draft_shard, spec_dtype dtype,
+                                     const int32_t* draft_tokens, const int32_t* verify_len,
+                                     const float* temperature, const spec_conf_args* conf, int B,
+                                     int k, int64_t V, int32_t* token_votes, cudaStream_t stream) {
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, rank, n_shards, target_shard, draft_shard, dtype,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  if (!blocks3 || !token_votes || !aligned(blocks3, 16) || !aligned(token_votes, 4))
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  const ShardSizes z = shard_sizes(B, k, sb);
+  p.shard_tok = token_votes;
+  sv::k_shard_unpack_refine<<<grid_for(static_cast<int64_t>(B) * p.n_chunks * sv::kSubsPerChunk), 256, 0, stream>>>(
+      p, sb, static_cast<const sv::RefRec*>(blocks3), z.nsub_max);
+  if (dtype == SPEC_BF16) sv::k_shard_refine_locate<true><<<B, sv::kThreads, 0, stream>>>(p);
+  else sv::k_shard_refine_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_shard_refine_finish(spec_verify_ctx* ctx, const int32_t* token_votes_max, int B,
+                                     int k, int32_t* out_tokens, int32_t* out_redo,
+                                     cudaStream_t stream) {
+  if (!ctx || B < 1 || B > ctx->max_batch || k < 0 || k > ctx->max_k || !token_votes_max ||
+      !out_tokens || !out_redo)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  sv::RunParams p{};
+  p.B = B;
+  p.k = k;
+  p.jobs = ctx->jobs;
+  p.fallback = ctx->fallback;
+  p.out_tok = out_tokens;
+  sv::k_shard_refine_finish<<<grid_for(B), 256, 0, stream>>>(p, token_votes_max);
   if (cudaMemcpyAsync(out_redo, ctx->fallback, static_cast<size_t>(B) * sizeof(int32_t),
                       cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
     return SPEC_ERR_CUDA;

@@ -39,8 +39,8 @@ def _run(single, w, n):
         kw = dict(verify_len=w.get("verify_len"), temperature=w.get("temperature"), conf=w.get("conf"),
                   seed=w["seed"])
         ref = single.run(w["target"], w.get("draft"), w["tokens"], **kw)
-        outs, final, redone, votes = binding.emulate_vocab_parallel(ranks, w["target"], w.get("draft"),
-                                                                    w["tokens"], **kw)
+        outs, final, info, votes = binding.emulate_vocab_parallel(ranks, w["target"], w.get("draft"),
+                                                                  w["tokens"], **kw)
         torch.cuda.synchronize()
         # every rank reaches the same decisions before the token exchange
         for o in outs[1:]:
@@ -50,7 +50,7 @@ def _run(single, w, n):
         v = votes.cpu().numpy()
         assert np.all((v >= 0).sum(axis=0) <= 1)
         _check_equal(ref, final, "n=%d" % n)
-        return redone
+        return info
     finally:
         for r in ranks:
             r.close()
@@ -64,9 +64,11 @@ def test_stochastic_b64_matches_single_rank(single, n):
 
 def test_headline_two_ranks(single):
     w = workloads.headline("cuda", seed=1)
-    redone = _run(single, w, 2)
-    # the fp32 filter certifies most samples; the rest are redone whole
-    assert len(redone) < 64
+    info = _run(single, w, 2)
+    # the fp32 filter certifies most samples; the others go through the
+    # vocabulary-parallel fp64 refinement, and none needs a whole redo here
+    assert 0 < len(info["refined"]) < 64
+    assert len(info["redone"]) == 0
 
 
 def test_mixed_temperatures_and_greedy(single):
@@ -96,3 +98,11 @@ def test_confidence_head_and_errors(single):
 def test_layout_refuses_too_many_shards():
     with pytest.raises(binding.SpecVerifyError):
         binding.shard_layout(4, 2, 40000, torch.float32, 4)  # only 3 segments
+
+
+def test_refinement_three_ranks(single):
+    """The vocabulary-parallel fp64 refinement with the drawn sub-chunks spread
+    over three ranks (the headline batch: 18 uncertified samples)."""
+    w = workloads.headline("cuda", seed=1)
+    info = _run(single, w, 3)
+    assert len(info["refined"]) > 0 and len(info["redone"]) == 0
