@@ -138,7 +138,7 @@ __device__ void enqueue_sample(const RunParams& p, int i, unsigned* s_base) {
 // task decides.
 template <bool BF16>
 __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, StatsShared& st,
-                             DecideShared& dec, unsigned* s_base) {
+                             DecideShared& dec, unsigned* s_base, uint4* stage_buf) {
   const ReqInfo ri = request_info(p, i);
   const bool is_draft = slot > p.k;
   const int j = is_draft ? slot - (p.k + 1) : slot;
@@ -151,10 +151,10 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     const int64_t rec = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs + seg;
     const void* row = is_draft ? draft_row(p, i, j, BF16) : target_row(p, i, j, BF16);
     if (ri.greedy) {
-      greedy_segment<BF16>(row, p.V, seg, p.meta + rec, st);
+      greedy_segment_staged<BF16>(row, p.V, seg, p.meta + rec, st, stage_buf);
     } else {
       const float cc = static_cast<float>(1.4426950408889634 / static_cast<double>(ri.T));
-      stochastic_segment<BF16>(row, p.V, seg, cc, p.meta + rec, p.ssum + rec, st);
+      stochastic_segment_staged<BF16>(row, p.V, seg, cc, p.meta + rec, p.ssum + rec, st, stage_buf);
     }
   }
   unsigned expected;
@@ -188,9 +188,9 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
 
 template <bool BF16>
 __device__ void engine_sample(const RunParams& p, int i, int seg, SampleShared& sa,
-                              unsigned* s_base) {
+                              unsigned* s_base, uint4* stage_buf) {
   const Job jb = load_job(p.jobs + i);
-  segment_masses<BF16>(p, i, jb, seg, sa);
+  segment_masses_staged<BF16>(p, i, jb, seg, sa, stage_buf);
   if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_segs), &sa.flag)) return;
   __threadfence();
   locate_sample<BF16>(p, i, jb, sa);
@@ -214,6 +214,7 @@ __device__ void engine_refine(const RunParams& p, int slot, int sub, RefineShare
 
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams p) {
+  extern __shared__ __align__(16) uint4 stage_buf[];  // kStageBytes, per-thread staging
   __shared__ StatsShared st;
   __shared__ DecideShared dec;
   __shared__ SampleShared sa;
@@ -230,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
     const int a = static_cast<int>((it >> 14) & 0xFFFFu);
     const int b = static_cast<int>(it & 0x3FFFu);
     switch (it >> 30) {
-      case kItemStats: engine_stats<BF16>(p, a, b >> 8, b & 0xFF, st, dec, &s_base); break;
-      case kItemSample: engine_sample<BF16>(p, a, b, sa, &s_base); break;
+      case kItemStats: engine_stats<BF16>(p, a, b >> 8, b & 0xFF, st, dec, &s_base, stage_buf); break;
+      case kItemSample: engine_sample<BF16>(p, a, b, sa, &s_base, stage_buf); break;
       default: engine_refine<BF16>(p, a, b, rf); break;
     }
     __syncthreads();

@@ -15,6 +15,7 @@
 // fp64 rule defines them.
 #pragma once
 #include "common.cuh"
+#include "stage.cuh"
 #include "stats.cuh"
 
 namespace sv {
@@ -270,6 +271,90 @@ __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const 
       r.mass = m;
       // the bound was accumulated in fp32 per batch (inflate for its own
       // rounding), plus the pairwise rounding of the fp32 batch sums
+      r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
+      p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
+    }
+  }
+}
+
+// The same masses fed by per-thread asynchronous staging: step s of the
+// segment (chunk c0 + s / 4, batch s % 4) stages the target's two vectors in
+// slots 0-1 and the draft's in slots 2-3 (bonus jobs: the target's only).
+static_assert(2 * kVecsPerBatch == kStepVecs, "a staging step is one batch of both rows");
+
+template <bool BF16>
+__device__ __forceinline__ void stage_sample_step(Stager& sg, const void* ra, const void* rb,
+                                                  int64_t nvec, int c0, int s) {
+  using G = Geo<BF16>;
+  const int c = c0 + s / kBatchesPerChunk, b = s % kBatchesPerChunk;
+  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads;
+    const bool valid = idx < nvec;
+    cp_async16(sg.slot(s, u), static_cast<const uint4*>(ra) + (valid ? idx : 0), valid);
+    if (rb) cp_async16(sg.slot(s, kVecsPerBatch + u), static_cast<const uint4*>(rb) + (valid ? idx : 0), valid);
+  }
+  cp_async_commit();
+  ++sg.issued;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void segment_masses_staged(const RunParams& p, int i, const Job& jb, int seg,
+                                                      SampleShared& sh, uint4* stage_buf) {
+  using G = Geo<BF16>;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const JobF32 j = job_f32(jb);
+  const void* ra = target_row(p, i, jb.row, BF16);
+  const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
+  const int64_t nvec = p.V / G::kPerVec;
+  constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
+  const int c0 = seg * kChunksPerSeg;
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int st = 0; st < kStageSlots; ++st) stage_sample_step<BF16>(sg, ra, rb, nvec, c0, st);
+  double cmass = 0.0, cbound = 0.0;
+#pragma unroll 1
+  for (int st = 0; st < kSteps; ++st) {
+    cp_async_wait(sg.issued - st - 1);
+    const int c = c0 + st / kBatchesPerChunk, b = st % kBatchesPerChunk;
+    const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
+    uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+#pragma unroll
+    for (int u = 0; u < kVecsPerBatch; ++u) {
+      const bool valid = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads < nvec;
+      va[u] = valid ? *sg.slot(st, u) : neg_inf_vec<BF16>();
+      vb[u] = rb ? (valid ? *sg.slot(st, kVecsPerBatch + u) : neg_inf_vec<BF16>()) : va[u];
+    }
+    float sum, bound;
+    double unused;
+    batch_weights<BF16, false>(j, va, vb, sum, unused, bound);
+    cmass += static_cast<double>(sum);
+    cbound += static_cast<double>(bound);
+    if (st + kStageSlots < kSteps) stage_sample_step<BF16>(sg, ra, rb, nvec, c0, st + kStageSlots);
+    if ((st + 1) % kBatchesPerChunk == 0) {
+      const double m = warp_sum_d(cmass);
+      const double bb = warp_sum_d(cbound);
+      if (lane == 0) {
+        sh.cm[st / kBatchesPerChunk][warp] = m;
+        sh.cb[st / kBatchesPerChunk][warp] = bb;
+      }
+      cmass = 0.0;
+      cbound = 0.0;
+    }
+  }
+  sync_compute();
+  if (threadIdx.x < kChunksPerSeg) {
+    const int bc = threadIdx.x;
+    const int c = c0 + bc;
+    if (c < p.n_chunks) {
+      double m = 0.0, bb = 0.0;
+      for (int w2 = 0; w2 < kWarps; ++w2) {
+        m += sh.cm[bc][w2];
+        bb += sh.cb[bc][w2];
+      }
+      SampleChunk r;
+      r.mass = m;
       r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
       p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
     }

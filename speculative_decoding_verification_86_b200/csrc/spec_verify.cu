@@ -384,8 +384,8 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   if (n_init > 0xFFFF0000ull) return SPEC_ERR_INVALID_ARG;
   p.n_init = static_cast<unsigned>(n_init);
   timing_mark(c, kClassStats, true, s);
-  if (bf16) sv::k_engine<true><<<c->engine_grid, sv::kThreads, 0, s>>>(p);
-  else sv::k_engine<false><<<c->engine_grid, sv::kThreads, 0, s>>>(p);
+  if (bf16) sv::k_engine<true><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
+  else sv::k_engine<false><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
   timing_mark(c, kClassStats, false, s);
   if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
   return SPEC_OK;
@@ -533,10 +533,14 @@ spec_status spec_verify_init(spec_verify_ctx** out, int device, int max_batch, i
     return st;
   }
   int occ_a = 0, occ_b = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, sv::k_engine<true>, sv::kThreads, 0) !=
-          cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, sv::k_engine<false>, sv::kThreads, 0) !=
-          cudaSuccess) {
+  if (cudaFuncSetAttribute(sv::k_engine<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
+      cudaFuncSetAttribute(sv::k_engine<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, sv::k_engine<true>, sv::kThreads,
+                                                    sv::kStageBytes) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, sv::k_engine<false>, sv::kThreads,
+                                                    sv::kStageBytes) != cudaSuccess) {
     cudaFree(c->ws);
     delete c;
     return SPEC_ERR_CUDA;

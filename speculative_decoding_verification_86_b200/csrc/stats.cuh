@@ -19,6 +19,7 @@
 #pragma once
 #include "common.cuh"
 #include "philox.cuh"
+#include "stage.cuh"
 
 namespace sv {
 
@@ -266,6 +267,57 @@ __device__ __forceinline__ void stochastic_segment(const void* row, int64_t V, i
   soft_merge_block(acc, sh, meta_out, sum_out);
 }
 
+// The segment passes fed by per-thread asynchronous staging (stage.cuh):
+// batch b of the segment is staging step b, three steps in flight.  Thread t
+// gets the same vectors as from load_batch.
+static_assert(kBatchVecs == kStepVecs, "a staging step is one batch");
+
+__device__ __forceinline__ void stage_segment_batch(Stager& sg, const uint4* rv, int64_t nvec,
+                                                    int64_t seg0, int b) {
+#pragma unroll
+  for (int u = 0; u < kBatchVecs; ++u) {
+    const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
+    const bool valid = idx < nvec;
+    cp_async16(sg.slot(b, u), valid ? rv + idx : rv, valid);
+  }
+  cp_async_commit();
+  ++sg.issued;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void staged_batch(Stager& sg, int64_t nvec, int64_t seg0, int b,
+                                             uint4 (&v)[kBatchVecs]) {
+  cp_async_wait(sg.issued - b - 1);
+#pragma unroll
+  for (int u = 0; u < kBatchVecs; ++u) {
+    const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
+    v[u] = idx < nvec ? *sg.slot(b, u) : neg_inf_vec<BF16>();
+  }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void stochastic_segment_staged(const void* row, int64_t V, int seg, float cc,
+                                                          ChunkMeta* meta_out, double* sum_out,
+                                                          StatsShared& sh, uint4* stage_buf) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch(sg, rv, nvec, seg0, b);
+  SoftAcc acc;
+#pragma unroll 1
+  for (int b = 0; b < kBatches; ++b) {
+    uint4 v[kBatchVecs];
+    staged_batch<BF16>(sg, nvec, seg0, b, v);
+    soft_batch<BF16>(acc, v, cc);
+    // refill this step's slot once its values have been used
+    if (b + kStageSlots < kBatches) stage_segment_batch(sg, rv, nvec, seg0, b + kStageSlots);
+  }
+  soft_merge_block(acc, sh, meta_out, sum_out);
+}
+
 // Max and lowest arg-max of one segment of a greedy row: each thread keeps its
 // running maximum and the lowest index attaining it (batches arrive in index
 // order per thread), then the CTA reduces (larger value wins, ties go to the
@@ -352,6 +404,28 @@ __device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int s
     g.scan(va, seg0, b);
     if (b + 2 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 2, va);
     if (b + 1 < kBatches) g.scan(vb, seg0, b + 1);
+  }
+  g.finish(meta_out, sh);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void greedy_segment_staged(const void* row, int64_t V, int seg,
+                                                      ChunkMeta* meta_out, StatsShared& sh,
+                                                      uint4* stage_buf) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch(sg, rv, nvec, seg0, b);
+  GreedyScan<BF16> g;
+#pragma unroll 1
+  for (int b = 0; b < kBatches; ++b) {
+    uint4 v[kBatchVecs];
+    staged_batch<BF16>(sg, nvec, seg0, b, v);
+    g.scan(v, seg0, b);
+    if (b + kStageSlots < kBatches) stage_segment_batch(sg, rv, nvec, seg0, b + kStageSlots);
   }
   g.finish(meta_out, sh);
 }
