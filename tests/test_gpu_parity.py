@@ -408,3 +408,27 @@ def test_hand_worked_golden_cases(ver, dtype):
         assert g["status"][0] == 0, c["name"]
         assert g["accepted"][0] == c["n"], c["name"]
         assert g["tokens"][0].tolist() == c["out_tokens"].tolist(), c["name"]
+
+
+# --------------------------------------------------------- maximum sizes ----
+
+@pytest.mark.parametrize("dtype,V", [(torch.bfloat16, 2097152), (torch.float32, 1048576)])
+def test_maximum_block_and_vocabulary(cuda_device, dtype, V):
+    """k = 16 (the largest block) and the largest vocabulary a context takes
+    (2^21 logits; fp32 at half that to bound memory), B = 2, against the oracle."""
+    build.build()
+    g = torch.Generator(device="cuda").manual_seed(17)
+    B, k = 2, 16
+    target = (torch.randn(B, k + 1, V, generator=g, device="cuda") * 2.5).to(dtype)
+    draft = (0.9 * target[:, :k].float() + 0.5 * torch.randn(B, k, V, generator=g, device="cuda")).to(dtype)
+    # drafted tokens: the target's arg-max (accepted often, so the chain runs long)
+    tokens = target[:, :k].float().argmax(dim=2).to(torch.int32)
+    w = dict(target=target, draft=draft, tokens=tokens, verify_len=None, temperature=None, conf=None,
+             seed=21)
+    v = binding.SpecVerifier(cuda_device, max_batch=B, max_k=k, max_vocab=2097152)
+    try:
+        for mode in ("prefix", "dense"):
+            v.set_mode(mode)
+            compare(run_gpu(v, w), run_oracle(w))
+    finally:
+        v.close()
