@@ -289,8 +289,9 @@ spec_status spec_verify_run_host(spec_verify_ctx* ctx, const void* target_logits
 
 /* Per-kernel timing: launches of the kernel classes selected by `class_mask`
  * (bit c selects class c: 0 = the verification engine (statistics, chain,
- * sampling and fp64 refinement in one launch), 1 and 2 = unused, 3 =
- * confidence head; 0 turns timing off) are
+ * sampling and fp64 refinement in one launch), 1 = the LM head's statistics
+ * GEMM, 2 = the LM head's row-writing GEMM, 3 = confidence head; 0 turns
+ * timing off) are
  * bracketed by CUDA events on the caller's stream.  spec_verify_timing_read
  * synchronises on those events and returns, for class `which`, the number of
  * launches and their total milliseconds since timing was last enabled (enabling
@@ -315,6 +316,69 @@ spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
  * the kernels assume; the measured maximum must not exceed it. */
 spec_status spec_verify_selfcheck_ex2(int device, float lo, float hi, double* max_rel_err);
 double spec_verify_ex2_error_bound(void);
+
+/* ---------------------------------------------------------------------------
+ * LM head with verification fused into its epilogue.
+ *
+ * The drafter shares the target's frozen output head ("Speculative decoding
+ * becomes standard: DSpark and multi-token drafters", section "What DSpark
+ * adds"), so the logits of every verified row are l = h W^T with one bf16
+ * matrix W [V, H]: target rows from the target's last hidden states, drafter
+ * rows from the drafter's.  These entry points take the hidden states instead
+ * of logits.  The GEMM runs on the tensor cores (tcgen05, bf16 operands, fp32
+ * accumulation); the logits are the fp32 accumulator values.
+ *
+ * spec_lmhead_verify computes exactly what spec_verify_run (dtype SPEC_F32,
+ * dense order) computes on the logits [B, k+1, V] = hidden_target W^T and
+ * [B, k, V] = hidden_draft W^T, without writing those logits: the GEMM's
+ * epilogue reduces each accumulator tile to the row statistics and picks the
+ * drafted tokens' logits; after the accept chains only the rows a request
+ * samples from (the rejected pair, or the bonus row) are written, as fp32
+ * logits, and the sample is drawn from them with the vocabulary-parallel
+ * protocol's phases run as a single shard.  Outputs and random draws are those
+ * of spec_verify_run.
+ * --------------------------------------------------------------------------- */
+typedef struct spec_lmhead_ctx spec_lmhead_ctx;
+
+/* Create the LM-head workspace for verification context `vctx` (which must
+ * outlive it and is used by it: one stream at a time for both).  Sizes follow
+ * vctx's max_batch, max_k and max_vocab, and max_hidden (a multiple of 8, at
+ * most 65536): about max_batch * (2 max_k + 1) * (4 max_vocab + 2 max_hidden)
+ * bytes of device memory. */
+spec_status spec_lmhead_init(spec_lmhead_ctx** ctx, spec_verify_ctx* vctx, int max_hidden);
+spec_status spec_lmhead_destroy(spec_lmhead_ctx* ctx);
+
+/* logits [rows, V] fp32 (row-major, caller-owned, 16-byte aligned) =
+ * hidden [rows, H] bf16 (row-major, 16-byte aligned) x head [V, H] bf16
+ * (row-major, 16-byte aligned)^T.  H a multiple of 8 (<= max_hidden), V a
+ * multiple of 4 (<= max_vocab).  Asynchronous on `stream`. */
+spec_status spec_lmhead_logits(spec_lmhead_ctx* ctx, const void* hidden, int rows,
+                               const void* head, int H, int64_t V, float* out_logits,
+                               cudaStream_t stream);
+
+/* Fused verification.  hidden_target [B, k+1, H] bf16 and hidden_draft
+ * [B, k, H] bf16 (NULL iff no sampled request verifies a position) are the
+ * last hidden states of the two models, head [V, H] bf16 the shared output
+ * head; every other argument and output is that of spec_verify_run.
+ * out_redo [B] (device) receives 0 for every request whose outputs are final,
+ * or 1 for a request whose decision needs rows this pass did not produce (an
+ * accept draw inside its certified fp32 bound, or a refined sample whose
+ * support stayed unsettled -- about one in 10^5 decisions): its outputs are to
+ * be recomputed, e.g. spec_lmhead_logits of its rows then spec_verify_run with
+ * request_offset + i.  Asynchronous on `stream`. */
+spec_status spec_lmhead_verify(spec_lmhead_ctx* ctx, const void* hidden_target,
+                               const void* hidden_draft, const void* head, int H,
+                               const int32_t* draft_tokens, const int32_t* verify_len,
+                               const float* temperature, const spec_conf_args* conf, int B, int k,
+                               int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                               int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                               float* out_q, uint32_t* out_status, int32_t* out_redo,
+                               cudaStream_t stream);
+
+/* Error word of the LM-head kernels since the context was created
+ * (synchronises the device): bit 0 set = a wait inside a GEMM timed out and
+ * that launch's outputs are not to be used. */
+spec_status spec_lmhead_errors(spec_lmhead_ctx* ctx, uint32_t* out);
 
 const char* spec_status_string(spec_status s);
 

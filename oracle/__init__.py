@@ -154,6 +154,34 @@ def conf_budget(hidden: np.ndarray, w: np.ndarray, bias: float, threshold: float
     return out_len, surv, pref
 
 
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) widened exactly to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+    return b.view(np.float32).astype(np.float64)
+
+
+def lmhead_logits(hidden: np.ndarray, head: np.ndarray) -> np.ndarray:
+    """Logits of the shared output head, l = h W^T ("Speculative decoding
+    becomes standard: DSpark and multi-token drafters", section "What DSpark
+    adds": the drafter shares the target's frozen output head), in fp64 from
+    the bf16 inputs: hidden [..., H] and head [V, H] as uint16 bits ->
+    float64 [..., V].  One library matmul is the whole step; every product of
+    two bf16 values is exact in fp64."""
+    h = bf16_to_f64(hidden)
+    w = bf16_to_f64(head)
+    return h @ w.T
+
+
+def verify_lmhead(hidden_target, hidden_draft, head, draft_tokens, **kw):
+    """Verification of the rows the shared head produces: the fp64 logits of
+    ``lmhead_logits`` rounded to fp32 (the precision the fused path holds its
+    accumulators in; on inputs whose partial sums are exact in fp32 the
+    rounding is exact too), then ``verify`` with dtype fp32."""
+    t = lmhead_logits(hidden_target, head).astype(np.float32)
+    d = None if hidden_draft is None else lmhead_logits(hidden_draft, head).astype(np.float32)
+    return verify(t, d, draft_tokens, dtype=DTYPE_F32, **kw)
+
+
 def row_softmax(row: np.ndarray, dtype: int, T: float) -> np.ndarray:
     row = np.ascontiguousarray(row)
     out = np.zeros(row.shape[-1], dtype=np.float64)

@@ -37,7 +37,7 @@ DEV_NONFINITE = 2
 DEV_BAD_TEMPERATURE = 4
 DEV_INTERNAL = 16
 
-TIMING_ENGINE, TIMING_CONF = 0, 3
+TIMING_ENGINE, TIMING_LM_STATS, TIMING_LM_ROWS, TIMING_CONF = 0, 1, 2, 3
 TIMING_STATS = TIMING_ENGINE
 
 
@@ -94,6 +94,13 @@ def lib():
         _u64, _u32, _u32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_shard_locate.argtypes = shard_common + [_vp] + shard_inputs + [_vp, _vp]
     L.spec_shard_finish.argtypes = [_vp, _vp, _i32, _i32, _vp, _vp, _vp]
+    L.spec_lmhead_init.argtypes = [ctypes.POINTER(_vp), _vp, _i32]
+    L.spec_lmhead_destroy.argtypes = [_vp]
+    L.spec_lmhead_errors.argtypes = [_vp, ctypes.POINTER(_u32)]
+    L.spec_lmhead_logits.argtypes = [_vp, _vp, _i32, _vp, _i32, _i64, _vp, _vp]
+    L.spec_lmhead_verify.argtypes = [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
+                                     ctypes.POINTER(ConfArgs), _i32, _i32, _i64, _u64, _u32, _u32,
+                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_verify_set_mode.argtypes = [_vp, _i32]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
@@ -108,6 +115,8 @@ def lib():
                  "spec_shard_layout", "spec_shard_stats", "spec_shard_decide", "spec_shard_locate",
                  "spec_shard_finish", "spec_shard_refine_partials", "spec_shard_refine_locate",
                  "spec_shard_refine_finish",
+                 "spec_lmhead_init", "spec_lmhead_destroy", "spec_lmhead_errors",
+                 "spec_lmhead_logits", "spec_lmhead_verify",
                  "spec_verify_set_mode",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
@@ -650,3 +659,90 @@ def emulate_vocab_parallel(ranks, target, draft, tokens, verify_len=None, temper
     redone = _redo_requests(ranks[0].ver, redo, rows_of, tokens, verify_len, temperature, conf,
                             seed, step, request_offset, final)
     return outs, final, dict(redone=redone, refined=refined), votes
+
+
+class LmHeadVerifier:
+    """The LM head with verification fused into its epilogue
+    (spec_lmhead_*): takes the two models' last hidden states and the shared
+    output head instead of logits.  Uses (and must not outlive) ``ver``."""
+
+    def __init__(self, ver: SpecVerifier, max_hidden=4096):
+        self.ver = ver
+        self.device = ver.device
+        self.max_hidden = max_hidden
+        h = _vp()
+        _check(lib().spec_lmhead_init(ctypes.byref(h), ver._h, int(max_hidden)), "spec_lmhead_init")
+        self._h = h
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().spec_lmhead_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def errors(self):
+        out = _u32(0)
+        _check(lib().spec_lmhead_errors(self._h, ctypes.byref(out)), "spec_lmhead_errors")
+        return int(out.value)
+
+    def logits(self, hidden, head, stream=None, out=None):
+        """fp32 logits [..., V] = hidden [..., H] (bf16) x head [V, H] (bf16)^T."""
+        H = hidden.shape[-1]
+        V = head.shape[0]
+        rows = hidden.numel() // H
+        if tuple(head.shape) != (V, H):
+            raise ValueError("head must be [V, H] with H = %d" % H)
+        if out is None:
+            out = torch.empty(tuple(hidden.shape[:-1]) + (V,), dtype=torch.float32, device=self.device)
+        st = lib().spec_lmhead_logits(self._h, _dev_ptr(hidden, torch.bfloat16, self.device, "hidden"),
+                                      rows, _dev_ptr(head, torch.bfloat16, self.device, "head"), H, V,
+                                      _dev_ptr(out, torch.float32, self.device, "out"),
+                                      _stream_handle(stream, self.device))
+        _check(st, "spec_lmhead_logits")
+        return out
+
+    def verify(self, hidden_target, hidden_draft, head, tokens, verify_len=None, temperature=None,
+               conf=None, seed=0, step=0, request_offset=0, stream=None, out=None, redo_whole=True):
+        """spec_lmhead_verify; with ``redo_whole`` the (rare) requests it
+        flags are verified again on their full rows (spec_lmhead_logits, then
+        the single-context path).  Returns the outputs of spec_verify_run,
+        plus "redo" [B] int32."""
+        B, kp1, H = hidden_target.shape
+        k = kp1 - 1
+        V = head.shape[0]
+        if hidden_draft is not None and tuple(hidden_draft.shape) != (B, k, H):
+            raise ValueError("hidden_draft must be [B, k, H] = %s" % ((B, k, H),))
+        if tuple(tokens.shape) != (B, k):
+            raise ValueError("draft tokens must be [B, k] = %s" % ((B, k),))
+        o = self.ver._outputs(B, k, True, out)
+        redo = o.get("redo")
+        if redo is None:
+            redo = o["redo"] = torch.empty(B, dtype=torch.int32, device=self.device)
+        cref, _keep = self.ver._conf(conf)
+        st = lib().spec_lmhead_verify(
+            self._h, _dev_ptr(hidden_target, torch.bfloat16, self.device, "hidden_target"),
+            _dev_ptr(hidden_draft, torch.bfloat16, self.device, "hidden_draft"),
+            _dev_ptr(head, torch.bfloat16, self.device, "head"), H,
+            _dev_ptr(tokens, torch.int32, self.device, "tokens"),
+            _dev_ptr(verify_len, torch.int32, self.device, "verify_len"),
+            _dev_ptr(temperature, torch.float32, self.device, "temperature"), cref, B, k, V,
+            int(seed), int(step), int(request_offset),
+            _dev_ptr(o["accepted"], torch.int32), _dev_ptr(o["tokens"], torch.int32),
+            _dev_ptr(o.get("p")), _dev_ptr(o.get("q")), _dev_ptr(o["status"]),
+            _dev_ptr(redo, torch.int32), _stream_handle(stream, self.device))
+        _check(st, "spec_lmhead_verify")
+        if redo_whole:
+            def rows_of(i):
+                t = self.logits(hidden_target[i:i + 1], head, stream)
+                d = None if hidden_draft is None else self.logits(hidden_draft[i:i + 1], head, stream)
+                return t, d
+
+            keys = {key: o[key] for key in o if key != "redo"}
+            _redo_requests(self.ver, redo, rows_of, tokens, verify_len, temperature, conf, seed,
+                           step, request_offset, keys)
+        return o

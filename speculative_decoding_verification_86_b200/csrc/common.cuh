@@ -166,6 +166,7 @@ struct RunParams {
   int32_t* fallback;       // [B]: set when a decision needs rows held by other ranks
   int32_t* shard_tok;      // [B]: located token, -1 to redo the request whole, -2 not here
   int c_lo, c_hi;          // chunks whose logits the buffers hold (c_hi = 0: all)
+  int rows_whole;          // the protocol runs as one shard over complete rows in memory
 
   // engine
   int mode;                        // kModeDense / kModePrefix

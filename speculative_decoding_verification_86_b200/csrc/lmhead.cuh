@@ -1,0 +1,653 @@
+// The target's LM head with the verification's row statistics in its epilogue.
+//
+// The drafter shares the target's frozen output head ("Speculative decoding
+// becomes standard: DSpark and multi-token drafters", section "What DSpark
+// adds"), so every verified row -- target position j, or drafter position j --
+// has logits l = h W^T with the same W [V, H].  Verification needs of most rows
+// only their softmax statistics and one logit (the drafted token's), so the
+// GEMM's epilogue reduces each accumulator tile straight into the statistics
+// records the accept chain merges; the logits never reach HBM.  Only the rows
+// a request samples from (the rejected pair, or the bonus row) are produced as
+// logits, by the same kernel in its row-writing mode, after the chain decided.
+//
+// Kernel: one CTA per SM, persistent over work units (128 rows x a run of
+// 128 x 256 tiles along the vocabulary).  Warp roles:
+//   warp 0     TMA producer: A (hidden rows, 128 x 64 bf16) and B (W rows,
+//              256 x 64 bf16) tiles, 128-byte swizzle, 4-stage ring;
+//   warp 1     TMEM owner (512 columns: two 128 x 256 fp32 accumulators) and
+//              MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
+//              M = 128, N = 256, K = 16 per instruction, one thread;
+//   warps 2-5  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, so each
+//              thread owns one row of the tile and walks its 256 columns in
+//              batches of 16 (tcgen05.ld 32x32b.x16), while the MMA warp fills
+//              the other accumulator.
+// Every wait on an mbarrier is bounded in time; a wait that runs out raises
+// the CTA's abort flag and the error word, drains what this CTA issued, frees
+// TMEM and returns.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "stats.cuh"
+
+namespace sv {
+
+constexpr int kLmBM = 128;  // rows per tile (UMMA M)
+constexpr int kLmBN = 256;  // vocabulary columns per tile (UMMA N)
+constexpr int kLmBK = 64;   // hidden elements per stage: one 128-byte swizzle row of bf16
+constexpr int kLmUK = 16;   // K of one kind::f16 instruction
+constexpr int kLmStages = 4;
+constexpr uint32_t kLmABytes = kLmBM * kLmBK * 2;  // 16 KB
+constexpr uint32_t kLmBBytes = kLmBN * kLmBK * 2;  // 32 KB
+constexpr uint32_t kLmStageBytes = kLmABytes + kLmBBytes;
+constexpr int kLmThreads = 192;
+constexpr uint32_t kLmTmemCols = 2 * kLmBN;
+// A work unit covers `part_tiles` N tiles (a power of two up to kLmSegTiles);
+// the statistics records of a unit ("parts") then tile the fp32 statistics
+// segment exactly.
+constexpr int kLmSegTiles = SegGeo<false>::kSeg / kLmBN;  // 64 tiles per statistics segment
+static_assert(SegGeo<false>::kSeg % kLmBN == 0, "tiles divide the fp32 statistics segment");
+constexpr size_t kLmBarrierBytes = 256;
+constexpr size_t kLmSmemBytes = 1024 + kLmStages * kLmStageBytes + kLmBarrierBytes;
+constexpr unsigned long long kLmWaitNs = 2000000000ull;  // 2 s: legitimate waits are microseconds
+
+constexpr int kLmModeStats = 0;  // epilogue -> statistics partial records + token logits
+constexpr int kLmModeRows = 1;   // epilogue -> fp32 logits of listed rows
+
+// Statistics of one row over one part (the columns of one work unit): the
+// fields of a segment record before the parts are merged.
+struct alignas(16) LmPart {
+  float K;     // stochastic: integer exponent frame (-inf: nothing finite)
+  float mraw;  // raw maximum
+  float er;    // stochastic: sum e |a_then|
+  float w;     // stochastic: om; greedy: lowest arg-max (int bits)
+  double s;    // stochastic: sum of 2^(l c - K) terms
+  int bad;     // NaN or +inf seen
+  int pad;
+};
+static_assert(sizeof(LmPart) == 32, "part record layout");
+
+struct LmParams {
+  int mode;
+  int H;
+  int64_t V;
+  int rows0, rows1;       // rows of A matrix 0 (target) and 1 (drafter); rows mode: rows0 = max rows
+  const int* rows_dev;    // rows mode: the row count on the device (nullptr: rows0)
+  // statistics mode
+  int B, k;
+  const int32_t* tokens;  // [B, k]
+  const float* temp;      // [B] or nullptr (1.0)
+  LmPart* parts;          // [rows0 + rows1, n_parts]
+  int n_parts;
+  int part_tiles;         // N tiles per work unit (both modes)
+  float* tok_logits;      // [B, k, 2] (target, drafter)
+  // rows mode
+  const int64_t* dst;     // per row: element offset of its logits in `out` (-1: skip); nullptr: row * V
+  float* out;
+  unsigned* error;        // bit 1: a wait timed out
+};
+
+// ------------------------------------------------------------ PTX helpers --
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long lm_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `parity` to complete.  Gives up (false) when another
+// role raised *abort, or after kLmWaitNs, raising *abort and the error word.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned* error) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = lm_now();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (lm_now() - t0 > kLmWaitNs) {
+        *abort = 1;
+        atomicOr(error, 1u);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ void tma_prefetch(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+// 2-D tiled TMA load (no multicast): box at (x = hidden offset, y = row).
+__device__ __forceinline__ void tma_load(void* dst, const CUtensorMap* m, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_addr(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: 8-row groups 1024 bytes apart (stride byte offset), the
+// leading byte offset unused for swizzled K-major layouts, descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kLmIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                              (static_cast<uint32_t>(kLmBN >> 3) << 17) |
+                              (static_cast<uint32_t>(kLmBM >> 4) << 24);
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kLmIdesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` once every tcgen05 operation this thread issued has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_addr(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------- work division --
+struct LmWork {
+  int mt0, n_mt, n_nt, pt, n_parts, units, n_kb;
+  __device__ LmWork(int rows0, int rows1, int64_t V, int H, int part_tiles) {
+    mt0 = (rows0 + kLmBM - 1) / kLmBM;
+    n_mt = mt0 + (rows1 + kLmBM - 1) / kLmBM;
+    n_nt = static_cast<int>((V + kLmBN - 1) / kLmBN);
+    pt = part_tiles;
+    n_parts = (n_nt + pt - 1) / pt;
+    units = n_mt * n_parts;
+    n_kb = (H + kLmBK - 1) / kLmBK;
+  }
+  // unit u: M tile u % n_mt, part u / n_mt (the CTAs at work at one time share W columns)
+  __device__ int mt(int u) const { return u % n_mt; }
+  __device__ int part(int u) const { return u / n_mt; }
+  __device__ int nt_lo(int u) const { return part(u) * pt; }
+  __device__ int nt_hi(int u) const { return min(nt_lo(u) + pt, n_nt); }
+};
+
+struct LmShared {
+  uint64_t full[kLmStages];
+  uint64_t empty[kLmStages];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t drain;
+  uint32_t tmem;
+  int abort;
+  int rows0;
+};
+static_assert(sizeof(LmShared) <= kLmBarrierBytes, "barrier block");
+
+// ---------------------------------------------------------------- epilogue --
+// Per-thread row state of the statistics mode.
+struct LmRowState {
+  bool valid = false;
+  bool greedy = false;
+  bool draft = false;
+  int i = 0, j = 0;
+  int64_t tok = -1;
+  float cc = 1.0f;
+  SoftAcc acc;
+  float best = -INFINITY;
+  int best_idx = INT_MAX;
+  int gbad = 0;
+};
+
+__device__ __forceinline__ void lm_row_init(const LmParams& p, int mt, int mt0, int r_in_tile,
+                                            LmRowState& st) {
+  st = LmRowState();
+  const bool draft = mt >= mt0;
+  const int r = (draft ? mt - mt0 : mt) * kLmBM + r_in_tile;
+  const int rows = draft ? p.rows1 : p.rows0;
+  if (r >= rows) return;
+  st.valid = true;
+  st.draft = draft;
+  if (draft) {
+    st.i = r / p.k;
+    st.j = r - st.i * p.k;
+  } else {
+    st.i = r / (p.k + 1);
+    st.j = r - st.i * (p.k + 1);
+  }
+  if (st.j < p.k) st.tok = __ldg(p.tokens + static_cast<int64_t>(st.i) * p.k + st.j);
+  float T = p.temp ? __ldg(p.temp + st.i) : 1.0f;
+  if (!temperature_valid(T)) T = 1.0f;  // the chain reports the request; any record will do
+  st.greedy = T == 0.0f;
+  if (!st.greedy) st.cc = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+}
+
+// 16 consecutive logits of the thread's row, starting at column `col`.
+__device__ __forceinline__ void lm_consume_stats(const LmParams& p, LmRowState& st,
+                                                 const uint32_t (&r)[16], int64_t col) {
+  const int64_t nvalid = p.V - col;  // >= 1
+  if (st.tok >= col && st.tok < col + 16) {
+    float x = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (col + q == st.tok) x = __uint_as_float(r[q]);
+    p.tok_logits[(static_cast<int64_t>(st.i) * p.k + st.j) * 2 + (st.draft ? 1 : 0)] = x;
+  }
+  if (st.greedy) {
+    float bm = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (q < nvalid) bm = fmax_nan(bm, __uint_as_float(r[q]));
+    if (isnan(bm)) st.gbad = 1;
+    if (bm > st.best || st.best_idx == INT_MAX) {
+      int first = INT_MAX;
+#pragma unroll
+      for (int q = 15; q >= 0; --q)
+        if (q < nvalid && __uint_as_float(r[q]) == bm) first = static_cast<int>(col) + q;
+      if (first != INT_MAX) {
+        st.best = bm;
+        st.best_idx = first;
+      }
+    }
+    return;
+  }
+  uint4 v[kBatchVecs];
+#pragma unroll
+  for (int u = 0; u < kBatchVecs; ++u) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w[e] = (4 * u + e) < nvalid ? r[4 * u + e] : 0xff800000u;
+    v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  soft_batch<false>(st.acc, v, st.cc);
+}
+
+__device__ __forceinline__ void lm_write_part(const LmParams& p, const LmRowState& st, int mt,
+                                              int mt0, int r_in_tile, int part) {
+  const bool draft = mt >= mt0;
+  const int r = (draft ? mt - mt0 : mt) * kLmBM + r_in_tile;
+  const int64_t g = draft ? static_cast<int64_t>(p.rows0) + r : r;
+  LmPart o;
+  if (st.greedy) {
+    o.K = 0.0f;
+    o.mraw = st.best;
+    o.er = 0.0f;
+    o.w = __int_as_float(st.best_idx == INT_MAX ? -1 : st.best_idx);
+    o.s = 0.0;
+    o.bad = st.gbad;
+  } else {
+    o.K = st.acc.K;
+    o.mraw = st.acc.mraw;
+    o.er = st.acc.er;
+    o.w = st.acc.om;
+    o.s = st.acc.s;
+    o.bad = st.acc.bad;
+  }
+  o.pad = 0;
+  p.parts[g * p.n_parts + part] = o;
+}
+
+__device__ __forceinline__ void lm_consume_rows(const LmParams& p, int64_t dst,
+                                                const uint32_t (&r)[16], int64_t col) {
+  float* o = p.out + dst + col;
+  if (col + 16 <= p.V) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      reinterpret_cast<uint4*>(o)[u] = make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 16; ++q)
+      if (col + q < p.V) o[q] = __uint_as_float(r[q]);
+  }
+}
+
+// ------------------------------------------------------------------ roles --
+__device__ __forceinline__ void lm_producer(const LmParams& p, const LmWork& w, LmShared& sh,
+                                            uint8_t* stages, const CUtensorMap* ma0,
+                                            const CUtensorMap* ma1, const CUtensorMap* mw) {
+  uint32_t g = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; ok && u < w.units; u += gridDim.x) {
+    const int mt = w.mt(u);
+    const CUtensorMap* ma = mt < w.mt0 ? ma0 : ma1;
+    const int arow = (mt < w.mt0 ? mt : mt - w.mt0) * kLmBM;
+    for (int nt = w.nt_lo(u); ok && nt < w.nt_hi(u); ++nt) {
+      for (int kb = 0; kb < w.n_kb; ++kb, ++g) {
+        const int s = static_cast<int>(g % kLmStages);
+        const uint32_t ph = (g / kLmStages) & 1u;
+        if (!mbar_wait(&sh.empty[s], ph ^ 1u, &sh.abort, p.error)) {
+          ok = false;
+          break;
+        }
+        uint8_t* a = stages + static_cast<size_t>(s) * kLmStageBytes;
+        mbar_expect_tx(&sh.full[s], kLmStageBytes);
+        tma_load(a, ma, &sh.full[s], kb * kLmBK, arow);
+        tma_load(a + kLmABytes, mw, &sh.full[s], kb * kLmBK, nt * kLmBN);
+      }
+    }
+  }
+  if (!ok) {
+    // drain: the loads this thread issued land before the CTA's memory goes away
+    for (uint32_t q = g > kLmStages ? g - kLmStages : 0; q < g; ++q) {
+      volatile int no_abort = 0;
+      mbar_wait(&sh.full[q % kLmStages], (q / kLmStages) & 1u, &no_abort, p.error);
+    }
+  }
+}
+
+__device__ __forceinline__ void lm_mma(const LmParams& p, const LmWork& w, LmShared& sh,
+                                       uint8_t* stages) {
+  uint32_t g = 0, t = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; ok && u < w.units; u += gridDim.x) {
+    for (int nt = w.nt_lo(u); ok && nt < w.nt_hi(u); ++nt, ++t) {
+      const uint32_t a = t & 1u;
+      if (!mbar_wait(&sh.tempty[a], ((t >> 1) & 1u) ^ 1u, &sh.abort, p.error)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d = sh.tmem + a * kLmBN;
+      for (int kb = 0; kb < w.n_kb; ++kb, ++g) {
+        const int s = static_cast<int>(g % kLmStages);
+        if (!mbar_wait(&sh.full[s], (g / kLmStages) & 1u, &sh.abort, p.error)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_addr(stages + static_cast<size_t>(s) * kLmStageBytes);
+        const uint64_t adesc = sw128_desc(sa);
+        const uint64_t bdesc = sw128_desc(sa + kLmABytes);
+#pragma unroll
+        for (int kk = 0; kk < kLmBK / kLmUK; ++kk) {
+          // advance along K inside the swizzled 128-byte rows: 32 bytes per step
+          umma_bf16(d, adesc + 2 * kk, bdesc + 2 * kk, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&sh.empty[s]);  // the stage is free once these MMAs have read it
+      }
+      if (ok) umma_commit(&sh.tfull[a]);
+    }
+  }
+  if (!ok) {  // every MMA issued so far completes before TMEM is released
+    umma_commit(&sh.drain);
+    volatile int no_abort = 0;
+    mbar_wait(&sh.drain, 0, &no_abort, p.error);
+  }
+}
+
+__device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork& w, LmShared& sh) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3;  // TMEM lanes this warp may read
+  const int r_in_tile = quarter * 32 + lane;
+  uint32_t t = 0;
+  for (int u = blockIdx.x; u < w.units; u += gridDim.x) {
+    const int mt = w.mt(u);
+    LmRowState st;
+    int64_t dst = -1;
+    if (p.mode == kLmModeStats) {
+      lm_row_init(p, mt, w.mt0, r_in_tile, st);
+    } else {
+      const int r = mt * kLmBM + r_in_tile;
+      if (r < sh.rows0) dst = p.dst ? __ldg(p.dst + r) : static_cast<int64_t>(r) * p.V;
+    }
+    for (int nt = w.nt_lo(u); nt < w.nt_hi(u); ++nt, ++t) {
+      const uint32_t a = t & 1u;
+      // every lane waits (bounded), then the warp votes: it leaves together,
+      // and stays converged for the .sync.aligned TMEM loads
+      const bool ready = mbar_wait(&sh.tfull[a], (t >> 1) & 1u, &sh.abort, p.error);
+      if (!__all_sync(0xffffffffu, ready)) return;
+      tc_fence_after();
+      const uint32_t taddr = sh.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * kLmBN;
+#pragma unroll 1
+      for (int c = 0; c < kLmBN; c += 32) {
+        uint32_t v0[16], v1[16];
+        tmem_ld16(taddr + c, v0);
+        tmem_ld16(taddr + c + 16, v1);
+        tmem_ld_wait();
+        const int64_t col = static_cast<int64_t>(nt) * kLmBN + c;
+        if (col < p.V) {
+          if (p.mode == kLmModeStats) {
+            if (st.valid) lm_consume_stats(p, st, v0, col);
+          } else if (dst >= 0) {
+            lm_consume_rows(p, dst, v0, col);
+          }
+        }
+        if (col + 16 < p.V) {
+          if (p.mode == kLmModeStats) {
+            if (st.valid) lm_consume_stats(p, st, v1, col + 16);
+          } else if (dst >= 0) {
+            lm_consume_rows(p, dst, v1, col + 16);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.tempty[a]);
+    }
+    if (p.mode == kLmModeStats && st.valid)
+      lm_write_part(p, st, mt, w.mt0, r_in_tile, w.part(u));
+  }
+}
+
+__global__ void __launch_bounds__(kLmThreads, 1)
+    k_lmhead(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUtensorMap ma1,
+             const __grid_constant__ CUtensorMap mw, LmParams p) {
+  extern __shared__ uint8_t lm_smem[];
+  const uint32_t pad = (1024u - (smem_addr(lm_smem) & 1023u)) & 1023u;
+  uint8_t* stages = lm_smem + pad;  // 1024-byte aligned: the swizzle atoms of every stage
+  LmShared& sh = *reinterpret_cast<LmShared*>(stages + kLmStages * kLmStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kLmStages; ++s) {
+      mbar_init(&sh.full[s], 1);
+      mbar_init(&sh.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sh.tfull[a], 1);
+      mbar_init(&sh.tempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&sh.drain, 1);
+    sh.abort = 0;
+    int rows0 = p.rows0;
+    if (p.mode == kLmModeRows && p.rows_dev) rows0 = max(0, min(__ldcg(p.rows_dev), p.rows0));
+    sh.rows0 = rows0;
+    mbar_init_fence();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&ma0);
+    tma_prefetch(&ma1);
+    tma_prefetch(&mw);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_addr(&sh.tmem)),
+                 "r"(kLmTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const LmWork w(sh.rows0, p.mode == kLmModeStats ? p.rows1 : 0, p.V, p.H, p.part_tiles);
+  if (warp == 0) {
+    if (lane == 0) lm_producer(p, w, sh, stages, &ma0, &ma1, &mw);
+  } else if (warp == 1) {
+    if (lane == 0) lm_mma(p, w, sh, stages);
+  } else {
+    lm_epilogue(p, w, sh);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sh.tmem),
+                 "r"(kLmTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------ side kernels --
+// Merge the parts of every (request, row slot, statistics segment) into the
+// segment record the accept chain reads (the same merge as across a CTA's
+// threads: rebase to the largest frame, then add).
+__global__ void k_lm_combine(RunParams p, const LmPart* parts, int n_parts, int parts_per_seg,
+                             int rows0) {
+  const int rows = 2 * p.k + 1;
+  const int64_t n = static_cast<int64_t>(p.B) * rows * p.n_segs;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int seg = static_cast<int>(e % p.n_segs);
+    const int64_t rs = e / p.n_segs;
+    const int i = static_cast<int>(rs / rows);
+    const int slot = static_cast<int>(rs - static_cast<int64_t>(i) * rows);
+    const int64_t g = slot <= p.k ? static_cast<int64_t>(i) * (p.k + 1) + slot
+                                  : rows0 + static_cast<int64_t>(i) * p.k + (slot - p.k - 1);
+    float T = p.temp ? __ldg(p.temp + i) : 1.0f;
+    if (!temperature_valid(T)) T = 1.0f;
+    const int q0 = seg * parts_per_seg, q1 = min(q0 + parts_per_seg, n_parts);
+    const LmPart* src = parts + g * n_parts;
+    ChunkMeta r;
+    if (T == 0.0f) {
+      float best = -INFINITY;
+      int arg = INT_MAX, bad = 0;
+      for (int q = q0; q < q1; ++q) {
+        const LmPart c = src[q];
+        bad |= c.bad;
+        const int a = __float_as_int(c.w);
+        if (a >= 0 && (c.mraw > best || (c.mraw == best && a < arg))) {
+          best = c.mraw;
+          arg = a;
+        }
+      }
+      r.K = 0.0f;
+      r.mraw = bad ? __int_as_float(0x7fc00000) : best;
+      r.err = 0.0f;
+      r.arg = arg == INT_MAX ? -1 : arg;
+      p.meta[e] = r;
+      continue;
+    }
+    float K = -INFINITY, mraw = -INFINITY;
+    int bad = 0;
+    for (int q = q0; q < q1; ++q) {
+      const LmPart c = src[q];
+      bad |= c.bad;
+      K = fmaxf(K, c.K);
+      mraw = fmax_nan(mraw, c.mraw);
+    }
+    double s = 0.0;
+    float er = 0.0f, om = 0.0f;
+    if (!bad && K > -INFINITY) {
+      for (int q = q0; q < q1; ++q) {
+        const LmPart c = src[q];
+        if (!(c.K > -INFINITY)) continue;
+        const double f = pow2_exact(c.K - K);
+        const float ff = static_cast<float>(f);
+        s += c.s * f;
+        er += c.er * ff;
+        om += (c.w + (K - c.K) * static_cast<float>(c.s)) * ff;
+      }
+    }
+    if (bad || isnan(mraw) || mraw == INFINITY) {
+      r.K = __int_as_float(0x7fc00000);
+      p.ssum[e] = __longlong_as_double(0x7ff8000000000000LL);
+    } else {
+      r.K = K;
+      p.ssum[e] = K == -INFINITY ? 0.0 : s;
+    }
+    r.mraw = mraw;
+    r.err = er;
+    r.arg = __float_as_int(om);
+    p.meta[e] = r;
+  }
+}
+
+// After the chain: the rows each request samples from (the rejected pair, or
+// the bonus row), listed for the row-writing GEMM.  src: the hidden row (target
+// rows first, then the drafter's, as the statistics pass numbers them); dst:
+// the element offset of the row's logits in the row buffer, laid out as
+// [B, k+1, V] target rows followed by [B, k, V] drafter rows.
+__global__ void k_lm_rowlist(RunParams p, int* count, int* src, int64_t* dst) {
+  const int rows0 = p.B * (p.k + 1);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < p.B; i += gridDim.x * blockDim.x) {
+    if (__ldcg(p.fallback + i)) continue;
+    const int kind = __ldcg(&p.jobs[i].kind);
+    if (kind == kJobNone) continue;
+    const int j = __ldcg(&p.jobs[i].row);
+    const int n = kind == kJobResidual ? 2 : 1;
+    const int at = atomicAdd(count, n);
+    const int rt = i * (p.k + 1) + j;
+    src[at] = rt;
+    dst[at] = static_cast<int64_t>(rt) * p.V;
+    if (n == 2) {
+      const int rd = i * p.k + j;
+      src[at + 1] = rows0 + rd;
+      dst[at + 1] = (static_cast<int64_t>(rows0) + rd) * p.V;
+    }
+  }
+}
+
+// Copy the listed hidden rows (H bf16, 16-byte vectors) into one compact matrix.
+__global__ void k_lm_gather(const int* count, const int* src, const uint4* hid_t, const uint4* hid_d,
+                            int rows0, int H, int max_rows, uint4* out) {
+  const int n = min(max(__ldcg(count), 0), max_rows);
+  const int hv = H / 8;
+  const int64_t total = static_cast<int64_t>(n) * hv;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(e / hv), c = static_cast<int>(e % hv);
+    const int s = __ldcg(src + r);
+    const uint4* from = s < rows0 ? hid_t + static_cast<int64_t>(s) * hv
+                                  : hid_d + static_cast<int64_t>(s - rows0) * hv;
+    out[e] = __ldg(from + c);
+  }
+}
+
+}  // namespace sv

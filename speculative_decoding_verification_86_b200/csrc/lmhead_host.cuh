@@ -1,0 +1,316 @@
+// Host side of the LM-head entry points (included at the end of
+// spec_verify.cu, whose argument checks and launch helpers it uses): the
+// context's buffers, the TMA tensor maps, and the launch sequence of the fused
+// verification -- statistics GEMM, part merge, accept chain, sampled rows,
+// then the vocabulary-parallel protocol's sample and refinement phases run
+// with a single shard.
+#include <cudaTypedefs.h>
+
+#include "lmhead.cuh"
+
+struct spec_lmhead_ctx {
+  spec_verify_ctx* vctx = nullptr;
+  int max_hidden = 0;
+  int max_rows = 0;  // max_batch * (2 max_k + 1)
+  int max_parts = 0;
+  void* ws = nullptr;
+  sv::LmPart* parts = nullptr;  // [max_rows, max_parts]
+  float* rows = nullptr;        // [max_rows, max_vocab] fp32: logits of the sampled rows
+  uint4* hc = nullptr;          // [max_rows, max_hidden] bf16: their hidden states
+  int* src = nullptr;           // [max_rows]
+  int64_t* dst = nullptr;       // [max_rows]
+  int* count = nullptr;
+  int32_t* votes = nullptr;     // [max_batch]
+  unsigned* error = nullptr;
+};
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, H] as 2-D tiles of box_rows x 64 (128 bytes,
+// the 128-byte swizzle); out-of-range rows and columns read as zero.
+bool bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int H, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc || rows < 1) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(sv::kLmBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int lm_tiles(int64_t V) { return static_cast<int>((V + sv::kLmBN - 1) / sv::kLmBN); }
+int lm_parts(int64_t V, int part_tiles) { return (lm_tiles(V) + part_tiles - 1) / part_tiles; }
+
+// Smallest statistics part the kernel is given (largest record count).
+constexpr int kLmMinPartTiles = 2;
+
+// Work-unit width of the statistics GEMM: the largest of 16, 8, 4, 2 tiles
+// whose unit count comes within 2% of filling its last wave as well as the
+// best of them (a wider unit writes fewer records).
+int lm_stats_part_tiles(int n_mt, int64_t V, int grid) {
+  double best = 0.0;
+  double eff[4];
+  const int cand[4] = {16, 8, 4, kLmMinPartTiles};
+  for (int q = 0; q < 4; ++q) {
+    const int64_t units = static_cast<int64_t>(n_mt) * lm_parts(V, cand[q]);
+    const int64_t waves = (units + grid - 1) / grid;
+    eff[q] = static_cast<double>(units) / static_cast<double>(waves * grid);
+    best = std::max(best, eff[q]);
+  }
+  for (int q = 0; q < 4; ++q)
+    if (eff[q] >= best - 0.02) return cand[q];
+  return kLmMinPartTiles;
+}
+
+int lm_grid(const spec_lmhead_ctx* lm, int64_t units) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, lm->vctx->num_sms)));
+}
+
+spec_status lm_check(const spec_lmhead_ctx* lm, int H, int64_t V, const void* head) {
+  if (!lm || !head || H < 8 || H > lm->max_hidden || V < 1 || V > lm->vctx->max_vocab)
+    return SPEC_ERR_INVALID_ARG;
+  if (H % 8 != 0 || V % 4 != 0 || !aligned(head, 16)) return SPEC_ERR_UNSUPPORTED;
+  return SPEC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+spec_status spec_lmhead_init(spec_lmhead_ctx** out, spec_verify_ctx* vctx, int max_hidden) {
+  if (!out) return SPEC_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!vctx || max_hidden < 8 || max_hidden > 65536 || max_hidden % 8 != 0)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(vctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  if (!tensor_map_encoder()) return SPEC_ERR_UNSUPPORTED;
+  auto* lm = new (std::nothrow) spec_lmhead_ctx();
+  if (!lm) return SPEC_ERR_NOMEM;
+  lm->vctx = vctx;
+  lm->max_hidden = max_hidden;
+  lm->max_rows = vctx->max_batch * (2 * vctx->max_k + 1);
+  lm->max_parts = lm_parts(vctx->max_vocab, kLmMinPartTiles);
+  const size_t R = static_cast<size_t>(lm->max_rows);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes, 256);
+    return at;
+  };
+  const size_t o_parts = take(R * lm->max_parts * sizeof(sv::LmPart));
+  const size_t o_rows = take(R * static_cast<size_t>(vctx->max_vocab) * sizeof(float));
+  const size_t o_hc = take(R * static_cast<size_t>(max_hidden) * 2);
+  const size_t o_src = take(R * sizeof(int));
+  const size_t o_dst = take(R * sizeof(int64_t));
+  const size_t o_cnt = take(sizeof(int));
+  const size_t o_votes = take(static_cast<size_t>(vctx->max_batch) * sizeof(int32_t));
+  const size_t o_err = take(sizeof(unsigned));
+  if (cudaMalloc(&lm->ws, off) != cudaSuccess) {
+    cudaGetLastError();
+    delete lm;
+    return SPEC_ERR_NOMEM;
+  }
+  char* b = static_cast<char*>(lm->ws);
+  lm->parts = reinterpret_cast<sv::LmPart*>(b + o_parts);
+  lm->rows = reinterpret_cast<float*>(b + o_rows);
+  lm->hc = reinterpret_cast<uint4*>(b + o_hc);
+  lm->src = reinterpret_cast<int*>(b + o_src);
+  lm->dst = reinterpret_cast<int64_t*>(b + o_dst);
+  lm->count = reinterpret_cast<int*>(b + o_cnt);
+  lm->votes = reinterpret_cast<int32_t*>(b + o_votes);
+  lm->error = reinterpret_cast<unsigned*>(b + o_err);
+  if (cudaMemset(lm->ws, 0, off) != cudaSuccess ||
+      cudaFuncSetAttribute(sv::k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sv::kLmSmemBytes)) != cudaSuccess) {
+    cudaFree(lm->ws);
+    delete lm;
+    return SPEC_ERR_CUDA;
+  }
+  *out = lm;
+  return SPEC_OK;
+}
+
+spec_status spec_lmhead_destroy(spec_lmhead_ctx* lm) {
+  if (!lm) return SPEC_OK;
+  DeviceGuard g(lm->vctx->device);
+  cudaDeviceSynchronize();
+  cudaFree(lm->ws);
+  delete lm;
+  return SPEC_OK;
+}
+
+spec_status spec_lmhead_errors(spec_lmhead_ctx* lm, uint32_t* out) {
+  if (!lm || !out) return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(lm->vctx->device);
+  if (cudaDeviceSynchronize() != cudaSuccess) return SPEC_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, lm->error, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return SPEC_ERR_CUDA;
+  *out = h;
+  return SPEC_OK;
+}
+
+spec_status spec_lmhead_logits(spec_lmhead_ctx* lm, const void* hidden, int rows, const void* head,
+                               int H, int64_t V, float* out_logits, cudaStream_t stream) {
+  if (spec_status st = lm_check(lm, H, V, head); st != SPEC_OK) return st;
+  if (rows < 1 || !hidden || !out_logits) return SPEC_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(out_logits, 16)) return SPEC_ERR_UNSUPPORTED;
+  DeviceGuard g(lm->vctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  CUtensorMap ma, mw;
+  if (!bf16_tile_map(&ma, hidden, rows, H, sv::kLmBM) || !bf16_tile_map(&mw, head, V, H, sv::kLmBN))
+    return SPEC_ERR_UNSUPPORTED;
+  sv::LmParams p{};
+  p.mode = sv::kLmModeRows;
+  p.H = H;
+  p.V = V;
+  p.rows0 = rows;
+  p.out = out_logits;
+  p.error = lm->error;
+  p.part_tiles = 1;  // no records: single-tile units balance the waves best
+  const int64_t units = static_cast<int64_t>((rows + sv::kLmBM - 1) / sv::kLmBM) * lm_tiles(V);
+  timing_mark(lm->vctx, kClassLmRows, true, stream);
+  sv::k_lmhead<<<lm_grid(lm, units), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(ma, ma, mw, p);
+  timing_mark(lm->vctx, kClassLmRows, false, stream);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
+                               const void* hidden_draft, const void* head, int H,
+                               const int32_t* draft_tokens, const int32_t* verify_len,
+                               const float* temperature, const spec_conf_args* conf, int B, int k,
+                               int64_t V, uint64_t seed, uint32_t step, uint32_t request_offset,
+                               int32_t* out_accepted, int32_t* out_tokens, float* out_p,
+                               float* out_q, uint32_t* out_status, int32_t* out_redo,
+                               cudaStream_t stream) {
+  if (spec_status st = lm_check(lm, H, V, head); st != SPEC_OK) return st;
+  spec_verify_ctx* ctx = lm->vctx;
+  if (B < 1 || B > ctx->max_batch || k < 0 || k > ctx->max_k || !hidden_target || !out_accepted ||
+      !out_tokens || !out_redo || (k > 0 && !draft_tokens))
+    return SPEC_ERR_INVALID_ARG;
+  if (!aligned(hidden_target, 16) || (hidden_draft && !aligned(hidden_draft, 16)))
+    return SPEC_ERR_UNSUPPORTED;
+  const int rows0 = B * (k + 1), rows1 = hidden_draft ? B * k : 0;
+  float* rows_t = lm->rows;
+  float* rows_d = lm->rows + static_cast<int64_t>(rows0) * V;
+  sv::RunParams p;
+  sv::ShardBounds sb;
+  int64_t segl = 0;
+  if (spec_status st = shard_params(ctx, 0, 1, rows_t, hidden_draft ? rows_d : nullptr, SPEC_F32,
+                                    draft_tokens, verify_len, temperature, conf, B, k, V, &p, &sb,
+                                    &segl);
+      st != SPEC_OK)
+    return st;
+  const int rows = 2 * k + 1;
+  if (static_cast<int64_t>(B) * rows * p.n_segs >
+      static_cast<int64_t>(ctx->max_batch) * (2 * ctx->max_k + 1) * ctx->max_chunks)
+    return SPEC_ERR_INVALID_ARG;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  CUtensorMap ma0, ma1, mw, mc;
+  if (!bf16_tile_map(&ma0, hidden_target, rows0, H, sv::kLmBM) ||
+      (rows1 > 0 && !bf16_tile_map(&ma1, hidden_draft, rows1, H, sv::kLmBM)) ||
+      !bf16_tile_map(&mw, head, V, H, sv::kLmBN) ||
+      !bf16_tile_map(&mc, lm->hc, static_cast<int64_t>(B) * rows, H, sv::kLmBM))
+    return SPEC_ERR_UNSUPPORTED;
+  if (rows1 == 0) ma1 = ma0;
+  p.rows_whole = 1;  // sampled rows are materialised in full before the sample phases
+  p.seed = seed;
+  p.step = step;
+  p.req_off = request_offset;
+  p.out_acc = out_accepted;
+  p.out_tok = out_tokens;
+  p.out_p = out_p;
+  p.out_q = out_q;
+  p.out_status = out_status;
+  const int n_mt1 = (rows0 + sv::kLmBM - 1) / sv::kLmBM + (rows1 + sv::kLmBM - 1) / sv::kLmBM;
+  const int part_tiles = lm_stats_part_tiles(n_mt1, V, ctx->num_sms);
+  const int n_parts = lm_parts(V, part_tiles);
+  if (conf) launch_conf(ctx, conf, B, k, verify_len, ctx->conf_len, nullptr, stream);
+  if (k > 0 && cudaMemsetAsync(ctx->tok_logits, 0, static_cast<size_t>(B) * k * 2 * sizeof(float),
+                               stream) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  if (cudaMemsetAsync(lm->count, 0, sizeof(int), stream) != cudaSuccess) return SPEC_ERR_CUDA;
+
+  // 1. statistics of every verified row, straight from the accumulators
+  sv::LmParams lp{};
+  lp.mode = sv::kLmModeStats;
+  lp.H = H;
+  lp.V = V;
+  lp.rows0 = rows0;
+  lp.rows1 = rows1;
+  lp.B = B;
+  lp.k = k;
+  lp.tokens = draft_tokens;
+  lp.temp = temperature;
+  lp.parts = lm->parts;
+  lp.n_parts = n_parts;
+  lp.part_tiles = part_tiles;
+  lp.tok_logits = ctx->tok_logits;
+  lp.error = lm->error;
+  const int64_t units1 = static_cast<int64_t>(n_mt1) * n_parts;
+  timing_mark(ctx, kClassLmStats, true, stream);
+  sv::k_lmhead<<<lm_grid(lm, units1), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(ma0, ma1, mw, lp);
+  timing_mark(ctx, kClassLmStats, false, stream);
+  sv::k_lm_combine<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
+      p, lm->parts, n_parts, sv::kLmSegTiles / part_tiles, rows0);
+
+  // 2. the accept chains (every request, dense order)
+  sv::k_shard_decide<false><<<B, sv::kThreads, 0, stream>>>(p);
+
+  // 3. logits of the rows each request samples from
+  sv::k_lm_rowlist<<<grid_for(B), 256, 0, stream>>>(p, lm->count, lm->src, lm->dst);
+  sv::k_lm_gather<<<grid_for(static_cast<int64_t>(2) * B * (H / 8)), 256, 0, stream>>>(
+      lm->count, lm->src, static_cast<const uint4*>(hidden_target),
+      static_cast<const uint4*>(hidden_draft ? hidden_draft : hidden_target), rows0, H, B * rows,
+      lm->hc);
+  sv::LmParams lr{};
+  lr.mode = sv::kLmModeRows;
+  lr.H = H;
+  lr.V = V;
+  lr.rows0 = 2 * B;  // at most a row pair per request
+  lr.rows_dev = lm->count;
+  lr.dst = lm->dst;
+  lr.out = lm->rows;
+  lr.error = lm->error;
+  lr.part_tiles = 1;
+  const int64_t units2 = static_cast<int64_t>((2 * B + sv::kLmBM - 1) / sv::kLmBM) * lm_tiles(V);
+  timing_mark(ctx, kClassLmRows, true, stream);
+  sv::k_lmhead<<<lm_grid(lm, units2), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(mc, mc, mw, lr);
+  timing_mark(ctx, kClassLmRows, false, stream);
+
+  // 4. sample: chunk masses, locate and certify, fp64 refinement where needed
+  sv::k_shard_masses<false><<<B * p.n_segs, sv::kThreads, 0, stream>>>(p, 0, p.n_segs);
+  p.shard_tok = lm->votes;
+  sv::k_shard_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
+  sv::k_shard_finish<<<grid_for(B), 256, 0, stream>>>(p, lm->votes);
+  const int nsub = p.n_chunks * sv::kSubsPerChunk;
+  sv::k_shard_refine_partials<false><<<B * nsub, sv::kThreads, 0, stream>>>(p, 0, nsub);
+  sv::k_shard_refine_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
+  sv::k_shard_refine_finish<<<grid_for(B), 256, 0, stream>>>(p, lm->votes);
+  if (cudaMemcpyAsync(out_redo, ctx->fallback, static_cast<size_t>(B) * sizeof(int32_t),
+                      cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+    return SPEC_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+}  // extern "C"

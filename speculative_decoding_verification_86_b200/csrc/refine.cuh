@@ -209,7 +209,7 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
   // sub-chunks whose support was not settled: recompute outright (rare).  A
   // vocabulary shard holds only its own sub-chunks: the request is redone whole.
   const bool sharded = p.c_hi > 0;
-  if (sharded) {
+  if (sharded && !p.rows_whole) {
     if (sync_compute_or(flagged)) {
       if (threadIdx.x == 0) p.shard_tok[i] = -1;
       sync_compute();

@@ -233,10 +233,10 @@ static_assert(sizeof(RefRec) == 48, "exchange record layout");
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) k_shard_refine_partials(RunParams p, int sub_lo, int nsub) {
   __shared__ RefineShared rf;
-  exp2_table_init(rf.tab);
   const int i = static_cast<int>(blockIdx.x / nsub);
   const int ls = static_cast<int>(blockIdx.x % nsub);
-  if (__ldcg(p.fallback + i) != kShardRefine) return;
+  if (__ldcg(p.fallback + i) != kShardRefine) return;  // (uniform over the CTA)
+  exp2_table_init(rf.tab);
   refine_item<BF16>(p, i, sub_lo + ls, rf);
 }
 
@@ -280,12 +280,12 @@ __global__ void k_shard_unpack_refine(RunParams p, ShardBounds sb, const RefRec*
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) k_shard_refine_locate(RunParams p) {
   __shared__ RefineShared rf;
-  exp2_table_init(rf.tab);
   const int i = blockIdx.x;
-  if (__ldcg(p.fallback + i) != kShardRefine) {
+  if (__ldcg(p.fallback + i) != kShardRefine) {  // (uniform over the CTA)
     if (threadIdx.x == 0) p.shard_tok[i] = -2;
     return;
   }
+  exp2_table_init(rf.tab);
   refine_finalize<BF16>(p, i, rf);
 }
 

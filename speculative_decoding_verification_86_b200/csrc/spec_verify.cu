@@ -31,7 +31,9 @@ namespace {
 // require it to stay at or below this bound.
 constexpr float kEpsEx2 = 1.5e-7f;
 
-constexpr int kClassStats = 0, kClassConf = 3;  // timing classes (1, 2: unused)
+// timing classes: the verification kernel, the LM head's statistics and
+// row-writing GEMMs, the confidence head
+constexpr int kClassStats = 0, kClassLmStats = 1, kClassLmRows = 2, kClassConf = 3;
 constexpr int kTimingClasses = 4;
 constexpr int kMaxTimed = 4096;
 
@@ -322,7 +324,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   const int segl = bf16 ? sv::SegGeo<true>::kSeg : sv::SegGeo<false>::kSeg;
   const int n_segs = static_cast<int>((V + segl - 1) / segl);
 
-  sv::RunParams p;
+  sv::RunParams p{};
   p.target = target;
   p.draft = force_greedy ? nullptr : draft;
   p.tokens = tokens;
@@ -1088,3 +1090,5 @@ spec_status spec_shard_refine_finish(spec_verify_ctx* ctx, const int32_t* token_
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
 }  // extern "C"
+
+#include "lmhead_host.cuh"

@@ -170,6 +170,47 @@ def sweep(device="cpu", seed=4, B=128, k=5, V=VOCAB_QWEN):
 
 SWEEP_BATCHES = (1, 8, 32, 128, 512, 1024)
 
+HIDDEN_QWEN3_4B = 2560
+
+
+def lmhead(device="cpu", seed=5, B=256, k=5, V=VOCAB_QWEN, H=HIDDEN_QWEN3_4B, grid=False,
+           temperature=None, verify_len=None, w_levels=1):
+    """Inputs of verification fused into the shared LM head: the two models'
+    last hidden states and the output head W [V, H] (the drafter shares the
+    target's head), all bf16.
+
+    Real-valued recipe: target hidden h_t ~ N(0, 1); drafter hidden
+    h_d = 0.8 h_t + 0.6 N(0, 1); W ~ N(0, (3 / sqrt(H))^2), so logits have a
+    standard deviation near 3 and the two models' rows are correlated, as in
+    the logit recipes.  ``grid=True`` draws instead small integers times powers
+    of two (h_t in {-3..3}/4, h_d = clamp(round(0.8 h_t + N(0, 0.6^2)))/4,
+    W in {-w_levels..w_levels}/8): every product and every partial sum of h W^T
+    is then exact in fp32, so the logits do not depend on summation order.
+    Drafted tokens are sampled from the drafter's own logits (fp32 matmul of
+    the bf16 inputs) at each request's temperature."""
+    g = _gen(device, seed)
+    if grid:
+        ht = torch.randint(-3, 4, (B, k + 1, H), generator=g, device=device).float()
+        hd = torch.clamp(torch.round(0.8 * ht[:, :k] + 0.6 * _normal((B, k, H), 1.0, g, device)), -3, 3)
+        W = torch.randint(-w_levels, w_levels + 1, (V, H), generator=g, device=device).float()
+        ht, hd, W = ht * 0.25, hd * 0.25, W * 0.125
+    else:
+        ht = _normal((B, k + 1, H), 1.0, g, device)
+        hd = 0.8 * ht[:, :k] + 0.6 * _normal((B, k, H), 1.0, g, device)
+        W = _normal((V, H), 3.0 / math.sqrt(H), g, device)
+    ht, hd, W = ht.to(torch.bfloat16), hd.to(torch.bfloat16), W.to(torch.bfloat16)
+    tokens = torch.empty((B, k), dtype=torch.int32, device=device)
+    Wt = W.float().T
+    for lo in range(0, B, 16):
+        hi = min(B, lo + 16)
+        d = hd[lo:hi].float() @ Wt
+        t = None if temperature is None else temperature[lo:hi]
+        tokens[lo:hi] = _draft_tokens(d, t, g, device)
+    return dict(hidden_target=ht.contiguous(), hidden_draft=hd.contiguous(), head=W.contiguous(),
+                tokens=tokens, verify_len=verify_len, temperature=temperature, conf=None,
+                seed=seed, name="LM-head fused B=%d k=%d V=%d H=%d%s" % (B, k, V, H,
+                                                                        " (exact grid)" if grid else ""))
+
 
 def to_numpy_inputs(w):
     """Host copies in the oracle's formats (bf16 as raw uint16 bits)."""
