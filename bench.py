@@ -12,7 +12,13 @@ per second (sum of L_i over the batch / step time), plus the HBM bandwidth
 the step sustains.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload headline|stochastic|greedy|conf|conf_budget|sweep:B]
+                  [--workload headline|stochastic|greedy|conf|conf_budget|sweep:B|lmhead]
+
+``--workload lmhead`` times verification fused into the shared LM head
+instead: the inputs are the two models' last hidden states (B=256, k=5,
+H=2560, bf16) and the output head W [151936, 2560] bf16; one step is the
+tcgen05 GEMM with the statistics epilogue, the accept chains, the GEMM of the
+sampled rows and the sample.  Its roofline is the tensor-core one.
 
 With N > 1 (launched by torch.distributed.run) every rank verifies its own
 batch of the same shape (weak scaling, no collective on the data path); the
@@ -569,9 +575,261 @@ def run_vocab_parallel(args):
         rk.close()
 
 
+LM_METRIC = ("verified draft positions/s, verification fused into the shared LM head "
+             "(B=256 k=5 V=151936 H=2560)")
+LM_LAUNCHES_PER_STEP = 12  # kernels spec_lmhead_verify launches
+
+
+def lm_config(w, n):
+    B, kp1, H = w["hidden_target"].shape
+    return {"workload": w["name"], "B": int(B), "k": int(kp1 - 1), "V": int(w["head"].shape[0]),
+            "H": int(H), "hidden": "bf16", "logits": "fp32 accumulators (never stored)",
+            "temperature": 1.0, "mean_L": float(kp1 - 1),
+            "l2": "no flush: the head alone is %.0f MB, more than the 126 MB L2"
+                  % (w["head"].numel() * 2 / 1e6),
+            "parallelism": "replicas%d" % n if n > 1 else "single", "global_batch": int(B) * n}
+
+
+def lm_oracle_sample(w, n_requests, threads):
+    """fp64 oracle on the first n_requests: the head's logits of their rows, then
+    the verification; returns (seconds, positions)."""
+    import numpy as np
+    import oracle
+
+    def bits(t):
+        return t.detach().cpu().contiguous().view(torch_int16()).numpy().view(np.uint16)
+
+    hs = bits(w["hidden_target"][:n_requests])
+    hd = bits(w["hidden_draft"][:n_requests])
+    W = bits(w["head"])
+    tok = w["tokens"][:n_requests].cpu().numpy()
+    t0 = time.perf_counter()
+    res = oracle.verify_lmhead(hs, hd, W, tok, seed=w["seed"], threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, int(res["verify_len_used"].sum())
+
+
+def blas_threads():
+    """Threads numpy's BLAS runs the oracle's matmul on."""
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def torch_int16():
+    import torch
+    return torch.int16
+
+
+def run_lmhead(args):
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_86_b200 import binding, build, ranks, workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    build.build()
+    w = W.lmhead(dev, seed=5)
+    ht, hd, head, tok = w["hidden_target"], w["hidden_draft"], w["head"], w["tokens"]
+    B, kp1, H = ht.shape
+    k = kp1 - 1
+    V = head.shape[0]
+    ver = binding.SpecVerifier(dev, max_batch=B, max_k=k, max_vocab=V, mode="dense")
+    lm = binding.LmHeadVerifier(ver, max_hidden=H)
+    positions = B * k
+    out = ver._outputs(B, k, True)
+    stream = torch.cuda.current_stream(dev)
+    off = ranks.weak_offset(B, rank)
+
+    def step():
+        lm.verify(ht, hd, head, tok, seed=w["seed"], request_offset=off, out=out, redo_whole=False)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    redo_warm = int(out["redo"].sum().item())
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    phys = int(visible.split(",")[local]) if visible else local
+    clocks = ClockSampler(phys)
+    clocks.start()
+    time.sleep(0.2)
+    ver.timing_enable([binding.TIMING_LM_STATS, binding.TIMING_LM_ROWS])
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark()
+    if world > 1:
+        dist.barrier()
+    ms_local = e0.elapsed_time(e1)
+    n_st, ms_st = ver.timing_read(binding.TIMING_LM_STATS)
+    n_rw, ms_rw = ver.timing_read(binding.TIMING_LM_ROWS)
+    ver.timing_enable([])
+    clk = clocks.stop()
+    redo_last = int(out["redo"].sum().item())
+    ms_per_step = ranks.max_over_ranks(ms_local, dev) / args.steps
+    value = positions * world / (ms_per_step / 1e3)
+
+    # the unfused pipeline on the same inputs (this GEMM writing fp32 logits,
+    # then the verifier), and cuBLAS's bf16 GEMM of the same shape, for context
+    tl = torch.empty((B, k + 1, V), dtype=torch.float32, device=dev)
+    dl = torch.empty((B, k, V), dtype=torch.float32, device=dev)
+    hall = torch.cat([ht.reshape(-1, H), hd.reshape(-1, H)]).contiguous()
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n
+
+    def unfused():
+        lm.logits(ht, head, out=tl)
+        lm.logits(hd, head, out=dl)
+        ver.run(tl, dl, tok, seed=w["seed"], request_offset=off)
+
+    nb = max(3, min(args.steps, 50))
+    unfused_ms = timed(unfused, nb)
+    cublas_ms = timed(lambda: torch.matmul(hall, head.T), nb)
+    del tl, dl
+
+    # end to end: hidden states and tokens from pinned host memory, outputs back
+    e2e = None
+    if args.e2e_steps > 0:
+        h_ht, h_hd, h_tok = ht.cpu().pin_memory(), hd.cpu().pin_memory(), tok.cpu().pin_memory()
+        d_ht, d_hd, d_tok = torch.empty_like(ht), torch.empty_like(hd), torch.empty_like(tok)
+        hout = {key: torch.empty(v.shape, dtype=v.dtype).pin_memory() for key, v in out.items()}
+
+        def hstep():
+            d_ht.copy_(h_ht, non_blocking=True)
+            d_hd.copy_(h_hd, non_blocking=True)
+            d_tok.copy_(h_tok, non_blocking=True)
+            o = lm.verify(d_ht, d_hd, head, d_tok, seed=w["seed"], request_offset=off, out=out)
+            for key in hout:
+                hout[key].copy_(o[key], non_blocking=True)
+
+        hstep()
+        torch.cuda.synchronize(dev)
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.e2e_steps):
+            hstep()
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = ranks.max_over_ranks(a0.elapsed_time(a1), dev) / args.e2e_steps
+        h2d = sum(t.numel() * t.element_size() for t in (h_ht, h_hd, h_tok))
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        e2e = {"value": positions * world / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "note": "the public call with its whole-request redo check (one host sync per step)"}
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        dt, pos = lm_oracle_sample(w, 1, 1)
+        cpu = {"value": pos / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": "request 0 of %d: fp64 head logits of its 11 rows (numpy matmul on the "
+                         "BLAS threads) then the fp64 C oracle on one thread, %.1f s" % (B, dt)}
+
+    peaks = measured_peaks()
+    if peaks and peaks.get("bf16_tflops"):
+        peak, peak_src = float(peaks["bf16_tflops"]), "measured burst (cuBLAS bf16)"
+    else:
+        peak, peak_src = 1590.0, "fallback"
+    rows = B * (2 * k + 1)
+    flops = 2.0 * rows * V * H
+    st_ms = ms_st / max(n_st, 1)
+    achieved = flops / (st_ms * 1e-3) / 1e12
+    line = {
+        "metric": LM_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": lm_config(w, world),
+        "roofline": {"bound": "tensor", "kernel": "k_lmhead (statistics epilogue)",
+                     "achieved": achieved, "peak": peak, "peak_source": peak_src,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "frac_of_sustained": (achieved / float(peaks["bf16_tflops_sustained"])
+                                           if peaks and peaks.get("bf16_tflops_sustained") else None),
+                     "traffic": profiled_traffic("k_lmhead", "lmhead_stats"),
+                     "flops_per_launch": flops, "launch_ms": st_ms, "launches_timed": n_st},
+        "rows_gemm_ms": ms_rw / max(n_rw, 1),
+        "unfused_ms_per_step": unfused_ms,
+        "unfused_value": positions * world / (unfused_ms / 1e3),
+        "cublas_bf16_gemm_ms": cublas_ms,
+        "cublas_bf16_gemm_tflops": flops / (cublas_ms * 1e-3) / 1e12,
+        "requests_redone": {"warmup_last_step": redo_warm, "timed_last_step": redo_last},
+        "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": LM_LAUNCHES_PER_STEP * args.steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    lm.close()
+    ver.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_lmhead_reference(args):
+    """The fp64 oracle on the LM-head workload (reference arm), host cores."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+    import torch
+    from speculative_decoding_verification_86_b200 import workloads as W
+    oracle.build()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = W.lmhead(dev, seed=5)
+    for _ in range(max(0, min(args.warmup, 1))):
+        lm_oracle_sample(w, 1, 1)
+    tot_t, tot_pos = 0.0, 0
+    for _ in range(args.steps):
+        dt, pos = lm_oracle_sample(w, 1, 1)
+        tot_t += dt
+        tot_pos += pos
+    value = tot_pos / tot_t
+    line = {
+        "impl": "reference", "metric": LM_METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": lm_config(w, 1),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": "one request per step: fp64 head logits of its rows (BLAS "
+                                   "threads), then the oracle on one thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.workload == "lmhead":
+        if args.impl == "reference":
+            run_lmhead_reference(args)
+        else:
+            run_lmhead(args)
+    elif args.impl == "reference":
         run_reference(args)
     elif args.vocab_shards > 1:
         run_vocab_parallel(args)
