@@ -304,7 +304,7 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   sv::k_shard_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
   sv::k_shard_finish<<<grid_for(B), 256, 0, stream>>>(p, lm->votes);
   const int nsub = p.n_chunks * sv::kSubsPerChunk;
-  sv::k_shard_refine_partials<false><<<B * nsub, sv::kThreads, 0, stream>>>(p, 0, nsub);
+  sv::k_shard_refine_partials<false><<<refine_grid(ctx, B, nsub), sv::kThreads, 0, stream>>>(p, 0, nsub);
   sv::k_shard_refine_locate<false><<<B, sv::kThreads, 0, stream>>>(p);
   sv::k_shard_refine_finish<<<grid_for(B), 256, 0, stream>>>(p, lm->votes);
   if (cudaMemcpyAsync(out_redo, ctx->fallback, static_cast<size_t>(B) * sizeof(int32_t),

@@ -230,14 +230,25 @@ struct alignas(16) RefRec {
 };
 static_assert(sizeof(RefRec) == 48, "exchange record layout");
 
+// Grid-stride over the B x nsub (request, sub-chunk) items: most requests need
+// no refinement, so a small grid skips their items instead of launching a CTA
+// for each.
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) k_shard_refine_partials(RunParams p, int sub_lo, int nsub) {
   __shared__ RefineShared rf;
-  const int i = static_cast<int>(blockIdx.x / nsub);
-  const int ls = static_cast<int>(blockIdx.x % nsub);
-  if (__ldcg(p.fallback + i) != kShardRefine) return;  // (uniform over the CTA)
-  exp2_table_init(rf.tab);
-  refine_item<BF16>(p, i, sub_lo + ls, rf);
+  bool table = false;
+  const int64_t n = static_cast<int64_t>(p.B) * nsub;
+  for (int64_t b = blockIdx.x; b < n; b += gridDim.x) {
+    const int i = static_cast<int>(b / nsub);
+    const int ls = static_cast<int>(b % nsub);
+    if (__ldcg(p.fallback + i) != kShardRefine) continue;  // (uniform over the CTA)
+    if (!table) {
+      exp2_table_init(rf.tab);
+      table = true;
+    }
+    refine_item<BF16>(p, i, sub_lo + ls, rf);
+    sync_compute();  // rf is reused by the next item
+  }
 }
 
 __global__ void k_shard_pack_refine(RunParams p, int sub_lo, int nsub, int nsub_max, RefRec* out) {

@@ -485,6 +485,12 @@ spec_status shard_params(spec_verify_ctx* c, int rank, int n_shards, const void*
 }
 
 int grid_for(int64_t n) { return static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)); }
+
+// Grid of the refinement partials: grid-strides over B x nsub items, eight CTAs per SM.
+int refine_grid(const spec_verify_ctx* c, int B, int nsub) {
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(B) * nsub,
+                                                                  8LL * c->num_sms)));
+}
 }  // namespace
 
 extern "C" {
@@ -1032,8 +1038,9 @@ spec_status spec_shard_refine_partials(spec_verify_ctx* ctx, int rank, int n_sha
   const int sub_lo = p.c_lo * sv::kSubsPerChunk;
   const int nsub = (p.c_hi - p.c_lo) * sv::kSubsPerChunk;
   if (nsub > 0) {
-    if (dtype == SPEC_BF16) sv::k_shard_refine_partials<true><<<B * nsub, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
-    else sv::k_shard_refine_partials<false><<<B * nsub, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
+    const int grid = refine_grid(ctx, B, nsub);
+    if (dtype == SPEC_BF16) sv::k_shard_refine_partials<true><<<grid, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
+    else sv::k_shard_refine_partials<false><<<grid, sv::kThreads, 0, stream>>>(p, sub_lo, nsub);
   }
   sv::k_shard_pack_refine<<<grid_for(static_cast<int64_t>(B) * z.nsub_max), 256, 0, stream>>>(
       p, sub_lo, nsub, z.nsub_max, static_cast<sv::RefRec*>(block3));
