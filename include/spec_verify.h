@@ -10,15 +10,15 @@
  * section "Why draft-and-verify does not change the output"):
  *   - stochastic (T > 0): accept drafted token x with probability
  *     min(1, p(x)/q(x)), p = softmax(target/T), q = softmax(draft/T); at the
- *     first rejection emit a sample from the corrected residual
+ *     first rejection emit a sample from the residual
  *     norm(max(0, p - q)) and drop the rest of the block; if every verified
  *     position is accepted emit a bonus token drawn from the target's next row;
  *   - greedy (T == 0): keep x while it is the target's argmax (lowest index on
  *     ties); at the first disagreement emit the argmax; if all agree emit the
  *     argmax of the next row.
- * The confidence head (same page, section "What DSpark adds") is a linear
- * projection with a sigmoid giving each position's survival probability given
- * that the earlier positions survived; the prefix product of these
+ * The confidence head (same page, section "What DSpark adds") maps each
+ * position's hidden state to s_j = sigmoid(w . h_j + b), the estimated chance
+ * that position j passes once all earlier positions have; the prefix product of these
  * probabilities, compared with a threshold, truncates the verified length.
  *
  * Readings where the pages are silent (all shared with the CPU oracle):
@@ -74,8 +74,8 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 /* Order in which the statistics pass reads a request's rows.  Both give the
  * same outputs, bit for bit:
  *   SPEC_MODE_PREFIX (default): position j+1's rows are read only once position
- *     j was accepted ("at the first disagreement ... throw away the rest of
- *     the draft"), so rows past the first rejection are never touched;
+ *     j was accepted (the block ends at its first rejected position), so rows
+ *     past the first rejection are never touched;
  *   SPEC_MODE_DENSE: every verified position's target and draft rows are
  *     reduced, then the chain is walked. */
 typedef enum { SPEC_MODE_DENSE = 0, SPEC_MODE_PREFIX = 1 } spec_mode;

@@ -9,14 +9,14 @@
  * What it computes (sources, by page title and section):
  *  - "Speculative decoding becomes standard: DSpark and multi-token drafters",
  *    section "Why draft-and-verify does not change the output": the target
- *    scores the drafted block; a drafted token is accepted with probability
- *    min(1, p/q) (p = target, q = drafter); the first rejection is replaced by a
- *    sample from a corrected residual distribution and the rest of the draft is
- *    thrown away; at temperature 0 a token is kept while the target agrees with
- *    it and the target's own token is taken at the first disagreement.
- *  - same page, section "What DSpark adds": a confidence head (linear
- *    projection + sigmoid) gives each position's survival probability given
- *    that the earlier positions survived; the verified length is set from it.
+ *    scores the drafted block; the token drafted at position j is kept with probability
+ *    min(1, p/q) (p = target, q = drafter); at the first rejection a token is
+ *    drawn from a residual distribution instead and the block ends there; at
+ *    temperature 0 a token is kept while it is the target's own choice, and
+ *    the target's choice replaces the first token that is not.
+ *  - same page, section "What DSpark adds": a confidence head,
+ *    s_j = sigmoid(w . h_j + b), estimates whether position j passes once the
+ *    positions before it have; the verified length is derived from it.
  *  - The residual is norm(max(0, p - q)) (Leviathan, Kalman, Matias 2022); a
  *    bonus token is drawn from the target when the whole block survives.
  *

@@ -1,7 +1,7 @@
 // Confidence head ("Speculative decoding becomes standard: DSpark and
-// multi-token drafters", section "What DSpark adds"): a linear projection with
-// a sigmoid estimates, for each drafted position, the probability that its
-// token survives verification given that the earlier ones did.  The chance
+// multi-token drafters", section "What DSpark adds"): s_j = sigmoid(w . h_j + b)
+// is the head's estimate that drafted position j passes verification when all
+// positions before it have passed.  The chance
 // that the first j positions all survive is the prefix product; the request's
 // budget is the number of leading positions whose prefix product stays at or
 // above the threshold.

@@ -14,7 +14,7 @@
 //
 // Two orders of the statistics ("Speculative decoding becomes standard: DSpark
 // and multi-token drafters", section "Why draft-and-verify does not change the
-// output": at the first disagreement the rest of the draft is thrown away):
+// output": the block ends at its first rejected position):
 //   dense  : every verified position's rows are statistics items from the start
 //            and the chain is walked once they are all in;
 //   prefix : a request's position j+1 rows are read only after position j was

@@ -1,5 +1,5 @@
 // Pass 2: the one sample each stochastic request still needs -- from the
-// corrected residual norm(max(0, p - q)) of the rejected row pair, or from the
+// residual distribution norm(max(0, p - q)) of the rejected row pair, or from the
 // target's bonus row when the whole block survived ("Speculative decoding
 // becomes standard: DSpark and multi-token drafters", section "Why
 // draft-and-verify does not change the output").

@@ -7,8 +7,8 @@
   against sigmoid(h @ w + b).cumprod in fp64.
 * The exactness invariant of rejection sampling ("Speculative decoding becomes
   standard: DSpark and multi-token drafters", section "Why draft-and-verify does
-  not change the output": the accepted sequence has exactly the target's
-  distribution) by exhaustive enumeration of draft tokens and of the oracle's
+  not change the output": the emitted tokens follow the target's law exactly)
+  by exhaustive enumeration of draft tokens and of the oracle's
   own decision cells on tiny vocabularies, to 1e-12; the probability of
   reaching position j equals prod_{j'<j} sum_t min(p, q) (closed form).
 * The same laws from 10^6 Philox-driven runs (chi-square, p > 1e-4).
