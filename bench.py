@@ -56,7 +56,7 @@ def parse_args():
     ap.add_argument("--workload", default="headline")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="prefix", choices=["prefix", "dense"])
+    ap.add_argument("--mode", default="prefix", choices=["prefix", "dense", "auto"])
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every step (cold L2) and report the "
                          "kernel time of each launch")
@@ -363,7 +363,7 @@ def run_ours(args):
     clk = clocks.stop()
     counters = ver.last_counters()
     # the other statistics order, timed the same way on the same batch
-    other = "dense" if ver.mode == "prefix" else "prefix"
+    other = "prefix" if ver.mode == "dense" else "dense"
     ver.set_mode(other)
     for _ in range(3):
         step()

@@ -71,14 +71,19 @@ typedef enum {
 
 typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
 
-/* Order in which the statistics pass reads a request's rows.  Both give the
+/* Order in which the statistics pass reads a request's rows.  All give the
  * same outputs, bit for bit:
- *   SPEC_MODE_PREFIX (default): position j+1's rows are read only once position
- *     j was accepted (the block ends at its first rejected position), so rows
- *     past the first rejection are never touched;
+ *   SPEC_MODE_PREFIX: position j+1's rows are read only once position j was
+ *     accepted (the block ends at its first rejected position), so rows past
+ *     the first rejection are never touched;
  *   SPEC_MODE_DENSE: every verified position's target and draft rows are
- *     reduced, then the chain is walked. */
-typedef enum { SPEC_MODE_DENSE = 0, SPEC_MODE_PREFIX = 1 } spec_mode;
+ *     reduced, then the chain is walked;
+ *   SPEC_MODE_AUTO (default): dense when the B * (2k + 1) rows, cut into
+ *     segments of 32768 bf16 or 16384 fp32 logits, make at most one segment
+ *     per CTA of the kernel's grid (the extra rows then cost no time and the
+ *     waits between positions go), prefix otherwise.  spec_verify_greedy
+ *     always uses the prefix order. */
+typedef enum { SPEC_MODE_DENSE = 0, SPEC_MODE_PREFIX = 1, SPEC_MODE_AUTO = 2 } spec_mode;
 
 /* Per-request device status bits (out_status[i]); 0 means success. */
 #define SPEC_DEV_BAD_TOKEN 1u       /* a drafted token the chain reached is outside [0, V) */

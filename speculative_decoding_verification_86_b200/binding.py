@@ -30,7 +30,8 @@ SPEC_BF16 = 1
 
 SPEC_MODE_DENSE = 0
 SPEC_MODE_PREFIX = 1
-MODES = {"dense": SPEC_MODE_DENSE, "prefix": SPEC_MODE_PREFIX}
+SPEC_MODE_AUTO = 2
+MODES = {"dense": SPEC_MODE_DENSE, "prefix": SPEC_MODE_PREFIX, "auto": SPEC_MODE_AUTO}
 
 DEV_BAD_TOKEN = 1
 DEV_NONFINITE = 2
@@ -177,7 +178,7 @@ class SpecVerifier:
     (default: current) torch stream and return output tensors.
     """
 
-    def __init__(self, device=None, max_batch=1024, max_k=8, max_vocab=262144, mode="prefix"):
+    def __init__(self, device=None, max_batch=1024, max_k=8, max_vocab=262144, mode="auto"):
         dev = torch.device("cuda") if device is None else torch.device(device)
         if dev.type != "cuda":
             raise ValueError("SpecVerifier needs a CUDA device, got %s" % dev)
@@ -192,8 +193,10 @@ class SpecVerifier:
         self.set_mode(mode)
 
     def set_mode(self, mode):
-        """Statistics order: "prefix" (default: rows past the first rejection
-        are never read) or "dense" (every verified position's rows)."""
+        """Statistics order: "auto" (default: dense when every row the batch
+        may verify fits in one wave of the grid, else prefix), "prefix" (rows
+        past the first rejection are never read) or "dense" (every verified
+        position's rows)."""
         _check(lib().spec_verify_set_mode(self._h, MODES[mode]), "spec_verify_set_mode")
         self.mode = mode
 

@@ -138,7 +138,7 @@ struct spec_verify_ctx {
   unsigned q_capacity = 0;
   unsigned* q_ctl = nullptr;
   int engine_grid = 0;
-  int mode = sv::kModePrefix;
+  int mode = SPEC_MODE_AUTO;  // as set by spec_verify_set_mode
   unsigned run_id = 0;
 
   unsigned timing_mask = 0;  // bit c set: bracket launches of class c with events
@@ -376,7 +376,15 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     launch_conf(c, conf, B, k, vlen, c->conf_len, nullptr, s);
     p.conf_len = c->conf_len;
   }
-  p.mode = force_greedy ? sv::kModePrefix : c->mode;
+  // Order of the statistics.  Automatic: the prefix order saves reads when the
+  // batch's rows compete for the grid; when every row the batch may verify
+  // fits in one wave of the grid, reading them all at once costs no extra time
+  // and removes the waits between positions, so the dense order is faster.
+  int mode = c->mode;
+  if (mode == SPEC_MODE_AUTO)
+    mode = static_cast<int64_t>(B) * (2 * k + 1) * n_segs <= c->engine_grid ? SPEC_MODE_DENSE
+                                                                           : SPEC_MODE_PREFIX;
+  p.mode = (force_greedy || mode == SPEC_MODE_PREFIX) ? sv::kModePrefix : sv::kModeDense;
   p.q_slots = c->q_slots;
   p.q_capacity = c->q_capacity;
   p.q_ctl = c->q_ctl;
@@ -816,8 +824,9 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
 }
 
 spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode) {
-  if (!ctx || (mode != SPEC_MODE_DENSE && mode != SPEC_MODE_PREFIX)) return SPEC_ERR_INVALID_ARG;
-  ctx->mode = mode == SPEC_MODE_DENSE ? sv::kModeDense : sv::kModePrefix;
+  if (!ctx || (mode != SPEC_MODE_DENSE && mode != SPEC_MODE_PREFIX && mode != SPEC_MODE_AUTO))
+    return SPEC_ERR_INVALID_ARG;
+  ctx->mode = mode;
   return SPEC_OK;
 }
 

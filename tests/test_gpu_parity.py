@@ -21,7 +21,7 @@ pytestmark = pytest.mark.gpu
 THREADS = max(1, min(32, os.cpu_count() or 1))
 
 
-@pytest.fixture(scope="module", params=["prefix", "dense"])
+@pytest.fixture(scope="module", params=["prefix", "dense", "auto"])
 def ver(cuda_device, request):
     build.build()
     v = binding.SpecVerifier(cuda_device, max_batch=1024, max_k=16, max_vocab=262144,
