@@ -380,6 +380,15 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* ctx, const void* hidden_target,
                                float* out_q, uint32_t* out_status, int32_t* out_redo,
                                cudaStream_t stream);
 
+/* Tile configuration of the LM-head GEMMs.  One CTA per SM with 128 x 256
+ * tiles (tcgen05.mma.cta_group::1), or clusters of two CTAs sharing 256 x 256
+ * tiles (tcgen05.mma.cta_group::2: each CTA loads its 128 rows and half of the
+ * tile's W rows, a third fewer bytes per flop).  pairs = 0: one CTA per tile
+ * everywhere; 1: CTA pairs everywhere; 2 (default): CTA pairs for the
+ * row-writing GEMM only (measured faster there; the statistics GEMM is not).
+ * Results are identical in every configuration. */
+spec_status spec_lmhead_set_cta_pairs(spec_lmhead_ctx* ctx, int pairs);
+
 /* Error word of the LM-head kernels since the context was created
  * (synchronises the device): bit 0 set = a wait inside a GEMM timed out and
  * that launch's outputs are not to be used. */

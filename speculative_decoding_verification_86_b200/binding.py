@@ -98,6 +98,7 @@ def lib():
     L.spec_lmhead_init.argtypes = [ctypes.POINTER(_vp), _vp, _i32]
     L.spec_lmhead_destroy.argtypes = [_vp]
     L.spec_lmhead_errors.argtypes = [_vp, ctypes.POINTER(_u32)]
+    L.spec_lmhead_set_cta_pairs.argtypes = [_vp, _i32]
     L.spec_lmhead_logits.argtypes = [_vp, _vp, _i32, _vp, _i32, _i64, _vp, _vp]
     L.spec_lmhead_verify.argtypes = [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                      ctypes.POINTER(ConfArgs), _i32, _i32, _i64, _u64, _u32, _u32,
@@ -117,7 +118,7 @@ def lib():
                  "spec_shard_finish", "spec_shard_refine_partials", "spec_shard_refine_locate",
                  "spec_shard_refine_finish",
                  "spec_lmhead_init", "spec_lmhead_destroy", "spec_lmhead_errors",
-                 "spec_lmhead_logits", "spec_lmhead_verify",
+                 "spec_lmhead_logits", "spec_lmhead_verify", "spec_lmhead_set_cta_pairs",
                  "spec_verify_set_mode",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
@@ -669,13 +670,20 @@ class LmHeadVerifier:
     (spec_lmhead_*): takes the two models' last hidden states and the shared
     output head instead of logits.  Uses (and must not outlive) ``ver``."""
 
-    def __init__(self, ver: SpecVerifier, max_hidden=4096):
+    def __init__(self, ver: SpecVerifier, max_hidden=4096, cta_pairs=2):
         self.ver = ver
         self.device = ver.device
         self.max_hidden = max_hidden
         h = _vp()
         _check(lib().spec_lmhead_init(ctypes.byref(h), ver._h, int(max_hidden)), "spec_lmhead_init")
         self._h = h
+        self.set_cta_pairs(cta_pairs)
+
+    def set_cta_pairs(self, pairs):
+        """GEMM tiles: 0 one CTA per tile, 1 CTA pairs (cta_group::2) for both
+        GEMMs, 2 (default) CTA pairs for the row-writing GEMM only."""
+        _check(lib().spec_lmhead_set_cta_pairs(self._h, int(pairs)), "spec_lmhead_set_cta_pairs")
+        self.cta_pairs = int(pairs)
 
     def close(self):
         if getattr(self, "_h", None):

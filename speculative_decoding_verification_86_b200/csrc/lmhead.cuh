@@ -36,10 +36,7 @@ constexpr int kLmBM = 128;  // rows per tile (UMMA M)
 constexpr int kLmBN = 256;  // vocabulary columns per tile (UMMA N)
 constexpr int kLmBK = 64;   // hidden elements per stage: one 128-byte swizzle row of bf16
 constexpr int kLmUK = 16;   // K of one kind::f16 instruction
-constexpr int kLmStages = 4;
-constexpr uint32_t kLmABytes = kLmBM * kLmBK * 2;  // 16 KB
-constexpr uint32_t kLmBBytes = kLmBN * kLmBK * 2;  // 32 KB
-constexpr uint32_t kLmStageBytes = kLmABytes + kLmBBytes;
+constexpr uint32_t kLmABytes = kLmBM * kLmBK * 2;  // 16 KB: this CTA's 128 rows
 constexpr int kLmThreads = 192;
 constexpr uint32_t kLmTmemCols = 2 * kLmBN;
 // A work unit covers `part_tiles` N tiles (a power of two up to kLmSegTiles);
@@ -48,7 +45,21 @@ constexpr uint32_t kLmTmemCols = 2 * kLmBN;
 constexpr int kLmSegTiles = SegGeo<false>::kSeg / kLmBN;  // 64 tiles per statistics segment
 static_assert(SegGeo<false>::kSeg % kLmBN == 0, "tiles divide the fp32 statistics segment");
 constexpr size_t kLmBarrierBytes = 256;
-constexpr size_t kLmSmemBytes = 1024 + kLmStages * kLmStageBytes + kLmBarrierBytes;
+
+// Geometry of the kernel with CG CTAs per MMA (1, or 2 for a CTA pair running
+// tcgen05.mma.cta_group::2 on a 256 x 256 tile: each CTA holds its 128 rows of
+// A and half of the 256 W rows, and gets its 128 rows of the accumulator).
+template <int CG>
+struct LmGeo {
+  static constexpr int kRowsPerUnit = kLmBM * CG;              // M tile of one MMA
+  static constexpr int kBRows = kLmBN / CG;                    // W rows per CTA and stage
+  static constexpr uint32_t kBBytes = kBRows * kLmBK * 2;      // 32 KB or 16 KB
+  static constexpr uint32_t kStageBytes = kLmABytes + kBBytes;  // 48 KB or 32 KB
+  static constexpr int kStages = CG == 1 ? 4 : 6;
+  static constexpr uint32_t kTxBytes = kStageBytes * CG;       // bytes the MMA CTA waits for
+  static constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kLmBarrierBytes;
+};
+constexpr int kLmMaxStages = 6;
 constexpr unsigned long long kLmWaitNs = 2000000000ull;  // 2 s: legitimate waits are microseconds
 
 constexpr int kLmModeStats = 0;  // epilogue -> statistics partial records + token logits
@@ -168,24 +179,47 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, N = 256, M = 128.
-constexpr uint32_t kLmIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                              (static_cast<uint32_t>(kLmBN >> 3) << 17) |
-                              (static_cast<uint32_t>(kLmBM >> 4) << 24);
+// K-major, N = 256, M = 128 per CTA of the group.
+template <int CG>
+__device__ __forceinline__ constexpr uint32_t lm_idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(kLmBN >> 3) << 17) |
+         (static_cast<uint32_t>((kLmBM * CG) >> 4) << 24);
+}
+template <int CG>
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kLmIdesc), "r"(accumulate)
-      : "memory");
+  if constexpr (CG == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(lm_idesc<1>()), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(lm_idesc<2>()), "r"(accumulate)
+        : "memory");
+  }
 }
-// Arrive on `bar` once every tcgen05 operation this thread issued has completed.
+// Arrive on `bar` (in every CTA of the group) once every tcgen05 operation
+// this thread issued has completed.
+template <int CG>
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_addr(bar))
-               : "memory");
+  if constexpr (CG == 1) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+  } else {
+    const uint16_t mask = 0x3;
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(smem_addr(bar)),
+        "h"(mask)
+        : "memory");
+  }
 }
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -200,17 +234,52 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------- CTA pair helpers --
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+  return r;
+}
+// Every thread of both CTAs (the non-.aligned form: warps may arrive diverged).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// 2-D tiled TMA load of this CTA's half of a pair's operands, completing on
+// the MMA CTA's barrier (a shared::cluster address); no multicast.
+__device__ __forceinline__ void tma_load_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
+                                              int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%3, %4}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+
 // ---------------------------------------------------------- work division --
+template <int CG>
 struct LmWork {
-  int mt0, n_mt, n_nt, pt, n_parts, units, n_kb;
+  int mt0, n_mt, n_nt, pt, n_parts, units, n_kb, first, stride;
   __device__ LmWork(int rows0, int rows1, int64_t V, int H, int part_tiles) {
-    mt0 = (rows0 + kLmBM - 1) / kLmBM;
-    n_mt = mt0 + (rows1 + kLmBM - 1) / kLmBM;
+    constexpr int R = LmGeo<CG>::kRowsPerUnit;
+    mt0 = (rows0 + R - 1) / R;
+    n_mt = mt0 + (rows1 + R - 1) / R;
     n_nt = static_cast<int>((V + kLmBN - 1) / kLmBN);
     pt = part_tiles;
     n_parts = (n_nt + pt - 1) / pt;
     units = n_mt * n_parts;
     n_kb = (H + kLmBK - 1) / kLmBK;
+    first = static_cast<int>(blockIdx.x) / CG;  // the CTAs of a group take the same units
+    stride = static_cast<int>(gridDim.x) / CG;
   }
   // unit u: M tile u % n_mt, part u / n_mt (the CTAs at work at one time share W columns)
   __device__ int mt(int u) const { return u % n_mt; }
@@ -220,8 +289,8 @@ struct LmWork {
 };
 
 struct LmShared {
-  uint64_t full[kLmStages];
-  uint64_t empty[kLmStages];
+  uint64_t full[kLmMaxStages];
+  uint64_t empty[kLmMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -246,13 +315,21 @@ struct LmRowState {
   int gbad = 0;
 };
 
-__device__ __forceinline__ void lm_row_init(const LmParams& p, int mt, int mt0, int r_in_tile,
-                                            LmRowState& st) {
+// Row of the batch (target rows, then the drafter's) held by TMEM lane
+// `r_in_unit` of M tile mt; false past the end of its matrix.
+__device__ __forceinline__ bool lm_row_of(const LmParams& p, int mt, int mt0, int rows_per_unit,
+                                          int r_in_unit, bool& draft, int& r) {
+  draft = mt >= mt0;
+  r = (draft ? mt - mt0 : mt) * rows_per_unit + r_in_unit;
+  return r < (draft ? p.rows1 : p.rows0);
+}
+
+__device__ __forceinline__ void lm_row_init(const LmParams& p, int mt, int mt0, int rows_per_unit,
+                                            int r_in_unit, LmRowState& st) {
   st = LmRowState();
-  const bool draft = mt >= mt0;
-  const int r = (draft ? mt - mt0 : mt) * kLmBM + r_in_tile;
-  const int rows = draft ? p.rows1 : p.rows0;
-  if (r >= rows) return;
+  bool draft;
+  int r;
+  if (!lm_row_of(p, mt, mt0, rows_per_unit, r_in_unit, draft, r)) return;
   st.valid = true;
   st.draft = draft;
   if (draft) {
@@ -310,9 +387,11 @@ __device__ __forceinline__ void lm_consume_stats(const LmParams& p, LmRowState& 
 }
 
 __device__ __forceinline__ void lm_write_part(const LmParams& p, const LmRowState& st, int mt,
-                                              int mt0, int r_in_tile, int part) {
-  const bool draft = mt >= mt0;
-  const int r = (draft ? mt - mt0 : mt) * kLmBM + r_in_tile;
+                                              int mt0, int rows_per_unit, int r_in_unit,
+                                              int part) {
+  bool draft;
+  int r;
+  lm_row_of(p, mt, mt0, rows_per_unit, r_in_unit, draft, r);
   const int64_t g = draft ? static_cast<int64_t>(p.rows0) + r : r;
   LmPart o;
   if (st.greedy) {
@@ -349,44 +428,65 @@ __device__ __forceinline__ void lm_consume_rows(const LmParams& p, int64_t dst,
 }
 
 // ------------------------------------------------------------------ roles --
-__device__ __forceinline__ void lm_producer(const LmParams& p, const LmWork& w, LmShared& sh,
+// With a CTA pair (CG = 2) both CTAs load their halves; the MMA CTA (rank 0)
+// arms its full barrier for both halves' bytes, and the loads complete there.
+template <int CG>
+__device__ __forceinline__ void lm_producer(const LmParams& p, const LmWork<CG>& w, LmShared& sh,
                                             uint8_t* stages, const CUtensorMap* ma0,
-                                            const CUtensorMap* ma1, const CUtensorMap* mw) {
+                                            const CUtensorMap* ma1, const CUtensorMap* mw,
+                                            uint32_t rank) {
+  using G = LmGeo<CG>;
   uint32_t g = 0;
   bool ok = true;
-  for (int u = blockIdx.x; ok && u < w.units; u += gridDim.x) {
+  for (int u = w.first; ok && u < w.units; u += w.stride) {
     const int mt = w.mt(u);
     const CUtensorMap* ma = mt < w.mt0 ? ma0 : ma1;
-    const int arow = (mt < w.mt0 ? mt : mt - w.mt0) * kLmBM;
+    const int arow = (mt < w.mt0 ? mt : mt - w.mt0) * G::kRowsPerUnit + static_cast<int>(rank) * kLmBM;
     for (int nt = w.nt_lo(u); ok && nt < w.nt_hi(u); ++nt) {
+      const int brow = nt * kLmBN + static_cast<int>(rank) * G::kBRows;
       for (int kb = 0; kb < w.n_kb; ++kb, ++g) {
-        const int s = static_cast<int>(g % kLmStages);
-        const uint32_t ph = (g / kLmStages) & 1u;
+        const int s = static_cast<int>(g % G::kStages);
+        const uint32_t ph = (g / G::kStages) & 1u;
         if (!mbar_wait(&sh.empty[s], ph ^ 1u, &sh.abort, p.error)) {
           ok = false;
           break;
         }
-        uint8_t* a = stages + static_cast<size_t>(s) * kLmStageBytes;
-        mbar_expect_tx(&sh.full[s], kLmStageBytes);
-        tma_load(a, ma, &sh.full[s], kb * kLmBK, arow);
-        tma_load(a + kLmABytes, mw, &sh.full[s], kb * kLmBK, nt * kLmBN);
+        uint8_t* a = stages + static_cast<size_t>(s) * G::kStageBytes;
+        if constexpr (CG == 1) {
+          mbar_expect_tx(&sh.full[s], G::kTxBytes);
+          tma_load(a, ma, &sh.full[s], kb * kLmBK, arow);
+          tma_load(a + kLmABytes, mw, &sh.full[s], kb * kLmBK, brow);
+        } else {
+          if (rank == 0) mbar_expect_tx(&sh.full[s], G::kTxBytes);
+          const uint32_t bar = peer_addr(&sh.full[s], 0);
+          tma_load_pair(a, ma, bar, kb * kLmBK, arow);
+          tma_load_pair(a + kLmABytes, mw, bar, kb * kLmBK, brow);
+        }
       }
     }
   }
   if (!ok) {
-    // drain: the loads this thread issued land before the CTA's memory goes away
-    for (uint32_t q = g > kLmStages ? g - kLmStages : 0; q < g; ++q) {
-      volatile int no_abort = 0;
-      mbar_wait(&sh.full[q % kLmStages], (q / kLmStages) & 1u, &no_abort, p.error);
+    if constexpr (CG == 1) {
+      // drain: the loads this thread issued land before the CTA's memory goes away
+      for (uint32_t q = g > G::kStages ? g - G::kStages : 0; q < g; ++q) {
+        volatile int no_abort = 0;
+        mbar_wait(&sh.full[q % G::kStages], (q / G::kStages) & 1u, &no_abort, p.error);
+      }
+    } else {
+      // this CTA's loads complete on the other CTA's barrier: give them time to land
+      const unsigned long long t0 = lm_now();
+      while (lm_now() - t0 < 200000ull) __nanosleep(1000);
     }
   }
 }
 
-__device__ __forceinline__ void lm_mma(const LmParams& p, const LmWork& w, LmShared& sh,
+template <int CG>
+__device__ __forceinline__ void lm_mma(const LmParams& p, const LmWork<CG>& w, LmShared& sh,
                                        uint8_t* stages) {
+  using G = LmGeo<CG>;
   uint32_t g = 0, t = 0;
   bool ok = true;
-  for (int u = blockIdx.x; ok && u < w.units; u += gridDim.x) {
+  for (int u = w.first; ok && u < w.units; u += w.stride) {
     for (int nt = w.nt_lo(u); ok && nt < w.nt_hi(u); ++nt, ++t) {
       const uint32_t a = t & 1u;
       if (!mbar_wait(&sh.tempty[a], ((t >> 1) & 1u) ^ 1u, &sh.abort, p.error)) {
@@ -396,45 +496,48 @@ __device__ __forceinline__ void lm_mma(const LmParams& p, const LmWork& w, LmSha
       tc_fence_after();
       const uint32_t d = sh.tmem + a * kLmBN;
       for (int kb = 0; kb < w.n_kb; ++kb, ++g) {
-        const int s = static_cast<int>(g % kLmStages);
-        if (!mbar_wait(&sh.full[s], (g / kLmStages) & 1u, &sh.abort, p.error)) {
+        const int s = static_cast<int>(g % G::kStages);
+        if (!mbar_wait(&sh.full[s], (g / G::kStages) & 1u, &sh.abort, p.error)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = smem_addr(stages + static_cast<size_t>(s) * kLmStageBytes);
+        const uint32_t sa = smem_addr(stages + static_cast<size_t>(s) * G::kStageBytes);
         const uint64_t adesc = sw128_desc(sa);
         const uint64_t bdesc = sw128_desc(sa + kLmABytes);
 #pragma unroll
         for (int kk = 0; kk < kLmBK / kLmUK; ++kk) {
           // advance along K inside the swizzled 128-byte rows: 32 bytes per step
-          umma_bf16(d, adesc + 2 * kk, bdesc + 2 * kk, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16<CG>(d, adesc + 2 * kk, bdesc + 2 * kk, (kb > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&sh.empty[s]);  // the stage is free once these MMAs have read it
+        umma_commit<CG>(&sh.empty[s]);  // the stage is free once these MMAs have read it
       }
-      if (ok) umma_commit(&sh.tfull[a]);
+      if (ok) umma_commit<CG>(&sh.tfull[a]);
     }
   }
   if (!ok) {  // every MMA issued so far completes before TMEM is released
-    umma_commit(&sh.drain);
+    umma_commit<CG>(&sh.drain);
     volatile int no_abort = 0;
     mbar_wait(&sh.drain, 0, &no_abort, p.error);
   }
 }
 
-__device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork& w, LmShared& sh) {
+template <int CG>
+__device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>& w, LmShared& sh,
+                                            uint32_t rank) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3;  // TMEM lanes this warp may read
-  const int r_in_tile = quarter * 32 + lane;
+  const int r_in_unit = static_cast<int>(rank) * kLmBM + quarter * 32 + lane;
+  constexpr int R = LmGeo<CG>::kRowsPerUnit;
   uint32_t t = 0;
-  for (int u = blockIdx.x; u < w.units; u += gridDim.x) {
+  for (int u = w.first; u < w.units; u += w.stride) {
     const int mt = w.mt(u);
     LmRowState st;
     int64_t dst = -1;
     if (p.mode == kLmModeStats) {
-      lm_row_init(p, mt, w.mt0, r_in_tile, st);
+      lm_row_init(p, mt, w.mt0, R, r_in_unit, st);
     } else {
-      const int r = mt * kLmBM + r_in_tile;
+      const int r = mt * R + r_in_unit;
       if (r < sh.rows0) dst = p.dst ? __ldg(p.dst + r) : static_cast<int64_t>(r) * p.V;
     }
     for (int nt = w.nt_lo(u); nt < w.nt_hi(u); ++nt, ++t) {
@@ -469,29 +572,37 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork& w, 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.tempty[a]);
+      if (lane == 0) {
+        if constexpr (CG == 1) mbar_arrive(&sh.tempty[a]);
+        else mbar_arrive_cluster(peer_addr(&sh.tempty[a], 0));  // the MMA CTA's barrier
+      }
     }
     if (p.mode == kLmModeStats && st.valid)
-      lm_write_part(p, st, mt, w.mt0, r_in_tile, w.part(u));
+      lm_write_part(p, st, mt, w.mt0, R, r_in_unit, w.part(u));
   }
 }
 
+// CG = 1: one CTA per SM.  CG = 2: launched in clusters of two CTAs (a pair on
+// one TPC); rank 0 issues the MMAs of the pair's 256 x 256 tiles.
+template <int CG>
 __global__ void __launch_bounds__(kLmThreads, 1)
     k_lmhead(const __grid_constant__ CUtensorMap ma0, const __grid_constant__ CUtensorMap ma1,
              const __grid_constant__ CUtensorMap mw, LmParams p) {
+  using G = LmGeo<CG>;
   extern __shared__ uint8_t lm_smem[];
   const uint32_t pad = (1024u - (smem_addr(lm_smem) & 1023u)) & 1023u;
   uint8_t* stages = lm_smem + pad;  // 1024-byte aligned: the swizzle atoms of every stage
-  LmShared& sh = *reinterpret_cast<LmShared*>(stages + kLmStages * kLmStageBytes);
+  LmShared& sh = *reinterpret_cast<LmShared*>(stages + G::kStages * G::kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 1 ? 0u : cluster_rank();
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kLmStages; ++s) {
+    for (int s = 0; s < G::kStages; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&sh.tempty[a], 4 * CG);  // one arrival per epilogue warp of the group
     }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -506,31 +617,47 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     tma_prefetch(&mw);
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_addr(&sh.tmem)),
-                 "r"(kLmTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (CG == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_addr(&sh.tmem)),
+                   "r"(kLmTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_addr(&sh.tmem)),
+                   "r"(kLmTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1) __syncthreads();
+  else cluster_sync_all();  // barriers of both CTAs initialised before either signals the other
   tc_fence_after();
-  const LmWork w(sh.rows0, p.mode == kLmModeStats ? p.rows1 : 0, p.V, p.H, p.part_tiles);
+  const LmWork<CG> w(sh.rows0, p.mode == kLmModeStats ? p.rows1 : 0, p.V, p.H, p.part_tiles);
   if (warp == 0) {
-    if (lane == 0) lm_producer(p, w, sh, stages, &ma0, &ma1, &mw);
+    if (lane == 0) lm_producer<CG>(p, w, sh, stages, &ma0, &ma1, &mw, rank);
   } else if (warp == 1) {
-    if (lane == 0) lm_mma(p, w, sh, stages);
+    if (lane == 0 && rank == 0) lm_mma<CG>(p, w, sh, stages);
   } else {
-    lm_epilogue(p, w, sh);
+    lm_epilogue<CG>(p, w, sh, rank);
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 1) __syncthreads();
+  else cluster_sync_all();  // no CTA leaves while the other may still signal it
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sh.tmem),
-                 "r"(kLmTmemCols)
-                 : "memory");
+    if constexpr (CG == 1) {
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(sh.tmem),
+                   "r"(kLmTmemCols)
+                   : "memory");
+    } else {
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(sh.tmem),
+                   "r"(kLmTmemCols)
+                   : "memory");
+    }
   }
 }
 

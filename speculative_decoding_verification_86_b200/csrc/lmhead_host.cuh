@@ -22,7 +22,14 @@ struct spec_lmhead_ctx {
   int* count = nullptr;
   int32_t* votes = nullptr;     // [max_batch]
   unsigned* error = nullptr;
+  int cta_pairs = 2;            // spec_lmhead_set_cta_pairs: 0 never, 1 always, 2 row GEMM only
 };
+
+namespace {
+// CTAs per MMA of the statistics GEMM and of the row-writing GEMM.
+int stats_cta_group(const spec_lmhead_ctx* lm) { return lm->cta_pairs == 1 ? 2 : 1; }
+int rows_cta_group(const spec_lmhead_ctx* lm) { return lm->cta_pairs >= 1 ? 2 : 1; }
+}  // namespace
 
 namespace {
 
@@ -79,8 +86,45 @@ int lm_stats_part_tiles(int n_mt, int64_t V, int grid) {
   return kLmMinPartTiles;
 }
 
-int lm_grid(const spec_lmhead_ctx* lm, int64_t units) {
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, lm->vctx->num_sms)));
+// M tiles of the GEMM over rows0 (+ rows1) rows with `cg` CTAs per MMA.
+int lm_mtiles(int rows0, int rows1, int cg) {
+  const int r = sv::kLmBM * cg;
+  return (rows0 + r - 1) / r + (rows1 + r - 1) / r;
+}
+
+// Launch k_lmhead over n_mt M tiles x the vocabulary in units of p.part_tiles
+// tiles: one CTA per SM, or clusters of two CTAs (one pair per TPC).
+spec_status lm_launch(const spec_lmhead_ctx* lm, int cg, const CUtensorMap& ma0,
+                      const CUtensorMap& ma1, const void* head, int H, int64_t V,
+                      const sv::LmParams& p, int n_mt, int cls, cudaStream_t stream) {
+  CUtensorMap mw;
+  if (!bf16_tile_map(&mw, head, V, H, sv::kLmBN / cg)) return SPEC_ERR_UNSUPPORTED;
+  const int64_t units = static_cast<int64_t>(n_mt) * lm_parts(V, p.part_tiles);
+  const int groups = static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(units, lm->vctx->num_sms / cg)));
+  timing_mark(lm->vctx, cls, true, stream);
+  if (cg == 1) {
+    sv::k_lmhead<1><<<groups, sv::kLmThreads, sv::LmGeo<1>::kSmemBytes, stream>>>(ma0, ma1, mw, p);
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * groups);
+    cfg.blockDim = dim3(sv::kLmThreads);
+    cfg.dynamicSmemBytes = sv::LmGeo<2>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, sv::k_lmhead<2>, ma0, ma1, mw, p) != cudaSuccess) {
+      timing_mark(lm->vctx, cls, false, stream);
+      return SPEC_ERR_CUDA;
+    }
+  }
+  timing_mark(lm->vctx, cls, false, stream);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
 
 spec_status lm_check(const spec_lmhead_ctx* lm, int H, int64_t V, const void* head) {
@@ -138,8 +182,10 @@ spec_status spec_lmhead_init(spec_lmhead_ctx** out, spec_verify_ctx* vctx, int m
   lm->votes = reinterpret_cast<int32_t*>(b + o_votes);
   lm->error = reinterpret_cast<unsigned*>(b + o_err);
   if (cudaMemset(lm->ws, 0, off) != cudaSuccess ||
-      cudaFuncSetAttribute(sv::k_lmhead, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sv::kLmSmemBytes)) != cudaSuccess) {
+      cudaFuncSetAttribute(sv::k_lmhead<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sv::LmGeo<1>::kSmemBytes)) != cudaSuccess ||
+      cudaFuncSetAttribute(sv::k_lmhead<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(sv::LmGeo<2>::kSmemBytes)) != cudaSuccess) {
     cudaFree(lm->ws);
     delete lm;
     return SPEC_ERR_CUDA;
@@ -154,6 +200,12 @@ spec_status spec_lmhead_destroy(spec_lmhead_ctx* lm) {
   cudaDeviceSynchronize();
   cudaFree(lm->ws);
   delete lm;
+  return SPEC_OK;
+}
+
+spec_status spec_lmhead_set_cta_pairs(spec_lmhead_ctx* lm, int pairs) {
+  if (!lm || pairs < 0 || pairs > 2) return SPEC_ERR_INVALID_ARG;
+  lm->cta_pairs = pairs;
   return SPEC_OK;
 }
 
@@ -175,9 +227,8 @@ spec_status spec_lmhead_logits(spec_lmhead_ctx* lm, const void* hidden, int rows
   DeviceGuard g(lm->vctx->device);
   if (!g.ok) return SPEC_ERR_CUDA;
   cudaGetLastError();
-  CUtensorMap ma, mw;
-  if (!bf16_tile_map(&ma, hidden, rows, H, sv::kLmBM) || !bf16_tile_map(&mw, head, V, H, sv::kLmBN))
-    return SPEC_ERR_UNSUPPORTED;
+  CUtensorMap ma;
+  if (!bf16_tile_map(&ma, hidden, rows, H, sv::kLmBM)) return SPEC_ERR_UNSUPPORTED;
   sv::LmParams p{};
   p.mode = sv::kLmModeRows;
   p.H = H;
@@ -186,11 +237,8 @@ spec_status spec_lmhead_logits(spec_lmhead_ctx* lm, const void* hidden, int rows
   p.out = out_logits;
   p.error = lm->error;
   p.part_tiles = 1;  // no records: single-tile units balance the waves best
-  const int64_t units = static_cast<int64_t>((rows + sv::kLmBM - 1) / sv::kLmBM) * lm_tiles(V);
-  timing_mark(lm->vctx, kClassLmRows, true, stream);
-  sv::k_lmhead<<<lm_grid(lm, units), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(ma, ma, mw, p);
-  timing_mark(lm->vctx, kClassLmRows, false, stream);
-  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+  const int cg = rows_cta_group(lm);
+  return lm_launch(lm, cg, ma, ma, head, H, V, p, lm_mtiles(rows, 0, cg), kClassLmRows, stream);
 }
 
 spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
@@ -226,10 +274,9 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   DeviceGuard g(ctx->device);
   if (!g.ok) return SPEC_ERR_CUDA;
   cudaGetLastError();
-  CUtensorMap ma0, ma1, mw, mc;
+  CUtensorMap ma0, ma1, mc;
   if (!bf16_tile_map(&ma0, hidden_target, rows0, H, sv::kLmBM) ||
       (rows1 > 0 && !bf16_tile_map(&ma1, hidden_draft, rows1, H, sv::kLmBM)) ||
-      !bf16_tile_map(&mw, head, V, H, sv::kLmBN) ||
       !bf16_tile_map(&mc, lm->hc, static_cast<int64_t>(B) * rows, H, sv::kLmBM))
     return SPEC_ERR_UNSUPPORTED;
   if (rows1 == 0) ma1 = ma0;
@@ -242,8 +289,9 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   p.out_p = out_p;
   p.out_q = out_q;
   p.out_status = out_status;
-  const int n_mt1 = (rows0 + sv::kLmBM - 1) / sv::kLmBM + (rows1 + sv::kLmBM - 1) / sv::kLmBM;
-  const int part_tiles = lm_stats_part_tiles(n_mt1, V, ctx->num_sms);
+  const int cg1 = stats_cta_group(lm), cg2 = rows_cta_group(lm);
+  const int n_mt1 = lm_mtiles(rows0, rows1, cg1);
+  const int part_tiles = lm_stats_part_tiles(n_mt1, V, ctx->num_sms / cg1);
   const int n_parts = lm_parts(V, part_tiles);
   if (conf) launch_conf(ctx, conf, B, k, verify_len, ctx->conf_len, nullptr, stream);
   if (k > 0 && cudaMemsetAsync(ctx->tok_logits, 0, static_cast<size_t>(B) * k * 2 * sizeof(float),
@@ -267,10 +315,9 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   lp.part_tiles = part_tiles;
   lp.tok_logits = ctx->tok_logits;
   lp.error = lm->error;
-  const int64_t units1 = static_cast<int64_t>(n_mt1) * n_parts;
-  timing_mark(ctx, kClassLmStats, true, stream);
-  sv::k_lmhead<<<lm_grid(lm, units1), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(ma0, ma1, mw, lp);
-  timing_mark(ctx, kClassLmStats, false, stream);
+  if (spec_status st = lm_launch(lm, cg1, ma0, ma1, head, H, V, lp, n_mt1, kClassLmStats, stream);
+      st != SPEC_OK)
+    return st;
   sv::k_lm_combine<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
       p, lm->parts, n_parts, sv::kLmSegTiles / part_tiles, rows0);
 
@@ -293,10 +340,10 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   lr.out = lm->rows;
   lr.error = lm->error;
   lr.part_tiles = 1;
-  const int64_t units2 = static_cast<int64_t>((2 * B + sv::kLmBM - 1) / sv::kLmBM) * lm_tiles(V);
-  timing_mark(ctx, kClassLmRows, true, stream);
-  sv::k_lmhead<<<lm_grid(lm, units2), sv::kLmThreads, sv::kLmSmemBytes, stream>>>(mc, mc, mw, lr);
-  timing_mark(ctx, kClassLmRows, false, stream);
+  if (spec_status st = lm_launch(lm, cg2, mc, mc, head, H, V, lr, lm_mtiles(2 * B, 0, cg2),
+                                 kClassLmRows, stream);
+      st != SPEC_OK)
+    return st;
 
   // 4. sample: chunk masses, locate and certify, fp64 refinement where needed
   sv::k_shard_masses<false><<<B * p.n_segs, sv::kThreads, 0, stream>>>(p, 0, p.n_segs);

@@ -1,5 +1,5 @@
-"""The LM head with verification fused into its epilogue (tcgen05 GEMM),
-through the C ABI, against the fp64 oracle.
+"""The LM head with verification fused into its epilogue (tcgen05 GEMM, one
+CTA per tile and CTA pairs), through the C ABI, against the fp64 oracle.
 
 Logits: on integer grids (every product and partial sum exact in fp32) the
 GEMM's fp32 logits must equal the oracle's fp64 ones bit for bit; on
@@ -22,11 +22,11 @@ from test_gpu_parity import compare
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def lm(cuda_device):
+@pytest.fixture(scope="module", params=[0, 1, 2], ids=["cta", "cta_pairs", "default"])
+def lm(cuda_device, request):
     build.build()
     v = binding.SpecVerifier(cuda_device, max_batch=256, max_k=8, max_vocab=151936, mode="dense")
-    h = binding.LmHeadVerifier(v, max_hidden=2560)
+    h = binding.LmHeadVerifier(v, max_hidden=2560, cta_pairs=request.param)
     yield v, h
     assert h.errors() == 0
     h.close()
