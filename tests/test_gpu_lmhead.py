@@ -198,3 +198,43 @@ def test_redo_recomputes_the_same_outputs(lm):
     torch.cuda.synchronize()
     for key in keys:
         torch.testing.assert_close(keys[key], first[key], rtol=2e-6, atol=1e-9)
+
+
+def test_fused_greedy_without_drafter_hidden_states(lm):
+    """Temperature 0 everywhere: the drafter's hidden states are not needed
+    (None), the chain compares arg-maxes of the head's fp32 logits."""
+    _, h = lm
+    B, k = 12, 4
+    temps = torch.zeros(B, device="cuda")
+    w = workloads.lmhead("cuda", seed=31, B=B, k=k, V=20000, H=256, grid=True, w_levels=3,
+                         temperature=temps)
+    w = dict(w, hidden_draft=None)
+    o = h.verify(w["hidden_target"], None, w["head"], w["tokens"], temperature=temps, seed=w["seed"])
+    torch.cuda.synchronize()
+    g = {key: val.cpu().numpy() for key, val in o.items()}
+    want = oracle.verify_lmhead(_bits(w["hidden_target"]), None, _bits(w["head"]), _np(w["tokens"]),
+                                temperature=_np(temps), seed=w["seed"])
+    np.testing.assert_array_equal(g["accepted"], want["accepted"])
+    np.testing.assert_array_equal(g["tokens"], want["tokens"])
+    np.testing.assert_array_equal(g["status"], 0)
+
+
+def test_fused_with_confidence_head(lm):
+    """The confidence head truncates the verified lengths before the chain,
+    as in spec_verify_run."""
+    _, h = lm
+    B, k, Hc = 16, 5, 512
+    w = workloads.lmhead("cuda", seed=41, B=B, k=k, V=20000, H=256, grid=True, w_levels=3)
+    g = torch.Generator(device="cuda").manual_seed(41)
+    conf = dict(hidden=torch.randn((B, k, Hc), generator=g, device="cuda").to(torch.bfloat16),
+                w=(torch.randn(Hc, generator=g, device="cuda") / Hc ** 0.5).to(torch.bfloat16),
+                bias=0.5, threshold=0.3)
+    o = h.verify(w["hidden_target"], w["hidden_draft"], w["head"], w["tokens"], conf=conf,
+                 seed=w["seed"])
+    torch.cuda.synchronize()
+    gout = {key: val.cpu().numpy() for key, val in o.items()}
+    oc = dict(hidden=_bits(conf["hidden"]), w=_bits(conf["w"]), bias=0.5, threshold=0.3)
+    want = oracle.verify_lmhead(_bits(w["hidden_target"]), _bits(w["hidden_draft"]), _bits(w["head"]),
+                                _np(w["tokens"]), conf=oc, seed=w["seed"])
+    compare(gout, want)
+    assert (want["verify_len_used"] < k).any()  # the head cut some blocks
