@@ -335,12 +335,13 @@ double spec_verify_ex2_error_bound(void);
  *
  * spec_lmhead_verify computes exactly what spec_verify_run (dtype SPEC_F32,
  * dense order) computes on the logits [B, k+1, V] = hidden_target W^T and
- * [B, k, V] = hidden_draft W^T, without writing those logits: the GEMM's
- * epilogue reduces each accumulator tile to the row statistics and picks the
- * drafted tokens' logits; after the accept chains only the rows a request
- * samples from (the rejected pair, or the bonus row) are written, as fp32
- * logits, and the sample is drawn from them with the vocabulary-parallel
- * protocol's phases run as a single shard.  Outputs and random draws are those
+ * [B, k, V] = hidden_draft W^T, without writing most of those logits: the
+ * GEMM's epilogue reduces each accumulator tile to the row statistics, picks
+ * the drafted tokens' logits and writes only the position-0 rows (the rows a
+ * request samples from most often); after the accept chains a second pass
+ * writes the other rows a request samples from (the rejected pair, or the
+ * bonus row), as fp32 logits, and the sample is drawn from them with the
+ * vocabulary-parallel protocol's phases run as a single shard.  Outputs and random draws are those
  * of spec_verify_run.
  * --------------------------------------------------------------------------- */
 typedef struct spec_lmhead_ctx spec_lmhead_ctx;

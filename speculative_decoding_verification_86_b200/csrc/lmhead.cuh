@@ -6,9 +6,10 @@
 // has logits l = h W^T with the same W [V, H].  Verification needs of most rows
 // only their softmax statistics and one logit (the drafted token's), so the
 // GEMM's epilogue reduces each accumulator tile straight into the statistics
-// records the accept chain merges; the logits never reach HBM.  Only the rows
-// a request samples from (the rejected pair, or the bonus row) are produced as
-// logits, by the same kernel in its row-writing mode, after the chain decided.
+// records the accept chain merges; of all the logits only the position-0 rows
+// reach HBM (the rows most requests sample from).  The other rows a request
+// samples from (a later rejected pair, or the bonus row) are produced as
+// logits by the same kernel in its row-writing mode, after the chain decided.
 //
 // Kernel: one CTA per SM, persistent over work units (128 rows x a run of
 // 128 x 256 tiles along the vocabulary).  Warp roles:
@@ -92,9 +93,9 @@ struct LmParams {
   int n_parts;
   int part_tiles;         // N tiles per work unit (both modes)
   float* tok_logits;      // [B, k, 2] (target, drafter)
-  // rows mode
+  // rows mode (and, in statistics mode, the position-0 rows when `out` is set)
   const int64_t* dst;     // per row: element offset of its logits in `out` (-1: skip); nullptr: row * V
-  float* out;
+  float* out;             // statistics mode: the row buffer [B, k+1, V] then [B, k, V], or nullptr
   unsigned* error;        // bit 1: a wait timed out
 };
 
@@ -536,6 +537,14 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
     int64_t dst = -1;
     if (p.mode == kLmModeStats) {
       lm_row_init(p, mt, w.mt0, R, r_in_unit, st);
+      // Position 0 is the row a request samples from most often (a rejection
+      // there, or the bonus row when nothing is verified): write its logits
+      // now, so the row-writing pass only needs the rows of later positions.
+      if (p.out && st.valid && st.j == 0) {
+        const int64_t r = st.draft ? static_cast<int64_t>(p.rows0) + static_cast<int64_t>(st.i) * p.k
+                                   : static_cast<int64_t>(st.i) * (p.k + 1);
+        dst = r * p.V;
+      }
     } else {
       const int r = mt * R + r_in_unit;
       if (r < sh.rows0) dst = p.dst ? __ldg(p.dst + r) : static_cast<int64_t>(r) * p.V;
@@ -558,6 +567,7 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
         if (col < p.V) {
           if (p.mode == kLmModeStats) {
             if (st.valid) lm_consume_stats(p, st, v0, col);
+            if (dst >= 0) lm_consume_rows(p, dst, v0, col);
           } else if (dst >= 0) {
             lm_consume_rows(p, dst, v0, col);
           }
@@ -565,6 +575,7 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
         if (col + 16 < p.V) {
           if (p.mode == kLmModeStats) {
             if (st.valid) lm_consume_stats(p, st, v1, col + 16);
+            if (dst >= 0) lm_consume_rows(p, dst, v1, col + 16);
           } else if (dst >= 0) {
             lm_consume_rows(p, dst, v1, col + 16);
           }
@@ -737,7 +748,8 @@ __global__ void k_lm_combine(RunParams p, const LmPart* parts, int n_parts, int 
 }
 
 // After the chain: the rows each request samples from (the rejected pair, or
-// the bonus row), listed for the row-writing GEMM.  src: the hidden row (target
+// the bonus row), listed for the row-writing GEMM -- except position-0 rows,
+// which the statistics pass has written already.  src: the hidden row (target
 // rows first, then the drafter's, as the statistics pass numbers them); dst:
 // the element offset of the row's logits in the row buffer, laid out as
 // [B, k+1, V] target rows followed by [B, k, V] drafter rows.
@@ -748,6 +760,7 @@ __global__ void k_lm_rowlist(RunParams p, int* count, int* src, int64_t* dst) {
     const int kind = __ldcg(&p.jobs[i].kind);
     if (kind == kJobNone) continue;
     const int j = __ldcg(&p.jobs[i].row);
+    if (j == 0) continue;  // written by the statistics pass
     const int n = kind == kJobResidual ? 2 : 1;
     const int at = atomicAdd(count, n);
     const int rt = i * (p.k + 1) + j;

@@ -314,6 +314,7 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   lp.n_parts = n_parts;
   lp.part_tiles = part_tiles;
   lp.tok_logits = ctx->tok_logits;
+  lp.out = lm->rows;  // position-0 rows are written by this pass
   lp.error = lm->error;
   if (spec_status st = lm_launch(lm, cg1, ma0, ma1, head, H, V, lp, n_mt1, kClassLmStats, stream);
       st != SPEC_OK)
