@@ -238,3 +238,35 @@ def test_fused_with_confidence_head(lm):
                                 _np(w["tokens"]), conf=oc, seed=w["seed"])
     compare(gout, want)
     assert (want["verify_len_used"] < k).any()  # the head cut some blocks
+
+
+def test_fused_other_model_shapes(cuda_device):
+    """Another model family's shapes: V=262144 (a Gemma-size vocabulary),
+    H=3840, k=8 drafted positions, mixed temperatures and lengths, on the
+    exact grid: fused against the unfused path for every request and against
+    the oracle for sampled requests."""
+    build.build()
+    B, k, V, H = 32, 8, 262144, 3840
+    v = binding.SpecVerifier(cuda_device, max_batch=B, max_k=k, max_vocab=V, mode="dense")
+    h = binding.LmHeadVerifier(v, max_hidden=H)
+    try:
+        g = torch.Generator(device="cuda").manual_seed(8)
+        vlen = torch.randint(0, k + 1, (B,), generator=g, device="cuda", dtype=torch.int32)
+        temps = _temps(B, 8)
+        w = workloads.lmhead("cuda", seed=8, B=B, k=k, V=V, H=H, grid=True, temperature=temps,
+                             verify_len=vlen)
+        fused = _run_fused(h, w)
+        t = h.logits(w["hidden_target"], w["head"])
+        d = h.logits(w["hidden_draft"], w["head"])
+        o = v.run(t, d, w["tokens"], verify_len=vlen, temperature=temps, seed=w["seed"])
+        torch.cuda.synchronize()
+        o = {key: val.cpu().numpy() for key, val in o.items()}
+        for key in ("accepted", "tokens", "status"):
+            np.testing.assert_array_equal(fused[key], o[key])
+        for i in (0, 17, 31):
+            oi = _run_oracle(w, rows=slice(i, i + 1), request_offset=i)
+            compare({key: val[i:i + 1] for key, val in fused.items()}, oi)
+        assert h.errors() == 0
+    finally:
+        h.close()
+        v.close()
