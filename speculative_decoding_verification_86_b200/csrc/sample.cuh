@@ -282,7 +282,8 @@ __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const 
 // slots 0-1 and the draft's in slots 2-3 (bonus jobs: the target's only).
 static_assert(2 * kVecsPerBatch == kStepVecs, "a staging step is one batch of both rows");
 
-template <bool BF16>
+// FULL: the segment's two chunks lie inside the row, so no range checks.
+template <bool BF16, bool FULL>
 __device__ __forceinline__ void stage_sample_step(Stager& sg, const void* ra, const void* rb,
                                                   int64_t nvec, int c0, int s) {
   using G = Geo<BF16>;
@@ -291,12 +292,55 @@ __device__ __forceinline__ void stage_sample_step(Stager& sg, const void* ra, co
 #pragma unroll
   for (int u = 0; u < kVecsPerBatch; ++u) {
     const int64_t idx = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads;
-    const bool valid = idx < nvec;
+    const bool valid = FULL || idx < nvec;
     cp_async16(sg.slot(s, u), static_cast<const uint4*>(ra) + (valid ? idx : 0), valid);
     if (rb) cp_async16(sg.slot(s, kVecsPerBatch + u), static_cast<const uint4*>(rb) + (valid ? idx : 0), valid);
   }
   cp_async_commit();
   ++sg.issued;
+}
+
+// The streaming part of segment_masses_staged (FULL: no range checks).
+template <bool BF16, bool FULL>
+__device__ __forceinline__ void segment_masses_pass(const JobF32& j, const void* ra, const void* rb,
+                                                    int64_t nvec, int c0, SampleShared& sh,
+                                                    uint4* stage_buf) {
+  using G = Geo<BF16>;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int st = 0; st < kStageSlots; ++st) stage_sample_step<BF16, FULL>(sg, ra, rb, nvec, c0, st);
+  double cmass = 0.0, cbound = 0.0;
+#pragma unroll 1
+  for (int st = 0; st < kSteps; ++st) {
+    cp_async_wait(sg.issued - st - 1);
+    const int c = c0 + st / kBatchesPerChunk, b = st % kBatchesPerChunk;
+    const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
+    uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+#pragma unroll
+    for (int u = 0; u < kVecsPerBatch; ++u) {
+      const bool valid = FULL || base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads < nvec;
+      va[u] = valid ? *sg.slot(st, u) : neg_inf_vec<BF16>();
+      vb[u] = rb ? (valid ? *sg.slot(st, kVecsPerBatch + u) : neg_inf_vec<BF16>()) : va[u];
+    }
+    float sum, bound;
+    double unused;
+    batch_weights<BF16, false>(j, va, vb, sum, unused, bound);
+    cmass += static_cast<double>(sum);
+    cbound += static_cast<double>(bound);
+    if (st + kStageSlots < kSteps) stage_sample_step<BF16, FULL>(sg, ra, rb, nvec, c0, st + kStageSlots);
+    if ((st + 1) % kBatchesPerChunk == 0) {
+      const double m = warp_sum_d(cmass);
+      const double bb = warp_sum_d(cbound);
+      if (lane == 0) {
+        sh.cm[st / kBatchesPerChunk][warp] = m;
+        sh.cb[st / kBatchesPerChunk][warp] = bb;
+      }
+      cmass = 0.0;
+      cbound = 0.0;
+    }
+  }
 }
 
 template <bool BF16>
@@ -310,39 +354,10 @@ __device__ __forceinline__ void segment_masses_staged(const RunParams& p, int i,
   const int64_t nvec = p.V / G::kPerVec;
   constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
   const int c0 = seg * kChunksPerSeg;
-  Stager sg{stage_buf};
-#pragma unroll
-  for (int st = 0; st < kStageSlots; ++st) stage_sample_step<BF16>(sg, ra, rb, nvec, c0, st);
-  double cmass = 0.0, cbound = 0.0;
-#pragma unroll 1
-  for (int st = 0; st < kSteps; ++st) {
-    cp_async_wait(sg.issued - st - 1);
-    const int c = c0 + st / kBatchesPerChunk, b = st % kBatchesPerChunk;
-    const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
-    uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
-#pragma unroll
-    for (int u = 0; u < kVecsPerBatch; ++u) {
-      const bool valid = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads < nvec;
-      va[u] = valid ? *sg.slot(st, u) : neg_inf_vec<BF16>();
-      vb[u] = rb ? (valid ? *sg.slot(st, kVecsPerBatch + u) : neg_inf_vec<BF16>()) : va[u];
-    }
-    float sum, bound;
-    double unused;
-    batch_weights<BF16, false>(j, va, vb, sum, unused, bound);
-    cmass += static_cast<double>(sum);
-    cbound += static_cast<double>(bound);
-    if (st + kStageSlots < kSteps) stage_sample_step<BF16>(sg, ra, rb, nvec, c0, st + kStageSlots);
-    if ((st + 1) % kBatchesPerChunk == 0) {
-      const double m = warp_sum_d(cmass);
-      const double bb = warp_sum_d(cbound);
-      if (lane == 0) {
-        sh.cm[st / kBatchesPerChunk][warp] = m;
-        sh.cb[st / kBatchesPerChunk][warp] = bb;
-      }
-      cmass = 0.0;
-      cbound = 0.0;
-    }
-  }
+  if ((static_cast<int64_t>(c0) + kChunksPerSeg) * G::kChunkVecs <= nvec)
+    segment_masses_pass<BF16, true>(j, ra, rb, nvec, c0, sh, stage_buf);
+  else
+    segment_masses_pass<BF16, false>(j, ra, rb, nvec, c0, sh, stage_buf);
   sync_compute();
   if (threadIdx.x < kChunksPerSeg) {
     const int bc = threadIdx.x;

@@ -272,26 +272,53 @@ __device__ __forceinline__ void stochastic_segment(const void* row, int64_t V, i
 // gets the same vectors as from load_batch.
 static_assert(kBatchVecs == kStepVecs, "a staging step is one batch");
 
+// FULL: the whole segment lies inside the row (every segment but a row's
+// last), so no vector needs a range check.
+template <bool FULL = false>
 __device__ __forceinline__ void stage_segment_batch(Stager& sg, const uint4* rv, int64_t nvec,
                                                     int64_t seg0, int b) {
 #pragma unroll
   for (int u = 0; u < kBatchVecs; ++u) {
     const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
-    const bool valid = idx < nvec;
-    cp_async16(sg.slot(b, u), valid ? rv + idx : rv, valid);
+    if constexpr (FULL) {
+      cp_async16(sg.slot(b, u), rv + idx, true);
+    } else {
+      const bool valid = idx < nvec;
+      cp_async16(sg.slot(b, u), valid ? rv + idx : rv, valid);
+    }
   }
   cp_async_commit();
   ++sg.issued;
 }
 
-template <bool BF16>
+template <bool BF16, bool FULL = false>
 __device__ __forceinline__ void staged_batch(Stager& sg, int64_t nvec, int64_t seg0, int b,
                                              uint4 (&v)[kBatchVecs]) {
   cp_async_wait(sg.issued - b - 1);
 #pragma unroll
   for (int u = 0; u < kBatchVecs; ++u) {
-    const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
-    v[u] = idx < nvec ? *sg.slot(b, u) : neg_inf_vec<BF16>();
+    if constexpr (FULL) {
+      v[u] = *sg.slot(b, u);
+    } else {
+      const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
+      v[u] = idx < nvec ? *sg.slot(b, u) : neg_inf_vec<BF16>();
+    }
+  }
+}
+
+template <bool BF16, bool FULL>
+__device__ __forceinline__ void stochastic_segment_pass(const uint4* rv, int64_t nvec, int64_t seg0,
+                                                        float cc, SoftAcc& acc, uint4* stage_buf) {
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
+#pragma unroll 1
+  for (int b = 0; b < kBatches; ++b) {
+    uint4 v[kBatchVecs];
+    staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
+    soft_batch<BF16>(acc, v, cc);
+    // refill this step's slot once its values have been used
+    if (b + kStageSlots < kBatches) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
   }
 }
 
@@ -303,18 +330,9 @@ __device__ __forceinline__ void stochastic_segment_staged(const void* row, int64
   const uint4* rv = static_cast<const uint4*>(row);
   const int64_t nvec = V / G::kPerVec;
   const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
-  Stager sg{stage_buf};
-#pragma unroll
-  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch(sg, rv, nvec, seg0, b);
   SoftAcc acc;
-#pragma unroll 1
-  for (int b = 0; b < kBatches; ++b) {
-    uint4 v[kBatchVecs];
-    staged_batch<BF16>(sg, nvec, seg0, b, v);
-    soft_batch<BF16>(acc, v, cc);
-    // refill this step's slot once its values have been used
-    if (b + kStageSlots < kBatches) stage_segment_batch(sg, rv, nvec, seg0, b + kStageSlots);
-  }
+  if (seg0 + G::kSegVecs <= nvec) stochastic_segment_pass<BF16, true>(rv, nvec, seg0, cc, acc, stage_buf);
+  else stochastic_segment_pass<BF16, false>(rv, nvec, seg0, cc, acc, stage_buf);
   soft_merge_block(acc, sh, meta_out, sum_out);
 }
 
@@ -408,6 +426,21 @@ __device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int s
   g.finish(meta_out, sh);
 }
 
+template <bool BF16, bool FULL>
+__device__ __forceinline__ void greedy_segment_pass(const uint4* rv, int64_t nvec, int64_t seg0,
+                                                    GreedyScan<BF16>& g, uint4* stage_buf) {
+  Stager sg{stage_buf};
+#pragma unroll
+  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
+#pragma unroll 1
+  for (int b = 0; b < kBatches; ++b) {
+    uint4 v[kBatchVecs];
+    staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
+    g.scan(v, seg0, b);
+    if (b + kStageSlots < kBatches) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+  }
+}
+
 template <bool BF16>
 __device__ __forceinline__ void greedy_segment_staged(const void* row, int64_t V, int seg,
                                                       ChunkMeta* meta_out, StatsShared& sh,
@@ -416,17 +449,9 @@ __device__ __forceinline__ void greedy_segment_staged(const void* row, int64_t V
   const uint4* rv = static_cast<const uint4*>(row);
   const int64_t nvec = V / G::kPerVec;
   const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
-  Stager sg{stage_buf};
-#pragma unroll
-  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch(sg, rv, nvec, seg0, b);
   GreedyScan<BF16> g;
-#pragma unroll 1
-  for (int b = 0; b < kBatches; ++b) {
-    uint4 v[kBatchVecs];
-    staged_batch<BF16>(sg, nvec, seg0, b, v);
-    g.scan(v, seg0, b);
-    if (b + kStageSlots < kBatches) stage_segment_batch(sg, rv, nvec, seg0, b + kStageSlots);
-  }
+  if (seg0 + G::kSegVecs <= nvec) greedy_segment_pass<BF16, true>(rv, nvec, seg0, g, stage_buf);
+  else greedy_segment_pass<BF16, false>(rv, nvec, seg0, g, stage_buf);
   g.finish(meta_out, sh);
 }
 
