@@ -312,7 +312,8 @@ __device__ __forceinline__ void stochastic_segment_pass(const uint4* rv, int64_t
   Stager sg{stage_buf};
 #pragma unroll
   for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
-#pragma unroll 1
+  // full segments: unrolled, so slots and wait counts are compile-time constants
+#pragma unroll (FULL ? kBatches : 1)
   for (int b = 0; b < kBatches; ++b) {
     uint4 v[kBatchVecs];
     staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
