@@ -432,3 +432,16 @@ def test_maximum_block_and_vocabulary(cuda_device, dtype, V):
             compare(run_gpu(v, w), run_oracle(w))
     finally:
         v.close()
+
+
+def test_masked_logits_at_scale(ver):
+    """About 1 % of the logits of every row masked (-inf) in target and draft
+    rows: the statistics and sample passes meet masked arguments in most
+    segments (their unclamped fast paths must fall back to the clamped ones)."""
+    w = workloads.stochastic("cuda", seed=12, B=32)
+    g = torch.Generator(device="cuda").manual_seed(12)
+    for key in ("target", "draft"):
+        t = w[key]
+        mask = torch.rand(t.shape, generator=g, device="cuda") < 0.01
+        t.masked_fill_(mask, float("-inf"))
+    compare(run_gpu(ver, w), run_oracle(w))
