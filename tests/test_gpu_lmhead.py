@@ -45,7 +45,7 @@ def _grid(shape, lo, hi, scale, g):
     return (torch.randint(lo, hi + 1, shape, generator=g, device="cuda").float() * scale).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("rows,H,V", [(16, 256, 2000), (300, 200, 20000), (129, 64, 4100)])
+@pytest.mark.parametrize("rows,H,V", [(16, 256, 2000), (300, 200, 20000), (129, 64, 4100), (5, 8, 4100)])
 def test_logits_exact_grid(lm, rows, H, V):
     _, h = lm
     g = torch.Generator(device="cuda").manual_seed(rows + H)
@@ -115,6 +115,8 @@ def _temps(B, seed):
     (40, 3, 20000, 200, True),     # two M tiles per model, 5 parts over 2 segments, ragged K
     (24, 5, 151936, 256, True),    # the full head's vocabulary
     (8, 0, 4096, 128, False),      # k = 0: the bonus row only
+    (6, 2, 4100, 64, True),        # V % 16 = 4: a partial 16-column batch at every row's end
+    (1, 3, 2000, 8, False),        # B = 1, H = 8: one k-block, mostly zero-filled
 ])
 def test_fused_verify_grid_vs_oracle(lm, B, k, V, H, mixed):
     _, h = lm
