@@ -222,12 +222,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text):
+    """Source text without comments and with whitespace collapsed: a change of
+    comments alone does not change the machine code the counters describe."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel):
     from speculative_decoding_verification_86_b200 import build
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(build.CSRC, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(build.CSRC, name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

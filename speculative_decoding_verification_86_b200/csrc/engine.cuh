@@ -9,8 +9,7 @@
 // enqueues it: the chain decision after STATS (then the next position's rows,
 // the sample, or nothing), the inverse-CDF locate after SAMPLE (then nothing
 // or the fp64 refinement), the fp64 token after REFINE.  Requests advance
-// independently, and the sample pass of a request runs right after its rows
-// were streamed, while they are still in L2.
+// independently; new items join the one FIFO behind those already queued.
 //
 // Two orders of the statistics ("Speculative decoding becomes standard: DSpark
 // and multi-token drafters", section "Why draft-and-verify does not change the

@@ -12,12 +12,15 @@
 // logits by the same kernel in its row-writing mode, after the chain decided.
 //
 // Kernel: one CTA per SM, persistent over work units (128 rows x a run of
-// 128 x 256 tiles along the vocabulary).  Warp roles:
+// 128 x 256 tiles along the vocabulary), or -- the CTA-pair form -- clusters of
+// two CTAs sharing 256 x 256 tiles (see LmGeo).  Warp roles:
 //   warp 0     TMA producer: A (hidden rows, 128 x 64 bf16) and B (W rows,
-//              256 x 64 bf16) tiles, 128-byte swizzle, 4-stage ring;
+//              256 x 64 bf16, or this CTA's 128 of them in a pair) tiles,
+//              128-byte swizzle, 4-stage ring (6 stages in a pair);
 //   warp 1     TMEM owner (512 columns: two 128 x 256 fp32 accumulators) and
 //              MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
-//              M = 128, N = 256, K = 16 per instruction, one thread;
+//              M = 128 (256 for a pair, issued by rank 0), N = 256, K = 16 per
+//              instruction, one thread;
 //   warps 2-5  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, so each
 //              thread owns one row of the tile and walks its 256 columns in
 //              batches of 16 (tcgen05.ld 32x32b.x16), while the MMA warp fills
