@@ -161,6 +161,14 @@ spec_status spec_verify_run_with_uniforms(
     int32_t* out_accepted, int32_t* out_tokens, float* out_p, float* out_q,
     uint32_t* out_status, cudaStream_t stream);
 
+/* Test hook: the random draws spec_verify_run makes, written to `out`
+ * (device, [B, k+1, 2] fp64; entry [i, j, d] = U(seed, request_offset + i,
+ * position j, draw d, step)), so tests can compare the device generator with
+ * an independent one.  Asynchronous on `stream`. */
+spec_status spec_verify_draws(spec_verify_ctx* ctx, uint64_t seed, uint32_t step,
+                              uint32_t request_offset, int B, int k, double* out,
+                              cudaStream_t stream);
+
 /* Greedy (temperature 0) verification: target_logits [B, k+1, V], draft_tokens
  * [B, k]; no draft logits are read.  Outputs as in spec_verify_run. */
 spec_status spec_verify_greedy(spec_verify_ctx* ctx, const void* target_logits, spec_dtype dtype,

@@ -104,6 +104,7 @@ def lib():
                                      ctypes.POINTER(ConfArgs), _i32, _i32, _i64, _u64, _u32, _u32,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_verify_set_mode.argtypes = [_vp, _i32]
+    L.spec_verify_draws.argtypes = [_vp, _u64, _u32, _u32, _i32, _i32, _vp, _vp]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
     L.spec_verify_last_counters.argtypes = [_vp, _vp, ctypes.POINTER(_u32)]
@@ -119,7 +120,7 @@ def lib():
                  "spec_shard_refine_finish",
                  "spec_lmhead_init", "spec_lmhead_destroy", "spec_lmhead_errors",
                  "spec_lmhead_logits", "spec_lmhead_verify", "spec_lmhead_set_cta_pairs",
-                 "spec_verify_set_mode",
+                 "spec_verify_set_mode", "spec_verify_draws",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
         getattr(L, name).restype = _i32
@@ -281,6 +282,14 @@ class SpecVerifier:
             st = lib().spec_verify_run(*args, int(seed), int(step), int(request_offset), *outs)
             _check(st, "spec_verify_run")
         return o
+
+    def draws(self, B, k, seed=0, step=0, request_offset=0, stream=None):
+        """spec_verify_draws: the run's random draws, [B, k+1, 2] float64."""
+        out = torch.empty((B, k + 1, 2), dtype=torch.float64, device=self.device)
+        _check(lib().spec_verify_draws(self._h, int(seed), int(step), int(request_offset), int(B),
+                                       int(k), _dev_ptr(out), _stream_handle(stream, self.device)),
+               "spec_verify_draws")
+        return out
 
     def greedy(self, target, tokens, verify_len=None, stream=None, out=None):
         """spec_verify_greedy (temperature 0, no draft logits)."""

@@ -494,6 +494,19 @@ spec_status shard_params(spec_verify_ctx* c, int rank, int n_shards, const void*
 
 int grid_for(int64_t n) { return static_cast<int>(std::min<int64_t>((n + 255) / 256, 4096)); }
 
+// The draws of a run (spec_verify_draws).
+__global__ void k_draws(uint64_t seed, uint32_t step, uint32_t req_off, int B, int k, double* out) {
+  const int64_t n = static_cast<int64_t>(B) * (k + 1) * 2;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / 2;
+    const int d = static_cast<int>(e % 2);
+    const int i = static_cast<int>(r / (k + 1)), j = static_cast<int>(r % (k + 1));
+    out[e] = sv::draw_uniform(seed, req_off + static_cast<uint32_t>(i), static_cast<uint32_t>(j),
+                              static_cast<uint32_t>(d), step);
+  }
+}
+
 // Grid of the refinement partials: grid-strides over B x nsub items, eight CTAs per SM.
 int refine_grid(const spec_verify_ctx* c, int B, int nsub) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(static_cast<int64_t>(B) * nsub,
@@ -820,6 +833,19 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
   const int64_t ctas = static_cast<int64_t>(B) * (2 * k + 1) * n_segs;
   if (bf16) sv::k_stats<true><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
   else sv::k_stats<false><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
+}
+
+spec_status spec_verify_draws(spec_verify_ctx* ctx, uint64_t seed, uint32_t step,
+                              uint32_t request_offset, int B, int k, double* out,
+                              cudaStream_t stream) {
+  if (!ctx || !out || B < 1 || k < 0 || k > sv::kMaxK) return SPEC_ERR_INVALID_ARG;
+  if (!aligned(out, 8)) return SPEC_ERR_UNSUPPORTED;
+  DeviceGuard g(ctx->device);
+  if (!g.ok) return SPEC_ERR_CUDA;
+  cudaGetLastError();
+  k_draws<<<grid_for(static_cast<int64_t>(B) * (k + 1) * 2), 256, 0, stream>>>(seed, step,
+                                                                              request_offset, B, k, out);
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
 
