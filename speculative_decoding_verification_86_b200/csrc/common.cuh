@@ -153,9 +153,7 @@ struct RunParams {
   SampleChunk* smass;      // [B, n_chunks]
   int* refine_list;        // [B]
   unsigned* arrive_r1;     // [B]
-  unsigned* arrive_r2;     // [B]
   double2* rz;             // [B, 4 n_chunks] fp64 normaliser partials per sub-chunk
-  double2* rZ;             // [B] (unused)
   double2* rm;             // [B, 4 n_chunks] fp64 support masses (target, draft)
   int* runc;               // [B, 4 n_chunks] sub-chunks holding unsettled logits
   Counters* counters;      // this run's counters

@@ -36,10 +36,8 @@ namespace sv {
 
 constexpr uint32_t kItemStats = 0u, kItemSample = 1u, kItemRefine = 2u;
 constexpr uint32_t kItemExit = 0xFFFFFFFFu;
-constexpr unsigned kSpinLimit = 1u << 24;
+constexpr unsigned kSpinLimit = 1u << 24;  // polls of a queue slot before giving up (seconds)
 constexpr int kEngineMinBlocks = 4;  // 64 registers: four CTAs per SM (measured best)
-constexpr int kEngineThreads = kThreads;
-constexpr size_t kEngineDynSmem = 0;  // ~ seconds of polling at the sleep below
 
 __device__ __forceinline__ uint32_t item_stats(int i, int slot, int seg) {
   return (kItemStats << 30) | (static_cast<uint32_t>(i) << 14) |

@@ -119,12 +119,10 @@ struct spec_verify_ctx {
   unsigned* arrive_stats = nullptr;
   unsigned* arrive_sample = nullptr;
   unsigned* arrive_r1 = nullptr;
-  unsigned* arrive_r2 = nullptr;
   sv::Job* jobs = nullptr;
   sv::SampleChunk* smass = nullptr;
   int* refine_list = nullptr;
   double2* rz = nullptr;
-  double2* rZ = nullptr;
   double2* rm = nullptr;
   int* runc = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
@@ -181,12 +179,11 @@ spec_status carve(spec_verify_ctx* c) {
   };
   const size_t o_meta = take(recs * sizeof(sv::ChunkMeta));
   const size_t o_ssum = take(recs * sizeof(double));
-  const size_t o_arr = take(4 * static_cast<size_t>(c->max_batch) * sizeof(unsigned));
+  const size_t o_arr = take(3 * static_cast<size_t>(c->max_batch) * sizeof(unsigned));
   const size_t o_jobs = take(static_cast<size_t>(c->max_batch) * sizeof(sv::Job));
   const size_t o_smass = take(per_req_chunks * sizeof(sv::SampleChunk));
   const size_t o_rlist = take(static_cast<size_t>(c->max_batch) * sizeof(int));
   const size_t o_rz = take(per_req_subs * sizeof(double2));
-  const size_t o_rZ = take(static_cast<size_t>(c->max_batch) * sizeof(double2));
   const size_t o_rm = take(per_req_subs * sizeof(double2));
   const size_t o_runc = take(per_req_subs * sizeof(int));
   const size_t o_cnt = take(2 * sizeof(sv::Counters));
@@ -219,12 +216,10 @@ spec_status carve(spec_verify_ctx* c) {
   c->arrive_stats = arr;
   c->arrive_sample = arr + c->max_batch;
   c->arrive_r1 = arr + 2 * c->max_batch;
-  c->arrive_r2 = arr + 3 * c->max_batch;
   c->jobs = reinterpret_cast<sv::Job*>(b + o_jobs);
   c->smass = reinterpret_cast<sv::SampleChunk*>(b + o_smass);
   c->refine_list = reinterpret_cast<int*>(b + o_rlist);
   c->rz = reinterpret_cast<double2*>(b + o_rz);
-  c->rZ = reinterpret_cast<double2*>(b + o_rZ);
   c->rm = reinterpret_cast<double2*>(b + o_rm);
   c->runc = reinterpret_cast<int*>(b + o_runc);
   c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
@@ -362,9 +357,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.smass = c->smass;
   p.refine_list = c->refine_list;
   p.arrive_r1 = c->arrive_r1;
-  p.arrive_r2 = c->arrive_r2;
   p.rz = c->rz;
-  p.rZ = c->rZ;
   p.rm = c->rm;
   p.runc = c->runc;
   if (++c->run_id == 0) c->run_id = 1;
