@@ -445,3 +445,12 @@ def test_masked_logits_at_scale(ver):
         mask = torch.rand(t.shape, generator=g, device="cuda") < 0.01
         t.masked_fill_(mask, float("-inf"))
     compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_extreme_temperatures(ver):
+    """Temperatures from 1e-3 (nearly greedy: c = log2(e)/T ~ 1443, every
+    argument but the top few huge) to 100 (nearly uniform) on full-size rows."""
+    w = workloads.stochastic("cuda", seed=13, B=24)
+    temps = torch.tensor([1e-3, 5e-3, 0.02, 0.1, 3.0, 10.0, 30.0, 100.0] * 3, device="cuda")
+    w["temperature"] = temps.contiguous()
+    compare(run_gpu(ver, w), run_oracle(w))
