@@ -272,3 +272,21 @@ def test_fused_other_model_shapes(cuda_device):
     finally:
         h.close()
         v.close()
+
+
+@pytest.mark.parametrize("B,k,V,H,status", [
+    (2, 2, 2000, 12, "SPEC_ERR_UNSUPPORTED"),   # H % 8 != 0: a row is not a whole number of 16-byte units
+    (2, 2, 2002, 64, "SPEC_ERR_UNSUPPORTED"),   # V % 4 != 0
+    (2, 2, 2000, 2568, "SPEC_ERR_INVALID_ARG"),  # H above the context's max_hidden
+    (257, 1, 2000, 64, "SPEC_ERR_INVALID_ARG"),  # B above the verifier's max_batch
+    (2, 9, 2000, 64, "SPEC_ERR_INVALID_ARG"),    # k above the verifier's max_k
+])
+def test_unsupported_shapes_are_refused(lm, B, k, V, H, status):
+    """Refused before any launch, and the context stays usable afterwards."""
+    _, h = lm
+    w = workloads.lmhead("cuda", seed=1, B=B, k=k, V=V, H=H, grid=True)
+    with pytest.raises(binding.SpecVerifyError) as e:
+        _run_fused(h, w)
+    assert e.value.status == getattr(binding, status)
+    ok = workloads.lmhead("cuda", seed=2, B=4, k=3, V=2000, H=256, grid=True)
+    compare(_run_fused(h, ok), _run_oracle(ok))

@@ -454,3 +454,11 @@ def test_extreme_temperatures(ver):
     temps = torch.tensor([1e-3, 5e-3, 0.02, 0.1, 3.0, 10.0, 30.0, 100.0] * 3, device="cuda")
     w["temperature"] = temps.contiguous()
     compare(run_gpu(ver, w), run_oracle(w))
+
+
+def test_fp32_full_vocabulary_mixed_temperatures(ver):
+    """fp32 logits over the full 151936-token vocabulary with greedy and sampled
+    requests mixed in one batch."""
+    w = workloads.stochastic("cuda", seed=14, B=48, V=151936, dtype=torch.float32)
+    w["temperature"] = torch.tensor([0.0, 0.6, 1.0, 1.7] * 12, device="cuda")
+    compare(run_gpu(ver, w), run_oracle(w))
