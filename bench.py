@@ -49,14 +49,22 @@ NOMINAL_HBM_GBS = 8000.0
 
 def parse_args():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="headline")
-    ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="prefix", choices=["prefix", "dense", "auto"])
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="ranks (one per GPU, launched by torch.distributed.run when N > 1); "
+                         "each verifies its own batch (weak scaling)")
+    ap.add_argument("--steps", type=int, default=2000, help="timed steps")
+    ap.add_argument("--warmup", type=int, default=20, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
+                    help="ours: the CUDA library; reference: the fp64 CPU oracle on the host "
+                         "cores, on a bounded sample of the same workload")
+    ap.add_argument("--workload", default="headline",
+                    help="headline | stochastic | greedy | conf | conf_budget | sweep:B | lmhead")
+    ap.add_argument("--e2e-steps", type=int, default=5,
+                    help="steps of the end-to-end measurement through host buffers (0: skip)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip timing the oracle beside the GPU run")
+    ap.add_argument("--mode", default="prefix", choices=["prefix", "dense", "auto"],
+                    help="order of the statistics passes in the verification kernel")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every step (cold L2) and report the "
                          "kernel time of each launch")
@@ -303,7 +311,7 @@ def run_reference(args):
     value = tot_pos / tot_t
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": max(0, args.warmup),
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_dict(w, args.workload, 1, L),
@@ -473,7 +481,7 @@ def run_ours(args):
     step_gbs = algo_bytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
         "data": "synthetic", "config": dict(config_dict(w, args.workload, world, L), **(
             {"l2": "flushed (512 MB write) before every step; kernel time per launch"} if flush is not None else {})),
@@ -579,7 +587,7 @@ def run_vocab_parallel(args):
     line = {
         "metric": "vocabulary-parallel verification, %d ranks emulated on one GPU" % n,
         "value": positions / (slowest * 1e-3), "unit": "positions/s (slowest rank's phases)",
-        "n_gpus": 1, "steps": steps, "warmup": args.warmup, "ms_per_step_slowest_rank": slowest,
+        "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step_slowest_rank": slowest,
         "higher_is_better": True, "data": "synthetic", "dtype": "bf16" if w["target"].element_size() == 2 else "f32",
         "config": {"workload": w["name"], "vocab_bounds": bounds},
         "per_rank_ms": [{"stats": a, "decide_and_masses": b, "locate": c, "fp64_refinement": d}
@@ -782,7 +790,7 @@ def run_lmhead(args):
     achieved = flops / (st_ms * 1e-3) / 1e12
     line = {
         "metric": LM_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": lm_config(w, world),
         "roofline": {"bound": "tensor", "kernel": "k_lmhead (statistics epilogue)",
@@ -829,7 +837,7 @@ def run_lmhead_reference(args):
     value = tot_pos / tot_t
     line = {
         "impl": "reference", "metric": LM_METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": max(0, min(args.warmup, 1)),
         "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": lm_config(w, 1),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
