@@ -63,3 +63,41 @@ def test_integer_grid_is_exact():
     np.testing.assert_array_equal(got, exact)
     # the fp32 rounding the verification applies is exact on this grid
     np.testing.assert_array_equal(got.astype(np.float32).astype(np.float64), got)
+
+
+def _grid_case(seed, B, k, H, V):
+    rng = np.random.default_rng(seed)
+    ht = rng.integers(-3, 4, (B, k + 1, H))
+    hd = rng.integers(-3, 4, (B, k, H))
+    w = rng.integers(-2, 3, (V, H))
+    tokens = rng.integers(0, V, (B, k)).astype(np.int32)
+    # exact logits by integer arithmetic: (h/4)(w/8)^T = (h w^T)/32
+    lt = (np.einsum("bjh,vh->bjv", ht, w) / 32.0).astype(np.float32)
+    ld = (np.einsum("bjh,vh->bjv", hd, w) / 32.0).astype(np.float32)
+    to_bits = lambda a, s: _bits((a / s).astype(np.float32))
+    return to_bits(ht, 4.0), to_bits(hd, 4.0), to_bits(w, 8.0), tokens, lt, ld
+
+
+def test_verify_lmhead_is_verify_on_the_heads_logits():
+    """The target rows come from hidden_target, the drafter rows from
+    hidden_draft, and position j of request i from row (i, j): swapping the two
+    models, transposing the head or misaligning a position changes the result."""
+    ht, hd, w, tokens, lt, ld = _grid_case(3, B=6, k=3, H=24, V=50)
+    temps = np.array([1.0, 0.0, 0.7, 1.0, 1.3, 0.0], dtype=np.float32)
+    vlen = np.array([3, 2, 3, 0, 1, 3], dtype=np.int32)
+    got = oracle.verify_lmhead(ht, hd, w, tokens, temperature=temps, verify_len=vlen, seed=11)
+    want = oracle.verify(lt, ld, tokens, dtype=oracle.DTYPE_F32, temperature=temps,
+                         verify_len=vlen, seed=11)
+    for key in ("accepted", "tokens"):
+        np.testing.assert_array_equal(got[key], want[key])
+    np.testing.assert_array_equal(got["p_x"], want["p_x"])
+    np.testing.assert_array_equal(got["q_x"], want["q_x"])
+    # the pin is sensitive: drafter rows taken from the target's hidden states differ
+    wrong = oracle.verify(lt, lt[:, :3].copy(), tokens, dtype=oracle.DTYPE_F32,
+                          temperature=temps, verify_len=vlen, seed=11)
+    assert not np.array_equal(wrong["q_x"], want["q_x"])
+    zeros = np.zeros(6, dtype=np.float32)
+    want_greedy = oracle.verify(lt, None, tokens, dtype=oracle.DTYPE_F32, temperature=zeros)
+    greedy = oracle.verify_lmhead(ht, None, w, tokens, temperature=zeros)
+    np.testing.assert_array_equal(greedy["tokens"], want_greedy["tokens"])
+    np.testing.assert_array_equal(greedy["accepted"], want_greedy["accepted"])
