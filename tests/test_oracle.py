@@ -109,7 +109,7 @@ def _bf16_values(bits):
     return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
 
 
-@pytest.mark.parametrize("T", [0.7, 1.0, 2.5])
+@pytest.mark.parametrize("T", [1e-3, 0.7, 1.0, 2.5, 100.0])
 def test_row_softmax_matches_torch_fp64(oracle_lib, T):
     rng = np.random.default_rng(11)
     for V in (1, 7, 1000, 4099):
