@@ -7,6 +7,10 @@ imports this package, and nothing here imports the CUDA package.
 ``build()`` compiles ``oracle.c`` with gcc into ``liboracle.so`` beside it
 (no fast-math, no FMA contraction, so the arithmetic is the plain fp64 the
 source spells out).
+
+``ORACLE_LIB_OVERRIDE`` (environment) names another build of the same source
+to load instead; the mutation tests use it to check that the pins fail on a
+copy of the oracle with one planted mistake.
 """
 from __future__ import annotations
 
@@ -30,15 +34,21 @@ ERR_NONFINITE = 2
 ERR_BAD_TEMPERATURE = 4
 
 
+def compile_source(src: str, out: str) -> str:
+    """gcc with the oracle's flags: ``src`` (C) -> shared library ``out``."""
+    tmp = out + ".tmp.%d" % os.getpid()
+    subprocess.check_call([
+        "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+        "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, src, "-lm",
+    ])
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
     """Compile the oracle if the library is missing or older than its source."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call([
-            "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-            "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm",
-        ])
-        os.replace(tmp, _LIB)
+        compile_source(_SRC, _LIB)
     return _LIB
 
 
@@ -88,7 +98,7 @@ def lib():
     global _lib
     with _lock:
         if _lib is None:
-            _lib = ctypes.CDLL(build())
+            _lib = ctypes.CDLL(os.environ.get("ORACLE_LIB_OVERRIDE") or build())
             _lib.oracle_philox4x32_10.argtypes = [ctypes.c_void_p] * 3
             _lib.oracle_philox4x32_10.restype = None
             _lib.oracle_uniform.argtypes = [ctypes.c_uint64] + [ctypes.c_uint32] * 4

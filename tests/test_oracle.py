@@ -172,6 +172,20 @@ def test_conf_budget_matches_torch_fp64(oracle_lib):
     assert np.all(oracle.conf_budget(hb, wb, bias, 1.5)[0] == 0)
 
 
+def test_conf_budget_threshold_is_inclusive(oracle_lib):
+    """A survival product equal to the threshold keeps its position (P_j >= tau).
+    With h = 0 and b = 0 every s_j is sigmoid(0) = 1/2 exactly, so P_j = 2^-(j+1)
+    exactly and tau = 2^-m keeps exactly m positions."""
+    kb, H = 6, 16
+    h = np.zeros((1, kb, H), dtype=np.uint16)   # bf16 +0
+    w = np.full(H, 0x3F80, dtype=np.uint16)     # bf16 1.0 (any w gives w . 0 = 0)
+    for m in range(1, kb + 1):
+        L, surv, pref = oracle.conf_budget(h, w, 0.0, 2.0 ** -m)
+        assert surv.tolist() == [[0.5] * kb]
+        assert pref.tolist() == [[2.0 ** -(j + 1) for j in range(kb)]]
+        assert L.tolist() == [m]
+
+
 # ------------------------------------------------------- exact enumeration ----
 
 def _softmax(x, T):
@@ -380,12 +394,14 @@ def test_errors_are_found_lazily_in_chain_order(oracle_lib):
 def test_residual_floor_and_inverse_cdf_fallback(oracle_lib):
     # p and q differ by ~1e-14: rejection needs u within 1e-13 of 1 and the
     # residual mass is below the 1e-12 floor, so the token comes from p.
+    # u' = 0.2 picks token 0 of p (uniform over 4); token 0 has no residual
+    # weight (q_0 > p_0), so sampling the residual instead would give token 1.
     tgt = np.zeros((1, 2, 4), dtype=np.float32)
     drf = np.zeros((1, 1, 4), dtype=np.float32)
     drf[0, 0, 0] = np.float32(1e-13)
-    u = np.array([[[1.0 - 2.0 ** -50, 0.6], [0.5, 0.5]]])
+    u = np.array([[[1.0 - 2.0 ** -50, 0.2], [0.5, 0.5]]])
     res = oracle.verify(tgt, drf, np.array([[0]], dtype=np.int32), dtype=F32, u_override=u)
-    assert res["accepted"][0] == 0 and res["tokens"][0, 0] == 2
+    assert res["accepted"][0] == 0 and res["tokens"][0, 0] == 0
     # u = 1 lies past every cell: the largest index with positive weight is taken
     tgt = np.array([[[0.0, 1.0, -np.inf, 2.0, -np.inf]]], dtype=np.float32)
     u = np.array([[[0.5, 1.0]]])
