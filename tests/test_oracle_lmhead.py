@@ -2,10 +2,12 @@
 against what fixes them independently: exact widening of known bf16 bit
 patterns, a brute-force correctly rounded sum per logit, one-hot rows that
 select a column of W, and integer grids whose product is an exact integer
-matmul."""
+matmul.  The last test plants mistakes in the oracle's shared-head functions
+(in this process, by monkeypatch) and checks that a pin fails on each."""
 import math
 
 import numpy as np
+import pytest
 
 import oracle
 
@@ -101,3 +103,47 @@ def test_verify_lmhead_is_verify_on_the_heads_logits():
     greedy = oracle.verify_lmhead(ht, None, w, tokens, temperature=zeros)
     np.testing.assert_array_equal(greedy["tokens"], want_greedy["tokens"])
     np.testing.assert_array_equal(greedy["accepted"], want_greedy["accepted"])
+
+
+# ------------------------------------------ the pins catch planted mistakes --
+
+def _bf16_round(a):
+    """float64 -> nearest bf16 value (round to nearest even), as float64."""
+    u = np.asarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+_PINS = [test_bf16_widening_known_patterns, test_logits_brute_force, test_one_hot_rows_select_a_column,
+         test_integer_grid_is_exact, test_verify_lmhead_is_verify_on_the_heads_logits]
+
+
+def _mutants():
+    good_widen, good_logits, good_verify = oracle.bf16_to_f64, oracle.lmhead_logits, oracle.verify
+    return {
+        "bf16 widened from the wrong half": ("bf16_to_f64", lambda b: (
+            (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(15))
+            .view(np.float32).astype(np.float64))),
+        "logits accumulated in fp32": ("lmhead_logits", lambda h, w: (
+            good_widen(h).astype(np.float32) @ good_widen(w).astype(np.float32).T).astype(np.float64)),
+        "head not transposed": ("lmhead_logits", lambda h, w: good_widen(h) @ good_widen(w)),
+        "logits rounded to bf16": ("lmhead_logits", lambda h, w: _bf16_round(good_logits(h, w))),
+        "drafter rows from the target's hidden states": ("verify_lmhead", lambda ht, hd, w, tok, **kw: (
+            good_verify(good_logits(ht, w).astype(np.float32),
+                        None if hd is None else good_logits(ht[..., :hd.shape[1], :], w).astype(np.float32),
+                        tok, dtype=oracle.DTYPE_F32, **kw))),
+    }
+
+
+@pytest.mark.parametrize("name", list(_mutants()))
+def test_planted_mistakes_fail_a_pin(monkeypatch, name):
+    attr, fn = _mutants()[name]
+    monkeypatch.setattr(oracle, attr, fn)
+    caught = 0
+    for pin in _PINS:
+        try:
+            with np.errstate(all="ignore"):  # a mutant may overflow
+                pin()
+        except (AssertionError, ValueError):
+            caught += 1
+    assert caught > 0, name
