@@ -410,6 +410,24 @@ def test_residual_floor_and_inverse_cdf_fallback(oracle_lib):
     assert res["accepted"][0] == 0 and res["tokens"][0, 0] == 3
 
 
+def test_verify_len_is_clamped_to_the_block(oracle_lib):
+    """L_i = verify_len_i clamped to [0, k] (a negative length verifies
+    nothing); with L_i = 0 a request emits one token from target row 0 and
+    accepts none."""
+    rng = np.random.default_rng(17)
+    B, k, V = 6, 3, 16
+    target = rng.standard_normal((B, k + 1, V)).astype(np.float32)
+    draft = rng.standard_normal((B, k, V)).astype(np.float32)
+    tokens = rng.integers(0, V, (B, k)).astype(np.int32)
+    vlen = np.array([-5, -1, 0, 2, 3, 9], dtype=np.int32)
+    res = oracle.verify(target, draft, tokens, dtype=F32, verify_len=vlen, seed=4)
+    assert res["verify_len_used"].tolist() == [0, 0, 0, 2, 3, 3]
+    assert np.all(res["accepted"] <= res["verify_len_used"])
+    for i in range(3):
+        assert res["accepted"][i] == 0
+        assert 0 <= res["tokens"][i, 0] < V and np.all(res["tokens"][i, 1:] == -1)
+
+
 def test_empty_batch(oracle_lib):
     res = oracle.verify(np.zeros((0, 3, 8), dtype=np.float32), np.zeros((0, 2, 8), dtype=np.float32),
                         np.zeros((0, 2), dtype=np.int32), dtype=F32)

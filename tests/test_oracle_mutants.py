@@ -14,7 +14,9 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_budget.py"]
 
-# name -> (exact text in oracle.c, its mutated form)
+# name -> (exact text in oracle.c, its mutated form).  Only mistakes that change
+# a result belong here: for example, counting every position with P_j >= tau
+# instead of the leading run would change nothing, since P never grows.
 MUTANTS = {
     # accept / reject rule
     "accept comparison not strict": ("if (u * q < p) {", "if (u * q <= p) {"),
@@ -61,13 +63,31 @@ MUTANTS = {
                                             "if (x->P != y->P) return x->P < y->P ? -1 : 1;"),
     "budget ties to the higher request": ("if (x->i != y->i) return x->i < y->i ? -1 : 1;",
                                           "if (x->i != y->i) return x->i > y->i ? -1 : 1;"),
+    "negative verify_len not clamped": ("if (L < 0) L = 0;", "if (L < 0) L = -L;"),
+    # the accept test's probabilities
+    "q of the drafted token read from the target row": (
+        "double q = exp(load_logit(drow, in->dtype, x[j]) / T - mq) / Zq;",
+        "double q = exp(load_logit(trow, in->dtype, x[j]) / T - mq) / Zq;"),
+    "p normalised by the drafter's sum": (
+        "double p = exp(load_logit(trow, in->dtype, x[j]) / T - mp) / Zp;",
+        "double p = exp(load_logit(trow, in->dtype, x[j]) / T - mp) / Zq;"),
+    "residual q normalised by the target's sum": (
+        "double q = exp(load_logit(c->drow, c->dtype, t) / c->T - c->mq) / c->Zq;",
+        "double q = exp(load_logit(c->drow, c->dtype, t) / c->T - c->mq) / c->Zp;"),
+    # the uniform's 53 bits
+    "uniform scaled by 2^53 - 1": ("/ 9007199254740992.0;", "/ 9007199254740991.0;"),
+    "uniform high word shifted one bit less": ("double hi = (double)(w[0] >> 5);",
+                                               "double hi = (double)(w[0] >> 4);"),
+    # chain bookkeeping
+    "stochastic rejection counts the rejected position": ("            n = j;\n            break;\n        }\n        if (!err && n == L) {\n            /* 4.",
+                                                          "            n = j + 1;\n            break;\n        }\n        if (!err && n == L) {\n            /* 4."),
 }
 
 
-def _run_pins_on(name, old, new, tmp_path):
+def _run_pins_on(index, name, old, new, tmp_path):
     src = open(os.path.join(ROOT, "oracle", "oracle.c")).read()
     assert src.count(old) == 1, "mutation site not unique: %s" % name
-    d = tmp_path / ("m%d" % (abs(hash(name)) % 10 ** 8))
+    d = tmp_path / ("mutant%02d" % index)
     d.mkdir()
     c_path = d / "oracle.c"
     c_path.write_text(src.replace(old, new))
@@ -83,7 +103,8 @@ def _run_pins_on(name, old, new, tmp_path):
 def test_every_planted_mistake_fails_a_pin(tmp_path):
     oracle.build()
     with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
-        futs = {n: ex.submit(_run_pins_on, n, o, m, tmp_path) for n, (o, m) in MUTANTS.items()}
+        futs = {n: ex.submit(_run_pins_on, q, n, o, m, tmp_path)
+                for q, (n, (o, m)) in enumerate(MUTANTS.items())}
         results = {n: f.result() for n, f in futs.items()}
     survivors = sorted(n for n, (rc, _) in results.items() if rc == 0)
     broken = sorted(n for n, (rc, _) in results.items() if rc not in (0, 1))
