@@ -391,6 +391,27 @@ def test_errors_are_found_lazily_in_chain_order(oracle_lib):
     assert np.all(res["tokens"][[0, 2, 3]] == -1)
 
 
+def test_greedy_chain_fails_on_a_nonfinite_row(oracle_lib):
+    """T = 0 reads target rows only; NaN or +inf in a row it reads fails the
+    request, while -inf (a masked token) does not, and a bad value in a row
+    past the first disagreement is never read."""
+    V, k = 8, 2
+    tgt = np.zeros((4, k + 1, V), dtype=np.float32)
+    tgt[:, :, 5] = 1.0                   # arg-max 5 everywhere
+    toks = np.full((4, k), 5, dtype=np.int32)
+    tgt[0, 1, 2] = np.inf                # request 0: +inf in row 1, which the chain reads
+    tgt[1, 0, 6] = np.nan                # request 1: NaN in row 0
+    tgt[2, 0, 0] = -np.inf               # request 2: a masked token only
+    toks[3, 0] = 4                       # request 3: disagrees at position 0 ...
+    tgt[3, 1, 0] = np.inf                # ... so row 1's +inf is never read
+    with pytest.raises(ValueError):
+        oracle.row_argmax(np.array([0.0, np.inf, 1.0], dtype=np.float32), F32)
+    res = oracle.verify(tgt, None, toks, dtype=F32, temperature=np.zeros(4, dtype=np.float32))
+    assert res["status"].tolist() == [oracle.ERR_NONFINITE, oracle.ERR_NONFINITE, 0, 0]
+    assert res["accepted"].tolist() == [-1, -1, 2, 0]
+    assert res["tokens"][2].tolist() == [5, 5, 5] and res["tokens"][3].tolist() == [5, -1, -1]
+
+
 def test_residual_floor_and_inverse_cdf_fallback(oracle_lib):
     # p and q differ by ~1e-14: rejection needs u within 1e-13 of 1 and the
     # residual mass is below the 1e-12 floor, so the token comes from p.

@@ -16,7 +16,9 @@ PIN_FILES = ["tests/test_oracle.py", "tests/test_oracle_budget.py"]
 
 # name -> (exact text in oracle.c, its mutated form).  Only mistakes that change
 # a result belong here: for example, counting every position with P_j >= tau
-# instead of the leading run would change nothing, since P never grows.
+# instead of the leading run would change nothing, since P never grows; and a
+# NaN or +inf that the sampled rows' scan missed would still fail the request
+# through the checks on the maximum and the normaliser.
 MUTANTS = {
     # accept / reject rule
     "accept comparison not strict": ("if (u * q < p) {", "if (u * q <= p) {"),
@@ -78,6 +80,14 @@ MUTANTS = {
     "uniform scaled by 2^53 - 1": ("/ 9007199254740992.0;", "/ 9007199254740991.0;"),
     "uniform high word shifted one bit less": ("double hi = (double)(w[0] >> 5);",
                                                "double hi = (double)(w[0] >> 4);"),
+    # error semantics
+    "+inf in a greedy row not detected": (
+        "        if (isnan(v) || v == INFINITY) return ORC_ERR_NONFINITE;\n        if (best_t < 0",
+        "        if (isnan(v)) return ORC_ERR_NONFINITE;\n        if (best_t < 0"),
+    "drafted token V accepted as in range": (
+        "if (x[j] < 0 || (int64_t)x[j] >= V) { err = ORC_ERR_BAD_TOKEN; break; }\n            const void* trow",
+        "if (x[j] < 0 || (int64_t)x[j] > V) { err = ORC_ERR_BAD_TOKEN; break; }\n            const void* trow"),
+    "negative temperature accepted": ("if (!(T >= 0.0f) || isinf(T)) return 0;", "if (isinf(T)) return 0;"),
     # chain bookkeeping
     "stochastic rejection counts the rejected position": ("            n = j;\n            break;\n        }\n        if (!err && n == L) {\n            /* 4.",
                                                           "            n = j + 1;\n            break;\n        }\n        if (!err && n == L) {\n            /* 4."),
