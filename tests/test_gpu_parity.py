@@ -237,7 +237,8 @@ def test_draws_on_decision_boundaries_take_the_fp64_paths(ver):
     assert c["accept_fp64"] > 0 and c["sample_fp64"] > 0
 
 
-def test_residual_floor_and_fallback_through_refinement(ver):
+@pytest.mark.parametrize("u_floor,tok_floor", [(0.6, 38), (0.01, 0)])
+def test_residual_floor_and_fallback_through_refinement(ver, u_floor, tok_floor):
     V = 64
     t = torch.zeros((2, 2, V), dtype=torch.float32)
     d = torch.zeros((2, 1, V), dtype=torch.float32)
@@ -245,12 +246,14 @@ def test_residual_floor_and_fallback_through_refinement(ver):
     t[1, 0, 40:] = float("-inf")  # request 1: x = 50 is masked in the target -> rejected
     w = dict(target=t.cuda(), draft=d.cuda(), tokens=torch.tensor([[0], [50]], dtype=torch.int32).cuda(),
              verify_len=None, temperature=None, conf=None, seed=0)
-    u = np.array([[[1 - 2.0 ** -50, 0.6], [0.5, 0.5]],
+    u = np.array([[[1 - 2.0 ** -50, u_floor], [0.5, 0.5]],
                   [[0.5, 1.0], [0.5, 0.5]]])            # u' = 1: past every cell
     o = run_oracle(w, u_override=u)
     g = run_gpu(ver, w, uniforms=torch.from_numpy(u).cuda())
     compare(g, o, strict=True)
-    assert o["tokens"][0, 0] == 38       # floor: drawn from p (uniform over 64) at u' = 0.6
+    # floor: drawn from p (uniform over 64).  At u' = 0.01 the residual, which
+    # has no weight on token 0 (q_0 > p_0), would give token 1 instead.
+    assert o["tokens"][0, 0] == tok_floor
     assert o["tokens"][1, 0] == 39       # fallback: last index with positive residual
 
 
