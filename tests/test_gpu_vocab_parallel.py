@@ -1,12 +1,15 @@
 """Vocabulary-parallel verification (logits split by vocabulary over ranks),
 run on one device: every rank is its own context with its slice of the
 logits, the all-gathers are concatenations and the max over ranks a torch.max
-(no kernel waits on another).  The result must equal the single-rank run
-element for element; the single-rank run is itself pinned to the oracle."""
+(no kernel waits on another).  Every case is checked twice: against the fp64
+CPU oracle on the same inputs (the same bar as the single-rank parity tests),
+and against the single-rank run element for element, since the merged
+statistics records of the ranks equal the single-rank records exactly."""
 import numpy as np
 import pytest
 import torch
 
+from parity_helpers import compare, host, run_oracle
 from speculative_decoding_verification_86_b200 import binding, build, workloads
 
 pytestmark = pytest.mark.gpu
@@ -50,6 +53,8 @@ def _run(single, w, n):
         v = votes.cpu().numpy()
         assert np.all((v >= 0).sum(axis=0) <= 1)
         _check_equal(ref, final, "n=%d" % n)
+        # the sharded result against the oracle directly
+        compare(host(final), run_oracle(w))
         return info
     finally:
         for r in ranks:
