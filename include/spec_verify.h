@@ -184,10 +184,11 @@ spec_status spec_verify_greedy(spec_verify_ctx* ctx, const void* target_logits, 
  * cudaMalloc's implicit synchronisation.  It computes exactly what
  * spec_verify_greedy computes, with the same arguments minus the context; the
  * current device is used.
- * Working space: a fixed array inside the library (about 2.3 MB per GPU that
- * loads it, kept until the process exits).  Limits: 0 <= B <= 256, 0 <= k <= 8,
- * and B * (2k + 1) * ceil(V / chunk) <= 139264, with chunk = 8192 (bf16) or 4096
- * (fp32) logits -- V up to 262144 (bf16) / 131072 (fp32) at B = 256, k = 8.
+ * Working space: a fixed array inside the library (about 0.6 MB per GPU that
+ * loads it, kept until the process exits), holding one 16-byte statistics
+ * record per (request, row slot, segment).  Limits: 0 <= B <= 256, 0 <= k <= 8,
+ * and B * (2k + 1) * ceil(V / segment) <= 34816, with segment = 32768 (bf16) or
+ * 16384 (fp32) logits -- V up to 262144 (bf16) / 131072 (fp32) at B = 256, k = 8.
  * Larger calls return SPEC_ERR_INVALID_ARG without launching anything.
  * No cudaMalloc/cudaFree is made.  The first call on a device looks up the
  * array's device address (once per device; make that first call before any
@@ -317,10 +318,13 @@ spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launch
  * out[0] = accept decisions settled by the fp64 path, out[1] = samples refined
  * in fp64, out[2] = samples certified by the fp32 filter, out[3] = chunks the
  * fp64 refinement recomputed outright, out[4] = engine error bits (0 on a good
- * run; 1 a wait for work timed out, 2 the work queue overflowed -- the run's
- * outputs are then not to be used). */
+ * run; bit 1 the work queue overflowed, any other bit a bounded wait of the
+ * engine gave up -- the run's outputs are then not to be used), out[5] = where
+ * the first such wait gave up (0 if none): site << 28 | CTA << 16 | its stage
+ * or item count, the site being 1 + the index of its error bit.  `out` holds
+ * 6 values. */
 spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
-                                      uint32_t out[5]);
+                                      uint32_t out[6]);
 
 /* Self-check of the one hardware constant the fp32 filter relies on: the
  * maximum relative error of the ex2.approx.ftz.f32 instruction against fp64

@@ -383,11 +383,11 @@ class SpecVerifier:
         return n.value, ms.value
 
     def last_counters(self, stream=None):
-        out = (_u32 * 5)()
+        out = (_u32 * 6)()
         _check(lib().spec_verify_last_counters(self._h, _stream_handle(stream, self.device), out),
                "spec_verify_last_counters")
         return dict(accept_fp64=out[0], sample_fp64=out[1], sample_fp32=out[2], chunks_fp64=out[3],
-                    engine_error=out[4])
+                    engine_error=out[4], wait_fail=out[5])
 
 
 def greedy_noalloc(target, tokens, verify_len=None, stream=None, out=None):
@@ -558,16 +558,28 @@ def _redo_requests(ver, redo, rows_of, tokens, verify_len, temperature, conf, se
                     verify_len=None if verify_len is None else verify_len[sl].contiguous(),
                     temperature=None if temperature is None else temperature[sl].contiguous(),
                     conf=c, seed=seed, step=step, request_offset=request_offset + i)
-        for key in out:
+        for key in o:
             out[key][sl] = o[key]
+        if "redo" in out:
+            out["redo"][sl] = 0
     return idx
 
 
 def verify_vocab_parallel(rank_obj, target, draft, tokens, V, verify_len=None, temperature=None,
-                          conf=None, seed=0, step=0, request_offset=0, group=None):
+                          conf=None, seed=0, step=0, request_offset=0, group=None, redo_whole=True):
     """Vocabulary-parallel verification on this rank's shard with
     torch.distributed collectives (all ranks call it with the same arguments
-    apart from their shards).  Returns the outputs (identical on every rank)."""
+    apart from their shards).  Returns the outputs (identical on every rank).
+
+    Every phase always runs, the fp64 refinement included (its kernels skip
+    the requests that do not need it), so a step is kernel launches and
+    collectives with no host round trip.  The one exception is a request whose
+    decision needs rows of every rank (out["redo"] == 1 on the device: an
+    accept draw inside the fp32 bound, about one decision in 10^5, or a
+    refinement whose support was not settled).  With ``redo_whole`` (the
+    default) such requests are found on the host and verified whole from
+    gathered rows; ``redo_whole=False`` leaves that to the caller and keeps the
+    step free of host synchronisation."""
     import torch.distributed as dist
     n, r = rank_obj.n, rank_obj.rank
     B, kp1, _ = target.shape
@@ -588,15 +600,18 @@ def verify_vocab_parallel(rank_obj, target, draft, tokens, V, verify_len=None, t
     dist.all_gather_into_tensor(all2, blk2, group=group)
     rank_obj.locate(all2, target, draft, tokens, V, votes, **kw)
     dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
-    redo = rank_obj.finish(votes, out)
-    if bool((redo == 2).any()):  # the same on every rank: the decisions are replicated
-        blk3 = torch.empty(b3, dtype=torch.uint8, device=dev)
-        all3 = torch.empty(n * b3, dtype=torch.uint8, device=dev)
-        rank_obj.refine_partials(target, draft, tokens, V, blk3, **kw)
-        dist.all_gather_into_tensor(all3, blk3, group=group)
-        rank_obj.refine_locate(all3, target, draft, tokens, V, votes, **kw)
-        dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
-        redo = rank_obj.refine_finish(votes, out)
+    rank_obj.finish(votes, out)
+    # the fp64 refinement phase, a no-op for requests that do not need it
+    blk3 = torch.empty(b3, dtype=torch.uint8, device=dev)
+    all3 = torch.empty(n * b3, dtype=torch.uint8, device=dev)
+    rank_obj.refine_partials(target, draft, tokens, V, blk3, **kw)
+    dist.all_gather_into_tensor(all3, blk3, group=group)
+    rank_obj.refine_locate(all3, target, draft, tokens, V, votes, **kw)
+    dist.all_reduce(votes, op=dist.ReduceOp.MAX, group=group)
+    redo = rank_obj.refine_finish(votes, out)
+    out["redo"] = redo
+    if not redo_whole:
+        return out
 
     widths = [bounds[q + 1] - bounds[q] for q in range(n)]
     wmax = max(widths)

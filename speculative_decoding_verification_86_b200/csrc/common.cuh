@@ -108,16 +108,39 @@ struct Counters {
   unsigned accept_slow;    // accept decisions resolved in fp64
   unsigned sample_fast;    // samples certified by the fp32 filter
   unsigned chunks_redone;  // refinement chunks recomputed outright (support unsettled)
-  unsigned queue_error;    // engine: 1 a wait for work gave up, 2 the queue overflowed
-  unsigned pad[3];
+  unsigned queue_error;    // engine: bits of the waits that gave up (see engine.cuh), 2 the queue overflowed
+  unsigned wait_fail;      // engine: the first wait that gave up: site << 28 | CTA << 16 | stage (low 16 bits)
+  unsigned pad[2];
 };
 
 // Engine: orders of the statistics pass, and the queue's control words.
 constexpr int kModeDense = 0;
 constexpr int kModePrefix = 1;
-constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQWords = 8;
+// head: implicit tickets handed out; tail / gen_head: generated items reserved /
+// claimed; done: requests finished; exits: CTAs that left; conf_done: the
+// epoch of the run whose confidence budgets are published.
+constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQGenHead = 4, kQConfDone = 5,
+              kQWords = 8;
 
 // -------------------------------------------------------------- run params --
+struct ConfParams {
+  const uint16_t* hidden;  // [B, kb, H] bf16 bits
+  const uint16_t* w;       // [H]
+  float bias;
+  float threshold;
+  int B;
+  int kb;
+  int H;
+  int k;                   // verify_len cap applies when >= 0 (clamp to [0, k])
+  const int32_t* vlen;     // [B] or nullptr (=> k)
+  long long total;         // batch-wide verify budget; <= 0: none
+  double* prefix;          // [B, kb] workspace: prefix survival (total > 0)
+  int32_t* cap;            // [B] workspace: per-request limit before the batch budget
+  unsigned* arrive;        // arrival counter (self-resetting)
+  int32_t* out_len;        // [B]
+  float* out_survival;     // [B, kb] or nullptr
+};
+
 struct RunParams {
   const void* target;      // [B, k+1, V]
   const void* draft;       // [B, k, V] or nullptr
@@ -137,6 +160,7 @@ struct RunParams {
   uint32_t step;
   uint32_t req_off;
   int force_greedy;        // every request at T = 0 (spec_verify_greedy)
+  int launch_rows;         // k_stats: row slots per request in its grid (0: all 2k + 1)
   float eps_ex2;           // certified relative error of ex2.approx.ftz.f32
 
   int32_t* out_acc;
@@ -171,27 +195,12 @@ struct RunParams {
   unsigned long long* q_slots;     // queue: (epoch << 32) | payload
   unsigned q_capacity;
   unsigned q_epoch;                // this run's epoch, never 0
-  unsigned* q_ctl;                 // head, tail, done, exits
+  unsigned* q_ctl;                 // the queue's control words (kQ*)
   unsigned n_init;                 // implicit initial tickets
+  unsigned n_conf;                 // of which the confidence head's (one per request, or 0)
+  ConfParams cp;                   // the confidence head run inside the engine (n_conf > 0)
 };
 
-struct ConfParams {
-  const uint16_t* hidden;  // [B, kb, H] bf16 bits
-  const uint16_t* w;       // [H]
-  float bias;
-  float threshold;
-  int B;
-  int kb;
-  int H;
-  int k;                   // verify_len cap applies when >= 0 (clamp to [0, k])
-  const int32_t* vlen;     // [B] or nullptr (=> k)
-  long long total;         // batch-wide verify budget; <= 0: none
-  double* prefix;          // [B, kb] workspace: prefix survival (total > 0)
-  int32_t* cap;            // [B] workspace: per-request limit before the batch budget
-  unsigned* arrive;        // arrival counter (self-resetting)
-  int32_t* out_len;        // [B]
-  float* out_survival;     // [B, kb] or nullptr
-};
 
 // ------------------------------------------------------------ device utils --
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
@@ -385,23 +394,30 @@ __device__ __forceinline__ const void* draft_row(const RunParams& p, int i, int 
 }
 
 struct ReqInfo {
-  int L;        // verified positions
-  float T;      // temperature
+  int L;          // verified positions
+  int Lcap;       // verify_len clamped to [0, k]: L before the confidence head's budget
+  float T;        // temperature
   bool greedy;
-  bool bad_T;
+  bool bad_T;     // the request fails: invalid temperature, or sampled positions without drafter logits
+  bool invalid_T; // the temperature alone is invalid
+  bool no_draft;  // sampled request and no drafter logits in the call
 };
 
-__device__ __forceinline__ ReqInfo request_info(const RunParams& p, int i) {
+// with_conf: apply the confidence head's budget (conf_len, once published);
+// without it L = Lcap, which is what the plan of reads is built on.
+__device__ __forceinline__ ReqInfo request_info(const RunParams& p, int i, bool with_conf = true) {
   ReqInfo r;
   int L = p.vlen ? __ldg(p.vlen + i) : p.k;
   L = max(0, min(L, p.k));
-  if (p.conf_len) L = min(L, __ldg(p.conf_len + i));
+  r.Lcap = L;
+  if (p.conf_len && with_conf) L = min(L, __ldcg(p.conf_len + i));
   r.L = L;
   r.T = p.force_greedy ? 0.0f : (p.temp ? __ldg(p.temp + i) : 1.0f);
-  r.bad_T = !temperature_valid(r.T);
-  r.greedy = !r.bad_T && r.T == 0.0f;
+  r.invalid_T = !temperature_valid(r.T);
+  r.greedy = !r.invalid_T && r.T == 0.0f;
+  r.no_draft = !r.invalid_T && !r.greedy && p.draft == nullptr;
   // a sampled request that verifies any position needs the drafter's logits
-  if (!r.bad_T && !r.greedy && r.L > 0 && p.draft == nullptr) r.bad_T = true;
+  r.bad_T = r.invalid_T || (r.no_draft && r.L > 0);
   return r;
 }
 

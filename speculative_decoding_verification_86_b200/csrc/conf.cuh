@@ -25,24 +25,33 @@
 
 namespace sv {
 
-// Last CTA of k_conf: the batch-wide selection.  Reads the prefix products and
-// per-request limits every CTA published, writes out_len.  Batches of up to
-// kSelCache candidate slots are first copied to shared memory (one pass of
-// independent loads), so the eight radix passes and the final count run on
-// shared memory; larger batches stream the candidates from L2 in every pass.
-constexpr int kSelCache = 4096;
+// The batch-wide selection, run by the CTA that completes the last request's
+// budget.  Reads the prefix products and per-request limits every CTA
+// published, writes out_len.  Batches of up to `cache` candidate slots are
+// first copied to shared memory (one pass of independent loads), so the eight
+// radix passes and the final count run on shared memory; larger batches stream
+// the candidates from L2 in every pass.
+constexpr int kSelCache = 4096;        // candidate cache of the standalone k_conf
+constexpr int kSelCacheEngine = 1024;  // ... of the verification engine (shared memory is the ring's)
 constexpr unsigned long long kNoKey = ~0ull;  // not a candidate (valid keys are <= bits of 1.0)
 static_assert(kThreads == 256, "one radix bin per thread");
 
-__device__ void conf_select(const ConfParams& cp) {
-  __shared__ unsigned long long s_keys[kSelCache];
-  __shared__ unsigned hist[256];
-  __shared__ double sh_d[kWarps];
-  __shared__ unsigned long long s_key;
-  __shared__ long long s_rank;
+struct ConfSelectShared {
+  unsigned hist[256];
+  double sh_d[kWarps];
+  unsigned long long key;
+  long long rank;
+};
+
+__device__ void conf_select(const ConfParams& cp, ConfSelectShared& ss, unsigned long long* s_keys,
+                            int cache) {
+  unsigned* hist = ss.hist;
+  double* sh_d = ss.sh_d;
+  unsigned long long& s_key = ss.key;
+  long long& s_rank = ss.rank;
   const int B = cp.B, kb = cp.kb;
   const long long n = static_cast<long long>(B) * kb;
-  const bool cached = n <= kSelCache;
+  const bool cached = n <= cache;
   auto load_key = [&](long long e) -> unsigned long long {
     const int i = static_cast<int>(e / kb), j = static_cast<int>(e - static_cast<long long>(i) * kb);
     if (j >= __ldcg(cp.cap + i)) return kNoKey;
@@ -116,10 +125,10 @@ __device__ void conf_select(const ConfParams& cp) {
   }
 }
 
-__global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
-  __shared__ double s_surv[kMaxK];
-  __shared__ int s_last;
-  const int i = blockIdx.x;
+// Per-request part, one CTA (kThreads compute threads) per request: s_j for
+// each position (one warp per position, fp64 dot), then the prefix product,
+// the budget and, with a batch budget, the published prefix and limit.
+__device__ void conf_request(const ConfParams& cp, int i, double* s_surv) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int j = warp; j < cp.kb; j += kWarps) {
     const uint16_t* h = cp.hidden + (static_cast<int64_t>(i) * cp.kb + j) * cp.H;
@@ -132,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
     z = warp_sum_d(z);
     if (lane == 0) s_surv[j] = 1.0 / (1.0 + exp(-(z + static_cast<double>(cp.bias))));
   }
-  __syncthreads();
+  sync_compute();
   if (threadIdx.x == 0) {
     double prefix = 1.0;
     int budget = 0;
@@ -152,10 +161,19 @@ __global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
     if (cp.total > 0) cp.cap[i] = budget;
     else cp.out_len[i] = budget;
   }
+  sync_compute();
+}
+
+__global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
+  __shared__ double s_surv[kMaxK];
+  __shared__ int s_last;
+  __shared__ ConfSelectShared ss;
+  __shared__ unsigned long long s_keys[kSelCache];
+  conf_request(cp, blockIdx.x, s_surv);
   if (cp.total <= 0) return;
   if (!arrive_last(cp.arrive, static_cast<unsigned>(cp.B), &s_last)) return;
   __threadfence();
-  conf_select(cp);
+  conf_select(cp, ss, s_keys, kSelCache);
 }
 
 }  // namespace sv

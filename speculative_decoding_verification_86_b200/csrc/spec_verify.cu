@@ -57,15 +57,17 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // ---------------------------------------------------------------------------
 // Scratch of spec_verify_greedy_noalloc.  Callers that may not allocate device
 // memory get their working space from this fixed array instead of a context:
-// every GPU that loads the library holds it (about 2.3 MB) until the process
-// exits.  Limits: B <= 256, k <= 8, and B * (2k + 1) * ceil(V / chunk) <=
-// 256 * 17 * 32 chunk records (chunk = 8192 bf16 or 4096 fp32 logits), i.e.
+// every GPU that loads the library holds it (about 0.6 MB) until the process
+// exits.  The statistics kernel writes one 16-byte record per (request, row,
+// segment), a segment being 32768 bf16 or 16384 fp32 logits, and indexes the
+// records with a stride of 2k + 1 rows per request.  Limits: B <= 256, k <= 8,
+// and B * (2k + 1) * ceil(V / segment) <= 256 * 17 * 8 records, i.e.
 // V <= 262144 for bf16 and V <= 131072 for fp32 at the largest B and k.
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int kNoAllocMaxBatch = 256;
 constexpr int kNoAllocMaxK = 8;
-constexpr size_t kNoAllocMaxRecords = size_t(kNoAllocMaxBatch) * (2 * kNoAllocMaxK + 1) * 32;
+constexpr size_t kNoAllocMaxRecords = size_t(kNoAllocMaxBatch) * (2 * kNoAllocMaxK + 1) * 8;
 constexpr size_t kNoAllocMetaOff = 0;
 constexpr size_t kNoAllocJobsOff = kNoAllocMetaOff + kNoAllocMaxRecords * sizeof(sv::ChunkMeta);
 constexpr size_t kNoAllocArriveOff = kNoAllocJobsOff + size_t(kNoAllocMaxBatch) * sizeof(sv::Job);
@@ -777,11 +779,9 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
     return SPEC_ERR_INVALID_ARG;
   if (dtype != SPEC_F32 && dtype != SPEC_BF16) return SPEC_ERR_INVALID_ARG;
   const bool bf16 = dtype == SPEC_BF16;
-  const int64_t limit_chunk = bf16 ? 8192 : 4096;  // the documented limit's unit
-  const int64_t n_limit = (V + limit_chunk - 1) / limit_chunk;
   const int segl = bf16 ? sv::SegGeo<true>::kSeg : sv::SegGeo<false>::kSeg;
-  const int64_t n_segs = (V + segl - 1) / segl;
-  if (static_cast<size_t>(B) * (2 * k + 1) * static_cast<size_t>(n_limit) > kNoAllocMaxRecords)
+  const int64_t n_segs = (V + segl - 1) / segl;  // statistics records per row
+  if (static_cast<size_t>(B) * (2 * k + 1) * static_cast<size_t>(n_segs) > kNoAllocMaxRecords)
     return SPEC_ERR_INVALID_ARG;
   if (B == 0) return SPEC_OK;
   if (!target_logits || !out_accepted || !out_tokens || (k > 0 && !draft_tokens))
@@ -823,7 +823,9 @@ spec_status spec_verify_greedy_noalloc(const void* target_logits, spec_dtype dty
   if (cudaMemsetAsync(p.arrive_stats, 0, static_cast<size_t>(B) * sizeof(unsigned), stream) !=
       cudaSuccess)
     return SPEC_ERR_CUDA;
-  const int64_t ctas = static_cast<int64_t>(B) * (2 * k + 1) * n_segs;
+  // greedy reads target rows only: one CTA per (request, target row, segment)
+  p.launch_rows = k + 1;
+  const int64_t ctas = static_cast<int64_t>(B) * (k + 1) * n_segs;
   if (bf16) sv::k_stats<true><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
   else sv::k_stats<false><<<static_cast<unsigned>(ctas), sv::kThreads, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
@@ -875,7 +877,7 @@ spec_status spec_verify_timing_read(spec_verify_ctx* ctx, int which, int* launch
   return SPEC_OK;
 }
 
-spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream, uint32_t out[5]) {
+spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream, uint32_t out[6]) {
   if (!ctx || !out) return SPEC_ERR_INVALID_ARG;
   DeviceGuard g(ctx->device);
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SPEC_ERR_CUDA;
@@ -888,6 +890,7 @@ spec_status spec_verify_last_counters(spec_verify_ctx* ctx, cudaStream_t stream,
   out[2] = h.sample_fast;
   out[3] = h.chunks_redone;
   out[4] = h.queue_error;
+  out[5] = h.wait_fail;
   return SPEC_OK;
 }
 

@@ -985,19 +985,24 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
 }
 
 // ---------------------------------------------------------------------------
-// The kernel: one CTA per (request, row slot, segment).
+// The kernel: one CTA per (request, row slot, segment).  The grid covers the
+// first launch_rows slots of each request (all 2k + 1 when it is 0; k + 1,
+// the target rows, for a greedy-only run); records keep the stride of 2k + 1
+// slots per request either way.
 // ---------------------------------------------------------------------------
 template <bool BF16>
 __global__ void __launch_bounds__(kThreads) k_stats(RunParams p) {
   __shared__ StatsShared sh;
   __shared__ DecideShared dsh;
   const int rows_per_req = 2 * p.k + 1;
+  const int launched = p.launch_rows > 0 ? p.launch_rows : rows_per_req;
   const int64_t b = blockIdx.x;
   const int seg = static_cast<int>(b % p.n_segs);
-  const int64_t slot_global = b / p.n_segs;
-  const int i = static_cast<int>(slot_global / rows_per_req);
-  const int slot = static_cast<int>(slot_global - static_cast<int64_t>(i) * rows_per_req);
-  if (b == 0 && threadIdx.x == 0) *p.counters_next = Counters{0u, 0u, 0u, 0u};
+  const int64_t slot_launched = b / p.n_segs;
+  const int i = static_cast<int>(slot_launched / launched);
+  const int slot = static_cast<int>(slot_launched - static_cast<int64_t>(i) * launched);
+  const int64_t slot_global = static_cast<int64_t>(i) * rows_per_req + slot;
+  if (b == 0 && threadIdx.x == 0) *p.counters_next = Counters{};
 
   const ReqInfo ri = request_info(p, i);
   const bool is_draft = slot > p.k;
