@@ -211,6 +211,40 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "samples_in_timed_region": len(inside)}
 
 
+# ---------------------------------------------------------------- timing ----
+
+TIMED_SECONDS = 1.0  # the timed block of --steps steps repeats until this much has elapsed
+
+
+def timed_blocks(step, steps, stream, dev, world):
+    """Time blocks of `steps` steps with CUDA events on the launching stream,
+    a barrier and a device synchronisation on both sides of each, until about
+    TIMED_SECONDS have elapsed; each block's time is the max over ranks.
+    Returns the per-block milliseconds (every rank gets the same list)."""
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_86_b200 import ranks
+    out = []
+    t0 = time.perf_counter()
+    while True:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        out.append(ranks.max_over_ranks(e0.elapsed_time(e1), dev))
+        elapsed = ranks.max_over_ranks((time.perf_counter() - t0) * 1e3, dev) / 1e3
+        if elapsed >= TIMED_SECONDS:
+            return out
+
+
 # -------------------------------------------------------------- roofline ----
 
 def measured_peaks():
@@ -371,18 +405,9 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     clocks.mark()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
+    block_ms = timed_blocks(step, args.steps, stream, dev, world)
     clocks.mark()
-    if world > 1:
-        dist.barrier()
-    ms_local = e0.elapsed_time(e1)
     n_stats, ms_stats = ver.timing_read(binding.TIMING_STATS)
     n_conf, ms_conf = ver.timing_read(binding.TIMING_CONF)
     ver.timing_enable([])
@@ -409,8 +434,7 @@ def run_ours(args):
                   "value": positions * world / (other_ms / 1e3),
                   "hbm_gbs": dense_row_bytes(w, L) / (other_ms * 1e-3) / 1e9 if other == "dense" else None}
     ver.set_mode(args.mode)
-    ms_total = ranks.max_over_ranks(ms_local, dev)
-    ms_per_step = ms_total / args.steps
+    ms_per_step = statistics.median(block_ms) / args.steps
     if flush is not None and n_stats:
         # the step includes the flush: report the verification launches alone
         ms_per_step = ranks.max_over_ranks(ms_stats / n_stats + (ms_conf / n_conf if n_conf else 0.0), dev)
@@ -493,7 +517,10 @@ def run_ours(args):
                      "algorithmic_bytes_dense": step_bytes,
                      "launch_ms": ms_stats_avg, "launches_timed": n_stats},
         "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps * len(block_ms),
+        "timed_blocks": {"blocks": len(block_ms), "steps_per_block": args.steps,
+                         "ms_per_block_min": min(block_ms), "ms_per_block_median": statistics.median(block_ms),
+                         "ms_per_block_max": max(block_ms)},
         "fp64_paths": counters,
         "conf_launch_ms": (ms_conf / n_conf) if n_conf else None,
         "mode": args.mode,

@@ -99,7 +99,7 @@ class _FakeRank:
         return redo
 
 
-def _worker(rank, n, port, q):
+def _worker(rank, n, port, q, redo_whole=True):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=n)
     try:
@@ -110,11 +110,11 @@ def _worker(rank, n, port, q):
         tokens = torch.zeros((B, K), dtype=torch.int32)
         out = binding.verify_vocab_parallel(rk, target[:, :, lo:hi].contiguous(),
                                             draft[:, :, lo:hi].contiguous(), tokens, V,
-                                            seed=5, request_offset=40)
+                                            seed=5, request_offset=40, redo_whole=redo_whole)
         votes = [e[1] for e in rk.log if e[0] == "votes"][0]
         redo = [e for e in rk.log if e[0] == "redo"]
         q.put((rank, bounds, votes.tolist(), out["accepted"].tolist(),
-               [(t.numpy(), d.numpy(), off) for _, t, d, off in redo]))
+               [(t.numpy(), d.numpy(), off) for _, t, d, off in redo], out["redo"].tolist()))
     finally:
         dist.destroy_process_group()
 
@@ -132,7 +132,7 @@ def test_two_rank_choreography():
         p.join(timeout=60)
         assert p.exitcode == 0
     target, draft = _full_logits()
-    for rank, bounds, votes, accepted, redo in got:
+    for rank, bounds, votes, accepted, redo, flags in got:
         assert bounds[0] == 0 and bounds[-1] == V and bounds[1] - bounds[0] != bounds[2] - bounds[1]
         # the MAX picks the holder's vote; request 0 went on to the refinement
         assert votes[0] == -1
@@ -144,3 +144,23 @@ def test_two_rank_choreography():
         np.testing.assert_array_equal(d, draft[0:1].numpy())
         assert off == 40
         assert accepted[0] == 77 and accepted[1:] == [1] * (B - 1)
+
+
+def test_two_rank_step_without_host_redo():
+    """redo_whole=False: every phase runs (the refinement included) and the
+    request that needs rows of every rank is only flagged in out["redo"]."""
+    n = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, n, port, q, False)) for r in range(n)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(n)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, bounds, votes, accepted, redo, flags in got:
+        assert len(redo) == 0                     # nothing verified whole on the host
+        assert flags[0] == 1 and flags[1:] == [0] * (B - 1)
+        assert accepted == [1] * B
