@@ -192,6 +192,7 @@ struct RunParams {
 
   // engine
   int mode;                        // kModeDense / kModePrefix
+  int whole_rows;                  // dense order: a statistics item is a whole row (else a segment)
   unsigned long long* q_slots;     // queue: (epoch << 32) | payload
   unsigned q_capacity;
   unsigned q_epoch;                // this run's epoch, never 0
@@ -533,15 +534,17 @@ __device__ __forceinline__ double chunk_prefix(const double (&v)[4], double (&pr
   return total;
 }
 
-// Arrival on a per-request counter: returns true in exactly one CTA, the last
-// of `expected` arrivals, and resets the counter for the next launch.  Writes
+// Arrival of `weight` units on a per-request counter: returns true in exactly
+// one CTA, the one completing `expected` units, and resets the counter for the
+// next launch.  Writes
 // this CTA made before the call are visible to the last arriver afterwards.
-__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* sh_flag) {
+__device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* sh_flag,
+                                            unsigned weight = 1u) {
   sync_compute();
   if (threadIdx.x == 0) {
     __threadfence();
-    const unsigned old = atomicAdd(counter, 1u);
-    const bool last = (old == expected - 1u);
+    const unsigned old = atomicAdd(counter, weight);
+    const bool last = (old + weight == expected);
     if (last) {
       *counter = 0u;
       __threadfence();

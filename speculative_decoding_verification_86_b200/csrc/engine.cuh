@@ -1,7 +1,7 @@
 // The verification engine: one persistent kernel that drives every request of
 // the batch through its passes with a device-side work queue.
 //
-// Work items (32-bit payloads, ticketed by one atomic counter):
+// Work items (32-bit payloads):
 //   STATS  (request, row slot, segment)  softmax / arg-max statistics of one row segment
 //   SAMPLE (request, segment)            residual / bonus masses of one segment
 //   REFINE (refinement slot, sub-chunk)  fp64 recomputation of one sub-chunk
@@ -9,7 +9,7 @@
 // enqueues it: the chain decision after STATS (then the next position's rows,
 // the sample, or nothing), the inverse-CDF locate after SAMPLE (then nothing
 // or the fp64 refinement), the fp64 token after REFINE.  Requests advance
-// independently; new items join the one FIFO behind those already queued.
+// independently.
 //
 // Two orders of the statistics ("Speculative decoding becomes standard: DSpark
 // and multi-token drafters", section "Why draft-and-verify does not change the
@@ -19,25 +19,35 @@
 //   prefix : a request's position j+1 rows are read only after position j was
 //            accepted.  The outputs are identical; prefix reads fewer bytes.
 //
-// The first tickets (0 .. n_init-1) are implicit: the rows of position 0 (prefix)
+// The first tickets (0 .. n_init-1) are implicit: the confidence head of every
+// request when it runs in this launch, then the rows of position 0 (prefix)
 // or of every position (dense), decoded from the ticket number.  Later tickets
 // index the queue, whose slots carry the run's epoch in their upper 32 bits so
-// a slot left by an earlier run is never taken for a new item.  A CTA waiting
-// for a slot sleeps between polls and gives up after a bounded time (setting
+// a slot left by an earlier run is never taken for a new item.  New items join
+// the one FIFO behind those already queued (handing generated items out
+// first was measured slower on every workload).  A CTA waiting for a slot
+// sleeps between polls and gives up after a bounded number of polls (setting
 // the queue error), as does the whole kernel once every request is finished.
 // The last CTA to leave resets the queue counters for the next run.
 #pragma once
 #include "common.cuh"
+#include "conf.cuh"
 #include "refine.cuh"
 #include "sample.cuh"
 #include "stats.cuh"
 
 namespace sv {
 
-constexpr uint32_t kItemStats = 0u, kItemSample = 1u, kItemRefine = 2u;
+constexpr uint32_t kItemStats = 0u, kItemSample = 1u, kItemRefine = 2u, kItemConf = 3u;
 constexpr uint32_t kItemExit = 0xFFFFFFFFu;
+constexpr int kRowSeg = 0xFF;  // segment field of a STATS item that covers its whole row
 constexpr unsigned kSpinLimit = 1u << 24;  // polls of a queue slot before giving up (seconds)
 constexpr int kEngineMinBlocks = 4;  // 64 registers: four CTAs per SM (measured best)
+// candidate keys of the batch-wide selection held in the staging buffer
+constexpr int kConfKeysInStage = 4096;
+static_assert(kMaxK * sizeof(double) + sizeof(ConfSelectShared) + kConfKeysInStage * sizeof(unsigned long long) <=
+                  kStageBytes,
+              "the confidence head's scratch fits the staging buffer");
 
 __device__ __forceinline__ uint32_t item_stats(int i, int slot, int seg) {
   return (kItemStats << 30) | (static_cast<uint32_t>(i) << 14) |
@@ -48,6 +58,9 @@ __device__ __forceinline__ uint32_t item_sample(int i, int seg) {
 }
 __device__ __forceinline__ uint32_t item_refine(int slot, int sub) {
   return (kItemRefine << 30) | (static_cast<uint32_t>(slot) << 14) | static_cast<uint32_t>(sub);
+}
+__device__ __forceinline__ uint32_t item_conf(int i) {
+  return (kItemConf << 30) | (static_cast<uint32_t>(i) << 14);
 }
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* a) {
@@ -72,6 +85,12 @@ __device__ __forceinline__ int task_rows(const ReqInfo& ri, int j) {
 
 // The implicit item of ticket h < n_init.
 __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h) {
+  if (h < p.n_conf) return item_conf(static_cast<int>(h));
+  h -= p.n_conf;
+  if (p.mode == kModeDense && p.whole_rows) {  // a request's 2k + 1 whole rows
+    const unsigned per_req = static_cast<unsigned>(2 * p.k + 1);
+    return item_stats(static_cast<int>(h / per_req), static_cast<int>(h % per_req), kRowSeg);
+  }
   if (p.mode == kModeDense) {
     const unsigned per_req = static_cast<unsigned>(2 * p.k + 1) * p.n_segs;
     const unsigned i = h / per_req, r = h % per_req;
@@ -83,7 +102,8 @@ __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h
   return item_stats(static_cast<int>(i), slot, static_cast<int>(r % p.n_segs));
 }
 
-// Thread 0: the next item (or kItemExit).
+// Thread 0: the next item (or kItemExit).  Tickets are handed out in order by
+// one atomic add; a ticket past the implicit ones waits for its queue slot.
 __device__ uint32_t fetch_item(const RunParams& p) {
   const unsigned h = atomicAdd(p.q_ctl + kQHead, 1u);
   if (h < p.n_init) return implicit_item(p, h);
@@ -131,34 +151,75 @@ __device__ void enqueue_sample(const RunParams& p, int i, unsigned* s_base) {
   enqueue(p, p.n_segs, [&](int q) { return item_sample(i, q); }, s_base);
 }
 
+// Wait (thread 0) until the confidence head run in this launch has published
+// every budget; false if the wait gave up.
+__device__ __forceinline__ bool wait_conf(const RunParams& p) {
+  if (p.n_conf == 0) return true;
+  for (unsigned w = 0;; ++w) {
+    if (ld_acquire_u32(p.q_ctl + kQConfDone) == p.q_epoch) return true;
+    if (w >= kSpinLimit) {
+      atomicOr(&p.counters->queue_error, 4u);
+      return false;
+    }
+    __nanosleep(w < 32 ? 64 : 256);
+  }
+}
+
 // STATS item: one segment of one row of request i; the last segment of the
 // task decides.
+//
+// When the confidence head runs in the same launch (prefix order only), the
+// rows of position 0 are read before its budgets are known: their plan
+// follows verify_len alone (Lcap), reading the drafter's row 0 whenever a
+// sampled request may verify a position, and the decision waits for the
+// budgets.  Every later position exists only after a decision, so its plan
+// already has them.
 template <bool BF16>
 __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, StatsShared& st,
                              DecideShared& dec, unsigned* s_base, uint4* stage_buf) {
-  const ReqInfo ri = request_info(p, i);
   const bool is_draft = slot > p.k;
   const int j = is_draft ? slot - (p.k + 1) : slot;
-  bool needed;
-  if (ri.bad_T) needed = (slot == 0 && seg == 0);
-  else if (ri.greedy) needed = !is_draft && j <= ri.L;
-  else needed = is_draft ? (j < ri.L) : (j <= ri.L);
+  const bool early = p.n_conf > 0 && j == 0;  // planned before the head's budgets
+  const ReqInfo ri = request_info(p, i, !early);
+  bool needed, pass;
+  unsigned expected;
+  if (early) {
+    const bool target_only = ri.greedy || ri.no_draft;
+    if (ri.invalid_T) needed = (slot == 0 && seg == 0);
+    else if (target_only) needed = !is_draft;
+    else needed = !is_draft || ri.Lcap > 0;
+    pass = !ri.invalid_T;
+    expected = ri.invalid_T ? 1u
+                            : static_cast<unsigned>(((!target_only && ri.Lcap > 0) ? 2 : 1) * p.n_segs);
+  } else {
+    if (ri.bad_T) needed = (slot == 0 && seg == 0);
+    else if (ri.greedy) needed = !is_draft && j <= ri.L;
+    else needed = is_draft ? (j < ri.L) : (j <= ri.L);
+    pass = !ri.bad_T;
+    if (ri.bad_T) expected = 1u;
+    else if (p.mode == kModeDense) expected = static_cast<unsigned>(stats_expected(ri, p.n_segs));
+    else expected = static_cast<unsigned>(task_rows(ri, j) * p.n_segs);
+  }
+  // a whole-row item (dense order) stands for all of the row's segment items
+  const bool whole = seg == kRowSeg;
+  if (whole && ri.bad_T) needed = slot == 0;
   if (!needed) return;
-  if (!ri.bad_T) {
-    const int64_t rec = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs + seg;
+  unsigned weight = 1u;
+  if (pass) {
+    const int64_t rec0 = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
     const void* row = is_draft ? draft_row(p, i, j, BF16) : target_row(p, i, j, BF16);
-    if (ri.greedy) {
-      greedy_segment_staged<BF16>(row, p.V, seg, p.meta + rec, st, stage_buf);
+    const float cc = ri.greedy ? 0.0f : static_cast<float>(1.4426950408889634 / static_cast<double>(ri.T));
+    if (whole) {
+      weight = static_cast<unsigned>(p.n_segs);
+      if (ri.greedy) stats_row_staged<BF16, true>(row, p.V, p.n_segs, cc, p.meta + rec0, nullptr, st, stage_buf);
+      else stats_row_staged<BF16, false>(row, p.V, p.n_segs, cc, p.meta + rec0, p.ssum + rec0, st, stage_buf);
+    } else if (ri.greedy) {
+      greedy_segment_staged<BF16>(row, p.V, seg, p.meta + rec0 + seg, st, stage_buf);
     } else {
-      const float cc = static_cast<float>(1.4426950408889634 / static_cast<double>(ri.T));
-      stochastic_segment_staged<BF16>(row, p.V, seg, cc, p.meta + rec, p.ssum + rec, st, stage_buf);
+      stochastic_segment_staged<BF16>(row, p.V, seg, cc, p.meta + rec0 + seg, p.ssum + rec0 + seg, st, stage_buf);
     }
   }
-  unsigned expected;
-  if (ri.bad_T) expected = 1u;
-  else if (p.mode == kModeDense) expected = static_cast<unsigned>(stats_expected(ri, p.n_segs));
-  else expected = static_cast<unsigned>(task_rows(ri, j) * p.n_segs);
-  if (!arrive_last(p.arrive_stats + i, expected, &st.flag)) return;
+  if (!arrive_last(p.arrive_stats + i, expected, &st.flag, weight)) return;
   __threadfence();
   if (p.mode == kModeDense) {
     decide_request<BF16>(p, i, ri, dec);
@@ -167,11 +228,17 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     else finish_request(p);
     return;
   }
-  decide_position<BF16>(p, i, ri, j, dec);
+  if (early) {
+    if (threadIdx.x == 0) st.flag = wait_conf(p) ? 1 : 0;
+    __syncthreads();
+    if (!st.flag) return;  // the head never finished: the run reports the queue error
+  }
+  const ReqInfo rc = early ? request_info(p, i, true) : ri;
+  decide_position<BF16>(p, i, rc, j, dec);
   const int next = dec.state;
   if (next == 1) {
     const int jn = j + 1;
-    const int rows = task_rows(ri, jn);
+    const int rows = task_rows(rc, jn);
     const int ns = p.n_segs;
     enqueue(p, rows * ns, [&](int q) {
       return item_stats(i, (q / ns) == 0 ? jn : p.k + 1 + jn, q % ns);
@@ -180,6 +247,24 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     enqueue_sample<BF16>(p, i, s_base);
   } else {
     finish_request(p);
+  }
+}
+
+// CONF item: the confidence head of request i.  The CTA completing the last
+// request runs the batch-wide selection (if any) and publishes the budgets.
+// Its scratch is the staging buffer, idle between streaming passes.
+__device__ void engine_conf(const RunParams& p, int i, int* flag, uint4* stage_buf) {
+  double* s_surv = reinterpret_cast<double*>(stage_buf);
+  ConfSelectShared* ss = reinterpret_cast<ConfSelectShared*>(s_surv + kMaxK);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(ss + 1);
+  conf_request(p.cp, i, s_surv);
+  if (!arrive_last(p.cp.arrive, static_cast<unsigned>(p.B), flag)) return;
+  __threadfence();
+  if (p.cp.total > 0) conf_select(p.cp, *ss, keys, kConfKeysInStage);
+  sync_compute();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.q_ctl + kQConfDone), "r"(p.q_epoch) : "memory");
   }
 }
 
@@ -230,7 +315,8 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
     switch (it >> 30) {
       case kItemStats: engine_stats<BF16>(p, a, b >> 8, b & 0xFF, st, dec, &s_base, stage_buf); break;
       case kItemSample: engine_sample<BF16>(p, a, b, sa, &s_base, stage_buf); break;
-      default: engine_refine<BF16>(p, a, b, rf); break;
+      case kItemRefine: engine_refine<BF16>(p, a, b, rf); break;
+      default: engine_conf(p, a, &st.flag, stage_buf); break;
     }
     __syncthreads();
   }

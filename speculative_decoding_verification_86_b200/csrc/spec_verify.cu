@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/spec_verify.h: argument checks,
-// the context's device workspace, and the launches: [k_conf] then one
-// persistent k_engine (engine.cuh) per run.  Every launch goes to the caller's
+// the context's device workspace, and the launches: one persistent k_engine
+// (engine.cuh) per run -- the confidence head included in the prefix order,
+// k_conf before it in the dense order.  Every launch goes to the caller's
 // stream; nothing here synchronises except the host-buffer entry point, the
 // diagnostics and the timing read-out.
 #include "spec_verify.h"
@@ -367,10 +368,6 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.counters_next = c->counters + ((c->run_id + 1u) & 1u);
 
   cudaGetLastError();  // clear stale errors so the check below is ours
-  if (conf) {
-    launch_conf(c, conf, B, k, vlen, c->conf_len, nullptr, s);
-    p.conf_len = c->conf_len;
-  }
   // Order of the statistics.  Automatic: the prefix order saves reads when the
   // batch's rows compete for the grid; when every row the batch may verify
   // fits in one wave of the grid, reading them all at once costs no extra time
@@ -380,12 +377,48 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     mode = static_cast<int64_t>(B) * (2 * k + 1) * n_segs <= c->engine_grid ? SPEC_MODE_DENSE
                                                                            : SPEC_MODE_PREFIX;
   p.mode = (force_greedy || mode == SPEC_MODE_PREFIX) ? sv::kModePrefix : sv::kModeDense;
+  if (conf && p.mode == sv::kModePrefix) {
+    // the confidence head runs inside the verification launch, as its first B
+    // items (the prefix order reads position 0 before the budgets are needed)
+    sv::ConfParams& cp = p.cp;
+    cp.hidden = static_cast<const uint16_t*>(conf->hidden);
+    cp.w = static_cast<const uint16_t*>(conf->w);
+    cp.bias = conf->bias;
+    cp.threshold = conf->threshold;
+    cp.B = B;
+    cp.kb = conf->kb;
+    cp.H = conf->H;
+    cp.k = k;
+    cp.vlen = vlen;
+    cp.total = conf->total_budget > 0 ? conf->total_budget : 0;
+    cp.prefix = c->conf_prefix;
+    cp.cap = c->conf_cap;
+    cp.arrive = c->conf_arrive;
+    cp.out_len = c->conf_len;
+    cp.out_survival = nullptr;
+    p.conf_len = c->conf_len;
+    p.n_conf = static_cast<unsigned>(B);
+  } else if (conf) {
+    // the dense order plans every row up front: the budgets come first
+    launch_conf(c, conf, B, k, vlen, c->conf_len, nullptr, s);
+    p.conf_len = c->conf_len;
+  }
   p.q_slots = c->q_slots;
   p.q_capacity = c->q_capacity;
   p.q_ctl = c->q_ctl;
   p.q_epoch = c->run_id;  // >= 1: slots left by earlier runs carry older epochs
-  const uint64_t n_init = static_cast<uint64_t>(B) *
-                          (p.mode == sv::kModeDense ? (2 * k + 1) : 2) * n_segs;
+  // Dense order: a statistics item is a whole row when the batch has at least
+  // as many rows as the grid has CTAs (one staging pipeline per row, no drain
+  // between its segments), else a segment (small batches: every segment of
+  // every row in flight at once).
+  p.whole_rows = (p.mode == sv::kModeDense &&
+                  static_cast<int64_t>(B) * (2 * k + 1) >= c->engine_grid) ? 1 : 0;
+  // implicit tickets: the confidence head's items, then the statistics items
+  // of every row (dense) or of position 0's rows (prefix)
+  const uint64_t per_req = p.mode == sv::kModePrefix ? 2ull * n_segs
+                           : (p.whole_rows ? static_cast<uint64_t>(2 * k + 1)
+                                           : static_cast<uint64_t>(2 * k + 1) * n_segs);
+  const uint64_t n_init = static_cast<uint64_t>(p.n_conf) + static_cast<uint64_t>(B) * per_req;
   if (n_init > 0xFFFF0000ull) return SPEC_ERR_INVALID_ARG;
   p.n_init = static_cast<unsigned>(n_init);
   timing_mark(c, kClassStats, true, s);

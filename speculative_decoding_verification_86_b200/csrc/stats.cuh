@@ -457,6 +457,73 @@ __device__ __forceinline__ void greedy_segment_staged(const void* row, int64_t V
 }
 
 // ---------------------------------------------------------------------------
+// A whole row in one pass: its segments' staging steps form one pipeline, so
+// the first steps of segment s+1 are in flight while segment s is finished and
+// its record written -- the copies never drain between segments.  The records
+// are those of the per-segment passes (the same vectors per thread, merged the
+// same way).  GREEDY selects the arg-max scan instead of the softmax sums.
+// ---------------------------------------------------------------------------
+template <bool FULL>
+__device__ __forceinline__ void stage_row_step(Stager& sg, const uint4* rv, int64_t nvec, int g) {
+  const int seg = g / kBatches, b = g % kBatches;
+  const int64_t base = static_cast<int64_t>(seg) * SegGeo<true>::kSegVecs + threadIdx.x;
+#pragma unroll
+  for (int u = 0; u < kBatchVecs; ++u) {
+    const int64_t idx = base + static_cast<int64_t>(b * kBatchVecs + u) * kThreads;
+    const bool valid = FULL || idx < nvec;
+    cp_async16(sg.slot(g, u), valid ? rv + idx : rv, valid);
+  }
+  cp_async_commit();
+  ++sg.issued;
+}
+static_assert(SegGeo<true>::kSegVecs == SegGeo<false>::kSegVecs, "segments hold the same vector count");
+
+template <bool BF16, bool GREEDY>
+__device__ void stats_row_staged(const void* row, int64_t V, int n_segs, float cc, ChunkMeta* meta,
+                                 double* ssum, StatsShared& sh, uint4* stage_buf) {
+  using G = SegGeo<BF16>;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t nvec = V / G::kPerVec;
+  const int n_steps = n_segs * kBatches;
+  // steps of segments wholly inside the row need no range checks
+  const int full_steps = static_cast<int>(nvec / G::kSegVecs) * kBatches;
+  Stager sg{stage_buf};
+  for (int g = 0; g < kStageSlots && g < n_steps; ++g) {
+    if (g < full_steps) stage_row_step<true>(sg, rv, nvec, g);
+    else stage_row_step<false>(sg, rv, nvec, g);
+  }
+#pragma unroll 1
+  for (int seg = 0; seg < n_segs; ++seg) {
+    const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+    const bool full = (seg + 1) * kBatches <= full_steps;
+    SoftAcc acc;
+    GreedyScan<BF16> gs;
+#pragma unroll 1
+    for (int b = 0; b < kBatches; ++b) {
+      const int g = seg * kBatches + b;
+      cp_async_wait(sg.issued - g - 1);
+      uint4 v[kBatchVecs];
+#pragma unroll
+      for (int u = 0; u < kBatchVecs; ++u) {
+        const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
+        v[u] = (full || idx < nvec) ? *sg.slot(g, u) : neg_inf_vec<BF16>();
+      }
+      if constexpr (GREEDY) gs.scan(v, seg0, b);
+      else soft_batch<BF16>(acc, v, cc);
+      // refill this step's slot once its values have been used
+      const int gn = g + kStageSlots;
+      if (gn < n_steps) {
+        if (gn < full_steps) stage_row_step<true>(sg, rv, nvec, gn);
+        else stage_row_step<false>(sg, rv, nvec, gn);
+      }
+    }
+    if constexpr (GREEDY) gs.finish(meta + seg, sh);
+    else soft_merge_block(acc, sh, meta + seg, ssum + seg);
+    sync_compute();  // sh is reused by the next segment's merge
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Merged row records, built by the deciding CTA in shared memory.
 // ---------------------------------------------------------------------------
 struct RowMerged {
