@@ -59,6 +59,9 @@ def parse_args():
                          "cores, on a bounded sample of the same workload")
     ap.add_argument("--workload", default="headline",
                     help="headline | stochastic | greedy | conf | conf_budget | sweep:B | lmhead")
+    ap.add_argument("--timed-seconds", type=float, default=1.0,
+                    help="repeat the timed block of --steps steps until this much time has "
+                         "elapsed (0: one block, e.g. under a profiler)")
     ap.add_argument("--e2e-steps", type=int, default=5,
                     help="steps of the end-to-end measurement through host buffers (0: skip)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
@@ -213,13 +216,10 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- timing ----
 
-TIMED_SECONDS = 1.0  # the timed block of --steps steps repeats until this much has elapsed
-
-
-def timed_blocks(step, steps, stream, dev, world):
+def timed_blocks(step, steps, stream, dev, world, seconds=1.0):
     """Time blocks of `steps` steps with CUDA events on the launching stream,
     a barrier and a device synchronisation on both sides of each, until about
-    TIMED_SECONDS have elapsed; each block's time is the max over ranks.
+    `seconds` have elapsed; each block's time is the max over ranks.
     Returns the per-block milliseconds (every rank gets the same list)."""
     import torch
     import torch.distributed as dist
@@ -241,7 +241,7 @@ def timed_blocks(step, steps, stream, dev, world):
             dist.barrier()
         out.append(ranks.max_over_ranks(e0.elapsed_time(e1), dev))
         elapsed = ranks.max_over_ranks((time.perf_counter() - t0) * 1e3, dev) / 1e3
-        if elapsed >= TIMED_SECONDS:
+        if elapsed >= seconds:
             return out
 
 
@@ -258,8 +258,8 @@ def measured_peaks():
 # The device sources each profiled kernel is compiled from (host code, the C
 # header and the other kernels' files do not change its machine code).
 KERNEL_SOURCES = {
-    "k_engine": ["common.cuh", "engine.cuh", "fp64.cuh", "philox.cuh", "refine.cuh", "sample.cuh",
-                 "stage.cuh", "stats.cuh"],
+    "k_engine": ["common.cuh", "conf.cuh", "engine.cuh", "fp64.cuh", "philox.cuh", "refine.cuh",
+                 "sample.cuh", "stage.cuh", "stats.cuh"],
     "k_lmhead": ["common.cuh", "philox.cuh", "stage.cuh", "stats.cuh", "lmhead.cuh"],
 }
 
@@ -406,7 +406,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.mark()
-    block_ms = timed_blocks(step, args.steps, stream, dev, world)
+    block_ms = timed_blocks(step, args.steps, stream, dev, world, args.timed_seconds)
     clocks.mark()
     n_stats, ms_stats = ver.timing_read(binding.TIMING_STATS)
     n_conf, ms_conf = ver.timing_read(binding.TIMING_CONF)

@@ -26,7 +26,13 @@ struct Geo {
   static constexpr int kBatchElems = kVecsPerBatch * kPerVec;                    // per thread and batch
   static constexpr int kPerThread = kBatchElems * kBatchesPerChunk;              // per thread and chunk
   static constexpr int kSumLevels = BF16 ? 4 : 3;                                // pairwise depth of a batch sum
+  static constexpr int kPartVecs = kChunkVecs / kWarps;                          // 256 vectors: one warp's part
+  static constexpr int kPart = kPartVecs * kPerVec;                              // logits per part
 };
+// The sampling passes split a chunk into kWarps contiguous parts, warp w of
+// the CTA streaming part w, and keep one mass record per part, so the inverse
+// CDF rescans a single part (one vector per thread) in the end.
+constexpr int kSampleParts = kWarps;
 
 constexpr int kChunkBf16 = Geo<true>::kChunk;   // 16384
 constexpr int kChunkF32 = Geo<false>::kChunk;   // 8192
@@ -99,7 +105,7 @@ __device__ __forceinline__ Job load_job(const Job* src) {
 }
 
 struct SampleChunk {
-  double mass;   // sum of fp32 weights over the chunk (fp64 accumulation of pairwise groups)
+  double mass;   // sum of fp32 weights over a part of a chunk (fp64 accumulation of pairwise groups)
   double bound;  // certified bound on |mass - exact mass|
 };
 
@@ -116,11 +122,16 @@ struct Counters {
 // Engine: orders of the statistics pass, and the queue's control words.
 constexpr int kModeDense = 0;
 constexpr int kModePrefix = 1;
-// head: implicit tickets handed out; tail / gen_head: generated items reserved /
-// claimed; done: requests finished; exits: CTAs that left; conf_done: the
-// epoch of the run whose confidence budgets are published.
-constexpr int kQHead = 0, kQTail = 1, kQDone = 2, kQExits = 3, kQGenHead = 4, kQConfDone = 5,
-              kQWords = 8;
+// head: implicit tickets handed out; done: requests finished; exits: CTAs that
+// left; conf_done: the epoch of the run whose confidence budgets are
+// published.  Generated items sit in one queue per class (statistics of a
+// later position, sample segments, refinement sub-chunks), each with its own
+// reserved (tail), claimed (claim) and published-but-unclaimed (avail, signed)
+// counts.
+constexpr int kQClasses = 3;
+constexpr int kQHead = 0, kQDone = 1, kQExits = 2, kQConfDone = 3, kQTail0 = 4,
+              kQClaim0 = kQTail0 + kQClasses, kQAvail0 = kQClaim0 + kQClasses, kQWords = 16;
+static_assert(kQAvail0 + kQClasses <= kQWords, "queue control words");
 
 // -------------------------------------------------------------- run params --
 struct ConfParams {
@@ -174,7 +185,7 @@ struct RunParams {
   unsigned* arrive_stats;  // [B]
   unsigned* arrive_sample; // [B]
   Job* jobs;               // [B]
-  SampleChunk* smass;      // [B, n_chunks]
+  SampleChunk* smass;      // [B, n_chunks, kSampleParts] part masses
   int* refine_list;        // [B]
   unsigned* arrive_r1;     // [B]
   double2* rz;             // [B, 4 n_chunks] fp64 normaliser partials per sub-chunk
@@ -185,6 +196,7 @@ struct RunParams {
 
   // vocabulary-parallel runs (nullptr / 0 otherwise)
   const float* tok_logits; // [B, k, 2]: target and draft logit of each drafted token
+  float* tok_cache;        // engine: the same, left by the statistics items (else nullptr)
   int32_t* fallback;       // [B]: set when a decision needs rows held by other ranks
   int32_t* shard_tok;      // [B]: located token, -1 to redo the request whole, -2 not here
   int c_lo, c_hi;          // chunks whose logits the buffers hold (c_hi = 0: all)
@@ -195,6 +207,8 @@ struct RunParams {
   int whole_rows;                  // dense order: a statistics item is a whole row (else a segment)
   unsigned long long* q_slots;     // queue: (epoch << 32) | payload
   unsigned q_capacity;
+  unsigned q_off[kQClasses];       // each class's region of q_slots
+  unsigned q_cap[kQClasses];
   unsigned q_epoch;                // this run's epoch, never 0
   unsigned* q_ctl;                 // the queue's control words (kQ*)
   unsigned n_init;                 // implicit initial tickets
@@ -350,6 +364,30 @@ __device__ __forceinline__ void load_batch_coalesced(const void* row, int64_t V,
 #pragma unroll
   for (int u = 0; u < kVecsPerBatch; ++u) {
     const int64_t idx = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads;
+    v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
+  }
+}
+
+// Batch b of chunk c, part layout: warp w streams part w (vectors
+// w * kPartVecs .. of the chunk), lane l holding vectors
+// l + (b * kVecsPerBatch + u) * 32 of it, so each load instruction of a warp
+// covers 512 contiguous bytes and a warp's sums cover one contiguous range.
+// Vectors past the row end read as -inf (weight 0).
+template <bool BF16>
+__device__ __forceinline__ int64_t part_vec_index(int c, int b, int u) {
+  using G = Geo<BF16>;
+  return static_cast<int64_t>(c) * G::kChunkVecs + (threadIdx.x >> 5) * G::kPartVecs + (threadIdx.x & 31) +
+         (b * kVecsPerBatch + u) * 32;
+}
+template <bool BF16>
+__device__ __forceinline__ void load_batch_parts(const void* row, int64_t V, int c, int b,
+                                                 uint4 (&v)[kVecsPerBatch]) {
+  using G = Geo<BF16>;
+  const int64_t nvec = V / G::kPerVec;
+  const uint4* rv = static_cast<const uint4*>(row);
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = part_vec_index<BF16>(c, b, u);
     v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
   }
 }
@@ -535,20 +573,21 @@ __device__ __forceinline__ double chunk_prefix(const double (&v)[4], double (&pr
 }
 
 // Arrival of `weight` units on a per-request counter: returns true in exactly
-// one CTA, the one completing `expected` units, and resets the counter for the
-// next launch.  Writes
-// this CTA made before the call are visible to the last arriver afterwards.
+// one CTA, the one completing `expected` units, and resets the counter for its
+// next use.  Thread 0's add is a release and acquire at GPU scope after a CTA
+// barrier, so everything the arriving CTAs wrote before the call is visible to
+// every thread of the last arriver once the call returns.  The reset reaches
+// the next use's arrivals through the release that announces their items (the
+// queue's slot stores) or through the end of the launch.
 __device__ __forceinline__ bool arrive_last(unsigned* counter, unsigned expected, int* sh_flag,
                                             unsigned weight = 1u) {
   sync_compute();
   if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned old = atomicAdd(counter, weight);
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
+                 : "=r"(old) : "l"(counter), "r"(weight) : "memory");
     const bool last = (old + weight == expected);
-    if (last) {
-      *counter = 0u;
-      __threadfence();
-    }
+    if (last) *counter = 0u;
     *sh_flag = last ? 1 : 0;
   }
   sync_compute();

@@ -172,7 +172,6 @@ __global__ void __launch_bounds__(kThreads) k_conf(ConfParams cp) {
   conf_request(cp, blockIdx.x, s_surv);
   if (cp.total <= 0) return;
   if (!arrive_last(cp.arrive, static_cast<unsigned>(cp.B), &s_last)) return;
-  __threadfence();
   conf_select(cp, ss, s_keys, kSelCache);
 }
 

@@ -3,7 +3,7 @@
 //
 // Work items (32-bit payloads):
 //   STATS  (request, row slot, segment)  softmax / arg-max statistics of one row segment
-//   SAMPLE (request, segment)            residual / bonus masses of one segment
+//   SAMPLE (request, chunk)              residual / bonus masses of one chunk
 //   REFINE (refinement slot, sub-chunk)  fp64 recomputation of one sub-chunk
 // The CTA completing the last item of a task decides what follows and
 // enqueues it: the chain decision after STATS (then the next position's rows,
@@ -21,13 +21,15 @@
 //
 // The first tickets (0 .. n_init-1) are implicit: the confidence head of every
 // request when it runs in this launch, then the rows of position 0 (prefix)
-// or of every position (dense), decoded from the ticket number.  Later tickets
-// index the queue, whose slots carry the run's epoch in their upper 32 bits so
-// a slot left by an earlier run is never taken for a new item.  New items join
-// the one FIFO behind those already queued (handing generated items out
-// first was measured slower on every workload).  A CTA waiting for a slot
-// sleeps between polls and gives up after a bounded number of polls (setting
-// the queue error), as does the whole kernel once every request is finished.
+// or of every position (dense), decoded from the ticket number.  Items the
+// run generates go to one queue per class, served after the implicit tickets
+// in the order: statistics of a later position, sample chunks, refinement
+// sub-chunks.  (One FIFO for all of them kept chain items waiting behind sample
+// items, and a request's chain of positions is the run's critical path.)  The
+// slots carry the run's epoch in their upper 32 bits so a slot left by an
+// earlier run is never taken for a new item.  A CTA waiting for work sleeps
+// between polls and gives up after a bounded number of polls (setting the
+// queue error), as does the whole kernel once every request is finished.
 // The last CTA to leave resets the queue counters for the next run.
 #pragma once
 #include "common.cuh"
@@ -102,19 +104,61 @@ __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h
   return item_stats(static_cast<int>(i), slot, static_cast<int>(r % p.n_segs));
 }
 
-// Thread 0: the next item (or kItemExit).  Tickets are handed out in order by
-// one atomic add; a ticket past the implicit ones waits for its queue slot.
-__device__ uint32_t fetch_item(const RunParams& p) {
-  const unsigned h = atomicAdd(p.q_ctl + kQHead, 1u);
-  if (h < p.n_init) return implicit_item(p, h);
-  const unsigned d = h - p.n_init;
+// Queue classes, in the order idle CTAs serve them once the implicit tickets
+// are gone: a later position's statistics first (they extend the longest
+// chains), then sample segments, then refinement sub-chunks.
+constexpr int kClassStats = 0, kClassSample = 1, kClassRefine = 2;
+static_assert(kClassRefine < kQClasses, "queue classes");
+// Sample items cover this many chunks of the row pair (shorter items keep the
+// sample step, which ends a request's chain, short).
+constexpr int kSampleChunksPerItem = 1;
+
+__device__ __forceinline__ int ld_volatile_s32(const unsigned* a) {
+  int v;
+  asm volatile("ld.volatile.global.s32 %0, [%1];" : "=r"(v) : "l"(a));
+  return v;
+}
+
+// Thread 0: the item behind ticket d of class c, once its producer wrote the
+// slot (it reserved the slot before publishing the count the claim came from,
+// so the wait is short); kItemExit if the wait gives up.
+__device__ uint32_t claim_slot(const RunParams& p, int c, unsigned d) {
+  const unsigned long long* slot = p.q_slots + p.q_off[c] + d;
   for (unsigned spin = 0;; ++spin) {
-    if (d < p.q_capacity) {
-      const unsigned long long v = ld_acquire_u64(p.q_slots + d);
-      if (static_cast<unsigned>(v >> 32) == p.q_epoch) return static_cast<uint32_t>(v);
+    const unsigned long long v = ld_acquire_u64(slot);
+    if (static_cast<unsigned>(v >> 32) == p.q_epoch) return static_cast<uint32_t>(v);
+    if (spin >= kSpinLimit) {
+      atomicOr(&p.counters->queue_error, 1u);
+      return kItemExit;
+    }
+    __nanosleep(64);
+  }
+}
+
+// Thread 0: the next item (or kItemExit).  Implicit tickets first (one atomic
+// add each; `implicit_left` turns false at the first ticket past them), then
+// the classes in order: a CTA claims an item of class c by taking one unit of
+// its published count (giving it back if there was none) and then a ticket of
+// the class, so it never holds a ticket whose item was not yet produced.
+__device__ uint32_t fetch_item(const RunParams& p, bool& implicit_left) {
+  if (implicit_left) {
+    const unsigned h = atomicAdd(p.q_ctl + kQHead, 1u);
+    if (h < p.n_init) return implicit_item(p, h);
+    implicit_left = false;
+  }
+  for (unsigned spin = 0;; ++spin) {
+#pragma unroll 1
+    for (int c = 0; c < kQClasses; ++c) {
+      unsigned* avail = p.q_ctl + kQAvail0 + c;
+      if (ld_volatile_s32(avail) <= 0) continue;
+      if (static_cast<int>(atomicSub(avail, 1u)) <= 0) {
+        atomicAdd(avail, 1u);
+        continue;
+      }
+      return claim_slot(p, c, atomicAdd(p.q_ctl + kQClaim0 + c, 1u));
     }
     if (ld_acquire_u32(p.q_ctl + kQDone) >= static_cast<unsigned>(p.B)) return kItemExit;
-    if (spin >= kSpinLimit) {
+    if (spin >= kSpinLimit || ld_volatile_s32(&p.counters->queue_error) != 0) {
       atomicOr(&p.counters->queue_error, 1u);
       return kItemExit;
     }
@@ -122,21 +166,28 @@ __device__ uint32_t fetch_item(const RunParams& p) {
   }
 }
 
-// Enqueue n items whose payloads gen(q) (q < n) produces (all threads call).
+// Enqueue n items of class c whose payloads gen(q) (q < n) produces (all
+// threads call): reserve slots, write them, then publish the count.
 template <typename Gen>
-__device__ __forceinline__ void enqueue(const RunParams& p, int n, Gen gen, unsigned* s_base) {
-  if (threadIdx.x == 0) *s_base = atomicAdd(p.q_ctl + kQTail, static_cast<unsigned>(n));
+__device__ __forceinline__ void enqueue(const RunParams& p, int c, int n, Gen gen, unsigned* s_base) {
+  if (threadIdx.x == 0) *s_base = atomicAdd(p.q_ctl + kQTail0 + c, static_cast<unsigned>(n));
   __syncthreads();
   const unsigned base = *s_base;
   for (int q = threadIdx.x; q < n; q += kThreads) {
     const unsigned d = base + static_cast<unsigned>(q);
-    if (d < p.q_capacity) {
-      st_release_u64(p.q_slots + d, (static_cast<unsigned long long>(p.q_epoch) << 32) | gen(q));
+    if (d < p.q_cap[c]) {
+      st_release_u64(p.q_slots + p.q_off[c] + d, (static_cast<unsigned long long>(p.q_epoch) << 32) | gen(q));
     } else {
       atomicOr(&p.counters->queue_error, 2u);
     }
   }
+  // The count needs no ordering against the slots: a claim waits for its
+  // slot's epoch tag anyway.
   __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned fits = base >= p.q_cap[c] ? 0u : min(static_cast<unsigned>(n), p.q_cap[c] - base);
+    atomicAdd(p.q_ctl + kQAvail0 + c, fits);
+  }
 }
 
 __device__ __forceinline__ void finish_request(const RunParams& p) {
@@ -148,7 +199,8 @@ __device__ __forceinline__ void finish_request(const RunParams& p) {
 
 template <bool BF16>
 __device__ void enqueue_sample(const RunParams& p, int i, unsigned* s_base) {
-  enqueue(p, p.n_segs, [&](int q) { return item_sample(i, q); }, s_base);
+  const int n = (p.n_chunks + kSampleChunksPerItem - 1) / kSampleChunksPerItem;
+  enqueue(p, kClassSample, n, [&](int q) { return item_sample(i, q); }, s_base);
 }
 
 // Wait (thread 0) until the confidence head run in this launch has published
@@ -218,9 +270,18 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     } else {
       stochastic_segment_staged<BF16>(row, p.V, seg, cc, p.meta + rec0 + seg, p.ssum + rec0 + seg, st, stage_buf);
     }
+    // The item holding the drafted token's logit leaves it for the decision
+    // (published by the arrival below), which then reads a small array
+    // instead of the row.
+    if (!ri.greedy && j < p.k && threadIdx.x == 0) {
+      const int64_t lo = whole ? 0 : static_cast<int64_t>(seg) * SegGeo<BF16>::kSeg;
+      const int64_t hi = whole ? p.V : min(p.V, lo + SegGeo<BF16>::kSeg);
+      const int xj = __ldg(p.tokens + static_cast<int64_t>(i) * p.k + j);
+      if (xj >= lo && xj < hi)
+        p.tok_cache[(static_cast<int64_t>(i) * p.k + j) * 2 + (is_draft ? 1 : 0)] = load_logit(row, xj, BF16);
+    }
   }
   if (!arrive_last(p.arrive_stats + i, expected, &st.flag, weight)) return;
-  __threadfence();
   if (p.mode == kModeDense) {
     decide_request<BF16>(p, i, ri, dec);
     __syncthreads();
@@ -240,7 +301,7 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     const int jn = j + 1;
     const int rows = task_rows(rc, jn);
     const int ns = p.n_segs;
-    enqueue(p, rows * ns, [&](int q) {
+    enqueue(p, kClassStats, rows * ns, [&](int q) {
       return item_stats(i, (q / ns) == 0 ? jn : p.k + 1 + jn, q % ns);
     }, s_base);
   } else if (next == 2) {
@@ -259,7 +320,6 @@ __device__ void engine_conf(const RunParams& p, int i, int* flag, uint4* stage_b
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(ss + 1);
   conf_request(p.cp, i, s_surv);
   if (!arrive_last(p.cp.arrive, static_cast<unsigned>(p.B), flag)) return;
-  __threadfence();
   if (p.cp.total > 0) conf_select(p.cp, *ss, keys, kConfKeysInStage);
   sync_compute();
   if (threadIdx.x == 0) {
@@ -269,12 +329,12 @@ __device__ void engine_conf(const RunParams& p, int i, int* flag, uint4* stage_b
 }
 
 template <bool BF16>
-__device__ void engine_sample(const RunParams& p, int i, int seg, SampleShared& sa,
+__device__ void engine_sample(const RunParams& p, int i, int part, SampleShared& sa,
                               unsigned* s_base, uint4* stage_buf) {
   const Job jb = load_job(p.jobs + i);
-  segment_masses_staged<BF16>(p, i, jb, seg, sa, stage_buf);
-  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(p.n_segs), &sa.flag)) return;
-  __threadfence();
+  chunk_masses_staged<BF16, kSampleChunksPerItem>(p, i, jb, part * kSampleChunksPerItem, stage_buf);
+  const int n_parts = (p.n_chunks + kSampleChunksPerItem - 1) / kSampleChunksPerItem;
+  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(n_parts), &sa.flag)) return;
   locate_sample<BF16>(p, i, jb, sa);
   const int slot = sa.refine_slot;
   if (slot < 0) {
@@ -282,14 +342,13 @@ __device__ void engine_sample(const RunParams& p, int i, int seg, SampleShared& 
     return;
   }
   const int n_subs = p.n_chunks * kSubsPerChunk;
-  enqueue(p, n_subs, [&](int q) { return item_refine(slot, q); }, s_base);
+  enqueue(p, kClassRefine, n_subs, [&](int q) { return item_refine(slot, q); }, s_base);
 }
 
 template <bool BF16>
 __device__ void engine_refine(const RunParams& p, int slot, int sub, RefineShared& rf) {
   refine_item<BF16>(p, slot, sub, rf);
   if (!arrive_last(p.arrive_r1 + slot, static_cast<unsigned>(p.n_chunks * kSubsPerChunk), &rf.flag)) return;
-  __threadfence();
   refine_finalize<BF16>(p, slot, rf);
   finish_request(p);
 }
@@ -304,9 +363,10 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
   __shared__ uint32_t s_item;
   __shared__ unsigned s_base;
   exp2_table_init(rf.tab);
+  bool implicit_left = true;  // thread 0: implicit tickets may remain
 #pragma unroll 1
   for (;;) {
-    if (threadIdx.x == 0) s_item = fetch_item(p);
+    if (threadIdx.x == 0) s_item = fetch_item(p, implicit_left);
     __syncthreads();
     const uint32_t it = s_item;
     if (it == kItemExit) break;
@@ -326,9 +386,13 @@ __global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams
     __threadfence();
     if (atomicAdd(p.q_ctl + kQExits, 1u) == gridDim.x - 1) {
       p.q_ctl[kQHead] = 0u;
-      p.q_ctl[kQTail] = 0u;
       p.q_ctl[kQDone] = 0u;
       p.q_ctl[kQExits] = 0u;
+      for (int c = 0; c < kQClasses; ++c) {
+        p.q_ctl[kQTail0 + c] = 0u;
+        p.q_ctl[kQClaim0 + c] = 0u;
+        p.q_ctl[kQAvail0 + c] = 0u;
+      }
       *p.counters_next = Counters{};
       __threadfence();
     }

@@ -5,14 +5,18 @@
 // draft-and-verify does not change the output").
 //
 // Inverse-CDF sampling in index order: the token is the smallest t whose
-// running weight exceeds u * (total weight).  One CTA per (request, segment of
-// kChunksPerSeg chunks) computes each chunk's weight mass in fp32 (fp64
-// accumulation) together with a certified bound on its error; the request's
-// last CTA prefixes the chunk masses block-wide, rescans the one chunk holding
-// u * total and checks that the chosen cell's edges sit farther from u * total
-// than the accumulated bound.  When they do not, the request is queued for the
-// fp64 refinement (refine.cuh), which recomputes the weights exactly as the
-// fp64 rule defines them.
+// running weight exceeds u * (total weight).  The row pair is streamed in
+// chunks (an engine item each; a segment of kChunksPerSeg chunks per CTA in
+// the vocabulary-parallel kernels), warp w of the CTA streaming part w of the
+// chunk, a contiguous eighth; every part's weight mass is summed in fp32 (fp64
+// accumulation) together with a certified bound on its error.  The request's
+// last CTA prefixes the part masses block-wide, rescans the one part holding
+// u * total (one vector per thread) and checks that the chosen cell's edges
+// sit farther from u * total than the bound on the error of
+// (prefix - u * total): each term's bound counts 1 - u times before the cell
+// and u times after it.  When they do not, the request is queued for the fp64
+// refinement (refine.cuh), which recomputes the weights exactly as the fp64
+// rule defines them.
 #pragma once
 #include "common.cuh"
 #include "stage.cuh"
@@ -26,8 +30,10 @@ namespace sv {
 // Fa, Fb are integer frames at or above the logits they serve (a batch's own
 // maximum), so the exponent argument, and with it its rounding, stays small.
 // Bound per term: p~ (epsa + kappa |xa|) + q~ (epsb + kappa |xb|) where eps
-// carries the ex2 error, the products' rounding, the normaliser's bound and the
-// frame's share of the temperature-rounding term.
+// carries the ex2 error, the products' rounding and the frame's share of the
+// temperature-rounding term; the error of the normalisers' ratio, the one part
+// of their errors that does not cancel from a scale-free sample, rides on the
+// draft terms (epsb).
 struct WeightCtx {
   float cc, Fa, Fb, Aeff, Beff, kappa, epsa, epsb;
   bool residual;
@@ -200,41 +206,54 @@ __device__ __forceinline__ void batch_weights(const JobF32& j, const uint4 (&va)
 constexpr int kChunksPerSeg = SegGeo<true>::kSegVecs / Geo<true>::kChunkVecs;  // 2
 static_assert(SegGeo<false>::kSegVecs / Geo<false>::kChunkVecs == kChunksPerSeg, "geometry");
 
+// Mass record of part (c, this warp) of request i (lane 0 of the warp that
+// streamed it): the bound was accumulated in fp32 per batch (inflated for its
+// own rounding), plus the pairwise rounding of the fp32 batch sums.
+template <bool BF16>
+__device__ __forceinline__ void write_part(const RunParams& p, int i, int c, double m, double bb) {
+  SampleChunk r;
+  r.mass = m;
+  r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
+  p.smass[(static_cast<int64_t>(i) * p.n_chunks + c) * kSampleParts + (threadIdx.x >> 5)] = r;
+}
+
 struct SampleShared {
   double d[kWarps];
-  double cm[kChunksPerSeg][kWarps];   // per chunk masses of each warp
-  double cb[kChunksPerSeg][kWarps];   // ... and bounds
   int flag;
   // locate
-  int cstar;
-  double base;        // weight before chunk cstar
-  double base_bound;  // bound before chunk cstar
-  int found;          // local index of the crossing in cstar, or -1
+  int pstar;          // the part holding u * total, or -1
+  double base;        // weight before part pstar
+  double base_bound;  // bound before part pstar
+  double pstar_bound; // the mass record's bound of part pstar
+  double after_bound; // bound of the parts after pstar
+  int found;          // index of the crossing inside part pstar, or -1
   int refine_slot;    // locate's outcome: -1 certain, else the refinement slot
-  double lo_gap, hi_gap, cell_bound;
+  double lo_gap, hi_gap;
+  double lo_bound, hi_bound;  // rescan bounds of part pstar's cells before / through the crossing
 };
 
-// One CTA per (request, segment of kChunksPerSeg chunks), coalesced loads, the
-// next batch's vectors in flight while the current one is reduced.
+// One CTA per (request, segment of kChunksPerSeg chunks), the next batch's
+// vectors in flight while the current one is reduced; each warp writes the
+// records of its parts.
 template <bool BF16>
 __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const Job& jb, int seg,
                                                SampleShared& sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const JobF32 j = job_f32(jb);
   const void* ra = target_row(p, i, jb.row, BF16);
   const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
   constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
   const int c0 = seg * kChunksPerSeg;
   uint4 va[kVecsPerBatch], vb[kVecsPerBatch], na[kVecsPerBatch], nb[kVecsPerBatch];
-  load_batch_coalesced<BF16>(ra, p.V, c0, 0, va);
-  if (j.residual) load_batch_coalesced<BF16>(rb, p.V, c0, 0, vb);
+  load_batch_parts<BF16>(ra, p.V, c0, 0, va);
+  if (j.residual) load_batch_parts<BF16>(rb, p.V, c0, 0, vb);
   double cmass = 0.0, cbound = 0.0;
 #pragma unroll 1
   for (int s = 0; s < kSteps; ++s) {
     if (s + 1 < kSteps) {
       const int c = c0 + (s + 1) / kBatchesPerChunk, b = (s + 1) % kBatchesPerChunk;
-      load_batch_coalesced<BF16>(ra, p.V, c, b, na);
-      if (j.residual) load_batch_coalesced<BF16>(rb, p.V, c, b, nb);
+      load_batch_parts<BF16>(ra, p.V, c, b, na);
+      if (j.residual) load_batch_parts<BF16>(rb, p.V, c, b, nb);
     }
     float sum, bound;
     double unused;
@@ -244,10 +263,8 @@ __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const 
     if ((s + 1) % kBatchesPerChunk == 0) {
       const double m = warp_sum_d(cmass);
       const double bb = warp_sum_d(cbound);
-      if (lane == 0) {
-        sh.cm[s / kBatchesPerChunk][warp] = m;
-        sh.cb[s / kBatchesPerChunk][warp] = bb;
-      }
+      const int c = c0 + s / kBatchesPerChunk;
+      if (lane == 0 && c < p.n_chunks) write_part<BF16>(p, i, c, m, bb);
       cmass = 0.0;
       cbound = 0.0;
     }
@@ -257,41 +274,21 @@ __device__ __forceinline__ void segment_masses(const RunParams& p, int i, const 
       if (j.residual) vb[u] = nb[u];
     }
   }
-  sync_compute();
-  if (threadIdx.x < kChunksPerSeg) {
-    const int b = threadIdx.x;
-    const int c = c0 + b;
-    if (c < p.n_chunks) {
-      double m = 0.0, bb = 0.0;
-      for (int w2 = 0; w2 < kWarps; ++w2) {
-        m += sh.cm[b][w2];
-        bb += sh.cb[b][w2];
-      }
-      SampleChunk r;
-      r.mass = m;
-      // the bound was accumulated in fp32 per batch (inflate for its own
-      // rounding), plus the pairwise rounding of the fp32 batch sums
-      r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
-      p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
-    }
-  }
 }
 
-// The same masses fed by per-thread asynchronous staging: step s of the
-// segment (chunk c0 + s / 4, batch s % 4) stages the target's two vectors in
-// slots 0-1 and the draft's in slots 2-3 (bonus jobs: the target's only).
+// The same masses fed by per-thread asynchronous staging: step s (chunk
+// c0 + s / 4, batch s % 4) stages the target's two vectors in slots 0-1 and
+// the draft's in slots 2-3 (bonus jobs: the target's only).
 static_assert(2 * kVecsPerBatch == kStepVecs, "a staging step is one batch of both rows");
 
-// FULL: the segment's two chunks lie inside the row, so no range checks.
+// FULL: the item's chunks lie inside the row, so no range checks.
 template <bool BF16, bool FULL>
 __device__ __forceinline__ void stage_sample_step(Stager& sg, const void* ra, const void* rb,
                                                   int64_t nvec, int c0, int s) {
-  using G = Geo<BF16>;
   const int c = c0 + s / kBatchesPerChunk, b = s % kBatchesPerChunk;
-  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
 #pragma unroll
   for (int u = 0; u < kVecsPerBatch; ++u) {
-    const int64_t idx = base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads;
+    const int64_t idx = part_vec_index<BF16>(c, b, u);
     const bool valid = FULL || idx < nvec;
     cp_async16(sg.slot(s, u), static_cast<const uint4*>(ra) + (valid ? idx : 0), valid);
     if (rb) cp_async16(sg.slot(s, kVecsPerBatch + u), static_cast<const uint4*>(rb) + (valid ? idx : 0), valid);
@@ -300,27 +297,26 @@ __device__ __forceinline__ void stage_sample_step(Stager& sg, const void* ra, co
   ++sg.issued;
 }
 
-// The streaming part of segment_masses_staged (FULL: no range checks).
-template <bool BF16, bool FULL>
-__device__ __forceinline__ void segment_masses_pass(const JobF32& j, const void* ra, const void* rb,
-                                                    int64_t nvec, int c0, SampleShared& sh,
-                                                    uint4* stage_buf) {
-  using G = Geo<BF16>;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
+// The streaming part of chunk_masses_staged over NC chunks from c0 (FULL: no
+// range checks).
+template <bool BF16, bool FULL, int NC>
+__device__ __forceinline__ void chunk_masses_pass(const RunParams& p, int i, const JobF32& j,
+                                                  const void* ra, const void* rb, int64_t nvec, int c0,
+                                                  uint4* stage_buf) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kSteps = NC * kBatchesPerChunk;
   Stager sg{stage_buf};
 #pragma unroll
-  for (int st = 0; st < kStageSlots; ++st) stage_sample_step<BF16, FULL>(sg, ra, rb, nvec, c0, st);
+  for (int st = 0; st < kStageSlots && st < kSteps; ++st) stage_sample_step<BF16, FULL>(sg, ra, rb, nvec, c0, st);
   double cmass = 0.0, cbound = 0.0;
 #pragma unroll 1
   for (int st = 0; st < kSteps; ++st) {
     cp_async_wait(sg.issued - st - 1);
     const int c = c0 + st / kBatchesPerChunk, b = st % kBatchesPerChunk;
-    const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + threadIdx.x;
     uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
 #pragma unroll
     for (int u = 0; u < kVecsPerBatch; ++u) {
-      const bool valid = FULL || base + static_cast<int64_t>(b * kVecsPerBatch + u) * kThreads < nvec;
+      const bool valid = FULL || part_vec_index<BF16>(c, b, u) < nvec;
       va[u] = valid ? *sg.slot(st, u) : neg_inf_vec<BF16>();
       vb[u] = rb ? (valid ? *sg.slot(st, kVecsPerBatch + u) : neg_inf_vec<BF16>()) : va[u];
     }
@@ -333,61 +329,49 @@ __device__ __forceinline__ void segment_masses_pass(const JobF32& j, const void*
     if ((st + 1) % kBatchesPerChunk == 0) {
       const double m = warp_sum_d(cmass);
       const double bb = warp_sum_d(cbound);
-      if (lane == 0) {
-        sh.cm[st / kBatchesPerChunk][warp] = m;
-        sh.cb[st / kBatchesPerChunk][warp] = bb;
-      }
+      if (lane == 0 && c < p.n_chunks) write_part<BF16>(p, i, c, m, bb);
       cmass = 0.0;
       cbound = 0.0;
     }
   }
 }
 
-template <bool BF16>
-__device__ __forceinline__ void segment_masses_staged(const RunParams& p, int i, const Job& jb, int seg,
-                                                      SampleShared& sh, uint4* stage_buf) {
+// The masses of the parts of NC chunks from c0 (one engine item), fed by the
+// staging.
+template <bool BF16, int NC>
+__device__ __forceinline__ void chunk_masses_staged(const RunParams& p, int i, const Job& jb, int c0,
+                                                    uint4* stage_buf) {
+  static_assert(NC >= 1 && NC <= kChunksPerSeg, "chunks per item");
   using G = Geo<BF16>;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const JobF32 j = job_f32(jb);
   const void* ra = target_row(p, i, jb.row, BF16);
   const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
   const int64_t nvec = p.V / G::kPerVec;
-  constexpr int kSteps = kChunksPerSeg * kBatchesPerChunk;
-  const int c0 = seg * kChunksPerSeg;
-  if ((static_cast<int64_t>(c0) + kChunksPerSeg) * G::kChunkVecs <= nvec)
-    segment_masses_pass<BF16, true>(j, ra, rb, nvec, c0, sh, stage_buf);
+  if ((static_cast<int64_t>(c0) + NC) * G::kChunkVecs <= nvec)
+    chunk_masses_pass<BF16, true, NC>(p, i, j, ra, rb, nvec, c0, stage_buf);
   else
-    segment_masses_pass<BF16, false>(j, ra, rb, nvec, c0, sh, stage_buf);
-  sync_compute();
-  if (threadIdx.x < kChunksPerSeg) {
-    const int bc = threadIdx.x;
-    const int c = c0 + bc;
-    if (c < p.n_chunks) {
-      double m = 0.0, bb = 0.0;
-      for (int w2 = 0; w2 < kWarps; ++w2) {
-        m += sh.cm[bc][w2];
-        bb += sh.cb[bc][w2];
-      }
-      SampleChunk r;
-      r.mass = m;
-      r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
-      p.smass[static_cast<int64_t>(i) * p.n_chunks + c] = r;
-    }
-  }
+    chunk_masses_pass<BF16, false, NC>(p, i, j, ra, rb, nvec, c0, stage_buf);
 }
+
+constexpr int kPartsPerThread = 8;  // records per thread in the locate prefix
+static_assert(kMaxChunksPerRow / kBatchesPerChunk * kSampleParts <= kPartsPerThread * kThreads,
+              "the locate prefix covers every part of the longest row");
 
 // Last CTA of request i: find the token or queue the request for refinement.
 template <bool BF16>
 __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleShared& sh) {
   using G = Geo<BF16>;
   const int tid = threadIdx.x;
-  const SampleChunk* sc = p.smass + static_cast<int64_t>(i) * p.n_chunks;
-  // 1. block-wide prefix of the chunk masses and bounds (thread t: chunks 4t..4t+3)
-  double m[4], b[4], pm[4], pb[4];
+  const int n_parts = p.n_chunks * kSampleParts;
+  const SampleChunk* sc = p.smass + static_cast<int64_t>(i) * n_parts;
+  // 1. block-wide prefix of the part masses and bounds (thread t: parts
+  //    8t .. 8t+7)
+  double m[kPartsPerThread], b[kPartsPerThread];
+  double mloc = 0.0, bloc = 0.0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = 4 * tid + q;
-    if (c < p.n_chunks) {
+  for (int q = 0; q < kPartsPerThread; ++q) {
+    const int c = kPartsPerThread * tid + q;
+    if (c < n_parts) {
       const double2 r = __ldcg(reinterpret_cast<const double2*>(sc + c));
       m[q] = r.x;
       b[q] = r.y;
@@ -395,28 +379,38 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
       m[q] = 0.0;
       b[q] = 0.0;
     }
+    mloc += m[q];
+    bloc += b[q];
   }
-  if (tid == 0) sh.cstar = -1;
-  const double total = chunk_prefix(m, pm, sh.d);
+  if (tid == 0) sh.pstar = -1;
+  double total, tball;
+  const double mbase = block_exclusive_scan_d(mloc, sh.d, total);
   sync_compute();
-  const double tb = chunk_prefix(b, pb, sh.d) + 1e-15 * total;
+  const double bbase = block_exclusive_scan_d(bloc, sh.d, tball);
+  const double tb = tball + 1e-15 * total;
   const double target = jb.u2 * total;
+  double pmq = mbase, pbq = bbase;  // prefixes before part q
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int c = 4 * tid + q;
-    if (c < p.n_chunks && pm[q] <= target && pm[q] + m[q] > target) {
-      sh.cstar = c;
-      sh.base = pm[q];
-      sh.base_bound = pb[q] + 1e-15 * pm[q];
+  for (int q = 0; q < kPartsPerThread; ++q) {
+    const int c = kPartsPerThread * tid + q;
+    if (c < n_parts && pmq <= target && pmq + m[q] > target) {
+      sh.pstar = c;
+      sh.base = pmq;
+      sh.base_bound = pbq + 1e-15 * pmq;
+      sh.pstar_bound = b[q];
+      sh.after_bound = fmax(0.0, tb - pbq - b[q]) + 1e-12 * tb;
     }
+    pmq += m[q];
+    pbq += b[q];
   }
   sync_compute();
-  int cstar = sh.cstar;
+  int pstar = sh.pstar;
   // residual mass must clear the 1e-12 floor with certainty
-  if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) cstar = -1;
-  // vocabulary-parallel: only the rank holding chunk cstar rescans it
+  if (jb.kind == kJobResidual && !(total - tb > 1e-12 * (1.0 + 1e-9))) pstar = -1;
+  // vocabulary-parallel: only the rank holding part pstar's chunk rescans it
   const bool sharded = p.c_hi > 0;
-  if (sharded && cstar >= 0 && (cstar < p.c_lo || cstar >= p.c_hi)) {
+  const int cstar = pstar / kSampleParts;
+  if (sharded && pstar >= 0 && (cstar < p.c_lo || cstar >= p.c_hi)) {
     if (tid == 0) {
       p.shard_tok[i] = -2;
       sh.refine_slot = -1;
@@ -426,24 +420,33 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
   }
   bool certain = false;
   int token = -1;
-  if (cstar >= 0) {
-    // 2. rescan chunk cstar in index order (contiguous runs per thread): exact
-    //    fp64 sums of the fp32 weights and their bounds
+  if (pstar >= 0) {
+    // 2. rescan part pstar in index order (thread t: vector t of the part):
+    //    exact fp64 sums of the fp32 weights and their bounds
     const JobF32 j = job_f32(jb);
-    const void* ra = target_row(p, i, jb.row, BF16);
-    const void* rb = j.residual ? draft_row(p, i, jb.row, BF16) : nullptr;
+    const uint4* ra = static_cast<const uint4*>(target_row(p, i, jb.row, BF16));
+    const uint4* rb = j.residual ? static_cast<const uint4*>(draft_row(p, i, jb.row, BF16)) : nullptr;
+    const int64_t nvec = p.V / G::kPerVec;
+    const int64_t vi = static_cast<int64_t>(pstar) * G::kPartVecs + tid;
+    const uint4 va = vi < nvec ? ld_stream(ra + vi) : neg_inf_vec<BF16>();
+    const uint4 vb = rb ? (vi < nvec ? ld_stream(rb + vi) : neg_inf_vec<BF16>()) : va;
+    uint4 fa[kVecsPerBatch], fb[kVecsPerBatch];  // the frames: this vector's own maxima
+#pragma unroll
+    for (int u = 0; u < kVecsPerBatch; ++u) {
+      fa[u] = va;
+      fb[u] = vb;
+    }
+    const WeightCtx w = weight_ctx(j, vec_max<BF16>(fa), j.residual ? vec_max<BF16>(fb) : 0.0f);
+    float xa[G::kPerVec], xb[G::kPerVec];
+    unpack<BF16>(va, xa);
+    unpack<BF16>(vb, xb);
     double tsum = 0.0, tbound = 0.0;
-#pragma unroll 1
-    for (int bt = 0; bt < kBatchesPerChunk; ++bt) {
-      uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
-      load_batch_contiguous<BF16>(ra, p.V, cstar, bt, va);
-      if (j.residual) load_batch_contiguous<BF16>(rb, p.V, cstar, bt, vb);
-      else for (int u = 0; u < kVecsPerBatch; ++u) vb[u] = va[u];
-      float s, bd;
-      double ex;
-      batch_weights<BF16, true>(j, va, vb, s, ex, bd);
-      tsum += ex;
-      tbound += static_cast<double>(bd);
+#pragma unroll
+    for (int q = 0; q < G::kPerVec; ++q) {
+      float wt, bq;
+      weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt, bq);
+      tsum += static_cast<double>(wt);
+      tbound += static_cast<double>(bq);
     }
     double all, allb;
     const double pre = block_exclusive_scan_d(tsum, sh.d, all);
@@ -454,42 +457,35 @@ __device__ void locate_sample(const RunParams& p, int i, const Job& jb, SampleSh
     sync_compute();
     if (start <= target && start + tsum > target) {
       // the one thread holding the crossing walks its logits again (same values)
-      double run = start, runb = sh.base_bound + preb * 1.001;
-      bool done = false;
-      for (int bt = 0; bt < kBatchesPerChunk && !done; ++bt) {
-        uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
-        const int off = load_batch_contiguous<BF16>(ra, p.V, cstar, bt, va);
-        if (j.residual) load_batch_contiguous<BF16>(rb, p.V, cstar, bt, vb);
-        else for (int u = 0; u < kVecsPerBatch; ++u) vb[u] = va[u];
-        const WeightCtx w = weight_ctx(j, vec_max<BF16>(va), j.residual ? vec_max<BF16>(vb) : 0.0f);
-        for (int u = 0; u < kVecsPerBatch && !done; ++u) {
-          float xa[G::kPerVec], xb[G::kPerVec];
-          unpack<BF16>(va[u], xa);
-          if (j.residual) unpack<BF16>(vb[u], xb);
-          for (int q = 0; q < G::kPerVec; ++q) {
-            float wt, bq;
-            weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt, bq);
-            const double before = run;
-            run += static_cast<double>(wt);
-            runb += static_cast<double>(bq) * 1.001;
-            if (run > target) {
-              sh.found = off + u * G::kPerVec + q;
-              sh.lo_gap = target - before;
-              sh.hi_gap = run - target;
-              sh.cell_bound = runb;
-              done = true;
-              break;
-            }
-          }
+      double run = start, runb = preb * 1.001;
+      for (int q = 0; q < G::kPerVec; ++q) {
+        float wt, bq;
+        weight_and_bound(w, xa[q], j.residual ? xb[q] : 0.0f, wt, bq);
+        const double before = run, before_b = runb;
+        run += static_cast<double>(wt);
+        runb += static_cast<double>(bq) * 1.001;
+        if (run > target) {
+          sh.found = tid * G::kPerVec + q;
+          sh.lo_gap = target - before;
+          sh.hi_gap = run - target;
+          sh.lo_bound = before_b;
+          sh.hi_bound = runb;
+          break;
         }
       }
     }
     sync_compute();
     if (tid == 0 && sh.found >= 0) {
-      const double slack = jb.u2 * tb + 1e-14 * total;
-      const double need = sh.cell_bound + slack;
-      certain = sh.lo_gap > need && sh.hi_gap > need;
-      token = static_cast<int>(static_cast<int64_t>(cstar) * G::kChunk + sh.found);
+      // The gaps are u W - S(<x) and S(<=x) - u W.  A term's error enters the
+      // prefix S with weight 1 and the target u W with weight u, so the
+      // parts before pstar count (1 - u) times, those after it u times.
+      // Part pstar's record enters the total (u times); its cells are
+      // recomputed by the rescan, whose own bounds enter the prefix.
+      const double u = jb.u2;
+      const double common = (1.0 - u) * sh.base_bound + u * (sh.after_bound + sh.pstar_bound) +
+                            1e-14 * total;
+      certain = sh.lo_gap > common + sh.lo_bound && sh.hi_gap > common + sh.hi_bound;
+      token = static_cast<int>(static_cast<int64_t>(pstar) * G::kPart + sh.found);
     }
   }
   if (tid == 0) {

@@ -158,30 +158,37 @@ __global__ void __launch_bounds__(kThreads) k_shard_masses(RunParams p, int s_lo
   segment_masses<BF16>(p, i, jb, s_lo + ls, sa);
 }
 
-// Phase 2 / 3: this rank's chunk masses to exchange block 2 ([B, nlc_max]),
-// and back from every rank's block into the whole-row layout.
+// Phase 2 / 3: this rank's part masses to exchange block 2
+// ([B, nlc_max * kSampleParts]), and back from every rank's block into the
+// whole-row layout.
 __global__ void k_shard_pack_masses(RunParams p, int c_lo, int nlc, int nlc_max, SampleChunk* out) {
-  const int64_t n = static_cast<int64_t>(p.B) * nlc_max;
+  const int64_t per_req = static_cast<int64_t>(nlc_max) * kSampleParts;
+  const int64_t n = static_cast<int64_t>(p.B) * per_req;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int i = static_cast<int>(e / nlc_max), lc = static_cast<int>(e % nlc_max);
+    const int i = static_cast<int>(e / per_req);
+    const int64_t lp = e % per_req;  // local part
     SampleChunk r{0.0, 0.0};
-    if (lc < nlc) r = p.smass[static_cast<int64_t>(i) * p.n_chunks + c_lo + lc];
+    if (lp < static_cast<int64_t>(nlc) * kSampleParts)
+      r = p.smass[(static_cast<int64_t>(i) * p.n_chunks + c_lo) * kSampleParts + lp];
     out[e] = r;
   }
 }
 
 __global__ void k_shard_unpack_masses(RunParams p, ShardBounds sb, const SampleChunk* blocks,
                                       int nlc_max) {
-  const int64_t n = static_cast<int64_t>(p.B) * p.n_chunks;
+  const int64_t per_row = static_cast<int64_t>(p.n_chunks) * kSampleParts;
+  const int64_t n = static_cast<int64_t>(p.B) * per_row;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int i = static_cast<int>(e / p.n_chunks), c = static_cast<int>(e % p.n_chunks);
+    const int i = static_cast<int>(e / per_row);
+    const int64_t part = e % per_row;
+    const int c = static_cast<int>(part / kSampleParts);
     const int seg = c / kChunksPerSeg;
     int r = 0;
     while (r + 1 < sb.n && seg >= sb.seg_lo[r + 1]) ++r;
-    const int lc = c - sb.seg_lo[r] * kChunksPerSeg;
-    const SampleChunk* src = blocks + (static_cast<int64_t>(r) * p.B + i) * nlc_max + lc;
+    const int64_t lp = part - static_cast<int64_t>(sb.seg_lo[r]) * kChunksPerSeg * kSampleParts;
+    const SampleChunk* src = blocks + (static_cast<int64_t>(r) * p.B + i) * nlc_max * kSampleParts + lp;
     p.smass[e] = SampleChunk{__ldcg(&src->mass), __ldcg(&src->bound)};
   }
 }

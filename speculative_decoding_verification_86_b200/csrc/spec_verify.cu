@@ -130,7 +130,7 @@ struct spec_verify_ctx {
   int* runc = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
   int32_t* conf_len = nullptr;
-  float* tok_logits = nullptr;    // [max_batch, max_k, 2] (vocabulary-parallel runs)
+  float* tok_logits = nullptr;    // [max_batch, max_k, 2] drafted tokens' logits
   int32_t* fallback = nullptr;    // [max_batch]
   double* conf_prefix = nullptr;  // [max_batch, kMaxK]
   int32_t* conf_cap = nullptr;    // [max_batch]
@@ -184,7 +184,7 @@ spec_status carve(spec_verify_ctx* c) {
   const size_t o_ssum = take(recs * sizeof(double));
   const size_t o_arr = take(3 * static_cast<size_t>(c->max_batch) * sizeof(unsigned));
   const size_t o_jobs = take(static_cast<size_t>(c->max_batch) * sizeof(sv::Job));
-  const size_t o_smass = take(per_req_chunks * sizeof(sv::SampleChunk));
+  const size_t o_smass = take(per_req_chunks * sv::kSampleParts * sizeof(sv::SampleChunk));
   const size_t o_rlist = take(static_cast<size_t>(c->max_batch) * sizeof(int));
   const size_t o_rz = take(per_req_subs * sizeof(double2));
   const size_t o_rm = take(per_req_subs * sizeof(double2));
@@ -202,7 +202,7 @@ spec_status carve(spec_verify_ctx* c) {
                                               sv::SegGeo<false>::kSeg);
   const size_t max_subs = static_cast<size_t>(c->max_chunks) * sv::kBatchesPerChunk;
   const size_t cap = static_cast<size_t>(c->max_batch) *
-                         ((2 * c->max_k + 1) * max_segs + max_segs + max_subs) + 8192;
+                         ((2 * c->max_k + 1) * max_segs + c->max_chunks + max_subs) + 8192;
   if (cap > 0xFFFFFFF0ull) return SPEC_ERR_INVALID_ARG;
   c->q_capacity = static_cast<unsigned>(cap);
   const size_t o_qs = take(cap * sizeof(unsigned long long));
@@ -336,6 +336,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.row_stride = V;
   p.v_lo = 0;
   p.tok_logits = nullptr;
+  p.tok_cache = c->tok_logits;  // the engine's statistics items leave the drafted tokens' logits here
   p.fallback = nullptr;
   p.shard_tok = nullptr;
   p.c_lo = 0;
@@ -406,6 +407,21 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.q_slots = c->q_slots;
   p.q_capacity = c->q_capacity;
   p.q_ctl = c->q_ctl;
+  {
+    // class regions: every later position's rows, every sample item and every
+    // refinement sub-chunk of the batch (each generated at most once)
+    const uint64_t caps[sv::kQClasses] = {
+        static_cast<uint64_t>(B) * (2 * k + 1) * n_segs,
+        static_cast<uint64_t>(B) * ((n_chunks + sv::kSampleChunksPerItem - 1) / sv::kSampleChunksPerItem),
+        static_cast<uint64_t>(B) * n_chunks * sv::kSubsPerChunk};
+    uint64_t off = 0;
+    for (int q = 0; q < sv::kQClasses; ++q) {
+      p.q_off[q] = static_cast<unsigned>(off);
+      p.q_cap[q] = static_cast<unsigned>(caps[q]);
+      off += caps[q];
+    }
+    if (off > c->q_capacity) return SPEC_ERR_INVALID_ARG;
+  }
   p.q_epoch = c->run_id;  // >= 1: slots left by earlier runs carry older epochs
   // Dense order: a statistics item is a whole row when the batch has at least
   // as many rows as the grid has CTAs (one staging pipeline per row, no drain
@@ -460,7 +476,7 @@ ShardSizes shard_sizes(int B, int k, const sv::ShardBounds& sb) {
   z.tok_off = align256(z.rec_bytes);
   z.block1 = z.tok_off + align256(static_cast<size_t>(B) * k * 2 * sizeof(float));
   z.nlc_max = sb.nls_max * sv::kChunksPerSeg;
-  z.block2 = static_cast<size_t>(B) * z.nlc_max * sizeof(sv::SampleChunk);
+  z.block2 = static_cast<size_t>(B) * z.nlc_max * sv::kSampleParts * sizeof(sv::SampleChunk);
   z.nsub_max = z.nlc_max * sv::kSubsPerChunk;
   z.block3 = static_cast<size_t>(B) * z.nsub_max * sizeof(sv::RefRec);
   return z;
@@ -1026,7 +1042,7 @@ spec_status spec_shard_decide(spec_verify_ctx* ctx, int rank, int n_shards, cons
     if (bf16) sv::k_shard_masses<true><<<B * nls, sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls);
     else sv::k_shard_masses<false><<<B * nls, sv::kThreads, 0, stream>>>(p, sb.seg_lo[rank], nls);
   }
-  sv::k_shard_pack_masses<<<grid_for(static_cast<int64_t>(B) * z.nlc_max), 256, 0, stream>>>(
+  sv::k_shard_pack_masses<<<grid_for(static_cast<int64_t>(B) * z.nlc_max * sv::kSampleParts), 256, 0, stream>>>(
       p, p.c_lo, p.c_hi - p.c_lo, z.nlc_max, static_cast<sv::SampleChunk*>(block2));
   return cudaGetLastError() == cudaSuccess ? SPEC_OK : SPEC_ERR_CUDA;
 }
@@ -1051,7 +1067,7 @@ spec_status spec_shard_locate(spec_verify_ctx* ctx, int rank, int n_shards, cons
   cudaGetLastError();
   const ShardSizes z = shard_sizes(B, k, sb);
   p.shard_tok = out_token_votes;
-  sv::k_shard_unpack_masses<<<grid_for(static_cast<int64_t>(B) * p.n_chunks), 256, 0, stream>>>(
+  sv::k_shard_unpack_masses<<<grid_for(static_cast<int64_t>(B) * p.n_chunks * sv::kSampleParts), 256, 0, stream>>>(
       p, sb, static_cast<const sv::SampleChunk*>(blocks2), z.nlc_max);
   if (dtype == SPEC_BF16) sv::k_shard_locate<true><<<B, sv::kThreads, 0, stream>>>(p);
   else sv::k_shard_locate<false><<<B, sv::kThreads, 0, stream>>>(p);

@@ -543,16 +543,33 @@ struct DecideShared {
   int state;        // 0 continue, 1 stop
   int need_exact;   // position whose accept test needs the fp64 row sums, or -1
   double exact_Za, exact_Zb;
+  // dense order: every position's accept test, evaluated at once
+  int dec[kMaxK];   // 1 accept, 0 reject, -1 inside the bound, 2 bad token, 3 non-finite rows
+  double pa[kMaxK], qb[kMaxK];
+  double u2[kMaxK + 1];  // the sample's draw of each position where the chain may end
+  // prefix order: position j's inputs, loaded while the rows are merged
+  int xj;
+  float la, lb;
+  double u;
 };
 
-// Merge the segment records of stochastic row `slot` with one warp.
+// Merge the segment records of stochastic row `slot` with one warp.  Lane l
+// loads the records of segments l, l + 32, ... once (one round trip for rows
+// of up to 32 segments) and keeps the first in registers for the sums.
 __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, int slot,
                                                      RowMerged& out) {
   const int lane = threadIdx.x & 31;
   const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
-  float K = -INFINITY, mraw = -INFINITY;
-  int bad = 0;
-  for (int c = lane; c < p.n_segs; c += 32) {
+  const bool have0 = lane < p.n_segs;
+  float4 m0 = make_float4(-INFINITY, -INFINITY, 0.0f, 0.0f);
+  double s0 = 0.0;
+  if (have0) {
+    m0 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + lane));
+    s0 = __ldcg(p.ssum + base + lane);
+  }
+  float K = m0.x, mraw = m0.y;
+  int bad = (isnan(m0.x) || m0.x == INFINITY) ? 1 : 0;
+  for (int c = lane + 32; c < p.n_segs; c += 32) {
     const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
     if (isnan(m4.x) || m4.x == INFINITY) bad = 1;
     K = fmaxf(K, m4.x);
@@ -565,17 +582,17 @@ __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, 
   double Z = 0.0, ER = 0.0, EA = 0.0;
   if (!bad) {
     for (int c = lane; c < p.n_segs; c += 32) {
-      const float4 m4 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
+      const float4 m4 = c == lane ? m0 : __ldcg(reinterpret_cast<const float4*>(p.meta + base + c));
       if (m4.x == -INFINITY) continue;
-      const double s = __ldcg(p.ssum + base + c);
+      const double sc = c == lane ? s0 : __ldcg(p.ssum + base + c);
       const double d = static_cast<double>(K) - static_cast<double>(m4.x);  // integer >= 0
       const double f = pow2_exact(static_cast<float>(-d));
-      Z += s * f;
+      Z += sc * f;
       ER += static_cast<double>(m4.z) * f;
       // |a| from K = |a_then| + (K_then's distance below K): the rounding weight,
       // plus the offsets recorded inside the segment, plus the segment's own offset.
       EA += (static_cast<double>(m4.z) + static_cast<double>(m4.w) +
-             d * s) * f;
+             d * sc) * f;
     }
   }
   Z = warp_sum_d(Z);
@@ -683,21 +700,18 @@ __device__ __forceinline__ double row_dZ(const TempConsts& t, const RowMerged& r
   return t.eps_base + kLn2 * kU24 * 1.0001 * r.ER / r.Z;
 }
 
-// Accept test of drafted token xj at position j from the fp32 statistics of
-// target row ra and draft row rb: 1 accept, 0 reject, -1 inside the bound.
-// Also returns p~(x), q~(x).  (Thread-local; any one thread may call it.)
+// Accept test of position j from the fp32 statistics of target row ra and
+// draft row rb, given the drafted token's logits la, lb and the draw u:
+// 1 accept, 0 reject, -1 inside the bound.  Also returns p~(x), q~(x).
+// (Thread-local; any one thread may call it.)
 template <bool BF16>
-__device__ __forceinline__ int accept_eval(const RunParams& p, int i, int j, int xj,
-                                          const RowMerged& ra, const RowMerged& rb,
-                                          const TempConsts& t, double& pa, double& qb) {
-  const int64_t tl = (static_cast<int64_t>(i) * p.k + j) * 2;
-  const float la = p.tok_logits ? __ldcg(p.tok_logits + tl) : load_logit(target_row(p, i, j, BF16), xj, BF16);
-  const float lb = p.tok_logits ? __ldcg(p.tok_logits + tl + 1) : load_logit(draft_row(p, i, j, BF16), xj, BF16);
+__device__ __forceinline__ int accept_eval(float la, float lb, double u, const RowMerged& ra,
+                                          const RowMerged& rb, const TempConsts& t, double& pa,
+                                          double& qb) {
   const double arg_a = static_cast<double>(la) * t.cc - static_cast<double>(ra.K);
   const double arg_b = static_cast<double>(lb) * t.cc - static_cast<double>(rb.K);
   pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) / ra.Z;
   qb = (lb == -INFINITY) ? 0.0 : exp2(arg_b) / rb.Z;
-  const double u = draw(p, i, j, 0);
   if (qb == 0.0) return pa > 0.0 ? 1 : 0;
   const double dp = row_dZ(t, ra) + kLn2 * t.eta * (fabs(arg_a + ra.EA / ra.Z) + 1e-3);
   const double dq = row_dZ(t, rb) + kLn2 * t.eta * (fabs(arg_b + rb.EA / rb.Z) + 1e-3);
@@ -706,6 +720,18 @@ __device__ __forceinline__ int accept_eval(const RunParams& p, int i, int j, int
   if (u < rho * (1.0 - delta)) return 1;
   if (u >= rho * (1.0 + delta)) return 0;
   return -1;
+}
+
+// The drafted token's logits at position j (target, draft): from the cache
+// the statistics items (or the vocabulary-parallel gather) filled, else from
+// the rows.
+template <bool BF16>
+__device__ __forceinline__ float2 token_logits(const RunParams& p, int i, int j, int xj) {
+  const int64_t tl = (static_cast<int64_t>(i) * p.k + j) * 2;
+  const float* cache = p.tok_logits ? p.tok_logits : p.tok_cache;
+  if (cache) return make_float2(__ldcg(cache + tl), __ldcg(cache + tl + 1));
+  return make_float2(load_logit(target_row(p, i, j, BF16), xj, BF16),
+                     load_logit(draft_row(p, i, j, BF16), xj, BF16));
 }
 
 // Slow path of an accept decision inside its bound: both normalisers in fp64
@@ -732,10 +758,11 @@ __device__ void accept_exact(const RunParams& p, int i, int j, int xj, const Row
 }
 
 // The job that samples position n of request i: the residual of row pair n
-// (n < L) or the bonus row L.  (Thread 0.)
+// (n < L) or the bonus row L; u2 is the sample's draw, draw(p, i, n, 1).
+// (Thread 0.)
 template <bool BF16>
 __device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerged& ra,
-                          const RowMerged* rb, const TempConsts& t) {
+                          const RowMerged* rb, const TempConsts& t, double u2) {
   Job jb;
   jb.n = n;
   jb.pad0 = 0;
@@ -743,7 +770,7 @@ __device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerg
   jb.kappa = static_cast<float>(t.kappa);
   jb.eta_ln2 = kLn2 * t.eta;
   jb.T = t.T;
-  jb.u2 = draw(p, i, n, 1);
+  jb.u2 = u2;
   jb.row = n;
   jb.Ka = ra.K;
   jb.mraw_a = ra.mraw;
@@ -753,11 +780,18 @@ __device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerg
     jb.mraw_b = rb->mraw;
     jb.A = static_cast<float>(1.0 / ra.Z);
     jb.Bq = static_cast<float>(1.0 / rb->Z);
-    // per term: ex2 error, rounding of 1/Z, of the scaled product and of the
-    // difference, the normaliser's own bound, and |mean exponent| of the
-    // temperature-rounding term (the frame adds its offset, the term its |a|).
-    jb.eps0a = static_cast<double>(p.eps_ex2) + 4 * kU24 + row_dZ(t, ra) + kLn2 * t.eta * ra.EA / ra.Z;
-    jb.eps0b = static_cast<double>(p.eps_ex2) + 4 * kU24 + row_dZ(t, *rb) + kLn2 * t.eta * rb->EA / rb->Z;
+    // Sampling is scale free, so the weights may be compared with
+    // (1 + alpha) max(0, p - q), alpha the relative error of the target's
+    // fp32 1/Za (its normaliser's bound plus the rounding to fp32).  The
+    // common factor then cancels from every target term, and what is left of
+    // it is gamma = beta - alpha, the error of the ratio of the two
+    // normalisers, which scales the draft terms only.  Per term: the ex2 error,
+    // the scaled product's rounding and (target) the difference's rounding,
+    // and |mean exponent| of the temperature-rounding term (the frame adds its
+    // offset, the term its |a|); the draft terms also carry |gamma|.
+    const double gamma = (kU24 + row_dZ(t, ra)) + (kU24 + row_dZ(t, *rb));
+    jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + kLn2 * t.eta * ra.EA / ra.Z;
+    jb.eps0b = static_cast<double>(p.eps_ex2) + kU24 + kLn2 * t.eta * rb->EA / rb->Z + gamma * 1.0001;
     // Bracket of rho = Z_a / Z_b in the refinement's frames (each row relative
     // to its own max at the true temperature): the fp32 sums' bounds, the
     // reshaping by the rounded temperature factor, and a factor 3 of margin.
@@ -865,69 +899,72 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     return;
   }
 
-  // Stochastic chain: thread 0 carries it; the block joins the fp64 slow path.
+  // Stochastic chain.  Thread j evaluates position j's accept test (all at
+  // once: each waits on its own token logits); then the walk takes them in
+  // order until the first rejection, the whole block settling a test inside
+  // its bound in fp64 before the walk goes on.
   const TempConsts t = temp_consts<BF16>(p, ri.T);
+  if (tid < L) {
+    const int j = tid;
+    const int xj = __ldg(x + j);
+    const RowMerged& ra = sh.rows[j];
+    const RowMerged& rb = sh.rows[k + 1 + j];
+    double pa = 0.0, qb = 0.0;
+    int d;
+    if (xj < 0 || static_cast<int64_t>(xj) >= p.V) {
+      d = 2;
+    } else if (ra.bad || rb.bad) {
+      d = 3;
+    } else {
+      const float2 l = token_logits<BF16>(p, i, j, xj);
+      d = accept_eval<BF16>(l.x, l.y, draw(p, i, j, 0), ra, rb, t, pa, qb);
+    }
+    sh.dec[j] = d;
+    sh.pa[j] = pa;
+    sh.qb[j] = qb;
+  }
+  if (tid <= L) sh.u2[tid] = draw(p, i, tid, 1);  // the sample's draw, wherever the chain ends
+  sync_compute();
   int n = L;
   uint32_t status = 0;
   for (int j = 0; j < L; ++j) {
-    int xj = 0;
-    if (tid == 0) {
-      sh.state = 0;
-      sh.need_exact = -1;
-      xj = __ldg(x + j);
-      const RowMerged& ra = sh.rows[j];
-      const RowMerged& rb = sh.rows[k + 1 + j];
-      if (xj < 0 || static_cast<int64_t>(xj) >= p.V) {
-        status = kDevBadToken;
-        sh.state = 1;
-      } else if (ra.bad || rb.bad) {
-        status = kDevNonfinite;
-        sh.state = 1;
-      } else {
-        double pa, qb;
-        const int decision = accept_eval<BF16>(p, i, j, xj, ra, rb, t, pa, qb);
-        if (op) op[j] = static_cast<float>(pa);
-        if (oq) oq[j] = static_cast<float>(qb);
-        if (decision < 0) {
-          sh.need_exact = j;
-        } else if (decision == 1) {
-          tok[j] = xj;
-        } else {
-          n = j;
-          sh.state = 1;
+    if (sh.dec[j] == -1) {
+      if (p.fallback) {
+        // the fp64 row sums need every rank's logits: the request is redone whole
+        if (tid == 0) {
+          for (int jj = 0; jj <= j; ++jj) {
+            if (op) op[jj] = static_cast<float>(sh.pa[jj]);
+            if (oq) oq[jj] = static_cast<float>(sh.qb[jj]);
+          }
+          p.fallback[i] = 1;
+          p.jobs[i].kind = kJobNone;
         }
+        return;
       }
-    }
-    sync_compute();
-    if (sh.need_exact >= 0 && p.fallback) {
-      // the fp64 row sums need every rank's logits: the request is redone whole
-      if (tid == 0) {
-        p.fallback[i] = 1;
-        p.jobs[i].kind = kJobNone;
-      }
-      return;
-    }
-    if (sh.need_exact >= 0) {
       bool accept = false;
       double pa = 0.0, qb = 0.0;
-      const int xs = __ldg(x + j);
-      accept_exact<BF16>(p, i, j, xs, sh.rows[j], sh.rows[k + 1 + j], t, sh.red, accept, pa, qb);
+      accept_exact<BF16>(p, i, j, __ldg(x + j), sh.rows[j], sh.rows[k + 1 + j], t, sh.red, accept, pa, qb);
       if (tid == 0) {
-        if (op) op[j] = static_cast<float>(pa);
-        if (oq) oq[j] = static_cast<float>(qb);
-        if (accept) {
-          tok[j] = xs;
-        } else {
-          n = j;
-          sh.state = 1;
-        }
-        sh.need_exact = -1;
+        sh.dec[j] = accept ? 1 : 0;
+        sh.pa[j] = pa;
+        sh.qb[j] = qb;
       }
       sync_compute();
     }
-    const int stop = sh.state;
-    sync_compute();
-    if (stop) break;
+    const int d = sh.dec[j];
+    if (d == 2 || d == 3) {
+      status = d == 2 ? kDevBadToken : kDevNonfinite;
+      break;
+    }
+    if (tid == 0) {
+      if (op) op[j] = static_cast<float>(sh.pa[j]);
+      if (oq) oq[j] = static_cast<float>(sh.qb[j]);
+      if (d == 1) tok[j] = __ldg(x + j);
+    }
+    if (d != 1) {
+      n = j;
+      break;
+    }
   }
 
   if (tid == 0) {
@@ -938,7 +975,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     }
     p.out_acc[i] = n;
     if (p.out_status) p.out_status[i] = 0;
-    write_job<BF16>(p, i, n, L, sh.rows[n], n < L ? &sh.rows[k + 1 + n] : nullptr, t);
+    write_job<BF16>(p, i, n, L, sh.rows[n], n < L ? &sh.rows[k + 1 + n] : nullptr, t, sh.u2[n]);
   }
 }
 
@@ -971,6 +1008,22 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
     else merge_stochastic_row(p, i, j, sh.rows[0]);
   } else if (warp == 1 && pair) {
     merge_stochastic_row(p, i, k + 1 + j, sh.rows[1]);
+  } else if (warp == 2) {
+    // the position's other inputs, loaded while the rows are merged
+    const int lane = tid & 31;
+    if (lane == 0 && j < L) {
+      const int xj = __ldg(x + j);
+      sh.xj = xj;
+      if (pair && xj >= 0 && static_cast<int64_t>(xj) < p.V) {
+        const float2 l = token_logits<BF16>(p, i, j, xj);
+        sh.la = l.x;
+        sh.lb = l.y;
+      }
+    } else if (lane == 1 && pair) {
+      sh.u = draw(p, i, j, 0);
+    } else if (lane == 2 && !ri.greedy) {
+      sh.u2[0] = draw(p, i, j, 1);
+    }
   }
   sync_compute();
   const RowMerged& ra = sh.rows[0];
@@ -989,12 +1042,12 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
         if (ri.greedy) {
           p.jobs[i].kind = kJobNone;
         } else {
-          write_job<BF16>(p, i, L, L, ra, nullptr, t);
+          write_job<BF16>(p, i, L, L, ra, nullptr, t, sh.u2[0]);
           sh.state = 2;
         }
       }
     } else {
-      const int xj = __ldg(x + j);
+      const int xj = sh.xj;
       if (xj < 0 || static_cast<int64_t>(xj) >= p.V) {
         status = kDevBadToken;
       } else if (ra.bad || (pair && rb.bad)) {
@@ -1011,7 +1064,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
         }
       } else {
         double pa, qb;
-        const int decision = accept_eval<BF16>(p, i, j, xj, ra, rb, t, pa, qb);
+        const int decision = accept_eval<BF16>(sh.la, sh.lb, sh.u, ra, rb, t, pa, qb);
         if (op) op[j] = static_cast<float>(pa);
         if (oq) oq[j] = static_cast<float>(qb);
         if (decision < 0) sh.need_exact = 1;
@@ -1021,7 +1074,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
         } else {
           p.out_acc[i] = j;
           if (p.out_status) p.out_status[i] = 0;
-          write_job<BF16>(p, i, j, L, ra, &rb, t);
+          write_job<BF16>(p, i, j, L, ra, &rb, t, sh.u2[0]);
           sh.state = 2;
         }
       }
@@ -1043,7 +1096,7 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
       } else {
         p.out_acc[i] = j;
         if (p.out_status) p.out_status[i] = 0;
-        write_job<BF16>(p, i, j, L, ra, &rb, t);
+        write_job<BF16>(p, i, j, L, ra, &rb, t, sh.u2[0]);
         sh.state = 2;
       }
     }
