@@ -191,6 +191,7 @@ struct RunParams {
   double2* rz;             // [B, 4 n_chunks] fp64 normaliser partials per sub-chunk
   double2* rm;             // [B, 4 n_chunks] fp64 support masses (target, draft)
   int* runc;               // [B, 4 n_chunks] sub-chunks holding unsettled logits
+  double4* rmp;            // [B, 4 n_chunks, kWarps] per-part (alpha, A, B) sums, or nullptr
   Counters* counters;      // this run's counters
   Counters* counters_next; // the other run's counters, reset here
 

@@ -32,6 +32,8 @@ struct RefineShared {
   int flag;
   int cstar;
   int redo_all;
+  int use_part, ppart;  // final rescan narrowed to part ppart of the sub-chunk
+  double pbase;
   int use_resid;
   int found;
   double base, target, Za, Zb;
@@ -50,6 +52,27 @@ __device__ __forceinline__ RefineRow refine_row(const Job& jb) {
 }
 
 constexpr int kSubsPerChunk = kBatchesPerChunk;  // a sub-chunk is one batch of a chunk
+constexpr int kSubVecs = kVecsPerBatch * kThreads;  // 512 contiguous vectors
+constexpr int kSubPartVecs = kSubVecs / kWarps;     // 64: one warp's part of a sub-chunk
+
+// Sub-chunk (c, bt), part layout: warp w holds the sub-chunk's vectors
+// 64 w .. 64 w + 63, lane l the two vectors 64 w + l and 64 w + 32 + l, so a
+// warp's sums cover one contiguous eighth of the sub-chunk.
+template <bool BF16>
+__device__ __forceinline__ void load_sub_parts(const void* row, int64_t V, int c, int bt,
+                                               uint4 (&v)[kVecsPerBatch]) {
+  using G = Geo<BF16>;
+  const int64_t nvec = V / G::kPerVec;
+  const uint4* rv = static_cast<const uint4*>(row);
+  const int64_t base = static_cast<int64_t>(c) * G::kChunkVecs + static_cast<int64_t>(bt) * kSubVecs +
+                       (threadIdx.x >> 5) * kSubPartVecs + (threadIdx.x & 31);
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    const int64_t idx = base + u * 32;
+    v[u] = idx < nvec ? ld_stream(rv + idx) : neg_inf_vec<BF16>();
+  }
+}
+static_assert(kVecsPerBatch * 32 == kSubPartVecs, "a warp's two loads cover its part");
 
 // One pass over sub-chunk (c, bt): alpha/beta sums and, for residual jobs, the
 // support sums A, B and the count of unsettled logits (alpha > 0 only: where
@@ -63,8 +86,8 @@ __device__ __forceinline__ void refine_sub_pass(const RunParams& p, int i, const
   const void* ra = target_row(p, i, jb.row, BF16);
   const void* rb = residual ? draft_row(p, i, jb.row, BF16) : nullptr;
   uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
-  load_batch_coalesced<BF16>(ra, p.V, c, bt, va);
-  if (residual) load_batch_coalesced<BF16>(rb, p.V, c, bt, vb);
+  load_sub_parts<BF16>(ra, p.V, c, bt, va);
+  if (residual) load_sub_parts<BF16>(rb, p.V, c, bt, vb);
 #pragma unroll
   for (int u = 0; u < kVecsPerBatch; ++u) {
     float xa[G::kPerVec], xb[G::kPerVec];
@@ -152,6 +175,11 @@ __device__ void refine_item(const RunParams& p, int slot, int sub, RefineShared&
   int unc = 0;
   refine_sub_pass<BF16>(p, i, jb, rr, sub / kSubsPerChunk, sub % kSubsPerChunk, residual, sh.tab,
                         za, zb, A, Bm, unc);
+  if (p.rmp) {  // the part sums, for a rescan of one part in the end
+    const double zw = warp_sum_d(za), aw = warp_sum_d(A), bw = warp_sum_d(Bm);
+    if ((threadIdx.x & 31) == 0)
+      p.rmp[(static_cast<int64_t>(slot) * n_subs + sub) * kWarps + (threadIdx.x >> 5)] = make_double4(zw, aw, bw, 0.0);
+  }
   za = block_sum_d(za, sh.d);
   zb = block_sum_d(zb, sh.d);
   A = block_sum_d(A, sh.d);
@@ -276,7 +304,83 @@ __device__ void refine_finalize(const RunParams& p, int slot, RefineShared& sh) 
     return;
   }
   int token = -1;
-  if (sstar >= 0) {
+  // With settled support the part sums narrow the draw to one eighth of the
+  // sub-chunk, and only that part is rescanned.
+  bool by_part = false;
+  if (sstar >= 0 && p.rmp && !fallback && !sharded) {
+    if (threadIdx.x == sstar / 4) sh.use_part = !((flagged >> (sstar % 4)) & 1);
+    sync_compute();
+    if (sh.use_part) {
+      if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        double m = 0.0;
+        if (lane < kWarps) {
+          const double2* r = reinterpret_cast<const double2*>(p.rmp + (rec0 + sstar) * kWarps + lane);
+          const double2 r0 = __ldcg(r), r1 = __ldcg(r + 1);  // (alpha, A), (B, -)
+          m = use_resid ? fmax(r0.y * iza - r1.x * izb, 0.0) : r0.x;
+        }
+        double incl = m;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const double y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const double pre = incl - m;
+        if (lane == 0) sh.ppart = -1;
+        __syncwarp();
+        if (lane < kWarps && sh.base + pre <= target && sh.base + pre + m > target) {
+          sh.ppart = lane;
+          sh.pbase = sh.base + pre;
+        }
+      }
+      sync_compute();
+      const int pp = sh.ppart;
+      if (pp >= 0) {
+        constexpr int kPartLogits = kSubPartVecs * G::kPerVec;  // 512 bf16 / 256 fp32
+        constexpr int kPer = kPartLogits / kThreads;           // logits per thread
+        static_assert(kPer * kThreads == kPartLogits, "a part spreads evenly over the block");
+        const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
+        const int off0 = bt * (kSubVecs * G::kPerVec) + pp * kPartLogits + threadIdx.x * kPer;  // in the chunk
+        const void* ra = target_row(p, i, jb.row, BF16);
+        const void* rb = use_resid ? draft_row(p, i, jb.row, BF16) : nullptr;
+        double w[kPer];
+        double tsum = 0.0;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+          const int64_t t = static_cast<int64_t>(c) * G::kChunk + off0 + e;
+          w[e] = 0.0;
+          if (t < p.V) {
+            const float a = load_logit(ra, t, BF16);
+            const float b = use_resid ? load_logit(rb, t, BF16) : 0.0f;
+            w[e] = exact_weight<BF16>(a, b, use_resid, rr, iza, izb, sh.tab);
+          }
+          tsum += w[e];
+        }
+        double all;
+        const double pre = block_exclusive_scan_d(tsum, sh.d, all);
+        if (threadIdx.x == 0) sh.found = -1;
+        sync_compute();
+        const double start = sh.pbase + pre;
+        if (start <= target && start + tsum > target) {
+          double run = start;
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) {
+            run += w[e];
+            if (run > target) {
+              sh.found = off0 + e;
+              break;
+            }
+          }
+        }
+        sync_compute();
+        if (sh.found >= 0) {
+          token = static_cast<int>(static_cast<int64_t>(c) * G::kChunk + sh.found);
+          by_part = true;
+        }
+      }
+    }
+  }
+  if (sstar >= 0 && !by_part) {
     const int c = sstar / kSubsPerChunk, bt = sstar % kSubsPerChunk;
     const void* ra = target_row(p, i, jb.row, BF16);
     const void* rb = use_resid ? draft_row(p, i, jb.row, BF16) : nullptr;

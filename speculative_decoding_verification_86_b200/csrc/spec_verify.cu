@@ -128,6 +128,7 @@ struct spec_verify_ctx {
   double2* rz = nullptr;
   double2* rm = nullptr;
   int* runc = nullptr;
+  double4* rmp = nullptr;
   sv::Counters* counters = nullptr;  // [2], alternating between runs
   int32_t* conf_len = nullptr;
   float* tok_logits = nullptr;    // [max_batch, max_k, 2] drafted tokens' logits
@@ -189,6 +190,7 @@ spec_status carve(spec_verify_ctx* c) {
   const size_t o_rz = take(per_req_subs * sizeof(double2));
   const size_t o_rm = take(per_req_subs * sizeof(double2));
   const size_t o_runc = take(per_req_subs * sizeof(int));
+  const size_t o_rmp = take(per_req_subs * sv::kWarps * sizeof(double4));
   const size_t o_cnt = take(2 * sizeof(sv::Counters));
   const size_t o_conf = take(static_cast<size_t>(c->max_batch) * sizeof(int32_t));
   const size_t o_tokl = take(static_cast<size_t>(c->max_batch) * c->max_k * 2 * sizeof(float));
@@ -225,6 +227,7 @@ spec_status carve(spec_verify_ctx* c) {
   c->rz = reinterpret_cast<double2*>(b + o_rz);
   c->rm = reinterpret_cast<double2*>(b + o_rm);
   c->runc = reinterpret_cast<int*>(b + o_runc);
+  c->rmp = reinterpret_cast<double4*>(b + o_rmp);
   c->counters = reinterpret_cast<sv::Counters*>(b + o_cnt);
   c->conf_len = reinterpret_cast<int32_t*>(b + o_conf);
   c->tok_logits = reinterpret_cast<float*>(b + o_tokl);
@@ -364,6 +367,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   p.rz = c->rz;
   p.rm = c->rm;
   p.runc = c->runc;
+  p.rmp = c->rmp;
   if (++c->run_id == 0) c->run_id = 1;
   p.counters = c->counters + (c->run_id & 1u);
   p.counters_next = c->counters + ((c->run_id + 1u) & 1u);

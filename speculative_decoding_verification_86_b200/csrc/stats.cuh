@@ -534,6 +534,18 @@ struct RowMerged {
   float mraw;    // raw max
   int arg;       // greedy: lowest arg-max
   int bad;       // NaN / +inf / all -inf
+  double invZ;   // 1 / Z, and ER / Z, EA / Z (stochastic rows that are not bad)
+  double erz, eaz;
+};
+
+// Constants of a request's temperature for the fp32 path and its bounds.
+struct TempConsts {
+  double T;         // temperature
+  double c_exact;   // log2(e) / T in fp64
+  double eta;       // |relative error| of cc
+  double kappa;     // ln2 (2^-24 + eta): bound per unit |exponent argument|
+  double eps_base;  // ex2 error + pairwise-sum rounding + slack
+  float cc;         // fp32 log2(e) / T used by the fp32 path
 };
 
 struct DecideShared {
@@ -551,6 +563,7 @@ struct DecideShared {
   int xj;
   float la, lb;
   double u;
+  TempConsts tc;
 };
 
 // Merge the segment records of stochastic row `slot` with one warp.  Lane l
@@ -607,6 +620,11 @@ __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, 
     out.mraw = mraw;
     out.arg = -1;
     out.bad = bad;
+    // the decision's divisions, done here while the other row merges
+    const double inv = bad ? 0.0 : 1.0 / Z;
+    out.invZ = inv;
+    out.erz = ER * inv;
+    out.eaz = EA * inv;
   }
 }
 
@@ -669,15 +687,6 @@ __device__ __forceinline__ double draw(const RunParams& p, int i, int j, int d) 
 constexpr double kU24 = 0x1p-24;
 constexpr double kLn2 = 0.69314718055994530942;
 
-// Constants of a request's temperature for the fp32 path and its bounds.
-struct TempConsts {
-  double T;         // temperature
-  double c_exact;   // log2(e) / T in fp64
-  double eta;       // |relative error| of cc
-  double kappa;     // ln2 (2^-24 + eta): bound per unit |exponent argument|
-  double eps_base;  // ex2 error + pairwise-sum rounding + slack
-  float cc;         // fp32 log2(e) / T used by the fp32 path
-};
 
 template <bool BF16>
 __device__ __forceinline__ TempConsts temp_consts(const RunParams& p, float Tf) {
@@ -697,7 +706,7 @@ __device__ __forceinline__ TempConsts temp_consts(const RunParams& p, float Tf) 
 // log p/p~ moves by at most ln2 * eta * |a_x - mean(a)|; that part is added
 // where p(x) is formed.
 __device__ __forceinline__ double row_dZ(const TempConsts& t, const RowMerged& r) {
-  return t.eps_base + kLn2 * kU24 * 1.0001 * r.ER / r.Z;
+  return t.eps_base + kLn2 * kU24 * 1.0002 * r.erz;
 }
 
 // Accept test of position j from the fp32 statistics of target row ra and
@@ -710,15 +719,16 @@ __device__ __forceinline__ int accept_eval(float la, float lb, double u, const R
                                           double& qb) {
   const double arg_a = static_cast<double>(la) * t.cc - static_cast<double>(ra.K);
   const double arg_b = static_cast<double>(lb) * t.cc - static_cast<double>(rb.K);
-  pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) / ra.Z;
-  qb = (lb == -INFINITY) ? 0.0 : exp2(arg_b) / rb.Z;
+  pa = (la == -INFINITY) ? 0.0 : exp2(arg_a) * ra.invZ;
+  qb = (lb == -INFINITY) ? 0.0 : exp2(arg_b) * rb.invZ;
   if (qb == 0.0) return pa > 0.0 ? 1 : 0;
-  const double dp = row_dZ(t, ra) + kLn2 * t.eta * (fabs(arg_a + ra.EA / ra.Z) + 1e-3);
-  const double dq = row_dZ(t, rb) + kLn2 * t.eta * (fabs(arg_b + rb.EA / rb.Z) + 1e-3);
+  const double dp = row_dZ(t, ra) + kLn2 * t.eta * (fabs(arg_a + ra.eaz) + 1e-3);
+  const double dq = row_dZ(t, rb) + kLn2 * t.eta * (fabs(arg_b + rb.eaz) + 1e-3);
   const double delta = (dp + dq) * 1.01 + 1e-13;
-  const double rho = pa / qb;
-  if (u < rho * (1.0 - delta)) return 1;
-  if (u >= rho * (1.0 + delta)) return 0;
+  // u against rho = p/q, compared as u q against p (q > 0)
+  const double uq = u * qb;
+  if (uq < pa * (1.0 - delta)) return 1;
+  if (uq >= pa * (1.0 + delta)) return 0;
   return -1;
 }
 
@@ -778,8 +788,8 @@ __device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerg
     jb.kind = kJobResidual;
     jb.Kb = rb->K;
     jb.mraw_b = rb->mraw;
-    jb.A = static_cast<float>(1.0 / ra.Z);
-    jb.Bq = static_cast<float>(1.0 / rb->Z);
+    jb.A = static_cast<float>(ra.invZ);
+    jb.Bq = static_cast<float>(rb->invZ);
     // Sampling is scale free, so the weights may be compared with
     // (1 + alpha) max(0, p - q), alpha the relative error of the target's
     // fp32 1/Za (its normaliser's bound plus the rounding to fp32).  The
@@ -790,17 +800,17 @@ __device__ void write_job(const RunParams& p, int i, int n, int L, const RowMerg
     // and |mean exponent| of the temperature-rounding term (the frame adds its
     // offset, the term its |a|); the draft terms also carry |gamma|.
     const double gamma = (kU24 + row_dZ(t, ra)) + (kU24 + row_dZ(t, *rb));
-    jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + kLn2 * t.eta * ra.EA / ra.Z;
-    jb.eps0b = static_cast<double>(p.eps_ex2) + kU24 + kLn2 * t.eta * rb->EA / rb->Z + gamma * 1.0001;
+    jb.eps0a = static_cast<double>(p.eps_ex2) + 2 * kU24 + kLn2 * t.eta * ra.eaz * 1.0001;
+    jb.eps0b = static_cast<double>(p.eps_ex2) + kU24 + kLn2 * t.eta * rb->eaz * 1.0001 + gamma * 1.0001;
     // Bracket of rho = Z_a / Z_b in the refinement's frames (each row relative
     // to its own max at the true temperature): the fp32 sums' bounds, the
     // reshaping by the rounded temperature factor, and a factor 3 of margin.
-    const double rho = (ra.Z / rb->Z) *
+    const double rho = (ra.Z * rb->invZ) *
         exp2((static_cast<double>(ra.K) - static_cast<double>(rb->K)) -
              (static_cast<double>(ra.mraw) - static_cast<double>(rb->mraw)) * t.c_exact);
     const double band = 3.0 * (row_dZ(t, ra) + row_dZ(t, *rb) +
         kLn2 * t.eta * (fabs(static_cast<double>(ra.mraw) - static_cast<double>(rb->mraw)) * t.c_exact +
-                        ra.EA / ra.Z + rb->EA / rb->Z + 1.0)) + 1e-12;
+                        ra.eaz + rb->eaz + 1.0)) + 1e-12;
     jb.rho_lo = rho * (1.0 - band);
     jb.rho_hi = rho * (1.0 + band);
   } else {
@@ -1012,9 +1022,15 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
     // the position's other inputs, loaded while the rows are merged
     const int lane = tid & 31;
     if (lane == 0 && j < L) {
+      const float* cache = p.tok_logits ? p.tok_logits : p.tok_cache;
+      const int64_t tl = (static_cast<int64_t>(i) * k + j) * 2;
+      if (pair && cache) {  // issued together with the token's load
+        sh.la = __ldcg(cache + tl);
+        sh.lb = __ldcg(cache + tl + 1);
+      }
       const int xj = __ldg(x + j);
       sh.xj = xj;
-      if (pair && xj >= 0 && static_cast<int64_t>(xj) < p.V) {
+      if (pair && !cache && xj >= 0 && static_cast<int64_t>(xj) < p.V) {
         const float2 l = token_logits<BF16>(p, i, j, xj);
         sh.la = l.x;
         sh.lb = l.y;
@@ -1023,12 +1039,14 @@ __device__ void decide_position(const RunParams& p, int i, const ReqInfo& ri, in
       sh.u = draw(p, i, j, 0);
     } else if (lane == 2 && !ri.greedy) {
       sh.u2[0] = draw(p, i, j, 1);
+    } else if (lane == 3) {
+      sh.tc = temp_consts<BF16>(p, ri.T);
     }
   }
   sync_compute();
   const RowMerged& ra = sh.rows[0];
   const RowMerged& rb = sh.rows[1];
-  const TempConsts t = temp_consts<BF16>(p, ri.T);
+  const TempConsts t = sh.tc;
   if (tid == 0) {
     sh.need_exact = -1;
     sh.state = 0;
