@@ -110,8 +110,15 @@ __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h
 constexpr int kClassStats = 0, kClassSample = 1, kClassRefine = 2;
 static_assert(kClassRefine < kQClasses, "queue classes");
 // Sample items cover this many chunks of the row pair (shorter items keep the
-// sample step, which ends a request's chain, short).
+// sample step, which ends a request's chain, short), or a single part of a
+// chunk when the batch is small enough for every part to get its own CTA.
 constexpr int kSampleChunksPerItem = 1;
+__host__ __device__ __forceinline__ int sample_items_of(int n_chunks, bool parts) {
+  return parts ? n_chunks * kSampleParts : (n_chunks + kSampleChunksPerItem - 1) / kSampleChunksPerItem;
+}
+__device__ __forceinline__ int sample_items(const RunParams& p) {
+  return sample_items_of(p.n_chunks, p.sample_parts != 0);
+}
 
 __device__ __forceinline__ int ld_volatile_s32(const unsigned* a) {
   int v;
@@ -199,8 +206,7 @@ __device__ __forceinline__ void finish_request(const RunParams& p) {
 
 template <bool BF16>
 __device__ void enqueue_sample(const RunParams& p, int i, unsigned* s_base) {
-  const int n = (p.n_chunks + kSampleChunksPerItem - 1) / kSampleChunksPerItem;
-  enqueue(p, kClassSample, n, [&](int q) { return item_sample(i, q); }, s_base);
+  enqueue(p, kClassSample, sample_items(p), [&](int q) { return item_sample(i, q); }, s_base);
 }
 
 // Wait (thread 0) until the confidence head run in this launch has published
@@ -332,9 +338,9 @@ template <bool BF16>
 __device__ void engine_sample(const RunParams& p, int i, int part, SampleShared& sa,
                               unsigned* s_base, uint4* stage_buf) {
   const Job jb = load_job(p.jobs + i);
-  chunk_masses_staged<BF16, kSampleChunksPerItem>(p, i, jb, part * kSampleChunksPerItem, stage_buf);
-  const int n_parts = (p.n_chunks + kSampleChunksPerItem - 1) / kSampleChunksPerItem;
-  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(n_parts), &sa.flag)) return;
+  if (p.sample_parts) part_mass_item<BF16>(p, i, jb, part, sa);
+  else chunk_masses_staged<BF16, kSampleChunksPerItem>(p, i, jb, part * kSampleChunksPerItem, stage_buf);
+  if (!arrive_last(p.arrive_sample + i, static_cast<unsigned>(sample_items(p)), &sa.flag)) return;
   locate_sample<BF16>(p, i, jb, sa);
   const int slot = sa.refine_slot;
   if (slot < 0) {

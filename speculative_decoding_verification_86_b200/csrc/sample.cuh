@@ -353,6 +353,41 @@ __device__ __forceinline__ void chunk_masses_staged(const RunParams& p, int i, c
     chunk_masses_pass<BF16, false, NC>(p, i, j, ra, rb, nvec, c0, stage_buf);
 }
 
+// The mass record of one part (`part` = chunk * kSampleParts + warp index)
+// computed by a whole CTA, for small batches whose chunk items would leave
+// most of the grid idle: thread t takes vector t of the part in each row.
+template <bool BF16>
+__device__ __forceinline__ void part_mass_item(const RunParams& p, int i, const Job& jb, int part,
+                                               SampleShared& sh) {
+  using G = Geo<BF16>;
+  const JobF32 j = job_f32(jb);
+  const uint4* ra = static_cast<const uint4*>(target_row(p, i, jb.row, BF16));
+  const uint4* rb = j.residual ? static_cast<const uint4*>(draft_row(p, i, jb.row, BF16)) : nullptr;
+  const int64_t nvec = p.V / G::kPerVec;
+  const int64_t vi = static_cast<int64_t>(part) * G::kPartVecs + threadIdx.x;
+  uint4 va[kVecsPerBatch], vb[kVecsPerBatch];
+#pragma unroll
+  for (int u = 0; u < kVecsPerBatch; ++u) {
+    va[u] = neg_inf_vec<BF16>();
+    vb[u] = neg_inf_vec<BF16>();
+  }
+  if (vi < nvec) {
+    va[0] = ld_stream(ra + vi);
+    vb[0] = rb ? ld_stream(rb + vi) : va[0];
+  }
+  float sum, bound;
+  double unused;
+  batch_weights<BF16, false>(j, va, vb, sum, unused, bound);
+  const double m = block_sum_d(static_cast<double>(sum), sh.d);
+  const double bb = block_sum_d(static_cast<double>(bound), sh.d);
+  if (threadIdx.x == 0) {
+    SampleChunk r;
+    r.mass = m;
+    r.bound = bb * 1.001 + Geo<BF16>::kSumLevels * kU24 * m;
+    p.smass[static_cast<int64_t>(i) * p.n_chunks * kSampleParts + part] = r;
+  }
+}
+
 constexpr int kPartsPerThread = 8;  // records per thread in the locate prefix
 static_assert(kMaxChunksPerRow / kBatchesPerChunk * kSampleParts <= kPartsPerThread * kThreads,
               "the locate prefix covers every part of the longest row");

@@ -204,7 +204,7 @@ spec_status carve(spec_verify_ctx* c) {
                                               sv::SegGeo<false>::kSeg);
   const size_t max_subs = static_cast<size_t>(c->max_chunks) * sv::kBatchesPerChunk;
   const size_t cap = static_cast<size_t>(c->max_batch) *
-                         ((2 * c->max_k + 1) * max_segs + c->max_chunks + max_subs) + 8192;
+                         ((2 * c->max_k + 1) * max_segs + c->max_chunks * sv::kSampleParts + max_subs) + 8192;
   if (cap > 0xFFFFFFF0ull) return SPEC_ERR_INVALID_ARG;
   c->q_capacity = static_cast<unsigned>(cap);
   const size_t o_qs = take(cap * sizeof(unsigned long long));
@@ -414,9 +414,12 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   {
     // class regions: every later position's rows, every sample item and every
     // refinement sub-chunk of the batch (each generated at most once)
+    // small batches: one sample item per part of a chunk when every part of
+    // every request fits the grid at once
+    p.sample_parts = static_cast<int64_t>(B) * n_chunks * sv::kSampleParts <= c->engine_grid ? 1 : 0;
     const uint64_t caps[sv::kQClasses] = {
         static_cast<uint64_t>(B) * (2 * k + 1) * n_segs,
-        static_cast<uint64_t>(B) * ((n_chunks + sv::kSampleChunksPerItem - 1) / sv::kSampleChunksPerItem),
+        static_cast<uint64_t>(B) * sv::sample_items_of(n_chunks, p.sample_parts != 0),
         static_cast<uint64_t>(B) * n_chunks * sv::kSubsPerChunk};
     uint64_t off = 0;
     for (int q = 0; q < sv::kQClasses; ++q) {

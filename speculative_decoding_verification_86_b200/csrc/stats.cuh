@@ -566,20 +566,32 @@ struct DecideShared {
   TempConsts tc;
 };
 
-// Merge the segment records of stochastic row `slot` with one warp.  Lane l
-// loads the records of segments l, l + 32, ... once (one round trip for rows
-// of up to 32 segments) and keeps the first in registers for the sums.
-__device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, int slot,
-                                                     RowMerged& out) {
+// A lane's first segment record of a row (segment = lane), loaded ahead of
+// the merge so a warp merging several rows waits for one round trip.
+struct SegRec {
+  float4 m;
+  double s;
+};
+__device__ __forceinline__ SegRec load_seg_rec(const RunParams& p, int i, int slot) {
   const int lane = threadIdx.x & 31;
   const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
-  const bool have0 = lane < p.n_segs;
-  float4 m0 = make_float4(-INFINITY, -INFINITY, 0.0f, 0.0f);
-  double s0 = 0.0;
-  if (have0) {
-    m0 = __ldcg(reinterpret_cast<const float4*>(p.meta + base + lane));
-    s0 = __ldcg(p.ssum + base + lane);
+  SegRec r{make_float4(-INFINITY, -INFINITY, 0.0f, 0.0f), 0.0};
+  if (lane < p.n_segs) {
+    r.m = __ldcg(reinterpret_cast<const float4*>(p.meta + base + lane));
+    r.s = __ldcg(p.ssum + base + lane);
   }
+  return r;
+}
+
+// Merge the segment records of stochastic row `slot` with one warp.  Lane l
+// holds the record of segment l (`first`, loaded by load_seg_rec) and loads
+// those of segments l + 32, ... itself.
+__device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, int slot,
+                                                     RowMerged& out, const SegRec& first) {
+  const int lane = threadIdx.x & 31;
+  const int64_t base = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
+  const float4 m0 = first.m;
+  const double s0 = first.s;
   float K = m0.x, mraw = m0.y;
   int bad = (isnan(m0.x) || m0.x == INFINITY) ? 1 : 0;
   for (int c = lane + 32; c < p.n_segs; c += 32) {
@@ -626,6 +638,11 @@ __device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, 
     out.erz = ER * inv;
     out.eaz = EA * inv;
   }
+}
+
+__device__ __forceinline__ void merge_stochastic_row(const RunParams& p, int i, int slot,
+                                                     RowMerged& out) {
+  merge_stochastic_row(p, i, slot, out, load_seg_rec(p, i, slot));
 }
 
 __device__ __forceinline__ void merge_greedy_row(const RunParams& p, int i, int slot,
@@ -872,11 +889,20 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   }
 
   // Merge the rows the chain can read: target rows 0..L, draft rows 0..L-1.
+  // A warp merging two rows loads both rows' records first.
   const int nrows = ri.greedy ? L + 1 : 2 * L + 1;
-  for (int r = warp; r < nrows; r += kWarps) {
-    const int slot = r <= L ? r : (k + 1) + (r - (L + 1));
-    if (ri.greedy) merge_greedy_row(p, i, slot, sh.rows[slot]);
-    else merge_stochastic_row(p, i, slot, sh.rows[slot]);
+  auto slot_of = [&](int r) { return r <= L ? r : (k + 1) + (r - (L + 1)); };
+  if (ri.greedy) {
+    for (int r = warp; r < nrows; r += kWarps) merge_greedy_row(p, i, slot_of(r), sh.rows[slot_of(r)]);
+  } else {
+    const int r0 = warp, r1 = warp + kWarps;
+    SegRec f0{}, f1{};
+    if (r0 < nrows) f0 = load_seg_rec(p, i, slot_of(r0));
+    if (r1 < nrows) f1 = load_seg_rec(p, i, slot_of(r1));
+    if (r0 < nrows) merge_stochastic_row(p, i, slot_of(r0), sh.rows[slot_of(r0)], f0);
+    if (r1 < nrows) merge_stochastic_row(p, i, slot_of(r1), sh.rows[slot_of(r1)], f1);
+    for (int r = warp + 2 * kWarps; r < nrows; r += kWarps)
+      merge_stochastic_row(p, i, slot_of(r), sh.rows[slot_of(r)]);
   }
   sync_compute();
 
@@ -916,6 +942,10 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   const TempConsts t = temp_consts<BF16>(p, ri.T);
   if (tid < L) {
     const int j = tid;
+    const float* cache = p.tok_logits ? p.tok_logits : p.tok_cache;
+    const int64_t tl = (static_cast<int64_t>(i) * k + j) * 2;
+    float2 l = make_float2(0.0f, 0.0f);
+    if (cache) l = make_float2(__ldcg(cache + tl), __ldcg(cache + tl + 1));  // with the token's load
     const int xj = __ldg(x + j);
     const RowMerged& ra = sh.rows[j];
     const RowMerged& rb = sh.rows[k + 1 + j];
@@ -926,14 +956,15 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     } else if (ra.bad || rb.bad) {
       d = 3;
     } else {
-      const float2 l = token_logits<BF16>(p, i, j, xj);
+      if (!cache) l = token_logits<BF16>(p, i, j, xj);
       d = accept_eval<BF16>(l.x, l.y, draw(p, i, j, 0), ra, rb, t, pa, qb);
     }
     sh.dec[j] = d;
     sh.pa[j] = pa;
     sh.qb[j] = qb;
+  } else if (tid >= 32 && tid - 32 <= L) {
+    sh.u2[tid - 32] = draw(p, i, tid - 32, 1);  // the sample's draw, wherever the chain ends
   }
-  if (tid <= L) sh.u2[tid] = draw(p, i, tid, 1);  // the sample's draw, wherever the chain ends
   sync_compute();
   int n = L;
   uint32_t status = 0;
