@@ -207,6 +207,8 @@ struct RunParams {
   int mode;                        // kModeDense / kModePrefix
   int whole_rows;                  // dense order: a statistics item is a whole row (else a segment)
   int sample_parts;                // a sample item is one part of a chunk (small batches), else a chunk
+  int short_segs;                  // statistics segments of one batch step (small dense batches)
+  int seg_len;                     // logits per statistics segment
   unsigned long long* q_slots;     // queue: (epoch << 32) | payload
   unsigned q_capacity;
   unsigned q_off[kQClasses];       // each class's region of q_slots

@@ -263,6 +263,10 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
   if (whole && ri.bad_T) needed = slot == 0;
   if (!needed) return;
   unsigned weight = 1u;
+  // the drafted token, loaded now (its logit is cached once the segment is in)
+  const bool cache_tok = pass && !ri.greedy && j < p.k;
+  int xj = -1;
+  if (cache_tok && threadIdx.x == 0) xj = __ldg(p.tokens + static_cast<int64_t>(i) * p.k + j);
   if (pass) {
     const int64_t rec0 = (static_cast<int64_t>(i) * (2 * p.k + 1) + slot) * p.n_segs;
     const void* row = is_draft ? draft_row(p, i, j, BF16) : target_row(p, i, j, BF16);
@@ -271,6 +275,10 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
       weight = static_cast<unsigned>(p.n_segs);
       if (ri.greedy) stats_row_staged<BF16, true>(row, p.V, p.n_segs, cc, p.meta + rec0, nullptr, st, stage_buf);
       else stats_row_staged<BF16, false>(row, p.V, p.n_segs, cc, p.meta + rec0, p.ssum + rec0, st, stage_buf);
+    } else if (p.short_segs) {
+      if (ri.greedy) greedy_segment_staged<BF16, kShortSegBatches>(row, p.V, seg, p.meta + rec0 + seg, st, stage_buf);
+      else stochastic_segment_staged<BF16, kShortSegBatches>(row, p.V, seg, cc, p.meta + rec0 + seg,
+                                                             p.ssum + rec0 + seg, st, stage_buf);
     } else if (ri.greedy) {
       greedy_segment_staged<BF16>(row, p.V, seg, p.meta + rec0 + seg, st, stage_buf);
     } else {
@@ -279,10 +287,9 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     // The item holding the drafted token's logit leaves it for the decision
     // (published by the arrival below), which then reads a small array
     // instead of the row.
-    if (!ri.greedy && j < p.k && threadIdx.x == 0) {
-      const int64_t lo = whole ? 0 : static_cast<int64_t>(seg) * SegGeo<BF16>::kSeg;
-      const int64_t hi = whole ? p.V : min(p.V, lo + SegGeo<BF16>::kSeg);
-      const int xj = __ldg(p.tokens + static_cast<int64_t>(i) * p.k + j);
+    if (cache_tok && threadIdx.x == 0) {
+      const int64_t lo = whole ? 0 : static_cast<int64_t>(seg) * p.seg_len;
+      const int64_t hi = whole ? p.V : min(p.V, lo + p.seg_len);
       if (xj >= lo && xj < hi)
         p.tok_cache[(static_cast<int64_t>(i) * p.k + j) * 2 + (is_draft ? 1 : 0)] = load_logit(row, xj, BF16);
     }

@@ -323,7 +323,7 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   const int chunk = bf16 ? sv::kChunkBf16 : sv::kChunkF32;
   const int n_chunks = static_cast<int>((V + chunk - 1) / chunk);
   const int segl = bf16 ? sv::SegGeo<true>::kSeg : sv::SegGeo<false>::kSeg;
-  const int n_segs = static_cast<int>((V + segl - 1) / segl);
+  int n_segs = static_cast<int>((V + segl - 1) / segl);
 
   sv::RunParams p{};
   p.target = target;
@@ -382,6 +382,23 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     mode = static_cast<int64_t>(B) * (2 * k + 1) * n_segs <= c->engine_grid ? SPEC_MODE_DENSE
                                                                            : SPEC_MODE_PREFIX;
   p.mode = (force_greedy || mode == SPEC_MODE_PREFIX) ? sv::kModePrefix : sv::kModeDense;
+  // Dense order: a statistics item is a whole row when the batch has at least
+  // as many rows as the grid has CTAs (one staging pipeline per row, no drain
+  // between its segments), else a segment (small batches: every segment of
+  // every row in flight at once) -- a short one when even those all fit.
+  p.whole_rows = (p.mode == sv::kModeDense &&
+                  static_cast<int64_t>(B) * (2 * k + 1) >= c->engine_grid) ? 1 : 0;
+  p.seg_len = segl;
+  if (p.mode == sv::kModeDense && !p.whole_rows) {
+    const int sl = segl / sv::kBatches * sv::kShortSegBatches;
+    const int ns = static_cast<int>((V + sl - 1) / sl);
+    if (static_cast<int64_t>(B) * (2 * k + 1) * ns <= c->engine_grid && ns <= c->max_chunks) {
+      p.short_segs = 1;
+      p.seg_len = sl;
+      n_segs = ns;
+      p.n_segs = ns;
+    }
+  }
   if (conf && p.mode == sv::kModePrefix) {
     // the confidence head runs inside the verification launch, as its first B
     // items (the prefix order reads position 0 before the budgets are needed)
@@ -414,9 +431,9 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   {
     // class regions: every later position's rows, every sample item and every
     // refinement sub-chunk of the batch (each generated at most once)
-    // small batches: one sample item per part of a chunk when every part of
-    // every request fits the grid at once
-    p.sample_parts = static_cast<int64_t>(B) * n_chunks * sv::kSampleParts <= c->engine_grid ? 1 : 0;
+    // small batches: one sample item per part of a chunk when the parts of
+    // every request fit two waves of the grid (usually only some requests sample)
+    p.sample_parts = static_cast<int64_t>(B) * n_chunks * sv::kSampleParts <= 2ll * c->engine_grid ? 1 : 0;
     const uint64_t caps[sv::kQClasses] = {
         static_cast<uint64_t>(B) * (2 * k + 1) * n_segs,
         static_cast<uint64_t>(B) * sv::sample_items_of(n_chunks, p.sample_parts != 0),
@@ -430,12 +447,6 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     if (off > c->q_capacity) return SPEC_ERR_INVALID_ARG;
   }
   p.q_epoch = c->run_id;  // >= 1: slots left by earlier runs carry older epochs
-  // Dense order: a statistics item is a whole row when the batch has at least
-  // as many rows as the grid has CTAs (one staging pipeline per row, no drain
-  // between its segments), else a segment (small batches: every segment of
-  // every row in flight at once).
-  p.whole_rows = (p.mode == sv::kModeDense &&
-                  static_cast<int64_t>(B) * (2 * k + 1) >= c->engine_grid) ? 1 : 0;
   // implicit tickets: the confidence head's items, then the statistics items
   // of every row (dense) or of position 0's rows (prefix)
   const uint64_t per_req = p.mode == sv::kModePrefix ? 2ull * n_segs

@@ -39,6 +39,9 @@ namespace sv {
 constexpr int kSegVecsPerThread = 16;
 constexpr int kBatchVecs = 4;
 constexpr int kBatches = kSegVecsPerThread / kBatchVecs;
+// Small dense batches use short segments of one batch step (8192 bf16 or 4096
+// fp32 logits): four times the items, each a quarter as long.
+constexpr int kShortSegBatches = 1;
 
 template <bool BF16>
 struct SegGeo {
@@ -306,34 +309,37 @@ __device__ __forceinline__ void staged_batch(Stager& sg, int64_t nvec, int64_t s
   }
 }
 
-template <bool BF16, bool FULL>
+// NB: batches per segment -- kBatches for the standard 64 KB segment, fewer
+// for the short segments small batches use (more CTAs per row, shorter items).
+template <bool BF16, bool FULL, int NB = kBatches>
 __device__ __forceinline__ void stochastic_segment_pass(const uint4* rv, int64_t nvec, int64_t seg0,
                                                         float cc, SoftAcc& acc, uint4* stage_buf) {
   Stager sg{stage_buf};
 #pragma unroll
-  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
+  for (int b = 0; b < kStageSlots && b < NB; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
   // full segments: unrolled, so slots and wait counts are compile-time constants
-#pragma unroll (FULL ? kBatches : 1)
-  for (int b = 0; b < kBatches; ++b) {
+#pragma unroll (FULL ? NB : 1)
+  for (int b = 0; b < NB; ++b) {
     uint4 v[kBatchVecs];
     staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
     soft_batch<BF16>(acc, v, cc);
     // refill this step's slot once its values have been used
-    if (b + kStageSlots < kBatches) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+    if (b + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
   }
 }
 
-template <bool BF16>
+template <bool BF16, int NB = kBatches>
 __device__ __forceinline__ void stochastic_segment_staged(const void* row, int64_t V, int seg, float cc,
                                                           ChunkMeta* meta_out, double* sum_out,
                                                           StatsShared& sh, uint4* stage_buf) {
   using G = SegGeo<BF16>;
+  constexpr int64_t kVecs = static_cast<int64_t>(kThreads) * kBatchVecs * NB;
   const uint4* rv = static_cast<const uint4*>(row);
   const int64_t nvec = V / G::kPerVec;
-  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  const int64_t seg0 = static_cast<int64_t>(seg) * kVecs;
   SoftAcc acc;
-  if (seg0 + G::kSegVecs <= nvec) stochastic_segment_pass<BF16, true>(rv, nvec, seg0, cc, acc, stage_buf);
-  else stochastic_segment_pass<BF16, false>(rv, nvec, seg0, cc, acc, stage_buf);
+  if (seg0 + kVecs <= nvec) stochastic_segment_pass<BF16, true, NB>(rv, nvec, seg0, cc, acc, stage_buf);
+  else stochastic_segment_pass<BF16, false, NB>(rv, nvec, seg0, cc, acc, stage_buf);
   soft_merge_block(acc, sh, meta_out, sum_out);
 }
 
@@ -427,32 +433,33 @@ __device__ __forceinline__ void greedy_segment(const void* row, int64_t V, int s
   g.finish(meta_out, sh);
 }
 
-template <bool BF16, bool FULL>
+template <bool BF16, bool FULL, int NB = kBatches>
 __device__ __forceinline__ void greedy_segment_pass(const uint4* rv, int64_t nvec, int64_t seg0,
                                                     GreedyScan<BF16>& g, uint4* stage_buf) {
   Stager sg{stage_buf};
 #pragma unroll
-  for (int b = 0; b < kStageSlots && b < kBatches; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
+  for (int b = 0; b < kStageSlots && b < NB; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
 #pragma unroll 1
-  for (int b = 0; b < kBatches; ++b) {
+  for (int b = 0; b < NB; ++b) {
     uint4 v[kBatchVecs];
     staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
     g.scan(v, seg0, b);
-    if (b + kStageSlots < kBatches) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+    if (b + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
   }
 }
 
-template <bool BF16>
+template <bool BF16, int NB = kBatches>
 __device__ __forceinline__ void greedy_segment_staged(const void* row, int64_t V, int seg,
                                                       ChunkMeta* meta_out, StatsShared& sh,
                                                       uint4* stage_buf) {
   using G = SegGeo<BF16>;
+  constexpr int64_t kVecs = static_cast<int64_t>(kThreads) * kBatchVecs * NB;
   const uint4* rv = static_cast<const uint4*>(row);
   const int64_t nvec = V / G::kPerVec;
-  const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
+  const int64_t seg0 = static_cast<int64_t>(seg) * kVecs;
   GreedyScan<BF16> g;
-  if (seg0 + G::kSegVecs <= nvec) greedy_segment_pass<BF16, true>(rv, nvec, seg0, g, stage_buf);
-  else greedy_segment_pass<BF16, false>(rv, nvec, seg0, g, stage_buf);
+  if (seg0 + kVecs <= nvec) greedy_segment_pass<BF16, true, NB>(rv, nvec, seg0, g, stage_buf);
+  else greedy_segment_pass<BF16, false, NB>(rv, nvec, seg0, g, stage_buf);
   g.finish(meta_out, sh);
 }
 
