@@ -488,10 +488,14 @@ def run_ours(args):
         t1, pos1, _ = oracle_sample(w, 1, 1)
         n = int(max(1, min(B, round(cores * 10.0 / max(t1, 1e-3)))))
         threads = min(cores, n)
-        dt, pos, _ = oracle_sample(w, n, threads)
+        # repeat the sample until about 10 s of CPU time have been measured
+        dt, pos, reps = 0.0, 0, 0
+        while reps == 0 or (dt < 10.0 and reps < 64):
+            d1, p1, _ = oracle_sample(w, n, threads)
+            dt, pos, reps = dt + d1, pos + p1, reps + 1
         cpu = {"value": pos / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
-               "sample": "first %d of %d requests of this batch, fp64 C oracle, %d threads, %.1f s"
-                         % (n, B, threads, dt)}
+               "sample": "first %d of %d requests of this batch, %d times, fp64 C oracle, %d threads, %.1f s"
+                         % (n, B, reps, threads, dt)}
 
     peaks = measured_peaks()
     if peaks and peaks.get("hbm_gbs"):
