@@ -226,12 +226,11 @@ __device__ __forceinline__ bool wait_conf(const RunParams& p) {
 // STATS item: one segment of one row of request i; the last segment of the
 // task decides.
 //
-// When the confidence head runs in the same launch (prefix order only), the
-// rows of position 0 are read before its budgets are known: their plan
-// follows verify_len alone (Lcap), reading the drafter's row 0 whenever a
-// sampled request may verify a position, and the decision waits for the
-// budgets.  Every later position exists only after a decision, so its plan
-// already has them.
+// When the confidence head runs in the same launch (prefix order), the rows of
+// position 0 are read before its budgets are known: their plan follows
+// verify_len alone (Lcap), reading the drafter's row 0 whenever a sampled
+// request may verify a position, and the decision waits for the budgets.  A
+// later position exists only after a decision, so its plan already has them.
 template <bool BF16>
 __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, StatsShared& st,
                              DecideShared& dec, unsigned* s_base, uint4* stage_buf) {
@@ -242,10 +241,11 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
   bool needed, pass;
   unsigned expected;
   if (early) {
+    // the plan cannot tell yet whether the head leaves a request without
+    // drafter logits any position to verify: its target row is read
     const bool target_only = ri.greedy || ri.no_draft;
     if (ri.invalid_T) needed = (slot == 0 && seg == 0);
-    else if (target_only) needed = !is_draft;
-    else needed = !is_draft || ri.Lcap > 0;
+    else needed = !is_draft || (!target_only && ri.Lcap > 0);
     pass = !ri.invalid_T;
     expected = ri.invalid_T ? 1u
                             : static_cast<unsigned>(((!target_only && ri.Lcap > 0) ? 2 : 1) * p.n_segs);
@@ -262,7 +262,8 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
   const bool whole = seg == kRowSeg;
   if (whole && ri.bad_T) needed = slot == 0;
   if (!needed) return;
-  unsigned weight = 1u;
+  // a whole row arrives for its n_segs segments (a failed request's one item for one)
+  const unsigned weight = (whole && pass) ? static_cast<unsigned>(p.n_segs) : 1u;
   // the drafted token, loaded now (its logit is cached once the segment is in)
   const bool cache_tok = pass && !ri.greedy && j < p.k;
   int xj = -1;
@@ -272,7 +273,6 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     const void* row = is_draft ? draft_row(p, i, j, BF16) : target_row(p, i, j, BF16);
     const float cc = ri.greedy ? 0.0f : static_cast<float>(1.4426950408889634 / static_cast<double>(ri.T));
     if (whole) {
-      weight = static_cast<unsigned>(p.n_segs);
       if (ri.greedy) stats_row_staged<BF16, true>(row, p.V, p.n_segs, cc, p.meta + rec0, nullptr, st, stage_buf);
       else stats_row_staged<BF16, false>(row, p.V, p.n_segs, cc, p.meta + rec0, p.ssum + rec0, st, stage_buf);
     } else if (p.short_segs) {
@@ -295,17 +295,17 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     }
   }
   if (!arrive_last(p.arrive_stats + i, expected, &st.flag, weight)) return;
-  if (p.mode == kModeDense) {
-    decide_request<BF16>(p, i, ri, dec);
-    __syncthreads();
-    if (__ldcg(&p.jobs[i].kind) != kJobNone) enqueue_sample<BF16>(p, i, s_base);
-    else finish_request(p);
-    return;
-  }
   if (early) {
     if (threadIdx.x == 0) st.flag = wait_conf(p) ? 1 : 0;
     __syncthreads();
     if (!st.flag) return;  // the head never finished: the run reports the queue error
+  }
+  if (p.mode == kModeDense) {
+    decide_request<BF16>(p, i, ri, dec);
+    __syncthreads();
+    if (dec.state == 2) enqueue_sample<BF16>(p, i, s_base);
+    else finish_request(p);
+    return;
   }
   const ReqInfo rc = early ? request_info(p, i, true) : ri;
   decide_position<BF16>(p, i, rc, j, dec);

@@ -888,6 +888,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   float* oq = p.out_q ? p.out_q + static_cast<int64_t>(i) * k : nullptr;
   const int32_t* x = p.tokens + static_cast<int64_t>(i) * k;
 
+  if (tid == 0) sh.state = 0;  // 2 once a sample job is written (read by the caller after a barrier)
   write_defaults(p, i);
   if (ri.bad_T) {
     sync_compute();
@@ -1024,6 +1025,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     p.out_acc[i] = n;
     if (p.out_status) p.out_status[i] = 0;
     write_job<BF16>(p, i, n, L, sh.rows[n], n < L ? &sh.rows[k + 1 + n] : nullptr, t, sh.u2[n]);
+    sh.state = 2;
   }
 }
 
