@@ -49,7 +49,7 @@ struct SegGeo {
   static constexpr int kSegVecs = kThreads * kSegVecsPerThread;   // 4096 vectors
   static constexpr int kSeg = kSegVecs * kPerVec;                 // logits per segment
   static constexpr int kBatchElems = kBatchVecs * kPerVec;        // per thread per batch
-  static constexpr int kSumLevels = BF16 ? 5 : 4;                 // pairwise depth of a batch sum
+  static constexpr int kSumLevels = BF16 ? 6 : 5;                 // pairwise depth of a batch sum (8 vectors)
 };
 
 template <bool BF16>
@@ -137,17 +137,44 @@ struct SoftAcc {
   }
 };
 
-// One batch of a thread's logits into its running statistics.  Logits are
-// taken in pairs (the two halves of a bf16x2 word, or two fp32 words) so the
-// exponent arguments, the bound terms and the sums use packed fp32x2
-// instructions; every lane is rounded as the scalar operation would be.  The
-// argument is formed negated, n = K - l c = -(l c - K) (the same rounding,
-// negated), clamped at 1024 so masked (-inf) logits give e = 0 and a finite
-// bound term.  The batch sum is a balanced pairwise tree: across the batch's
-// vectors, then across the pairs of a vector, then the two lanes.
-template <bool BF16>
-__device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatchVecs], float cc) {
-  const float bm = batch_max<BF16>(v);
+// One batch of NV vectors of a thread's logits into its running statistics,
+// given the batch's maximum bm (batch_max_n).  Logits are taken in pairs (the
+// two halves of a bf16x2 word, or two fp32 words) so the exponent arguments,
+// the bound terms and the sums use packed fp32x2 instructions; every lane is
+// rounded as the scalar operation would be.  The argument is formed negated,
+// n = K - l c = -(l c - K) (the same rounding, negated), clamped at 1024 so
+// masked (-inf) logits give e = 0 and a finite bound term.  The batch sum is a
+// balanced pairwise tree: across the batch's vectors, then across the pairs of
+// a vector, then the two lanes (depth log2(NV) + log2(pairs) + 1, at most
+// SegGeo::kSumLevels).
+template <bool BF16, int NV>
+__device__ __forceinline__ float batch_max_n(const uint4 (&v)[NV]) {
+  static_assert(NV == 4 || NV == 8, "batch of 4 or 8 vectors");
+  if constexpr (BF16) {
+    uint32_t m[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) m[u] = hmax2_nan(hmax2_nan(v[u].x, v[u].y), hmax2_nan(v[u].z, v[u].w));
+#pragma unroll
+    for (int w = 1; w < NV; w *= 2)
+#pragma unroll
+      for (int u = 0; u + w < NV; u += 2 * w) m[u] = hmax2_nan(m[u], m[u + w]);
+    return fmax_nan(bf16_lo(m[0]), bf16_hi(m[0]));
+  } else {
+    float m[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u)
+      m[u] = fmax_nan(fmax_nan(__uint_as_float(v[u].x), __uint_as_float(v[u].y)),
+                      fmax_nan(__uint_as_float(v[u].z), __uint_as_float(v[u].w)));
+#pragma unroll
+    for (int w = 1; w < NV; w *= 2)
+#pragma unroll
+      for (int u = 0; u + w < NV; u += 2 * w) m[u] = fmax_nan(m[u], m[u + w]);
+    return m[0];
+  }
+}
+
+template <bool BF16, int NV>
+__device__ __forceinline__ void soft_terms(SoftAcc& acc, const uint4 (&v)[NV], float cc, float bm) {
   acc.mraw = fmax_nan(acc.mraw, bm);
   if (isnan(bm) || bm == INFINITY) acc.bad = 1;
   const float Kb = ceilf(bm * cc);
@@ -157,9 +184,9 @@ __device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatch
   const float2 K2 = make_float2(acc.K, acc.K);
   float2 er2 = make_float2(acc.er, 0.0f);
   constexpr int kPairs = BF16 ? 4 : 2;  // logit pairs per 16-byte vector
-  float2 ps[kBatchVecs][kPairs];
+  float2 ps[NV][kPairs];
 #pragma unroll
-  for (int u = 0; u < kBatchVecs; ++u) {
+  for (int u = 0; u < NV; ++u) {
     const uint32_t wd[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
     for (int q = 0; q < kPairs; ++q) {
@@ -177,11 +204,13 @@ __device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatch
       ps[u][q] = e;
     }
   }
-  // across vectors (kBatchVecs = 4: two levels)
+  // across vectors
 #pragma unroll
-  for (int q = 0; q < kPairs; ++q) {
-    ps[0][q] = fadd2(fadd2(ps[0][q], ps[1][q]), fadd2(ps[2][q], ps[3][q]));
-  }
+  for (int w = 1; w < NV; w *= 2)
+#pragma unroll
+    for (int u = 0; u + w < NV; u += 2 * w)
+#pragma unroll
+      for (int q = 0; q < kPairs; ++q) ps[u][q] = fadd2(ps[u][q], ps[u + w][q]);
   float2 t;
   if constexpr (BF16) {
     t = fadd2(fadd2(ps[0][0], ps[0][1]), fadd2(ps[0][2], ps[0][3]));
@@ -190,6 +219,11 @@ __device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatch
   }
   acc.er = er2.x + er2.y;
   acc.s += static_cast<double>(t.x + t.y);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void soft_batch(SoftAcc& acc, const uint4 (&v)[kBatchVecs], float cc) {
+  soft_terms<BF16, kBatchVecs>(acc, v, cc, batch_max_n<BF16, kBatchVecs>(v));
 }
 
 // Merge `acc` of all threads of the CTA into one record (called by every thread).
@@ -258,15 +292,20 @@ __device__ __forceinline__ void stochastic_segment(const void* row, int64_t V, i
   const int64_t nvec = V / G::kPerVec;
   const int64_t seg0 = static_cast<int64_t>(seg) * G::kSegVecs;
   SoftAcc acc;
-  uint4 va[kBatchVecs], vb[kBatchVecs];
-  load_batch<BF16>(rv, nvec, seg0, 0, va);
-#pragma unroll
-  for (int b = 0; b < kBatches; b += 2) {
-    if (b + 1 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 1, vb);
-    soft_batch<BF16>(acc, va, cc);
-    if (b + 2 < kBatches) load_batch<BF16>(rv, nvec, seg0, b + 2, va);
-    if (b + 1 < kBatches) soft_batch<BF16>(acc, vb, cc);
-  }
+  // batches of two load steps (8 vectors), as in the staged pass, so both
+  // passes round the same sums in the same order
+  static_assert(kBatches == 4, "two batches of two steps");
+  uint4 v[2 * kBatchVecs], w[2 * kBatchVecs];
+  uint4 (&v0)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&v[0]);
+  uint4 (&v1)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&v[kBatchVecs]);
+  uint4 (&w0)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&w[0]);
+  uint4 (&w1)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&w[kBatchVecs]);
+  load_batch<BF16>(rv, nvec, seg0, 0, v0);
+  load_batch<BF16>(rv, nvec, seg0, 1, v1);
+  load_batch<BF16>(rv, nvec, seg0, 2, w0);
+  load_batch<BF16>(rv, nvec, seg0, 3, w1);
+  soft_terms<BF16, 2 * kBatchVecs>(acc, v, cc, batch_max_n<BF16, 2 * kBatchVecs>(v));
+  soft_terms<BF16, 2 * kBatchVecs>(acc, w, cc, batch_max_n<BF16, 2 * kBatchVecs>(w));
   soft_merge_block(acc, sh, meta_out, sum_out);
 }
 
@@ -317,14 +356,32 @@ __device__ __forceinline__ void stochastic_segment_pass(const uint4* rv, int64_t
   Stager sg{stage_buf};
 #pragma unroll
   for (int b = 0; b < kStageSlots && b < NB; ++b) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b);
-  // full segments: unrolled, so slots and wait counts are compile-time constants
+  if constexpr (NB % 2 == 0) {
+    // two staging steps per batch (64 bf16 / 32 fp32 logits a thread): half
+    // the per-batch work (maximum, frame check, fp64 accumulation)
+#pragma unroll (FULL ? NB / 2 : 1)
+    for (int b = 0; b < NB; b += 2) {
+      uint4 v[2 * kBatchVecs];
+      uint4 (&v0)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&v[0]);
+      uint4 (&v1)[kBatchVecs] = *reinterpret_cast<uint4 (*)[kBatchVecs]>(&v[kBatchVecs]);
+      staged_batch<BF16, FULL>(sg, nvec, seg0, b, v0);
+      staged_batch<BF16, FULL>(sg, nvec, seg0, b + 1, v1);
+      const float bm = batch_max_n<BF16, 2 * kBatchVecs>(v);  // every staged value is in registers
+      // refill both steps' slots
+      if (b + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+      if (b + 1 + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + 1 + kStageSlots);
+      soft_terms<BF16, 2 * kBatchVecs>(acc, v, cc, bm);
+    }
+  } else {
+    // full segments: unrolled, so slots and wait counts are compile-time constants
 #pragma unroll (FULL ? NB : 1)
-  for (int b = 0; b < NB; ++b) {
-    uint4 v[kBatchVecs];
-    staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
-    soft_batch<BF16>(acc, v, cc);
-    // refill this step's slot once its values have been used
-    if (b + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+    for (int b = 0; b < NB; ++b) {
+      uint4 v[kBatchVecs];
+      staged_batch<BF16, FULL>(sg, nvec, seg0, b, v);
+      soft_batch<BF16>(acc, v, cc);
+      // refill this step's slot once its values have been used
+      if (b + kStageSlots < NB) stage_segment_batch<FULL>(sg, rv, nvec, seg0, b + kStageSlots);
+    }
   }
 }
 
@@ -505,24 +562,35 @@ __device__ void stats_row_staged(const void* row, int64_t V, int n_segs, float c
     const bool full = (seg + 1) * kBatches <= full_steps;
     SoftAcc acc;
     GreedyScan<BF16> gs;
+    // greedy: one step per batch; stochastic: two (as in the segment pass)
+    constexpr int kSteps = GREEDY ? 1 : 2;
+    static_assert(kBatches % kSteps == 0, "steps per batch divide a segment");
 #pragma unroll 1
-    for (int b = 0; b < kBatches; ++b) {
-      const int g = seg * kBatches + b;
-      cp_async_wait(sg.issued - g - 1);
-      uint4 v[kBatchVecs];
+    for (int b = 0; b < kBatches; b += kSteps) {
+      uint4 v[kSteps * kBatchVecs];
 #pragma unroll
-      for (int u = 0; u < kBatchVecs; ++u) {
-        const int64_t idx = seg0 + static_cast<int64_t>(b * kBatchVecs + u) * kThreads + threadIdx.x;
-        v[u] = (full || idx < nvec) ? *sg.slot(g, u) : neg_inf_vec<BF16>();
+      for (int h = 0; h < kSteps; ++h) {
+        const int g = seg * kBatches + b + h;
+        cp_async_wait(sg.issued - g - 1);
+#pragma unroll
+        for (int u = 0; u < kBatchVecs; ++u) {
+          const int64_t idx = seg0 + static_cast<int64_t>((b + h) * kBatchVecs + u) * kThreads + threadIdx.x;
+          v[h * kBatchVecs + u] = (full || idx < nvec) ? *sg.slot(g, u) : neg_inf_vec<BF16>();
+        }
       }
+      float bm = 0.0f;
       if constexpr (GREEDY) gs.scan(v, seg0, b);
-      else soft_batch<BF16>(acc, v, cc);
-      // refill this step's slot once its values have been used
-      const int gn = g + kStageSlots;
-      if (gn < n_steps) {
-        if (gn < full_steps) stage_row_step<true>(sg, rv, nvec, gn);
-        else stage_row_step<false>(sg, rv, nvec, gn);
+      else bm = batch_max_n<BF16, kSteps * kBatchVecs>(v);  // every staged value is in registers
+      // refill the steps' slots once their values are in registers
+#pragma unroll
+      for (int h = 0; h < kSteps; ++h) {
+        const int gn = seg * kBatches + b + h + kStageSlots;
+        if (gn < n_steps) {
+          if (gn < full_steps) stage_row_step<true>(sg, rv, nvec, gn);
+          else stage_row_step<false>(sg, rv, nvec, gn);
+        }
       }
+      if constexpr (!GREEDY) soft_terms<BF16, kSteps * kBatchVecs>(acc, v, cc, bm);
     }
     if constexpr (GREEDY) gs.finish(meta + seg, sh);
     else soft_merge_block(acc, sh, meta + seg, ssum + seg);
