@@ -45,6 +45,10 @@ constexpr uint32_t kItemExit = 0xFFFFFFFFu;
 constexpr int kRowSeg = 0xFF;  // segment field of a STATS item that covers its whole row
 constexpr unsigned kSpinLimit = 1u << 24;  // polls of a queue slot before giving up (seconds)
 constexpr int kEngineMinBlocks = 4;  // 64 registers: four CTAs per SM (measured best)
+// Small, latency-bound batches run an instance with three CTAs per SM (80
+// registers, fewer spills on the serial decision paths; measured faster there,
+// slower for large batches).
+constexpr int kEngineMinBlocksSmall = 3;
 // candidate keys of the batch-wide selection held in the staging buffer
 constexpr int kConfKeysInStage = 4096;
 static_assert(kMaxK * sizeof(double) + sizeof(ConfSelectShared) + kConfKeysInStage * sizeof(unsigned long long) <=
@@ -366,8 +370,8 @@ __device__ void engine_refine(const RunParams& p, int slot, int sub, RefineShare
   finish_request(p);
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(kThreads, kEngineMinBlocks) k_engine(RunParams p) {
+template <bool BF16, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB) k_engine(RunParams p) {
   extern __shared__ __align__(16) uint4 stage_buf[];  // kStageBytes, per-thread staging
   __shared__ StatsShared st;
   __shared__ DecideShared dec;

@@ -139,7 +139,8 @@ struct spec_verify_ctx {
   unsigned long long* q_slots = nullptr;
   unsigned q_capacity = 0;
   unsigned* q_ctl = nullptr;
-  int engine_grid = 0;
+  int engine_grid = 0;        // CTAs of the k_engine instance for large batches
+  int engine_grid_small = 0;  // ... and of the one for small dense batches
   int mode = SPEC_MODE_AUTO;  // as set by spec_verify_set_mode
   unsigned run_id = 0;
 
@@ -458,8 +459,16 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   if (n_init > 0xFFFF0000ull) return SPEC_ERR_INVALID_ARG;
   p.n_init = static_cast<unsigned>(n_init);
   timing_mark(c, kClassStats, true, s);
-  if (bf16) sv::k_engine<true><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
-  else sv::k_engine<false><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
+  // a small dense batch (every item in the first wave) is latency bound:
+  // the instance with more registers per thread
+  const bool small = p.mode == sv::kModeDense && !p.whole_rows;
+  if (small) {
+    if (bf16) sv::k_engine<true, sv::kEngineMinBlocksSmall><<<c->engine_grid_small, sv::kThreads, sv::kStageBytes, s>>>(p);
+    else sv::k_engine<false, sv::kEngineMinBlocksSmall><<<c->engine_grid_small, sv::kThreads, sv::kStageBytes, s>>>(p);
+  } else {
+    if (bf16) sv::k_engine<true, sv::kEngineMinBlocks><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
+    else sv::k_engine<false, sv::kEngineMinBlocks><<<c->engine_grid, sv::kThreads, sv::kStageBytes, s>>>(p);
+  }
   timing_mark(c, kClassStats, false, s);
   if (cudaGetLastError() != cudaSuccess) return SPEC_ERR_CUDA;
   return SPEC_OK;
@@ -625,20 +634,26 @@ spec_status spec_verify_init(spec_verify_ctx** out, int device, int max_batch, i
     delete c;
     return st;
   }
-  int occ_a = 0, occ_b = 0;
-  if (cudaFuncSetAttribute(sv::k_engine<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
-      cudaFuncSetAttribute(sv::k_engine<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, sv::k_engine<true>, sv::kThreads,
-                                                    sv::kStageBytes) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, sv::k_engine<false>, sv::kThreads,
-                                                    sv::kStageBytes) != cudaSuccess) {
+  // one grid per instance: as many CTAs as are resident at once
+  auto grid_of = [&](auto kb, auto kf, int* grid) {
+    int occ_a = 0, occ_b = 0;
+    if (cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(sv::kStageBytes)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_a, kb, sv::kThreads, sv::kStageBytes) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ_b, kf, sv::kThreads, sv::kStageBytes) != cudaSuccess)
+      return false;
+    *grid = c->num_sms * std::max(1, std::min(occ_a, occ_b));
+    return true;
+  };
+  if (!grid_of(sv::k_engine<true, sv::kEngineMinBlocks>, sv::k_engine<false, sv::kEngineMinBlocks>, &c->engine_grid) ||
+      !grid_of(sv::k_engine<true, sv::kEngineMinBlocksSmall>, sv::k_engine<false, sv::kEngineMinBlocksSmall>,
+               &c->engine_grid_small)) {
     cudaFree(c->ws);
     delete c;
     return SPEC_ERR_CUDA;
   }
-  c->engine_grid = c->num_sms * std::max(1, std::min(occ_a, occ_b));
   *out = c;
   return SPEC_OK;
 }
