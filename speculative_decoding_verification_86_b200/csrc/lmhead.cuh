@@ -21,10 +21,14 @@
 //              MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
 //              M = 128 (256 for a pair, issued by rank 0), N = 256, K = 16 per
 //              instruction, one thread;
-//   warps 2-5  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31, so each
-//              thread owns one row of the tile and walks its 256 columns in
-//              batches of 16 (tcgen05.ld 32x32b.x16), while the MMA warp fills
-//              the other accumulator.
+//   warps 2-9  epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 and one
+//              half of the tile's columns (warps 2-5 the first 128, warps 6-9
+//              the last 128), so two threads share each row of the tile; each
+//              walks its 128 columns in batches of 16 (tcgen05.ld
+//              32x32b.x16) while the MMA warp fills the other accumulator.  At
+//              the end of a work unit the two halves' statistics are merged
+//              through shared memory (the merge k_lm_combine applies across
+//              parts) and one record per row is written.
 // Every wait on an mbarrier is bounded in time; a wait that runs out raises
 // the CTA's abort flag and the error word, drains what this CTA issued, frees
 // TMEM and returns.
@@ -41,7 +45,9 @@ constexpr int kLmBN = 256;  // vocabulary columns per tile (UMMA N)
 constexpr int kLmBK = 64;   // hidden elements per stage: one 128-byte swizzle row of bf16
 constexpr int kLmUK = 16;   // K of one kind::f16 instruction
 constexpr uint32_t kLmABytes = kLmBM * kLmBK * 2;  // 16 KB: this CTA's 128 rows
-constexpr int kLmThreads = 192;
+constexpr int kLmEpiWarps = 8;                   // two per TMEM lane quarter
+constexpr int kLmHalfN = kLmBN / 2;              // columns of a tile per epilogue warp
+constexpr int kLmThreads = 32 * (2 + kLmEpiWarps);
 constexpr uint32_t kLmTmemCols = 2 * kLmBN;
 // A work unit covers `part_tiles` N tiles (a power of two up to kLmSegTiles);
 // the statistics records of a unit ("parts") then tile the fp32 statistics
@@ -49,6 +55,17 @@ constexpr uint32_t kLmTmemCols = 2 * kLmBN;
 constexpr int kLmSegTiles = SegGeo<false>::kSeg / kLmBN;  // 64 tiles per statistics segment
 static_assert(SegGeo<false>::kSeg % kLmBN == 0, "tiles divide the fp32 statistics segment");
 constexpr size_t kLmBarrierBytes = 256;
+
+// One row's statistics over the columns of one epilogue warp, handed to the
+// warp holding the other half of the row (shared memory, one per TMEM lane).
+struct LmXchg {
+  double s;
+  float K, mraw, er, om;
+  float best;
+  int best_idx;
+  int bad, gbad;
+};
+constexpr size_t kLmXchgBytes = sizeof(LmXchg) * kLmBM;
 
 // Geometry of the kernel with CG CTAs per MMA (1, or 2 for a CTA pair running
 // tcgen05.mma.cta_group::2 on a 256 x 256 tile: each CTA holds its 128 rows of
@@ -61,7 +78,7 @@ struct LmGeo {
   static constexpr uint32_t kStageBytes = kLmABytes + kBBytes;  // 48 KB or 32 KB
   static constexpr int kStages = CG == 1 ? 4 : 6;
   static constexpr uint32_t kTxBytes = kStageBytes * CG;       // bytes the MMA CTA waits for
-  static constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kLmBarrierBytes;
+  static constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kLmBarrierBytes + kLmXchgBytes;
 };
 constexpr int kLmMaxStages = 6;
 constexpr unsigned long long kLmWaitNs = 2000000000ull;  // 2 s: legitimate waits are microseconds
@@ -297,6 +314,8 @@ struct LmShared {
   uint64_t empty[kLmMaxStages];
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t xfull[4];   // per lane quarter: the second half's statistics are in LmXchg
+  uint64_t xempty[4];  // per lane quarter: the first half has read them
   uint64_t drain;
   uint32_t tmem;
   int abort;
@@ -380,12 +399,17 @@ __device__ __forceinline__ void lm_consume_stats(const LmParams& p, LmRowState& 
     return;
   }
   uint4 v[kBatchVecs];
+  if (nvalid >= 16) {  // every batch but the vocabulary's ragged end
 #pragma unroll
-  for (int u = 0; u < kBatchVecs; ++u) {
-    uint32_t w[4];
+    for (int u = 0; u < kBatchVecs; ++u) v[u] = make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+  } else {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) w[e] = (4 * u + e) < nvalid ? r[4 * u + e] : 0xff800000u;
-    v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int u = 0; u < kBatchVecs; ++u) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) w[e] = (4 * u + e) < nvalid ? r[4 * u + e] : 0xff800000u;
+      v[u] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
   }
   soft_batch<false>(st.acc, v, st.cc);
 }
@@ -526,15 +550,60 @@ __device__ __forceinline__ void lm_mma(const LmParams& p, const LmWork<CG>& w, L
   }
 }
 
+// Fold the other column half's statistics of the same row into `st`: the
+// greedy maximum with the lowest column among equal values, and the stochastic
+// sums rebased to the larger frame and added -- the merge k_lm_combine applies
+// across parts, so the record is what two separate part records would combine to.
+__device__ __forceinline__ void lm_merge_half(LmRowState& st, const LmXchg& o) {
+  if (st.greedy) {
+    st.gbad |= o.gbad;
+    if (o.best_idx != INT_MAX &&
+        (st.best_idx == INT_MAX || o.best > st.best || (o.best == st.best && o.best_idx < st.best_idx))) {
+      st.best = o.best;
+      st.best_idx = o.best_idx;
+    }
+    return;
+  }
+  SoftAcc& a = st.acc;
+  const float K = fmaxf(a.K, o.K);
+  const int bad = a.bad | o.bad;
+  double s = 0.0;
+  float er = 0.0f, om = 0.0f;
+  if (!bad && K > -INFINITY) {
+    if (a.K > -INFINITY) {
+      const double f = pow2_exact(a.K - K);
+      const float ff = static_cast<float>(f);
+      s += a.s * f;
+      er += a.er * ff;
+      om += (a.om + (K - a.K) * static_cast<float>(a.s)) * ff;
+    }
+    if (o.K > -INFINITY) {
+      const double f = pow2_exact(o.K - K);
+      const float ff = static_cast<float>(f);
+      s += o.s * f;
+      er += o.er * ff;
+      om += (o.om + (K - o.K) * static_cast<float>(o.s)) * ff;
+    }
+  }
+  a.K = K;
+  a.mraw = fmax_nan(a.mraw, o.mraw);
+  a.bad = bad;
+  a.s = s;
+  a.er = er;
+  a.om = om;
+}
+
 template <int CG>
 __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>& w, LmShared& sh,
-                                            uint32_t rank) {
+                                            LmXchg* xchg, uint32_t rank) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quarter = warp & 3;  // TMEM lanes this warp may read
+  const int quarter = warp & 3;       // TMEM lanes this warp may read
+  const int half = (warp - 2) >> 2;   // columns [half * 128, half * 128 + 128) of every tile
   const int r_in_unit = static_cast<int>(rank) * kLmBM + quarter * 32 + lane;
   constexpr int R = LmGeo<CG>::kRowsPerUnit;
-  uint32_t t = 0;
-  for (int u = w.first; u < w.units; u += w.stride) {
+  LmXchg& xc = xchg[quarter * 32 + lane];
+  uint32_t t = 0, n_unit = 0;
+  for (int u = w.first; u < w.units; u += w.stride, ++n_unit) {
     const int mt = w.mt(u);
     LmRowState st;
     int64_t dst = -1;
@@ -561,7 +630,7 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
       tc_fence_after();
       const uint32_t taddr = sh.tmem + (static_cast<uint32_t>(quarter * 32) << 16) + a * kLmBN;
 #pragma unroll 1
-      for (int c = 0; c < kLmBN; c += 32) {
+      for (int c = half * kLmHalfN; c < (half + 1) * kLmHalfN; c += 32) {
         uint32_t v0[16], v1[16];
         tmem_ld16(taddr + c, v0);
         tmem_ld16(taddr + c + 16, v1);
@@ -591,8 +660,33 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
         else mbar_arrive_cluster(peer_addr(&sh.tempty[a], 0));  // the MMA CTA's barrier
       }
     }
-    if (p.mode == kLmModeStats && st.valid)
-      lm_write_part(p, st, mt, w.mt0, R, r_in_unit, w.part(u));
+    if (p.mode != kLmModeStats) continue;
+    // The second half hands its statistics over (once the first half has read
+    // the previous unit's); the first half merges them and writes the record.
+    const uint32_t par = n_unit & 1u;
+    if (half == 1) {
+      const bool free = mbar_wait(&sh.xempty[quarter], par ^ 1u, &sh.abort, p.error);
+      if (!__all_sync(0xffffffffu, free)) return;
+      xc.s = st.acc.s;
+      xc.K = st.acc.K;
+      xc.mraw = st.acc.mraw;
+      xc.er = st.acc.er;
+      xc.om = st.acc.om;
+      xc.bad = st.acc.bad;
+      xc.best = st.best;
+      xc.best_idx = st.best_idx;
+      xc.gbad = st.gbad;
+      mbar_arrive(&sh.xfull[quarter]);
+    } else {
+      const bool full = mbar_wait(&sh.xfull[quarter], par, &sh.abort, p.error);
+      if (!__all_sync(0xffffffffu, full)) return;
+      const LmXchg o = xc;
+      mbar_arrive(&sh.xempty[quarter]);
+      if (st.valid) {
+        lm_merge_half(st, o);
+        lm_write_part(p, st, mt, w.mt0, R, r_in_unit, w.part(u));
+      }
+    }
   }
 }
 
@@ -607,6 +701,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   const uint32_t pad = (1024u - (smem_addr(lm_smem) & 1023u)) & 1023u;
   uint8_t* stages = lm_smem + pad;  // 1024-byte aligned: the swizzle atoms of every stage
   LmShared& sh = *reinterpret_cast<LmShared*>(stages + G::kStages * G::kStageBytes);
+  LmXchg* xchg = reinterpret_cast<LmXchg*>(stages + G::kStages * G::kStageBytes + kLmBarrierBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = CG == 1 ? 0u : cluster_rank();
   if (threadIdx.x == 0) {
@@ -616,7 +711,11 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sh.tfull[a], 1);
-      mbar_init(&sh.tempty[a], 4 * CG);  // one arrival per epilogue warp of the group
+      mbar_init(&sh.tempty[a], kLmEpiWarps * CG);  // one arrival per epilogue warp of the group
+    }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&sh.xfull[q], 32);
+      mbar_init(&sh.xempty[q], 32);
     }
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
@@ -655,7 +754,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) lm_mma<CG>(p, w, sh, stages);
   } else {
-    lm_epilogue<CG>(p, w, sh, rank);
+    lm_epilogue<CG>(p, w, sh, xchg, rank);
   }
   tc_fence_before();
   if constexpr (CG == 1) __syncthreads();
