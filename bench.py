@@ -71,6 +71,9 @@ def parse_args():
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every step (cold L2) and report the "
                          "kernel time of each launch")
+    ap.add_argument("--lm-cta-pairs", type=int, default=2, choices=[0, 1, 2],
+                    help="lmhead: GEMM tile form (0 one CTA per tile, 1 CTA pairs for both "
+                         "GEMMs, 2 CTA pairs for the row-writing GEMM only)")
     ap.add_argument("--vocab-shards", type=int, default=1,
                     help="N > 1: time the vocabulary-parallel protocol with N ranks emulated "
                          "on this one GPU (one rank per context, exchanges as copies)")
@@ -706,7 +709,7 @@ def run_lmhead(args):
     k = kp1 - 1
     V = head.shape[0]
     ver = binding.SpecVerifier(dev, max_batch=B, max_k=k, max_vocab=V, mode="dense")
-    lm = binding.LmHeadVerifier(ver, max_hidden=H)
+    lm = binding.LmHeadVerifier(ver, max_hidden=H, cta_pairs=args.lm_cta_pairs)
     positions = B * k
     out = ver._outputs(B, k, True)
     stream = torch.cuda.current_stream(dev)
@@ -826,13 +829,14 @@ def run_lmhead(args):
         "metric": LM_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": lm_config(w, world),
+        "config": dict(lm_config(w, world), cta_pairs=args.lm_cta_pairs),
         "roofline": {"bound": "tensor", "kernel": "k_lmhead (statistics epilogue)",
                      "achieved": achieved, "peak": peak, "peak_source": peak_src,
                      "unit": "TFLOP/s", "frac": achieved / peak,
                      "frac_of_sustained": (achieved / float(peaks["bf16_tflops_sustained"])
                                            if peaks and peaks.get("bf16_tflops_sustained") else None),
-                     "traffic": profiled_traffic("k_lmhead", "lmhead_stats"),
+                     "traffic": profiled_traffic("k_lmhead", "lmhead_stats_pairs" if args.lm_cta_pairs == 1
+                                                  else "lmhead_stats"),
                      "flops_per_launch": flops, "launch_ms": st_ms, "launches_timed": n_st},
         "rows_gemm_ms": ms_rw / max(n_rw, 1),
         "unfused_ms_per_step": unfused_ms,
