@@ -68,6 +68,9 @@ def parse_args():
                     help="skip timing the oracle beside the GPU run")
     ap.add_argument("--mode", default="prefix", choices=["prefix", "dense", "auto"],
                     help="order of the statistics passes in the verification kernel")
+    ap.add_argument("--prefix-tail", type=int, default=None,
+                    help="prefix order: read a request's remaining positions together from "
+                         "this position on (1..17; default: the library's)")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 512 MB buffer before every step (cold L2) and report the "
                          "kernel time of each launch")
@@ -381,6 +384,8 @@ def run_ours(args):
     B, kp1, V = w["target"].shape
     k = kp1 - 1
     ver = binding.SpecVerifier(dev, max_batch=max(B, 1), max_k=max(k, 1), max_vocab=V, mode=args.mode)
+    if args.prefix_tail is not None:
+        ver.set_prefix_tail(args.prefix_tail)
     L = effective_lengths(w, ver)
     positions = int(L.sum().item())
     step_bytes = dense_row_bytes(w, L)
@@ -534,6 +539,7 @@ def run_ours(args):
         "fp64_paths": counters,
         "conf_launch_ms": (ms_conf / n_conf) if n_conf else None,
         "mode": args.mode,
+        "prefix_tail": args.prefix_tail,
         "other_mode": other_line,
     }
     if rank == 0:
@@ -829,8 +835,9 @@ def run_lmhead(args):
                      "traffic": profiled_traffic("k_lmhead", "lmhead_stats_pairs" if args.lm_cta_pairs == 1
                                                   else "lmhead_stats"),
                      "flops_per_launch": flops, "launch_ms": st_ms, "launches_timed": n_st},
-        "timed_blocks": {"n": len(block_ms), "steps_each": args.steps,
-                         "ms_per_block_min": min(block_ms), "ms_per_block_median": statistics.median(block_ms)},
+        "timed_blocks": {"blocks": len(block_ms), "steps_per_block": args.steps,
+                         "ms_per_block_min": min(block_ms), "ms_per_block_median": statistics.median(block_ms),
+                         "ms_per_block_max": max(block_ms)},
         "rows_gemm_ms": ms_rw / max(n_rw, 1),
         "unfused_ms_per_step": unfused_ms,
         "unfused_value": positions * world / (unfused_ms / 1e3),

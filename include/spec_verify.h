@@ -75,7 +75,9 @@ typedef enum { SPEC_F32 = 0, SPEC_BF16 = 1 } spec_dtype;
  * same outputs, bit for bit:
  *   SPEC_MODE_PREFIX: position j+1's rows are read only once position j was
  *     accepted (the block ends at its first rejected position), so rows past
- *     the first rejection are never touched;
+ *     the first rejection are never touched -- up to the dense tail
+ *     (spec_verify_set_prefix_tail): from that position on, a request's
+ *     remaining rows are read together;
  *   SPEC_MODE_DENSE: every verified position's target and draft rows are
  *     reduced, then the chain is walked;
  *   SPEC_MODE_AUTO (default): dense when the B * (2k + 1) rows, cut into
@@ -125,6 +127,20 @@ spec_status spec_verify_destroy(spec_verify_ctx* ctx);
 
 /* Select the statistics order for later runs on this context (spec_mode). */
 spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode);
+
+/* Prefix order's dense tail, for later runs on this context: once a request
+ * has accepted positions 0 .. position-1, the rows of all its remaining
+ * positions (target rows position..L, draft rows position..L-1) are read at
+ * once and its chain is walked from there, as in the dense order.  A request
+ * that accepts many positions then waits on fewer dependent statistics passes;
+ * the price is reading the rows of that tail past its first rejection.  The
+ * outputs do not depend on it.  `position` in [1, 17]; a value above the run's
+ * k reads every position separately; 0 (the default) chooses per run: 2 when
+ * the batch's rows (2k + 1 per request, k + 1 without draft logits), cut into
+ * segments of 32768 bf16 or 16384 fp32 logits, make at most 16 waves of the
+ * kernel's grid, else no tail.  SPEC_ERR_INVALID_ARG for a NULL context or a
+ * position outside [0, 17]. */
+spec_status spec_verify_set_prefix_tail(spec_verify_ctx* ctx, int position);
 
 /* Stochastic/mixed verification of B requests.
  *   target_logits [B, k+1, V]: row j scores drafted position j; row k is the bonus row.

@@ -104,6 +104,7 @@ def lib():
                                      ctypes.POINTER(ConfArgs), _i32, _i32, _i64, _u64, _u32, _u32,
                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp]
     L.spec_verify_set_mode.argtypes = [_vp, _i32]
+    L.spec_verify_set_prefix_tail.argtypes = [_vp, _i32]
     L.spec_verify_draws.argtypes = [_vp, _u64, _u32, _u32, _i32, _i32, _vp, _vp]
     L.spec_verify_timing_enable.argtypes = [_vp, _i32]
     L.spec_verify_timing_read.argtypes = [_vp, _i32, ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double)]
@@ -120,7 +121,7 @@ def lib():
                  "spec_shard_refine_finish",
                  "spec_lmhead_init", "spec_lmhead_destroy", "spec_lmhead_errors",
                  "spec_lmhead_logits", "spec_lmhead_verify", "spec_lmhead_set_cta_pairs",
-                 "spec_verify_set_mode", "spec_verify_draws",
+                 "spec_verify_set_mode", "spec_verify_set_prefix_tail", "spec_verify_draws",
                  "spec_verify_timing_enable", "spec_verify_timing_read",
                  "spec_verify_last_counters", "spec_verify_selfcheck_ex2"):
         getattr(L, name).restype = _i32
@@ -201,6 +202,13 @@ class SpecVerifier:
         position's rows)."""
         _check(lib().spec_verify_set_mode(self._h, MODES[mode]), "spec_verify_set_mode")
         self.mode = mode
+
+    def set_prefix_tail(self, position):
+        """Prefix order: read all remaining positions of a request at once
+        after it accepted positions 0 .. position-1 (1..17; above k: one
+        position at a time; 0, the default: chosen per run from the batch's
+        size against the grid).  The outputs do not depend on it."""
+        _check(lib().spec_verify_set_prefix_tail(self._h, int(position)), "spec_verify_set_prefix_tail")
 
     # -- lifecycle ------------------------------------------------------------
     def close(self):

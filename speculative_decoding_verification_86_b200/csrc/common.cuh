@@ -206,6 +206,8 @@ struct RunParams {
   // engine
   int mode;                        // kModeDense / kModePrefix
   int whole_rows;                  // dense order: a statistics item is a whole row (else a segment)
+  int tail_from;                   // prefix order: positions >= this (>= 1) are read together, once
+                                   // the position before it accepted (k + 1: one at a time)
   int sample_parts;                // a sample item is one part of a chunk (small batches), else a chunk
   int short_segs;                  // statistics segments of one batch step (small dense batches)
   int seg_len;                     // logits per statistics segment

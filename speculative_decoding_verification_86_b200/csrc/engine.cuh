@@ -88,6 +88,11 @@ __device__ __forceinline__ void st_release_u64(unsigned long long* a, unsigned l
 __device__ __forceinline__ int task_rows(const ReqInfo& ri, int j) {
   return (!ri.greedy && j < ri.L) ? 2 : 1;
 }
+// Rows of the prefix order's dense tail from position d <= L: target rows
+// d..L and, for a sampled request, draft rows d..L-1.
+__device__ __forceinline__ int tail_rows(const ReqInfo& ri, int d) {
+  return ri.greedy ? ri.L - d + 1 : 2 * (ri.L - d) + 1;
+}
 
 // The implicit item of ticket h < n_init.
 __device__ __forceinline__ uint32_t implicit_item(const RunParams& p, unsigned h) {
@@ -260,6 +265,7 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     pass = !ri.bad_T;
     if (ri.bad_T) expected = 1u;
     else if (p.mode == kModeDense) expected = static_cast<unsigned>(stats_expected(ri, p.n_segs));
+    else if (j >= p.tail_from) expected = static_cast<unsigned>(tail_rows(ri, p.tail_from) * p.n_segs);
     else expected = static_cast<unsigned>(task_rows(ri, j) * p.n_segs);
   }
   // a whole-row item (dense order) stands for all of the row's segment items
@@ -304,8 +310,8 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
     __syncthreads();
     if (!st.flag) return;  // the head never finished: the run reports the queue error
   }
-  if (p.mode == kModeDense) {
-    decide_request<BF16>(p, i, ri, dec);
+  if (p.mode == kModeDense || j >= p.tail_from) {
+    decide_request<BF16>(p, i, ri, dec, p.mode == kModeDense ? 0 : p.tail_from);
     __syncthreads();
     if (dec.state == 2) enqueue_sample<BF16>(p, i, s_base);
     else finish_request(p);
@@ -316,11 +322,20 @@ __device__ void engine_stats(const RunParams& p, int i, int slot, int seg, Stats
   const int next = dec.state;
   if (next == 1) {
     const int jn = j + 1;
-    const int rows = task_rows(rc, jn);
     const int ns = p.n_segs;
-    enqueue(p, kClassStats, rows * ns, [&](int q) {
-      return item_stats(i, (q / ns) == 0 ? jn : p.k + 1 + jn, q % ns);
-    }, s_base);
+    if (jn >= p.tail_from) {
+      // the rest of the request at once: target rows jn..L, then draft rows jn..L-1
+      const int nt = rc.L - jn + 1;
+      enqueue(p, kClassStats, tail_rows(rc, jn) * ns, [&](int q) {
+        const int r = q / ns;
+        return item_stats(i, r < nt ? jn + r : p.k + 1 + jn + (r - nt), q % ns);
+      }, s_base);
+    } else {
+      const int rows = task_rows(rc, jn);
+      enqueue(p, kClassStats, rows * ns, [&](int q) {
+        return item_stats(i, (q / ns) == 0 ? jn : p.k + 1 + jn, q % ns);
+      }, s_base);
+    }
   } else if (next == 2) {
     enqueue_sample<BF16>(p, i, s_base);
   } else {

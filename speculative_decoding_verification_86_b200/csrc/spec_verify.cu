@@ -37,6 +37,9 @@ constexpr float kEpsEx2 = 1.5e-7f;
 constexpr int kClassStats = 0, kClassLmStats = 1, kClassLmRows = 2, kClassConf = 3;
 constexpr int kTimingClasses = 4;
 constexpr int kMaxTimed = 4096;
+// Automatic prefix tail: batches whose row segments make at most this many
+// waves of the engine's grid read their requests' later positions together.
+constexpr int64_t kTailWaves = 16;
 
 struct DeviceGuard {
   int prev = -1;
@@ -142,6 +145,7 @@ struct spec_verify_ctx {
   int engine_grid = 0;        // CTAs of the k_engine instance for large batches
   int engine_grid_small = 0;  // ... and of the one for small dense batches
   int mode = SPEC_MODE_AUTO;  // as set by spec_verify_set_mode
+  int tail_from = 0;          // as set by spec_verify_set_prefix_tail (0: automatic)
   unsigned run_id = 0;
 
   unsigned timing_mask = 0;  // bit c set: bracket launches of class c with events
@@ -383,6 +387,18 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
     mode = static_cast<int64_t>(B) * (2 * k + 1) * n_segs <= c->engine_grid ? SPEC_MODE_DENSE
                                                                            : SPEC_MODE_PREFIX;
   p.mode = (force_greedy || mode == SPEC_MODE_PREFIX) ? sv::kModePrefix : sv::kModeDense;
+  {
+    // Prefix order's dense tail.  Automatic: from position 2 when the batch's
+    // rows, in segments, make at most kTailWaves waves of the grid (the grid
+    // then idles while long chains walk their positions one at a time), else
+    // none (every extra row read competes with other requests' rows).
+    int tail = c->tail_from;
+    if (tail == 0) {
+      const int64_t rows = static_cast<int64_t>(B) * (p.draft ? 2 * k + 1 : k + 1);
+      tail = rows * n_segs <= kTailWaves * static_cast<int64_t>(c->engine_grid) ? 2 : k + 1;
+    }
+    p.tail_from = std::min(tail, k + 1);
+  }
   // Dense order: a statistics item is a whole row when the batch has at least
   // as many rows as the grid has CTAs (one staging pipeline per row, no drain
   // between its segments), else a segment (small batches: every segment of
@@ -932,6 +948,12 @@ spec_status spec_verify_set_mode(spec_verify_ctx* ctx, int mode) {
   if (!ctx || (mode != SPEC_MODE_DENSE && mode != SPEC_MODE_PREFIX && mode != SPEC_MODE_AUTO))
     return SPEC_ERR_INVALID_ARG;
   ctx->mode = mode;
+  return SPEC_OK;
+}
+
+spec_status spec_verify_set_prefix_tail(spec_verify_ctx* ctx, int position) {
+  if (!ctx || position < 0 || position > sv::kMaxK + 1) return SPEC_ERR_INVALID_ARG;
+  ctx->tail_from = position;
   return SPEC_OK;
 }
 

@@ -944,11 +944,14 @@ __device__ __forceinline__ void fail_request(const RunParams& p, int i, uint32_t
   p.jobs[i].kind = kJobNone;
 }
 
-// Resolve request i after all its rows' statistics are in (dense order: every
-// verified position's rows were read).  Leaves p.jobs[i] describing the sample
+// Resolve request i from position j0 on, once the statistics of its rows from
+// j0 on are in (dense order: j0 = 0, every verified position's rows were read;
+// the prefix order's dense tail: positions before j0 were accepted one at a
+// time and their outputs are written).  Leaves p.jobs[i] describing the sample
 // still to draw (kind kJobNone when the request is finished).
 template <bool BF16>
-__device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, DecideShared& sh) {
+__device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, DecideShared& sh,
+                               int j0 = 0) {
   const int tid = threadIdx.x, warp = tid >> 5;
   const int k = p.k, L = ri.L;
   int32_t* tok = p.out_tok + static_cast<int64_t>(i) * (k + 1);
@@ -957,17 +960,18 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   const int32_t* x = p.tokens + static_cast<int64_t>(i) * k;
 
   if (tid == 0) sh.state = 0;  // 2 once a sample job is written (read by the caller after a barrier)
-  write_defaults(p, i);
+  if (j0 == 0) write_defaults(p, i);
   if (ri.bad_T) {
     sync_compute();
     if (tid == 0) fail_request(p, i, kDevBadTemperature);
     return;
   }
 
-  // Merge the rows the chain can read: target rows 0..L, draft rows 0..L-1.
+  // Merge the rows the chain can read: target rows j0..L, draft rows j0..L-1.
   // A warp merging two rows loads both rows' records first.
-  const int nrows = ri.greedy ? L + 1 : 2 * L + 1;
-  auto slot_of = [&](int r) { return r <= L ? r : (k + 1) + (r - (L + 1)); };
+  const int span = L - j0;
+  const int nrows = ri.greedy ? span + 1 : 2 * span + 1;
+  auto slot_of = [&](int r) { return r <= span ? j0 + r : (k + 1) + j0 + (r - (span + 1)); };
   if (ri.greedy) {
     for (int r = warp; r < nrows; r += kWarps) merge_greedy_row(p, i, slot_of(r), sh.rows[slot_of(r)]);
   } else {
@@ -986,7 +990,7 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     if (tid == 0) {
       uint32_t status = 0;
       int n = L;
-      for (int j = 0; j < L; ++j) {
+      for (int j = j0; j < L; ++j) {
         const int xj = __ldg(x + j);
         if (xj < 0 || static_cast<int64_t>(xj) >= p.V) { status = kDevBadToken; break; }
         if (sh.rows[j].bad) { status = kDevNonfinite; break; }
@@ -1016,8 +1020,8 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
   // order until the first rejection, the whole block settling a test inside
   // its bound in fp64 before the walk goes on.
   const TempConsts t = temp_consts<BF16>(p, ri.T);
-  if (tid < L) {
-    const int j = tid;
+  if (tid < span) {
+    const int j = j0 + tid;
     const float* cache = p.tok_logits ? p.tok_logits : p.tok_cache;
     const int64_t tl = (static_cast<int64_t>(i) * k + j) * 2;
     float2 l = make_float2(0.0f, 0.0f);
@@ -1038,18 +1042,19 @@ __device__ void decide_request(const RunParams& p, int i, const ReqInfo& ri, Dec
     sh.dec[j] = d;
     sh.pa[j] = pa;
     sh.qb[j] = qb;
-  } else if (tid >= 32 && tid - 32 <= L) {
-    sh.u2[tid - 32] = draw(p, i, tid - 32, 1);  // the sample's draw, wherever the chain ends
+  } else if (tid >= 32 && tid - 32 <= span) {
+    const int j = j0 + tid - 32;
+    sh.u2[j] = draw(p, i, j, 1);  // the sample's draw, wherever the chain ends
   }
   sync_compute();
   int n = L;
   uint32_t status = 0;
-  for (int j = 0; j < L; ++j) {
+  for (int j = j0; j < L; ++j) {
     if (sh.dec[j] == -1) {
       if (p.fallback) {
         // the fp64 row sums need every rank's logits: the request is redone whole
         if (tid == 0) {
-          for (int jj = 0; jj <= j; ++jj) {
+          for (int jj = j0; jj <= j; ++jj) {
             if (op) op[jj] = static_cast<float>(sh.pa[jj]);
             if (oq) oq[jj] = static_cast<float>(sh.qb[jj]);
           }
