@@ -755,16 +755,12 @@ def run_lmhead(args):
     hall = torch.cat([ht.reshape(-1, H), hd.reshape(-1, H)]).contiguous()
 
     def timed(fn, n):
+        # the same timed blocks as the fused pipeline above (median block), so
+        # all three are compared at the same settled power state
         for _ in range(3):
             fn()
         torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        return a.elapsed_time(b) / n
+        return statistics.median(timed_blocks(fn, n, stream, dev, world, args.timed_seconds)) / n
 
     def unfused():
         lm.logits(ht, head, out=tl)

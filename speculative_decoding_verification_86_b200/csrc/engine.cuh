@@ -45,10 +45,10 @@ constexpr uint32_t kItemExit = 0xFFFFFFFFu;
 constexpr int kRowSeg = 0xFF;  // segment field of a STATS item that covers its whole row
 constexpr unsigned kSpinLimit = 1u << 24;  // polls of a queue slot before giving up (seconds)
 constexpr int kEngineMinBlocks = 4;  // 64 registers: four CTAs per SM (measured best)
-// Small, latency-bound batches run an instance with three CTAs per SM (80
-// registers, fewer spills on the serial decision paths; measured faster there,
-// slower for large batches).
-constexpr int kEngineMinBlocksSmall = 3;
+// Small, latency-bound batches run an instance with two CTAs per SM (128
+// registers: no spills on the serial decision paths; measured faster there than
+// three CTAs per SM at 80 registers, which in turn beat four at 64).
+constexpr int kEngineMinBlocksSmall = 2;
 // candidate keys of the batch-wide selection held in the staging buffer
 constexpr int kConfKeysInStage = 4096;
 static_assert(kMaxK * sizeof(double) + sizeof(ConfSelectShared) + kConfKeysInStage * sizeof(unsigned long long) <=

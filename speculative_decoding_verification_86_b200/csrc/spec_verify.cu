@@ -475,9 +475,10 @@ spec_status run_impl(spec_verify_ctx* c, const void* target, const void* draft, 
   if (n_init > 0xFFFF0000ull) return SPEC_ERR_INVALID_ARG;
   p.n_init = static_cast<unsigned>(n_init);
   timing_mark(c, kClassStats, true, s);
-  // a small dense batch (every item in the first wave) is latency bound:
-  // the instance with more registers per thread
-  const bool small = p.mode == sv::kModeDense && !p.whole_rows;
+  // a small dense batch (its items within two waves of that instance's grid)
+  // is latency bound: the instance with more registers per thread
+  const bool small = p.mode == sv::kModeDense && !p.whole_rows &&
+                     static_cast<int64_t>(B) * (2 * k + 1) * p.n_segs <= 2ll * c->engine_grid_small;
   if (small) {
     if (bf16) sv::k_engine<true, sv::kEngineMinBlocksSmall><<<c->engine_grid_small, sv::kThreads, sv::kStageBytes, s>>>(p);
     else sv::k_engine<false, sv::kEngineMinBlocksSmall><<<c->engine_grid_small, sv::kThreads, sv::kStageBytes, s>>>(p);
