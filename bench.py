@@ -646,7 +646,7 @@ def run_vocab_parallel(args):
 
 LM_METRIC = ("verified draft positions/s, verification fused into the shared LM head "
              "(B=256 k=5 V=151936 H=2560)")
-LM_LAUNCHES_PER_STEP = 12  # kernels spec_lmhead_verify launches
+LM_LAUNCHES_PER_STEP = 16  # kernels spec_lmhead_verify launches (no confidence head)
 
 
 def lm_config(w, n):
@@ -814,10 +814,21 @@ def run_lmhead(args):
         peak, peak_src = float(peaks["bf16_tflops"]), "measured burst (cuBLAS bf16)"
     else:
         peak, peak_src = 1590.0, "fallback"
+    import numpy as np
     rows = B * (2 * k + 1)
-    flops = 2.0 * rows * V * H
-    st_ms = ms_st / max(n_st, 1)
-    achieved = flops / (st_ms * 1e-3) / 1e12
+    flops = 2.0 * rows * V * H  # the whole head applied to every row: the unfused GEMM, cuBLAS
+    # the rows the prefix-ordered statistics passes computed: position 0 of every
+    # request, then the other rows of the requests that accepted position 0
+    acc = out["accepted"].cpu().numpy()
+    temp = w.get("temperature")
+    tn = temp.cpu().numpy() if temp is not None else np.ones(B)
+    vl = w.get("verify_len")
+    lv = np.clip(vl.cpu().numpy(), 0, k) if vl is not None else np.full(B, k)
+    cont = acc >= 1
+    rows_done = B * (2 if k > 0 else 1) + int(np.sum(np.where(tn[cont] == 0, lv[cont], 2 * lv[cont] - 1)))
+    flops_done = 2.0 * rows_done * V * H
+    st_ms = ms_st / max(len(block_ms) * args.steps, 1)  # both statistics launches of a step
+    achieved = flops_done / (st_ms * 1e-3) / 1e12
     line = {
         "metric": LM_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -830,7 +841,8 @@ def run_lmhead(args):
                                            if peaks and peaks.get("bf16_tflops_sustained") else None),
                      "traffic": profiled_traffic("k_lmhead", "lmhead_stats_pairs" if args.lm_cta_pairs == 1
                                                   else "lmhead_stats"),
-                     "flops_per_launch": flops, "launch_ms": st_ms, "launches_timed": n_st},
+                     "flops_per_step": flops_done, "rows_per_step": rows_done, "rows_all": rows,
+                     "ms_per_step": st_ms, "launches_timed": n_st},
         "timed_blocks": {"blocks": len(block_ms), "steps_per_block": args.steps,
                          "ms_per_block_min": min(block_ms), "ms_per_block_median": statistics.median(block_ms),
                          "ms_per_block_max": max(block_ms)},

@@ -103,8 +103,14 @@ struct LmParams {
   int mode;
   int H;
   int64_t V;
-  int rows0, rows1;       // rows of A matrix 0 (target) and 1 (drafter); rows mode: rows0 = max rows
-  const int* rows_dev;    // rows mode: the row count on the device (nullptr: rows0)
+  int rows0, rows1;       // rows of A matrix 0 (target) and 1 (drafter); with rows_dev: rows0 = max rows
+  const int* rows_dev;    // the row count of matrix 0 on the device (nullptr: rows0)
+  // statistics mode: which rows the matrices hold.  pos0: matrix 0 holds the
+  // target rows (i, 0) and matrix 1 the drafter rows (i, 0), i < B; row_map:
+  // matrix 0 row r is batch row row_map[r] (target rows [B, k+1] then drafter
+  // rows [B, k] numbered together); neither: the whole [B, k+1] and [B, k].
+  int pos0;
+  const int* row_map;
   // statistics mode
   int B, k;
   const int32_t* tokens;  // [B, k]
@@ -330,6 +336,7 @@ struct LmRowState {
   bool greedy = false;
   bool draft = false;
   int i = 0, j = 0;
+  int64_t g = 0;  // batch row: target rows [B, k+1], then drafter rows [B, k]
   int64_t tok = -1;
   float cc = 1.0f;
   SoftAcc acc;
@@ -338,30 +345,41 @@ struct LmRowState {
   int gbad = 0;
 };
 
-// Row of the batch (target rows, then the drafter's) held by TMEM lane
-// `r_in_unit` of M tile mt; false past the end of its matrix.
-__device__ __forceinline__ bool lm_row_of(const LmParams& p, int mt, int mt0, int rows_per_unit,
-                                          int r_in_unit, bool& draft, int& r) {
-  draft = mt >= mt0;
-  r = (draft ? mt - mt0 : mt) * rows_per_unit + r_in_unit;
-  return r < (draft ? p.rows1 : p.rows0);
+// The batch row held by TMEM lane `r_in_unit` of M tile mt (matrix 0 holds
+// rows0 rows, matrix 1 p.rows1): its request i, position j, whether it is the
+// drafter's, and its index g among the target rows [B, k+1] then the drafter
+// rows [B, k]; false past the end of its matrix.
+__device__ __forceinline__ bool lm_row_of(const LmParams& p, int rows0, int mt, int mt0,
+                                          int rows_per_unit, int r_in_unit, LmRowState& st) {
+  const bool m1 = mt >= mt0;
+  const int r = (m1 ? mt - mt0 : mt) * rows_per_unit + r_in_unit;
+  if (r >= (m1 ? p.rows1 : rows0)) return false;
+  const int64_t nt = static_cast<int64_t>(p.B) * (p.k + 1);
+  if (p.pos0) {
+    st.draft = m1;
+    st.i = r;
+    st.j = 0;
+    st.g = m1 ? nt + static_cast<int64_t>(r) * p.k : static_cast<int64_t>(r) * (p.k + 1);
+    return true;
+  }
+  const int64_t g = p.row_map ? __ldg(p.row_map + r) : (m1 ? nt + r : r);
+  st.g = g;
+  st.draft = g >= nt;
+  if (st.draft) {
+    st.i = static_cast<int>((g - nt) / p.k);
+    st.j = static_cast<int>(g - nt - static_cast<int64_t>(st.i) * p.k);
+  } else {
+    st.i = static_cast<int>(g / (p.k + 1));
+    st.j = static_cast<int>(g - static_cast<int64_t>(st.i) * (p.k + 1));
+  }
+  return true;
 }
 
-__device__ __forceinline__ void lm_row_init(const LmParams& p, int mt, int mt0, int rows_per_unit,
-                                            int r_in_unit, LmRowState& st) {
+__device__ __forceinline__ void lm_row_init(const LmParams& p, int rows0, int mt, int mt0,
+                                            int rows_per_unit, int r_in_unit, LmRowState& st) {
   st = LmRowState();
-  bool draft;
-  int r;
-  if (!lm_row_of(p, mt, mt0, rows_per_unit, r_in_unit, draft, r)) return;
+  if (!lm_row_of(p, rows0, mt, mt0, rows_per_unit, r_in_unit, st)) return;
   st.valid = true;
-  st.draft = draft;
-  if (draft) {
-    st.i = r / p.k;
-    st.j = r - st.i * p.k;
-  } else {
-    st.i = r / (p.k + 1);
-    st.j = r - st.i * (p.k + 1);
-  }
   if (st.j < p.k) st.tok = __ldg(p.tokens + static_cast<int64_t>(st.i) * p.k + st.j);
   float T = p.temp ? __ldg(p.temp + st.i) : 1.0f;
   if (!temperature_valid(T)) T = 1.0f;  // the chain reports the request; any record will do
@@ -414,13 +432,8 @@ __device__ __forceinline__ void lm_consume_stats(const LmParams& p, LmRowState& 
   soft_batch<false>(st.acc, v, st.cc);
 }
 
-__device__ __forceinline__ void lm_write_part(const LmParams& p, const LmRowState& st, int mt,
-                                              int mt0, int rows_per_unit, int r_in_unit,
-                                              int part) {
-  bool draft;
-  int r;
-  lm_row_of(p, mt, mt0, rows_per_unit, r_in_unit, draft, r);
-  const int64_t g = draft ? static_cast<int64_t>(p.rows0) + r : r;
+__device__ __forceinline__ void lm_write_part(const LmParams& p, const LmRowState& st, int part) {
+  const int64_t g = st.g;
   LmPart o;
   if (st.greedy) {
     o.K = 0.0f;
@@ -608,15 +621,11 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
     LmRowState st;
     int64_t dst = -1;
     if (p.mode == kLmModeStats) {
-      lm_row_init(p, mt, w.mt0, R, r_in_unit, st);
+      lm_row_init(p, sh.rows0, mt, w.mt0, R, r_in_unit, st);
       // Position 0 is the row a request samples from most often (a rejection
       // there, or the bonus row when nothing is verified): write its logits
       // now, so the row-writing pass only needs the rows of later positions.
-      if (p.out && st.valid && st.j == 0) {
-        const int64_t r = st.draft ? static_cast<int64_t>(p.rows0) + static_cast<int64_t>(st.i) * p.k
-                                   : static_cast<int64_t>(st.i) * (p.k + 1);
-        dst = r * p.V;
-      }
+      if (p.out && st.valid && st.j == 0) dst = st.g * p.V;
     } else {
       const int r = mt * R + r_in_unit;
       if (r < sh.rows0) dst = p.dst ? __ldg(p.dst + r) : static_cast<int64_t>(r) * p.V;
@@ -684,7 +693,7 @@ __device__ __forceinline__ void lm_epilogue(const LmParams& p, const LmWork<CG>&
       mbar_arrive(&sh.xempty[quarter]);
       if (st.valid) {
         lm_merge_half(st, o);
-        lm_write_part(p, st, mt, w.mt0, R, r_in_unit, w.part(u));
+        lm_write_part(p, st, w.part(u));
       }
     }
   }
@@ -720,7 +729,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     mbar_init(&sh.drain, 1);
     sh.abort = 0;
     int rows0 = p.rows0;
-    if (p.mode == kLmModeRows && p.rows_dev) rows0 = max(0, min(__ldcg(p.rows_dev), p.rows0));
+    if (p.rows_dev) rows0 = max(0, min(__ldcg(p.rows_dev), p.rows0));
     sh.rows0 = rows0;
     mbar_init_fence();
   }
@@ -778,8 +787,10 @@ __global__ void __launch_bounds__(kLmThreads, 1)
 // Merge the parts of every (request, row slot, statistics segment) into the
 // segment record the accept chain reads (the same merge as across a CTA's
 // threads: rebase to the largest frame, then add).
+// slot_sel: 0 every row, 1 the position-0 rows (slots 0 and k + 1) only, 2 the
+// others only (a pass that computed some of the rows leaves the rest alone).
 __global__ void k_lm_combine(RunParams p, const LmPart* parts, int n_parts, int parts_per_seg,
-                             int rows0) {
+                             int rows0, int slot_sel) {
   const int rows = 2 * p.k + 1;
   const int64_t n = static_cast<int64_t>(p.B) * rows * p.n_segs;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
@@ -788,6 +799,8 @@ __global__ void k_lm_combine(RunParams p, const LmPart* parts, int n_parts, int 
     const int64_t rs = e / p.n_segs;
     const int i = static_cast<int>(rs / rows);
     const int slot = static_cast<int>(rs - static_cast<int64_t>(i) * rows);
+    const bool pos0 = slot == 0 || slot == p.k + 1;
+    if ((slot_sel == 1 && !pos0) || (slot_sel == 2 && pos0)) continue;
     const int64_t g = slot <= p.k ? static_cast<int64_t>(i) * (p.k + 1) + slot
                                   : rows0 + static_cast<int64_t>(i) * p.k + (slot - p.k - 1);
     float T = p.temp ? __ldg(p.temp + i) : 1.0f;
@@ -847,6 +860,47 @@ __global__ void k_lm_combine(RunParams p, const LmPart* parts, int n_parts, int 
     r.arg = __float_as_int(om);
     p.meta[e] = r;
   }
+}
+
+// The prefix-ordered LM head, first decision: position 0 of every request,
+// from the statistics of its two position-0 rows (their fp32 logits are
+// written, so a decision inside its bound is settled exactly here).  A request
+// that accepts position 0 lists the rest of its rows -- target rows 1..L, and
+// drafter rows 1..L-1 for a sampled request -- as batch rows (target rows
+// [B, k+1], then drafter rows [B, k]) for the second statistics pass.
+// state[i]: 0 finished, 1 continues, 2 a sample job was written.
+__global__ void __launch_bounds__(kThreads) k_lm_decide0(RunParams p, int* state, int* count,
+                                                         int* src) {
+  __shared__ DecideShared dsh;
+  const int i = blockIdx.x;
+  if (threadIdx.x == 0) p.fallback[i] = 0;
+  sync_compute();
+  const ReqInfo ri = request_info(p, i);
+  decide_position<false>(p, i, ri, 0, dsh);
+  if (threadIdx.x == 0) {
+    const int st = dsh.state;
+    state[i] = st;
+    if (st == 1) {
+      const int L = ri.L;
+      const int n = ri.greedy ? L : 2 * L - 1;
+      const int at = atomicAdd(count, n);
+      const int nt = p.B * (p.k + 1);
+      int q = at;
+      for (int j = 1; j <= L; ++j) src[q++] = i * (p.k + 1) + j;
+      if (!ri.greedy)
+        for (int j = 1; j < L; ++j) src[q++] = nt + i * p.k + j;
+    }
+  }
+}
+
+// Second decision: the chains of the requests that accepted position 0,
+// walked from position 1 (a decision inside its bound marks the request for a
+// whole redo: those rows' logits were never written).
+__global__ void __launch_bounds__(kThreads) k_lm_decide_rest(RunParams p, const int* state) {
+  __shared__ DecideShared dsh;
+  const int i = blockIdx.x;
+  if (__ldcg(state + i) != 1) return;
+  decide_request<false>(p, i, request_info(p, i), dsh, 1);
 }
 
 // After the chain: the rows each request samples from (the rejected pair, or

@@ -20,6 +20,8 @@ struct spec_lmhead_ctx {
   int* src = nullptr;           // [max_rows]
   int64_t* dst = nullptr;       // [max_rows]
   int* count = nullptr;
+  int* rest_count = nullptr;  // rows of the second statistics pass (prefix-ordered verify)
+  int* state = nullptr;       // [max_batch]: each request's state after its position 0
   int32_t* votes = nullptr;     // [max_batch]
   unsigned* error = nullptr;
   int cta_pairs = 2;            // spec_lmhead_set_cta_pairs: 0 never, 1 always, 2 row GEMM only
@@ -49,12 +51,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // Row-major bf16 matrix [rows, H] as 2-D tiles of box_rows x 64 (128 bytes,
-// the 128-byte swizzle); out-of-range rows and columns read as zero.
-bool bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int H, int box_rows) {
+// the 128-byte swizzle); out-of-range rows and columns read as zero.  Rows are
+// row_stride elements apart (0: H; a multiple of 8, so 16-byte aligned).
+bool bf16_tile_map(CUtensorMap* m, const void* base, int64_t rows, int H, int box_rows,
+                   int64_t row_stride = 0) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc || rows < 1) return false;
+  if (row_stride == 0) row_stride = H;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 2};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride) * 2};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(sv::kLmBK), static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -165,6 +170,8 @@ spec_status spec_lmhead_init(spec_lmhead_ctx** out, spec_verify_ctx* vctx, int m
   const size_t o_src = take(R * sizeof(int));
   const size_t o_dst = take(R * sizeof(int64_t));
   const size_t o_cnt = take(sizeof(int));
+  const size_t o_rcnt = take(sizeof(int));
+  const size_t o_state = take(static_cast<size_t>(vctx->max_batch) * sizeof(int));
   const size_t o_votes = take(static_cast<size_t>(vctx->max_batch) * sizeof(int32_t));
   const size_t o_err = take(sizeof(unsigned));
   if (cudaMalloc(&lm->ws, off) != cudaSuccess) {
@@ -179,6 +186,8 @@ spec_status spec_lmhead_init(spec_lmhead_ctx** out, spec_verify_ctx* vctx, int m
   lm->src = reinterpret_cast<int*>(b + o_src);
   lm->dst = reinterpret_cast<int64_t*>(b + o_dst);
   lm->count = reinterpret_cast<int*>(b + o_cnt);
+  lm->rest_count = reinterpret_cast<int*>(b + o_rcnt);
+  lm->state = reinterpret_cast<int*>(b + o_state);
   lm->votes = reinterpret_cast<int32_t*>(b + o_votes);
   lm->error = reinterpret_cast<unsigned*>(b + o_err);
   if (cudaMemset(lm->ws, 0, off) != cudaSuccess ||
@@ -274,12 +283,9 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   DeviceGuard g(ctx->device);
   if (!g.ok) return SPEC_ERR_CUDA;
   cudaGetLastError();
-  CUtensorMap ma0, ma1, mc;
-  if (!bf16_tile_map(&ma0, hidden_target, rows0, H, sv::kLmBM) ||
-      (rows1 > 0 && !bf16_tile_map(&ma1, hidden_draft, rows1, H, sv::kLmBM)) ||
-      !bf16_tile_map(&mc, lm->hc, static_cast<int64_t>(B) * rows, H, sv::kLmBM))
+  CUtensorMap mc;  // the gathered hidden rows
+  if (!bf16_tile_map(&mc, lm->hc, static_cast<int64_t>(B) * rows, H, sv::kLmBM))
     return SPEC_ERR_UNSUPPORTED;
-  if (rows1 == 0) ma1 = ma0;
   p.rows_whole = 1;  // sampled rows are materialised in full before the sample phases
   p.seed = seed;
   p.step = step;
@@ -290,40 +296,83 @@ spec_status spec_lmhead_verify(spec_lmhead_ctx* lm, const void* hidden_target,
   p.out_q = out_q;
   p.out_status = out_status;
   const int cg1 = stats_cta_group(lm), cg2 = rows_cta_group(lm);
-  const int n_mt1 = lm_mtiles(rows0, rows1, cg1);
-  const int part_tiles = lm_stats_part_tiles(n_mt1, V, ctx->num_sms / cg1);
-  const int n_parts = lm_parts(V, part_tiles);
   if (conf) launch_conf(ctx, conf, B, k, verify_len, ctx->conf_len, nullptr, stream);
   if (k > 0 && cudaMemsetAsync(ctx->tok_logits, 0, static_cast<size_t>(B) * k * 2 * sizeof(float),
                                stream) != cudaSuccess)
     return SPEC_ERR_CUDA;
-  if (cudaMemsetAsync(lm->count, 0, sizeof(int), stream) != cudaSuccess) return SPEC_ERR_CUDA;
+  if (cudaMemsetAsync(lm->count, 0, sizeof(int), stream) != cudaSuccess ||
+      cudaMemsetAsync(lm->rest_count, 0, sizeof(int), stream) != cudaSuccess)
+    return SPEC_ERR_CUDA;
 
-  // 1. statistics of every verified row, straight from the accumulators
+  // Prefix order, as in the verification of logits: position 0 first, then
+  // the other rows of the requests that accepted it (most requests stop at
+  // position 0, so most rows are never computed).
+  //
+  // 1. position 0 of every request: the statistics of its two rows, read in
+  //    place (rows (k+1) H and k H elements apart); their logits are written
   sv::LmParams lp{};
   lp.mode = sv::kLmModeStats;
   lp.H = H;
   lp.V = V;
-  lp.rows0 = rows0;
-  lp.rows1 = rows1;
   lp.B = B;
   lp.k = k;
   lp.tokens = draft_tokens;
   lp.temp = temperature;
   lp.parts = lm->parts;
-  lp.n_parts = n_parts;
-  lp.part_tiles = part_tiles;
   lp.tok_logits = ctx->tok_logits;
-  lp.out = lm->rows;  // position-0 rows are written by this pass
   lp.error = lm->error;
-  if (spec_status st = lm_launch(lm, cg1, ma0, ma1, head, H, V, lp, n_mt1, kClassLmStats, stream);
-      st != SPEC_OK)
-    return st;
-  sv::k_lm_combine<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
-      p, lm->parts, n_parts, sv::kLmSegTiles / part_tiles, rows0);
+  {
+    const int r1 = (rows1 > 0 && k > 0) ? B : 0;
+    CUtensorMap mp0, mp1;
+    if (!bf16_tile_map(&mp0, hidden_target, B, H, sv::kLmBM, static_cast<int64_t>(k + 1) * H) ||
+        (r1 > 0 && !bf16_tile_map(&mp1, hidden_draft, B, H, sv::kLmBM, static_cast<int64_t>(k) * H)))
+      return SPEC_ERR_UNSUPPORTED;
+    if (r1 == 0) mp1 = mp0;
+    const int n_mt = lm_mtiles(B, r1, cg1);
+    const int part_tiles = lm_stats_part_tiles(n_mt, V, ctx->num_sms / cg1);
+    const int n_parts = lm_parts(V, part_tiles);
+    lp.rows0 = B;
+    lp.rows1 = r1;
+    lp.pos0 = 1;
+    lp.n_parts = n_parts;
+    lp.part_tiles = part_tiles;
+    lp.out = lm->rows;  // position-0 rows: the rows most requests sample from
+    if (spec_status st = lm_launch(lm, cg1, mp0, mp1, head, H, V, lp, n_mt, kClassLmStats, stream);
+        st != SPEC_OK)
+      return st;
+    sv::k_lm_combine<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
+        p, lm->parts, n_parts, sv::kLmSegTiles / part_tiles, rows0, 1);
+  }
+  sv::k_lm_decide0<<<B, sv::kThreads, 0, stream>>>(p, lm->state, lm->rest_count, lm->src);
 
-  // 2. the accept chains (every request, dense order)
-  sv::k_shard_decide<false><<<B, sv::kThreads, 0, stream>>>(p);
+  // 2. the other rows of the requests that accepted position 0: gathered, then
+  //    one statistics pass over them (its row count is on the device), and
+  //    their chains walked from position 1
+  if (k > 0) {
+    const int max_rest = B * 2 * k;
+    sv::k_lm_gather<<<grid_for(static_cast<int64_t>(max_rest) * (H / 8)), 256, 0, stream>>>(
+        lm->rest_count, lm->src, static_cast<const uint4*>(hidden_target),
+        static_cast<const uint4*>(hidden_draft ? hidden_draft : hidden_target), rows0, H, max_rest,
+        lm->hc);
+    const int n_mt = lm_mtiles(max_rest, 0, cg1);
+    const int part_tiles = lm_stats_part_tiles(n_mt, V, ctx->num_sms / cg1);
+    const int n_parts = lm_parts(V, part_tiles);
+    sv::LmParams lq = lp;
+    lq.rows0 = max_rest;
+    lq.rows1 = 0;
+    lq.rows_dev = lm->rest_count;
+    lq.pos0 = 0;
+    lq.row_map = lm->src;
+    lq.n_parts = n_parts;
+    lq.part_tiles = part_tiles;
+    lq.out = nullptr;  // no position-0 rows in this pass
+    if (spec_status st = lm_launch(lm, cg1, mc, mc, head, H, V, lq, n_mt, kClassLmStats, stream);
+        st != SPEC_OK)
+      return st;
+    sv::k_lm_combine<<<grid_for(static_cast<int64_t>(B) * rows * p.n_segs), 256, 0, stream>>>(
+        p, lm->parts, n_parts, sv::kLmSegTiles / part_tiles, rows0, 2);
+    sv::k_lm_decide_rest<<<B, sv::kThreads, 0, stream>>>(p, lm->state);
+  }
 
   // 3. logits of the rows each request samples from
   sv::k_lm_rowlist<<<grid_for(B), 256, 0, stream>>>(p, lm->count, lm->src, lm->dst);
