@@ -361,16 +361,18 @@ double spec_verify_ex2_error_bound(void);
  * of logits.  The GEMM runs on the tensor cores (tcgen05, bf16 operands, fp32
  * accumulation); the logits are the fp32 accumulator values.
  *
- * spec_lmhead_verify computes exactly what spec_verify_run (dtype SPEC_F32,
- * dense order) computes on the logits [B, k+1, V] = hidden_target W^T and
- * [B, k, V] = hidden_draft W^T, without writing most of those logits: the
- * GEMM's epilogue reduces each accumulator tile to the row statistics, picks
- * the drafted tokens' logits and writes only the position-0 rows (the rows a
- * request samples from most often); after the accept chains a second pass
- * writes the other rows a request samples from (the rejected pair, or the
- * bonus row), as fp32 logits, and the sample is drawn from them with the
- * vocabulary-parallel protocol's phases run as a single shard.  Outputs and random draws are those
- * of spec_verify_run.
+ * spec_lmhead_verify computes exactly what spec_verify_run (dtype SPEC_F32)
+ * computes on the logits [B, k+1, V] = hidden_target W^T and [B, k, V] =
+ * hidden_draft W^T, without computing or writing most of those logits.  In
+ * prefix order: the GEMM over position 0's two rows of every request, whose
+ * epilogue reduces each accumulator tile to the row statistics, picks the
+ * drafted tokens' logits and writes these rows (the rows a request samples
+ * from most often); the decision of position 0; then the GEMM over the other
+ * rows of the requests that accepted it, and their chains.  A last pass writes
+ * the other rows a request samples from (the rejected pair, or the bonus row)
+ * as fp32 logits, and the sample is drawn from them with the
+ * vocabulary-parallel protocol's phases run as a single shard.  Outputs and
+ * random draws are those of spec_verify_run.
  * --------------------------------------------------------------------------- */
 typedef struct spec_lmhead_ctx spec_lmhead_ctx;
 

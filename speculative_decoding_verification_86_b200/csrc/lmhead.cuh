@@ -7,9 +7,12 @@
 // only their softmax statistics and one logit (the drafted token's), so the
 // GEMM's epilogue reduces each accumulator tile straight into the statistics
 // records the accept chain merges; of all the logits only the position-0 rows
-// reach HBM (the rows most requests sample from).  The other rows a request
-// samples from (a later rejected pair, or the bonus row) are produced as
-// logits by the same kernel in its row-writing mode, after the chain decided.
+// reach HBM (the rows most requests sample from).  The statistics run in
+// prefix order: position 0's rows of every request first, then, once position
+// 0 is decided, the other rows of the requests that accepted it.  The other
+// rows a request samples from (a later rejected pair, or the bonus row) are
+// produced as logits by the same kernel in its row-writing mode, after the
+// chain decided.
 //
 // Kernel: one CTA per SM, persistent over work units (128 rows x a run of
 // 128 x 256 tiles along the vocabulary), or -- the CTA-pair form -- clusters of
