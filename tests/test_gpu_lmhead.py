@@ -133,6 +133,42 @@ def test_fused_verify_grid_vs_oracle(lm, B, k, V, H, mixed):
     assert (g_out["redo"] == 0).all() or (g_out["redo"] == 1).sum() <= 1
 
 
+def test_fused_every_request_continues_past_position_0(lm):
+    """The drafter's hidden states are the target's: p = q at every position,
+    so every sampled request accepts its whole block, and greedy requests
+    whose drafted tokens are the target's lowest arg-max accept too: the second
+    statistics pass gets every remaining row (its largest row count)."""
+    _, h = lm
+    B, k, V, H = 24, 4, 20000, 128
+    temps = _temps(B, 11)
+    w = workloads.lmhead("cuda", seed=12, B=B, k=k, V=V, H=H, grid=True, temperature=temps)
+    w["hidden_draft"] = w["hidden_target"][:, :k].contiguous()
+    t = w["hidden_target"][:, :k].float() @ w["head"].float().T  # exact on the grid
+    greedy = temps == 0
+    w["tokens"] = torch.where(greedy[:, None], t.argmax(dim=2).to(torch.int32), w["tokens"]).contiguous()
+    g_out = _run_fused(h, w)
+    o = _run_oracle(w)
+    compare(g_out, o)
+    assert (g_out["accepted"] == k).all()
+
+
+def test_fused_every_request_stops_at_position_0(lm):
+    """Greedy requests whose drafted tokens are never the target's arg-max:
+    every request stops at position 0, and the second statistics pass runs
+    with no rows."""
+    _, h = lm
+    B, k, V, H = 16, 3, 4100, 64
+    w = workloads.lmhead("cuda", seed=13, B=B, k=k, V=V, H=H, grid=True,
+                         temperature=torch.zeros(B, device="cuda"))
+    t = w["hidden_target"][:, :k].float() @ w["head"].float().T  # exact on the grid
+    top = t.argmax(dim=2)
+    w["tokens"] = ((top + 1) % V).to(torch.int32).contiguous()
+    g_out = _run_fused(h, w)
+    o = _run_oracle(w)
+    compare(g_out, o)
+    assert (g_out["accepted"] == 0).all()
+
+
 def test_fused_matches_unfused_real_valued(lm):
     """Real-valued inputs: the fused path decides as the verifier does on the
     same GEMM's logits (decisions are certified, so summation order inside the
